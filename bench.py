@@ -1,0 +1,440 @@
+"""Benchmark: MXFP4 quantize+pack throughput on one or more B200s.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl mx|reference]
+    python -m torch.distributed.run --nproc-per-node N --master-addr 127.0.0.1 \
+        --master-port P bench.py --gpus N --steps K --warmup W
+
+One step = one MXFP4 (E2M1 elements, E8M0 scales) FLOOR quantize+pack of the
+MoE w13 expert stack [128, 1536, 2048] bf16 (N(0, 0.02^2) times a per-expert
+U(0.5, 2) factor, seeded, generated on the device): 805,306,368 input bytes,
+201,326,592 code bytes and 12,582,912 scale bytes. GB/s counts those
+algorithmic bytes (bf16 in + packed out). The input is far larger than L2
+(126 MB), so no flush is needed between steps. With N ranks every rank
+quantizes its own stack (weak scaling: rows are independent, there is no
+data exchange); the step time is the maximum over ranks.
+
+The JSON line also carries: the roofline of the kernel (CUDA-event duration of
+each launch inside the timed region against the measured HBM copy bandwidth),
+the end-to-end figure through the public API with host buffers (pinned input
+copied in, outputs copied out, inside the timed region), the oracle timed on
+the host cores on a bounded sample (`cpu_baseline`), SM clocks sampled with
+nvidia-smi during the timed region, and per-op figures for the other
+workloads (`ops`).
+
+--impl reference times the CPU oracle (the only other implementation of this
+path) on the same workload, a bounded sample per step, and prints the same
+line with "impl": "reference".
+"""
+
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import re
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "MXFP4 quantize+pack GB/s (bf16 in + packed out) and % of B200 HBM peak"
+WORKLOAD = "moe_w13 [128,1536,2048] bf16 -> MXFP4 (E2M1 codes [128,1536,1024] + E8M0 scales [128,1536,64]), FLOOR scaling"
+EXPERTS, INTER2, HIDDEN = 128, 1536, 2048
+N_ELEM = EXPERTS * INTER2 * HIDDEN
+BYTES_IN = 2 * N_ELEM
+BYTES_CODES = N_ELEM // 2
+BYTES_SCALES = N_ELEM // 32
+BYTES_STEP = BYTES_IN + BYTES_CODES + BYTES_SCALES            # 1,019,215,872
+FALLBACK_HBM_GBS = 6650.0
+KERNEL_SOURCES = ["fp8_quantization_mx_b200/csrc/mx_kernels.cu",
+                  "fp8_quantization_mx_b200/csrc/mx_device.cuh"]
+PROFILE = os.path.join(ROOT, "profiles", "quantize_fp4_floor_moe_w13.md")
+
+
+# ------------------------------------------------------------------ helpers --
+
+def kernel_source_hash() -> str:
+    h = hashlib.sha256()
+    for p in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, p), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def measured_peak():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured (MEASURED_PEAKS.json hbm_gbs, copy burst)"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def profiled_traffic():
+    """DRAM bytes per launch recorded by ncu for the timed kernel, if current."""
+    try:
+        text = open(PROFILE).read()
+    except OSError:
+        return None, "no profile"
+    t = re.search(r"traffic_bytes_per_launch:\s*([0-9]+)", text)
+    h = re.search(r"kernel_source_sha256_16:\s*([0-9a-f]+)", text)
+    if not t or not h:
+        return None, "profile lacks figures"
+    if h.group(1) != kernel_source_hash():
+        return None, "kernel changed since the capture"
+    return int(t.group(1)), "ncu dram__bytes_read.sum + dram__bytes_write.sum"
+
+
+class ClockSampler:
+    """nvidia-smi clocks/throttle reasons sampled while the timed region runs."""
+
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int, period_ms: int = 50):
+        self.index = index
+        self.period_ms = period_ms
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.QUERY}",
+                 "--format=csv,noheader,nounits", "-lms", str(self.period_ms)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+            time.sleep(0.3)
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            time.sleep(0.2)
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            f = [p.strip() for p in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                mx = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": [], "samples": 0}
+        sm.sort()
+        return {"sm_mhz": sm[len(sm) // 2], "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def oracle_baseline(x_host_rows, budget_s: float = 10.0):
+    """Times the CPU oracle on a bounded sample of the workload (rows of 2048)."""
+    import oracle
+    threads = len(os.sched_getaffinity(0))
+    oracle.set_threads(threads)
+    probe = x_host_rows[:256]
+    t0 = time.perf_counter()
+    oracle.quantize(probe, 0, 0)
+    rate = probe.shape[0] / max(time.perf_counter() - t0, 1e-6)        # rows per s
+    nrows = int(min(x_host_rows.shape[0], max(256, rate * budget_s)))
+    sample = x_host_rows[:nrows]
+    t0 = time.perf_counter()
+    oracle.quantize(sample, 0, 0)
+    dt = time.perf_counter() - t0
+    nbytes = sample.size * 2 + sample.size // 2 + sample.size // 32
+    return {"value": nbytes / dt / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
+            "sample": f"first {nrows} of {x_host_rows.shape[0]} rows of 2048 ({sample.size} elements), "
+                      f"{dt:.2f} s on {threads} threads, scalar C++ oracle"}
+
+
+# --------------------------------------------------------------- arms --
+
+def run_reference(args):
+    """The oracle on the host cores, one bounded sample of the workload per step."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    import numpy as np
+    import torch
+    import oracle
+    from fp8_quantization_mx_b200 import inputs
+    threads = len(os.sched_getaffinity(0))
+    oracle.set_threads(threads)
+    # a few experts of the same seeded stack, generated on the host
+    x = inputs.moe_w13(experts=4, device="cpu")
+    xb = inputs.bf16_bits_numpy(x).reshape(-1, HIDDEN)
+    t0 = time.perf_counter()
+    oracle.quantize(xb[:512], 0, 0)
+    rate = 512 / max(time.perf_counter() - t0, 1e-6)
+    budget = max(0.5, min(5.0, 120.0 / max(1, args.steps + args.warmup)))
+    nrows = int(min(xb.shape[0], max(64, rate * budget)))
+    sample = np.ascontiguousarray(xb[:nrows])
+    for _ in range(args.warmup):
+        oracle.quantize(sample, 0, 0)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.quantize(sample, 0, 0)
+    dt = (time.perf_counter() - t0) / args.steps
+    nbytes = sample.size * 2 + sample.size // 2 + sample.size // 32
+    value = nbytes / dt / 1e9
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": dt * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "sample_rows": nrows, "rows_total": EXPERTS * INTER2},
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": threads, "kind": "oracle",
+                         "sample": f"{nrows} rows of 2048 ({sample.size} elements) per step"},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def time_op(fn, reps, flush=None, stream=None):
+    """Mean kernel time (ms) of fn() over reps, CUDA events on the launching stream."""
+    import torch
+    stream = stream or torch.cuda.current_stream()
+    times = []
+    for _ in range(reps):
+        if flush is not None:
+            flush.zero_()
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record(stream)
+        fn()
+        e.record(stream)
+        e.synchronize()
+        times.append(s.elapsed_time(e))
+    times.sort()
+    return times[len(times) // 2]
+
+
+def other_ops(mx, inputs, dev, reps=10):
+    """GB/s of the other ops on their workloads (median of reps; L2 flushed before each)."""
+    import torch
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+    res = {}
+
+    def rec(name, nbytes, fn):
+        fn()
+        torch.cuda.synchronize()
+        ms = time_op(fn, reps, flush)
+        res[name] = {"ms": round(ms, 4), "GB/s": round(nbytes / ms / 1e6, 1)}
+
+    x1 = inputs.outlier_act(device=dev)
+    n1 = x1.numel()
+    c, s, _ = mx.quantize(x1)
+    rec("outlier_act_256x4096/fp4_floor_quantize", 2 * n1 + n1 // 2 + n1 // 32, lambda: mx.quantize(x1, out=(c, s, None)))
+    y1 = torch.empty_like(x1)
+    rec("outlier_act_256x4096/fp4_dequantize_bf16", 2 * n1 + n1 // 2 + n1 // 32,
+        lambda: mx.dequantize(c, s, None, out=y1))
+    del x1, y1
+    x2 = inputs.mlp_weight(device=dev)
+    n2 = x2.numel()
+    c2, s2, _ = mx.quantize(x2, mx.E4M3)
+    rec("mlp_weight_8192x3072/fp8_floor_quantize", 2 * n2 + n2 + n2 // 32,
+        lambda: mx.quantize(x2, mx.E4M3, out=(c2, s2, None)))
+    y2 = torch.empty_like(x2)
+    rec("mlp_weight_8192x3072/fp8_dequantize_bf16", 2 * n2 + n2 + n2 // 32,
+        lambda: mx.dequantize(c2, s2, None, mx.E4M3, out=y2))
+    del x2, y2, c2, s2
+    for name, gen in (("qat_act_16384x3072", inputs.qat_act), ("qat_weight_8192x3072", inputs.qat_weight)):
+        x3 = gen(device=dev)
+        n3 = x3.numel()
+        g3 = inputs.qat_grad(*x3.shape, device=dev)
+        y3 = torch.empty_like(x3)
+        rec(f"{name}/fp4_fake_quant_fwd", 4 * n3, lambda: mx.fake_quant(x3, out=y3))
+        rec(f"{name}/fp4_fake_quant_bwd", 6 * n3, lambda: mx.fake_quant_bwd(x3, g3, out=y3))
+        del x3, g3, y3
+    x4 = inputs.heavy_tail(device=dev)
+    n4 = x4.numel()
+    modes = [("FLOOR", 0), ("CEIL", 1), ("OAS_RULE", 2), ("OAS", 3), ("MBS_STATIC", 16),
+             ("MBS_DYNAMIC", 32), ("OAS+MBS_STATIC", 19), ("OAS+MBS_DYNAMIC", 35)]
+    for mname, m in modes:
+        bufs = mx.quantize(x4, mx.E2M1, m)
+        extra = n4 // 128 if m >> 4 else 0
+        rec(f"heavy_tail_8192x4096/fp4_{mname}_quantize", 2 * n4 + n4 // 2 + n4 // 32 + extra,
+            lambda: mx.quantize(x4, mx.E2M1, m, out=bufs))
+        _, tot = mx.block_error(x4, mx.E2M1, m, per_block=False)
+        rec(f"heavy_tail_8192x4096/fp4_{mname}_block_error", 2 * n4,
+            lambda: mx.block_error(x4, mx.E2M1, m, per_block=False))
+        t = tot.cpu().tolist()
+        res[f"heavy_tail_8192x4096/fp4_{mname}_block_error"].update(
+            {"mse": t[0] / n4, "sqnr_db": (10 * __import__("math").log10(t[1] / t[0])) if t[0] > 0 else None})
+    del x4
+    return res
+
+
+def run_mx(args):
+    import torch
+    import torch.distributed as dist
+
+    import fp8_quantization_mx_b200 as mx
+    from fp8_quantization_mx_b200 import build as mxbuild
+    from fp8_quantization_mx_b200 import inputs
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    if rank == 0:
+        mxbuild.build()
+    if world > 1:
+        dist.barrier()
+    mx.load_library()
+
+    # each rank quantizes its own stack (weak scaling, no exchange)
+    x = inputs.moe_w13(seed=4 + 1000 * rank, device=dev).view(-1, HIDDEN)
+    codes = torch.empty(x.shape[0], HIDDEN // 2, dtype=torch.uint8, device=dev)
+    scales = torch.empty(x.shape[0], HIDDEN // 32, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    rows, cols = x.shape
+    sh = stream.cuda_stream
+    xp, cp, sp = x.data_ptr(), codes.data_ptr(), scales.data_ptr()
+
+    def step():
+        st = mx.mx_quantize(xp, rows, cols, mx.E2M1, mx.FLOOR, cp, sp, None, sh)
+        if st != 0:
+            raise mx.MXError(st, "mx_quantize")
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clocks:
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        t_start.record(stream)
+        for s, e in ev:
+            s.record(stream)
+            step()
+            e.record(stream)
+        t_end.record(stream)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+    total_ms = t_start.elapsed_time(t_end)
+    launch_ms = sum(s.elapsed_time(e) for s, e in ev) / len(ev)
+    if world > 1:
+        t = torch.tensor([total_ms, launch_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        total_ms, launch_ms = t.tolist()
+    ms_per_step = total_ms / args.steps
+    value = world * BYTES_STEP / (ms_per_step * 1e-3) / 1e9
+
+    # end to end through the public API with host buffers (pinned in, pinned out)
+    xh = x.cpu().pin_memory()
+    e2e_steps = max(3, min(args.steps, 10))
+    mx.quantize(xh)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(e2e_steps):
+        hc, hs, _ = mx.quantize(xh)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / e2e_steps
+    if world > 1:
+        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        e2e_ms = t.item()
+    e2e = {"value": world * BYTES_STEP / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+           "h2d_bytes_per_step": BYTES_IN, "d2h_bytes_per_step": BYTES_CODES + BYTES_SCALES,
+           "ms_per_step": e2e_ms}
+    del xh, hc, hs
+
+    ops = None
+    if not args.no_ops and rank == 0:
+        ops = other_ops(mx, inputs, dev)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = oracle_baseline(inputs.bf16_bits_numpy(x[: 16 * INTER2]).reshape(-1, HIDDEN))
+
+    peak, peak_src = measured_peak()
+    achieved = BYTES_STEP / (launch_ms * 1e-3) / 1e9
+    traffic, traffic_src = profiled_traffic()
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": ms_per_step,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f32", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "elements_per_gpu": N_ELEM,
+                       "bytes_per_step_per_gpu": BYTES_STEP,
+                       "l2": "input (805 MB) larger than L2 (126 MB); no flush between steps",
+                       "parallelism": f"weak: {world} independent stacks, no data exchange"},
+            "elements_per_s": world * N_ELEM / (ms_per_step * 1e-3),
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "peak_source": peak_src,
+                         "frac_of_8000": achieved / 8000.0, "traffic": traffic,
+                         "traffic_source": traffic_src, "kernel": "stream_kernel<quantize, E2M1, FLOOR>",
+                         "launch_ms": launch_ms},
+            "e2e": e2e,
+            "gpu_launches": args.steps,
+            "clocks": clocks.summary(),
+        }
+        if cpu is not None:
+            line["cpu_baseline"] = cpu
+        if ops is not None:
+            line["ops"] = ops
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__, formatter_class=argparse.RawDescriptionHelpFormatter)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["mx", "reference"], default="mx")
+    ap.add_argument("--no-ops", action="store_true", help="skip the per-op figures")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_mx(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

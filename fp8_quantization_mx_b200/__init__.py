@@ -1,0 +1,280 @@
+"""B200-native OCP Microscaling (MX) block-32 quantization.
+
+A thin Python binding over ``libmx.so`` (C ABI in ``include/mx.h``): argument
+marshalling only. Every step of quantize / dequantize / fake-quant / error runs
+in the library's sm_100a kernels; PyTorch provides device memory and streams.
+There is no CPU fallback: without the built library, or on a machine whose
+tensors are not on a CUDA device, the calls raise.
+
+Two layers, both exported here:
+
+* ``mx_quantize``, ``mx_dequantize``, ``mx_fake_quant_fwd``,
+  ``mx_fake_quant_bwd``, ``mx_block_error``, ``mx_status_string``: the C
+  functions with their C names and arguments (raw pointers as ints, stream as
+  an int handle), returning the status code.
+* ``quantize``, ``dequantize``, ``fake_quant``, ``fake_quant_bwd``,
+  ``block_error``: tensor-level calls that check tensors, allocate outputs
+  with torch on the input's device, launch on the current CUDA stream and
+  raise ``MXError`` on a nonzero status. ``quantize`` and ``dequantize`` also
+  take CPU tensors: the binding then copies the input to the GPU, launches,
+  and copies the outputs back (pinned host memory makes those copies async).
+* ``MXFakeQuantize``: an autograd function (forward fake-quant, straight-
+  through backward) for quantization-aware training of activations and
+  weights alike.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+__all__ = [
+    "E2M1", "E4M3", "FLOOR", "CEIL", "OAS_RULE", "OAS", "MBS_STATIC", "MBS_DYNAMIC",
+    "MXError", "library_path", "load_library",
+    "mx_quantize", "mx_dequantize", "mx_fake_quant_fwd", "mx_fake_quant_bwd",
+    "mx_block_error", "mx_status_string", "mx_version",
+    "quantize", "dequantize", "fake_quant", "fake_quant_bwd", "block_error", "MXFakeQuantize",
+    "MXFP4_FORMAT", "MXFP8_FORMAT",
+]
+
+# formats (mx_format_t)
+E2M1 = 0
+E4M3 = 1
+MXFP4_FORMAT = E2M1
+MXFP8_FORMAT = E4M3
+# scaling (mx_scaling_t)
+FLOOR, CEIL, OAS_RULE, OAS = 0, 1, 2, 3
+MBS_STATIC, MBS_DYNAMIC = 1 << 4, 2 << 4
+
+_STATUS = {0: "MX_OK", 1: "MX_ERR_INVALID_ARG", 2: "MX_ERR_SHAPE", 3: "MX_ERR_ALIGN",
+           4: "MX_ERR_UNSUPPORTED", 5: "MX_ERR_CUDA"}
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_lib = None
+
+
+class MXError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {_STATUS.get(status, status)} ({mx_status_string(status)})")
+
+
+def library_path() -> str:
+    return os.path.join(_HERE, "libmx.so")
+
+
+def load_library():
+    """Loads libmx.so (raises if it has not been built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    path = library_path()
+    if not os.path.exists(path):
+        raise RuntimeError(f"{path} is missing: build it with `python -m fp8_quantization_mx_b200.build`")
+    lib = ctypes.CDLL(path)
+    vp, i64, c_int = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int
+    lib.mx_quantize.argtypes = [vp, i64, i64, c_int, c_int, vp, vp, vp, vp]
+    lib.mx_dequantize.argtypes = [vp, vp, vp, i64, i64, c_int, c_int, vp, vp]
+    lib.mx_fake_quant_fwd.argtypes = [vp, i64, i64, c_int, c_int, vp, vp, vp]
+    lib.mx_fake_quant_bwd.argtypes = [vp, vp, i64, i64, c_int, c_int, vp, vp]
+    lib.mx_block_error.argtypes = [vp, i64, i64, c_int, c_int, vp, vp, vp]
+    for f in ("mx_quantize", "mx_dequantize", "mx_fake_quant_fwd", "mx_fake_quant_bwd",
+              "mx_block_error"):
+        getattr(lib, f).restype = c_int
+    lib.mx_status_string.argtypes = [c_int]
+    lib.mx_status_string.restype = ctypes.c_char_p
+    lib.mx_version.restype = c_int
+    _lib = lib
+    return lib
+
+
+# ---------------------------------------------------------------- C layer --
+
+def mx_quantize(x, rows, cols, format, scaling, codes, scales, macro, stream=0) -> int:
+    return load_library().mx_quantize(x, rows, cols, format, scaling, codes, scales, macro, stream)
+
+
+def mx_dequantize(codes, scales, macro, rows, cols, format, out_fp32, out, stream=0) -> int:
+    return load_library().mx_dequantize(codes, scales, macro, rows, cols, format, out_fp32, out,
+                                        stream)
+
+
+def mx_fake_quant_fwd(x, rows, cols, format, scaling, y, scales_out, stream=0) -> int:
+    return load_library().mx_fake_quant_fwd(x, rows, cols, format, scaling, y, scales_out, stream)
+
+
+def mx_fake_quant_bwd(x, grad_y, rows, cols, format, scaling, grad_x, stream=0) -> int:
+    return load_library().mx_fake_quant_bwd(x, grad_y, rows, cols, format, scaling, grad_x, stream)
+
+
+def mx_block_error(x, rows, cols, format, scaling, block_sse, totals, stream=0) -> int:
+    return load_library().mx_block_error(x, rows, cols, format, scaling, block_sse, totals, stream)
+
+
+def mx_status_string(status: int) -> str:
+    return load_library().mx_status_string(int(status)).decode()
+
+
+def mx_version() -> int:
+    return load_library().mx_version()
+
+
+# ----------------------------------------------------------- tensor layer --
+
+def _ptr(t):
+    return None if t is None else t.data_ptr()
+
+
+def _stream(device) -> int:
+    return torch.cuda.current_stream(device).cuda_stream
+
+
+def _check(status: int, where: str):
+    if status != 0:
+        raise MXError(status, where)
+
+
+def _rows_cols(x: torch.Tensor):
+    if x.dim() == 0:
+        raise ValueError("expected at least a 1-D tensor")
+    cols = x.shape[-1]
+    rows = x.numel() // cols if cols else 0
+    return rows, cols
+
+
+def _cuda_bf16(x: torch.Tensor, name: str):
+    if not x.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if x.dtype != torch.bfloat16:
+        raise ValueError(f"{name} must be bfloat16, got {x.dtype}")
+    if not x.is_contiguous():
+        raise ValueError(f"{name} must be contiguous (row-major)")
+
+
+def quantize(x: torch.Tensor, format: int = E2M1, scaling: int = FLOOR, out=None):
+    """MX-quantizes bf16 ``x`` [..., cols] along its last dimension.
+
+    Returns ``(codes, scales, macro)``: codes uint8 [..., cols/2] (MXFP4, two
+    codes per byte, even element in the low nibble) or [..., cols] (MXFP8,
+    E4M3 bytes); scales uint8 [..., cols/32] (E8M0); macro uint8 [..., cols/128]
+    with Macro Block Scaling, else None. ``out`` may supply the three buffers.
+    A CPU ``x`` is copied to the current GPU and the outputs come back to the
+    CPU (pinned when ``x`` is pinned).
+    """
+    if not x.is_cuda:
+        dev = torch.device("cuda", torch.cuda.current_device())
+        xd = x.to(dev, non_blocking=x.is_pinned())
+        res = quantize(xd, format, scaling)
+        return tuple(None if t is None else _to_host(t, x.is_pinned()) for t in res)
+    _cuda_bf16(x, "x")
+    rows, cols = _rows_cols(x)
+    lead = x.shape[:-1]
+    mbs = (scaling >> 4) != 0
+    if out is None:
+        ccols = cols // 2 if format == E2M1 else cols
+        codes = torch.empty(*lead, ccols, dtype=torch.uint8, device=x.device)
+        scales = torch.empty(*lead, cols // 32, dtype=torch.uint8, device=x.device)
+        macro = torch.empty(*lead, cols // 128, dtype=torch.uint8, device=x.device) if mbs else None
+    else:
+        codes, scales, macro = out
+    with torch.cuda.device(x.device):
+        _check(mx_quantize(_ptr(x), rows, cols, format, scaling, _ptr(codes), _ptr(scales),
+                           _ptr(macro), _stream(x.device)), "mx_quantize")
+    return codes, scales, macro
+
+
+def _to_host(t: torch.Tensor, pinned: bool) -> torch.Tensor:
+    if pinned:
+        h = torch.empty(t.shape, dtype=t.dtype, pin_memory=True)
+        h.copy_(t, non_blocking=True)
+        return h
+    return t.cpu()
+
+
+def dequantize(codes: torch.Tensor, scales: torch.Tensor, macro=None, format: int = E2M1,
+               out_dtype=torch.bfloat16, out=None):
+    """Inverse of ``quantize``: value(code) * f * 2^(scale - 127) as bf16 or fp32."""
+    if not codes.is_cuda:
+        dev = torch.device("cuda", torch.cuda.current_device())
+        pinned = codes.is_pinned()
+        args = [None if t is None else t.to(dev, non_blocking=pinned) for t in (codes, scales, macro)]
+        return _to_host(dequantize(*args, format=format, out_dtype=out_dtype), pinned)
+    if codes.dtype != torch.uint8 or scales.dtype != torch.uint8:
+        raise ValueError("codes and scales must be uint8")
+    cols = codes.shape[-1] * 2 if format == E2M1 else codes.shape[-1]
+    rows = codes.numel() * (2 if format == E2M1 else 1) // cols if cols else 0
+    if out_dtype not in (torch.bfloat16, torch.float32):
+        raise ValueError("out_dtype must be bfloat16 or float32")
+    if out is None:
+        out = torch.empty(*codes.shape[:-1], cols, dtype=out_dtype, device=codes.device)
+    with torch.cuda.device(codes.device):
+        _check(mx_dequantize(_ptr(codes), _ptr(scales), _ptr(macro), rows, cols, format,
+                             int(out_dtype == torch.float32), _ptr(out), _stream(codes.device)),
+               "mx_dequantize")
+    return out
+
+
+def fake_quant(x: torch.Tensor, format: int = E2M1, scaling: int = FLOOR, out=None,
+               return_scales: bool = False):
+    """QAT forward: dequantize(quantize(x)) in one kernel, bf16 out."""
+    _cuda_bf16(x, "x")
+    rows, cols = _rows_cols(x)
+    y = torch.empty_like(x) if out is None else out
+    scales = (torch.empty(*x.shape[:-1], cols // 32, dtype=torch.uint8, device=x.device)
+              if return_scales else None)
+    with torch.cuda.device(x.device):
+        _check(mx_fake_quant_fwd(_ptr(x), rows, cols, format, scaling, _ptr(y), _ptr(scales),
+                                 _stream(x.device)), "mx_fake_quant_fwd")
+    return (y, scales) if return_scales else y
+
+
+def fake_quant_bwd(x: torch.Tensor, grad_y: torch.Tensor, format: int = E2M1,
+                   scaling: int = FLOOR, out=None):
+    """Straight-through backward: grad_y where |x| <= maxv * X, else 0."""
+    _cuda_bf16(x, "x")
+    _cuda_bf16(grad_y, "grad_y")
+    if grad_y.shape != x.shape:
+        raise ValueError("grad_y must have the shape of x")
+    rows, cols = _rows_cols(x)
+    gx = torch.empty_like(x) if out is None else out
+    with torch.cuda.device(x.device):
+        _check(mx_fake_quant_bwd(_ptr(x), _ptr(grad_y), rows, cols, format, scaling, _ptr(gx),
+                                 _stream(x.device)), "mx_fake_quant_bwd")
+    return gx
+
+
+def block_error(x: torch.Tensor, format: int = E2M1, scaling: int = FLOOR,
+                per_block: bool = True):
+    """Returns (block_sse float32 [..., cols/32] or None, totals float64 [2]).
+
+    totals = {sum (x - y)^2, sum x^2} with y the exact dequantized value;
+    MSE = totals[0] / numel, SQNR = 10 log10(totals[1] / totals[0]).
+    """
+    _cuda_bf16(x, "x")
+    rows, cols = _rows_cols(x)
+    bs = (torch.empty(*x.shape[:-1], cols // 32, dtype=torch.float32, device=x.device)
+          if per_block else None)
+    totals = torch.empty(2, dtype=torch.float64, device=x.device)
+    with torch.cuda.device(x.device):
+        _check(mx_block_error(_ptr(x), rows, cols, format, scaling, _ptr(bs), _ptr(totals),
+                              _stream(x.device)), "mx_block_error")
+    return bs, totals
+
+
+class MXFakeQuantize(torch.autograd.Function):
+    """y = fake_quant(x) with the straight-through gradient of the forward's mask."""
+
+    @staticmethod
+    def forward(ctx, x, format=E2M1, scaling=FLOOR):
+        ctx.save_for_backward(x)
+        ctx.format = format
+        ctx.scaling = scaling
+        return fake_quant(x.contiguous(), format, scaling)
+
+    @staticmethod
+    def backward(ctx, grad_y):
+        (x,) = ctx.saved_tensors
+        gx = fake_quant_bwd(x.contiguous(), grad_y.contiguous(), ctx.format, ctx.scaling)
+        return gx, None, None

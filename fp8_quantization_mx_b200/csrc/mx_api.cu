@@ -1,0 +1,140 @@
+// C entry points of libmx.so (declared in include/mx.h): argument checks on
+// the host, then one launch on the caller's stream. Nothing is allocated and
+// no state is kept between calls.
+//
+// The checks restate the sources' interface: block size 32 or an error
+// ("[Axolotl] MXFP4 quantization support", 2: a ValueError unless the block
+// size is 32), contiguous row-major input with the block along the last
+// dimension ("[vLLM] MXFP8/MXFP4", MXFP8 block-32 scaling), dynamic scaling
+// only (scales always come from the live tensor; there is no static-scale
+// argument), packed FP4 with the last dimension halved ("[vLLM]", MXFP4).
+
+#include <cstdint>
+
+#include "mx.h"
+#include "mx_launch.h"
+
+namespace {
+
+// Largest element count accepted: keeps every byte offset far inside int64.
+constexpr int64_t kMaxElems = int64_t(1) << 40;
+
+bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+int check_shape(int64_t rows, int64_t cols, bool mbs) {
+  if (rows < 0 || cols < 0) return MX_ERR_INVALID_ARG;
+  if (cols % 32 != 0) return MX_ERR_SHAPE;
+  if (mbs && cols % 128 != 0) return MX_ERR_SHAPE;
+  if (rows > 0 && cols > 0 && rows > kMaxElems / cols) return MX_ERR_INVALID_ARG;
+  return MX_OK;
+}
+
+// Format and scaling combinations the kernels implement.
+int check_mode(int format, int scaling) {
+  if (format != MX_FMT_E2M1 && format != MX_FMT_E4M3) return MX_ERR_UNSUPPORTED;
+  if (scaling < 0 || (scaling & ~0x3F) != 0) return MX_ERR_UNSUPPORTED;
+  const int rule = scaling & 0xF;
+  const int mbs = scaling >> 4;
+  if (rule > MX_SCALE_OAS || mbs > 2) return MX_ERR_UNSUPPORTED;
+  if (format == MX_FMT_E4M3 && (rule == MX_SCALE_OAS_RULE || rule == MX_SCALE_OAS || mbs != 0))
+    return MX_ERR_UNSUPPORTED;
+  if (mbs != 0 && rule != MX_SCALE_FLOOR && rule != MX_SCALE_OAS) return MX_ERR_UNSUPPORTED;
+  return MX_OK;
+}
+
+int from_cuda(cudaError_t e) { return e == cudaSuccess ? MX_OK : MX_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+int mx_version(void) { return (1 << 16) | 0; }
+
+const char* mx_status_string(int status) {
+  switch (status) {
+    case MX_OK: return "ok";
+    case MX_ERR_INVALID_ARG: return "invalid argument (null pointer or bad shape)";
+    case MX_ERR_SHAPE: return "cols must be a multiple of 32 (of 128 with macro block scaling)";
+    case MX_ERR_ALIGN: return "pointer is not aligned as required";
+    case MX_ERR_UNSUPPORTED: return "unsupported format / scaling combination";
+    case MX_ERR_CUDA: return "CUDA launch or stream operation failed";
+    default: return "unknown status";
+  }
+}
+
+int mx_quantize(const void* x, int64_t rows, int64_t cols, int format, int scaling, void* codes,
+                uint8_t* scales, uint8_t* macro, void* stream) {
+  int st = check_mode(format, scaling);
+  if (st != MX_OK) return st;
+  const bool mbs = (scaling >> 4) != 0;
+  st = check_shape(rows, cols, mbs);
+  if (st != MX_OK) return st;
+  const int64_t n = rows * cols;
+  if (n == 0) return MX_OK;
+  if (!x || !codes || !scales || (mbs && !macro)) return MX_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(codes, 16)) return MX_ERR_ALIGN;
+  return from_cuda(mxk::launch_quantize(x, n, format, scaling, codes, scales, mbs ? macro : nullptr,
+                                        static_cast<cudaStream_t>(stream)));
+}
+
+int mx_dequantize(const void* codes, const uint8_t* scales, const uint8_t* macro, int64_t rows,
+                  int64_t cols, int format, int out_fp32, void* out, void* stream) {
+  if (format != MX_FMT_E2M1 && format != MX_FMT_E4M3) return MX_ERR_UNSUPPORTED;
+  if (format == MX_FMT_E4M3 && macro) return MX_ERR_UNSUPPORTED;
+  if (out_fp32 != 0 && out_fp32 != 1) return MX_ERR_INVALID_ARG;
+  int st = check_shape(rows, cols, macro != nullptr);
+  if (st != MX_OK) return st;
+  const int64_t n = rows * cols;
+  if (n == 0) return MX_OK;
+  if (!codes || !scales || !out) return MX_ERR_INVALID_ARG;
+  if (!aligned(codes, 16) || !aligned(out, 16)) return MX_ERR_ALIGN;
+  return from_cuda(mxk::launch_dequantize(codes, scales, macro, n, format, out_fp32, out,
+                                          static_cast<cudaStream_t>(stream)));
+}
+
+int mx_fake_quant_fwd(const void* x, int64_t rows, int64_t cols, int format, int scaling, void* y,
+                      uint8_t* scales_out, void* stream) {
+  int st = check_mode(format, scaling);
+  if (st != MX_OK) return st;
+  st = check_shape(rows, cols, (scaling >> 4) != 0);
+  if (st != MX_OK) return st;
+  const int64_t n = rows * cols;
+  if (n == 0) return MX_OK;
+  if (!x || !y) return MX_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(y, 16)) return MX_ERR_ALIGN;
+  return from_cuda(mxk::launch_fake_fwd(x, n, format, scaling, y, scales_out,
+                                        static_cast<cudaStream_t>(stream)));
+}
+
+int mx_fake_quant_bwd(const void* x, const void* grad_y, int64_t rows, int64_t cols, int format,
+                      int scaling, void* grad_x, void* stream) {
+  int st = check_mode(format, scaling);
+  if (st != MX_OK) return st;
+  st = check_shape(rows, cols, (scaling >> 4) != 0);
+  if (st != MX_OK) return st;
+  const int64_t n = rows * cols;
+  if (n == 0) return MX_OK;
+  if (!x || !grad_y || !grad_x) return MX_ERR_INVALID_ARG;
+  if (!aligned(x, 16) || !aligned(grad_y, 16) || !aligned(grad_x, 16)) return MX_ERR_ALIGN;
+  return from_cuda(mxk::launch_fake_bwd(x, grad_y, n, format, scaling, grad_x,
+                                        static_cast<cudaStream_t>(stream)));
+}
+
+int mx_block_error(const void* x, int64_t rows, int64_t cols, int format, int scaling,
+                   float* block_sse, double* totals, void* stream) {
+  int st = check_mode(format, scaling);
+  if (st != MX_OK) return st;
+  st = check_shape(rows, cols, (scaling >> 4) != 0);
+  if (st != MX_OK) return st;
+  if (!totals) return MX_ERR_INVALID_ARG;
+  if (!aligned(totals, 8)) return MX_ERR_ALIGN;
+  const int64_t n = rows * cols;
+  if (n != 0) {
+    if (!x) return MX_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || (block_sse && !aligned(block_sse, 4))) return MX_ERR_ALIGN;
+  }
+  return from_cuda(mxk::launch_block_error(x, n, format, scaling, block_sse, totals,
+                                           static_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

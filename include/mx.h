@@ -1,0 +1,144 @@
+/*
+ * mx.h — C ABI of libmx.so: OCP Microscaling (MX) block-32 quantization of
+ * bf16 tensors on NVIDIA B200 (sm_100a).
+ *
+ * Sources restated (page titles; sections in brackets):
+ *  [AX] "[Axolotl] MXFP4 quantization support" (PR #3375 analysis) [2: config,
+ *       block_size must be 32 else ValueError; torch.float4_e2m1fn_x2 packs two
+ *       E2M1 codes per byte] [3: activation and weight share one fake-quantizer].
+ *  [VL] "[vLLM] MXFP8/MXFP4: microscaling format quantization" [MXFP8: block-32
+ *       scaling: contiguous weight -> (fp8 elements, uint8 scales), dynamic
+ *       scheme only] [MXFP4: uint8 storage, two FP4 values per byte, last dim
+ *       halved] [MX format table: E2M1 / E4M3 elements, E8M0 scale, block 32,
+ *       one scale byte per 32 elements].
+ *  [UP] "Unveiling the Potential of Quantization with MXFP4: Strategies for
+ *       Quantization Error Reduction" [technical summary 1: E8M0 = 2^k only]
+ *       [2.A Overflow-Aware Scaling] [2.B Macro Block Scaling] [3-4: QSNR].
+ *
+ * Layout (every call): x is row-major contiguous [rows, cols] bf16, cols a
+ * multiple of 32; block b of row r is elements [32b, 32b+32) of that row.
+ * A 3-D tensor [E, R, C] is passed as rows = E*R, cols = C.
+ *   codes  MXFP4: uint8 [rows, cols/2], element 2j in the low nibble and 2j+1
+ *                 in the high nibble of byte j; bit 3 of a nibble is the sign.
+ *          MXFP8: uint8 [rows, cols], one E4M3 ("fn": no Inf, S.1111.111 = NaN).
+ *   scales uint8 [rows, cols/32], E8M0: byte s means 2^(s-127); 255 is NaN.
+ *   macro  uint8 [rows, cols/128] (MBS only): k, the macro factor f = 1 + k/256
+ *          of the 128-element macro block [128m, 128m+128) of the row.
+ *
+ * Ownership: the caller allocates and owns every buffer (device memory unless
+ * stated). The library allocates nothing and keeps no state between calls.
+ * Streams: every call enqueues its kernels on `stream` (a cudaStream_t passed
+ * as void*; NULL = the legacy default stream) and returns without waiting.
+ * Errors: arguments are checked on the host before anything is enqueued; on
+ * any error nothing is launched and no output is written. A failed launch
+ * returns MX_ERR_CUDA. Faults inside a kernel surface at the caller's next
+ * synchronisation, as usual for CUDA. Kernels never trap, assert or wait on
+ * flags. All entry points are thread-safe.
+ * Empty inputs (rows == 0 or cols == 0) are valid and launch nothing (except
+ * that mx_block_error still zeroes its totals).
+ * Alignment: x, grad, y, out and codes pointers must be 16-byte aligned;
+ * block_sse 4-byte, totals 8-byte; scales and macro have no requirement.
+ */
+#ifndef MX_H_
+#define MX_H_
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Element formats ([VL] MX format table). */
+typedef enum {
+  MX_FMT_E2M1 = 0, /* MXFP4: magnitudes {0, .5, 1, 1.5, 2, 3, 4, 6} ([UP] 2.A: max 6.0) */
+  MX_FMT_E4M3 = 1  /* MXFP8: E4M3fn, max 448 */
+} mx_format_t;
+
+/* Scale selection. Low 4 bits: the base rule; bits 4-5: Macro Block Scaling.
+ * emax is the exponent of the element's largest value (2 for E2M1, 8 for E4M3)
+ * and e = floor(log2 amax) of the block. Every rule clamps E to [-127, 127];
+ * an all-zero block gets E = -127 (byte 0); a block holding NaN or Inf gets
+ * byte 255 and element codes that keep only the sign (E4M3: S.1111.111). */
+typedef enum {
+  /* OCP rule 2^(e - emax): amax lands in [4, 8) (E2M1) or [256, 512) (E4M3);
+   * values above the largest element saturate. FP4 and FP8. */
+  MX_SCALE_FLOOR = 0,
+  /* [UP] 2.A's "existing" scale: the smallest 2^E with amax <= maxv * 2^E
+   * (no element saturates). FP4 and FP8. */
+  MX_SCALE_CEIL = 1,
+  /* [UP] 2.A as a rule on the mantissa bits: under the no-overflow scale a
+   * block max in (3.0, 3.5] of the 6.0 range is mapped to (6.0, 7.0] instead,
+   * i.e. E = e - 2 when the amax significand is at most 1.75, else e - 1. FP4. */
+  MX_SCALE_OAS_RULE = 2,
+  /* Overflow-Aware Scaling as a per-block minimum-SSE choice between the
+   * FLOOR exponent and FLOOR + 1 (exact comparison; a tie keeps FLOOR). FP4. */
+  MX_SCALE_OAS = 3,
+  /* [UP] 2.B Macro Block Scaling, OR-able with MX_SCALE_FLOOR or MX_SCALE_OAS;
+   * FP4 only; cols must be a multiple of 128. Each 128-element macro block
+   * gets a factor f = 1 + k/256 (k stored in `macro`); each 32-block inside it
+   * takes its exponent from floor(log2(amax / f)) and its elements are rounded
+   * as x / (f * 2^E). STATIC: the smallest k that maps the macro-block max to
+   * at most 6. DYNAMIC: the k in 0..255 with the smallest macro-block SSE
+   * (double, summed in element order; a tie keeps the smaller k). */
+  MX_MBS_STATIC = 1 << 4,
+  MX_MBS_DYNAMIC = 2 << 4
+} mx_scaling_t;
+
+typedef enum {
+  MX_OK = 0,
+  MX_ERR_INVALID_ARG = 1, /* NULL required pointer, negative or oversized shape */
+  MX_ERR_SHAPE = 2,       /* cols % 32 != 0, or cols % 128 != 0 with MBS ([AX] 2) */
+  MX_ERR_ALIGN = 3,       /* a pointer below its stated alignment */
+  MX_ERR_UNSUPPORTED = 4, /* unknown format/scaling, or a scaling the format lacks */
+  MX_ERR_CUDA = 5         /* a kernel launch or stream operation failed */
+} mx_status_t;
+
+/* Quantize ([VL] MXFP8/MXFP4 sections; [UP] 2.A/2.B for the scaling modes).
+ * x: device bf16 [rows, cols]. codes: device, FP4 rows*cols/2 bytes or FP8
+ * rows*cols bytes. scales: device uint8 [rows, cols/32]. macro: device uint8
+ * [rows, cols/128] when scaling has an MBS bit (required then), else ignored
+ * and may be NULL. Elements: round to nearest, ties to the even code, values
+ * past the largest magnitude saturate, the sign is kept (small negatives -> -0). */
+int mx_quantize(const void* x, int64_t rows, int64_t cols, int format, int scaling,
+                void* codes, uint8_t* scales, uint8_t* macro, void* stream);
+
+/* Dequantize: out = value(code) * f * 2^(scale - 127), f = 1 + k/256 from
+ * `macro` (NULL means f = 1). out_fp32 = 0: bf16 (rounded to nearest even;
+ * exact for FP4 without MBS); 1: float (exact). A scale byte of 255 or an
+ * E4M3 NaN code gives the canonical NaN (0x7FC0 / 0x7FC00000). */
+int mx_dequantize(const void* codes, const uint8_t* scales, const uint8_t* macro,
+                  int64_t rows, int64_t cols, int format, int out_fp32, void* out,
+                  void* stream);
+
+/* QAT fake-quantization forward ([AX] 2-3): y = dequantize(quantize(x)) as
+ * bf16, in one pass. scales_out (nullable): the E8M0 bytes, as mx_quantize. */
+int mx_fake_quant_fwd(const void* x, int64_t rows, int64_t cols, int format, int scaling,
+                      void* y, uint8_t* scales_out, void* stream);
+
+/* Straight-through backward of the fake-quantizer: grad_x = grad_y where
+ * |x| <= maxv * X (X = f * 2^E, the scale the forward uses for that block;
+ * inclusive), else +0. NaN x, and every element of a NaN/Inf block, give +0.
+ * The grad_y bits pass unchanged. */
+int mx_fake_quant_bwd(const void* x, const void* grad_y, int64_t rows, int64_t cols,
+                      int format, int scaling, void* grad_x, void* stream);
+
+/* Quantization error ([UP] 3-4, QSNR): d = x - y with y the exact dequantized
+ * value (float, not rounded to bf16) under `scaling`. block_sse (nullable):
+ * device float [rows, cols/32], the per-block sum of d^2. totals: device
+ * double[2] = {sum d^2, sum x^2}; the call zeroes it on the stream first and
+ * then accumulates (atomically: the last bits may vary run to run). MSE =
+ * totals[0] / (rows*cols); SQNR dB = 10 log10(totals[1] / totals[0]). */
+int mx_block_error(const void* x, int64_t rows, int64_t cols, int format, int scaling,
+                   float* block_sse, double* totals, void* stream);
+
+/* Static description of a status code (never NULL). */
+const char* mx_status_string(int status);
+
+/* Library ABI version, (major << 16) | minor. */
+int mx_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MX_H_ */

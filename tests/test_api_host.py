@@ -1,0 +1,120 @@
+"""The C ABI on a host without a GPU: the library loads, exports every symbol
+include/mx.h declares, and rejects bad arguments before touching CUDA.
+
+Every call here fails validation (or is empty) and returns before any CUDA
+call, so no kernel is launched; the fake device addresses are never
+dereferenced.
+"""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "mx.h")
+
+OK, INVALID, SHAPE, ALIGN, UNSUPPORTED, CUDA_ERR = 0, 1, 2, 3, 4, 5
+A = 0x10000          # a 16-byte aligned fake device address (never dereferenced)
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(mx_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for n in ("mx_quantize", "mx_dequantize", "mx_fake_quant_fwd", "mx_fake_quant_bwd",
+              "mx_block_error", "mx_status_string", "mx_version"):
+        assert n in names
+
+
+def test_library_exports_every_declared_symbol(mx):
+    lib = ctypes.CDLL(mx.library_path())
+    for name in declared_functions():
+        assert hasattr(lib, name), name
+
+
+def test_status_strings(mx):
+    for s in range(6):
+        assert mx.mx_status_string(s)
+    assert mx.mx_status_string(99) == "unknown status"
+    assert mx.mx_version() >> 16 == 1
+
+
+def test_product_does_not_use_the_oracle():
+    """The package neither imports the oracle nor includes or loads its code."""
+    pkg = os.path.join(ROOT, "fp8_quantization_mx_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            path = os.path.join(dirpath, f)
+            if f.endswith(".py"):
+                text = open(path).read()
+                assert not re.search(r"^\s*(import|from)\s+oracle\b", text, re.M), f
+                assert "libmx_oracle" not in text and "mx_oracle" not in text, f
+            if f.endswith((".cu", ".cuh", ".h", ".cpp")):
+                text = open(path).read()
+                assert "oracle" not in text, f
+
+
+@pytest.mark.parametrize("fmt,scaling,status", [
+    (2, 0, UNSUPPORTED), (0, 4, UNSUPPORTED), (0, 0x30, UNSUPPORTED), (0, 0x40, UNSUPPORTED),
+    (1, 2, UNSUPPORTED), (1, 3, UNSUPPORTED), (1, 0x10, UNSUPPORTED), (0, 0x11, UNSUPPORTED),
+    (0, 0x12, UNSUPPORTED), (-1, 0, UNSUPPORTED), (0, -1, UNSUPPORTED),
+])
+def test_quantize_rejects_modes(mx, fmt, scaling, status):
+    assert mx.mx_quantize(A, 4, 128, fmt, scaling, A, A, A, 0) == status
+
+
+def test_quantize_rejects_shapes_and_pointers(mx):
+    q = mx.mx_quantize
+    assert q(A, 4, 33, 0, 0, A, A, None, 0) == SHAPE
+    assert q(A, 4, 96, 0, 0x10, A, A, A, 0) == SHAPE        # MBS needs cols % 128
+    assert q(A, -1, 32, 0, 0, A, A, None, 0) == INVALID
+    assert q(A, 4, -32, 0, 0, A, A, None, 0) == INVALID
+    assert q(A, 1 << 40, 1 << 10, 0, 0, A, A, None, 0) == INVALID   # too many elements
+    assert q(None, 4, 32, 0, 0, A, A, None, 0) == INVALID
+    assert q(A, 4, 32, 0, 0, None, A, None, 0) == INVALID
+    assert q(A, 4, 32, 0, 0, A, None, None, 0) == INVALID
+    assert q(A, 4, 128, 0, 0x10, A, A, None, 0) == INVALID   # MBS needs macro
+    assert q(A + 8, 4, 32, 0, 0, A, A, None, 0) == ALIGN
+    assert q(A, 4, 32, 0, 0, A + 4, A, None, 0) == ALIGN
+    # scales and macro may sit at any byte address: this one only fails on x
+    assert q(A + 2, 4, 128, 0, 0x10, A, A + 1, A + 3, 0) == ALIGN
+    # empty inputs are valid and launch nothing (pointers are not needed)
+    assert q(None, 0, 32, 0, 0, None, None, None, 0) == OK
+    assert q(None, 5, 0, 0, 0, None, None, None, 0) == OK
+
+
+def test_other_entry_points_validate(mx):
+    assert mx.mx_dequantize(A, A, None, 4, 33, 0, 0, A, 0) == SHAPE
+    assert mx.mx_dequantize(A, A, A, 4, 96, 0, 0, A, 0) == SHAPE
+    assert mx.mx_dequantize(A, A, A, 4, 128, 1, 0, A, 0) == UNSUPPORTED   # FP8 has no MBS
+    assert mx.mx_dequantize(A, A, None, 4, 32, 0, 2, A, 0) == INVALID
+    assert mx.mx_dequantize(A, A, None, 4, 32, 3, 0, A, 0) == UNSUPPORTED
+    assert mx.mx_dequantize(A + 8, A, None, 4, 32, 0, 0, A, 0) == ALIGN
+    assert mx.mx_dequantize(A, None, None, 4, 32, 0, 0, A, 0) == INVALID
+    assert mx.mx_dequantize(None, None, None, 0, 32, 0, 0, None, 0) == OK
+    assert mx.mx_fake_quant_fwd(A, 4, 32, 1, 3, A, None, 0) == UNSUPPORTED
+    assert mx.mx_fake_quant_fwd(A, 4, 48, 0, 0, A, None, 0) == SHAPE
+    assert mx.mx_fake_quant_fwd(A, 4, 32, 0, 0, None, None, 0) == INVALID
+    assert mx.mx_fake_quant_fwd(A, 4, 32, 0, 0, A + 8, None, 0) == ALIGN
+    assert mx.mx_fake_quant_bwd(A, A, 4, 32, 0, 0, A + 8, 0) == ALIGN
+    assert mx.mx_fake_quant_bwd(A, None, 4, 32, 0, 0, A, 0) == INVALID
+    assert mx.mx_fake_quant_bwd(A, A, 4, 64, 0, 0x20, A, 0) == SHAPE
+    assert mx.mx_block_error(A, 4, 32, 0, 0, None, None, 0) == INVALID
+    assert mx.mx_block_error(A, 4, 32, 0, 0, None, A + 4, 0) == ALIGN
+    assert mx.mx_block_error(A, 4, 32, 0, 0, A + 2, A, 0) == ALIGN
+    assert mx.mx_block_error(A, 4, 32, 1, 0x20, None, A, 0) == UNSUPPORTED
+
+
+def test_binding_refuses_cpu_tensors_for_device_only_calls(mx):
+    import torch
+    x = torch.zeros(2, 32, dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        mx.fake_quant(x)
+    with pytest.raises(ValueError):
+        mx.block_error(x)

@@ -1,0 +1,365 @@
+"""GPU parity: the CUDA path (through the C ABI) against the CPU oracle.
+
+Codes, scale bytes, macro bytes, dequantized bf16/float bits and straight-
+through gradients must be bit-identical; error statistics agree within a
+relative 1e-6 (the kernel sums per-block squares in double and atomically adds
+per-CTA double partials, the oracle sums sequentially in double). Inputs are
+seeded and synthetic (fp8_quantization_mx_b200.inputs); at the full workload
+sizes the oracle checks sampled rows and properties that hold at any size.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+from fp8_quantization_mx_b200 import inputs
+
+pytestmark = pytest.mark.gpu
+
+E2M1, E4M3 = 0, 1
+FLOOR, CEIL, OAS_RULE, OAS = 0, 1, 2, 3
+MBS_STATIC, MBS_DYNAMIC = 16, 32
+FP4_MODES = [FLOOR, CEIL, OAS_RULE, OAS, MBS_STATIC, MBS_DYNAMIC, OAS | MBS_STATIC, OAS | MBS_DYNAMIC]
+FP8_MODES = [FLOOR, CEIL]
+ALL = [(E2M1, m) for m in FP4_MODES] + [(E4M3, m) for m in FP8_MODES]
+REL = 1e-6
+
+
+def ids(fm):
+    fmt, m = fm
+    names = {0: "FLOOR", 1: "CEIL", 2: "OAS_RULE", 3: "OAS"}
+    s = names[m & 15]
+    if m >> 4:
+        s += "+MBS_" + ("STATIC" if m >> 4 == 1 else "DYNAMIC")
+    return ("fp4-" if fmt == 0 else "fp8-") + s
+
+
+def bits(t):
+    return inputs.bf16_bits_numpy(t)
+
+
+def host_u8(t):
+    return t.detach().cpu().numpy()
+
+
+def from_bits(b, device):
+    return torch.from_numpy(np.ascontiguousarray(b).view(np.int16)).view(torch.bfloat16).to(device)
+
+
+# ------------------------------------------------------------ small inputs --
+
+def special_blocks():
+    """Blocks with zeros, signed zeros, NaN, Inf, subnormals, extremes and ties."""
+    rows = []
+    z = np.zeros(32, np.uint16)
+    rows.append(z.copy())
+    b = z.copy(); b[3] = 0x8000; rows.append(b)                       # -0
+    b = z.copy(); b[0] = 0x7FC0; b[1] = 0x3F80; b[2] = 0xC000; rows.append(b)   # NaN
+    b = z.copy(); b[5] = 0xFF80; b[6] = 0x4000; rows.append(b)         # -Inf
+    b = z.copy(); b[0] = 0x7F80; rows.append(b)                        # +Inf
+    b = np.arange(1, 33, dtype=np.uint16); rows.append(b)              # subnormals only
+    b = (np.arange(32, dtype=np.uint16) + 0x8001); rows.append(b)      # negative subnormals
+    b = z.copy(); b[0] = 0x7F7F; b[1:] = 0x0001; rows.append(b)        # max bf16 with tiny tail
+    b = z.copy(); b[0] = 0x0080; b[1] = 0x0040; rows.append(b)         # smallest normal amax
+    ties = np.array([4.0, .25, .75, 1.25, 1.75, 2.5, 3.5, 5.0, -0.125, 7.0, 6.0, 3.0], np.float32)
+    b = z.copy(); b[:12] = torch.from_numpy(ties).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    rows.append(b)
+    for e in (-126, -100, -3, 0, 5, 60, 120, 125):
+        v = np.full(32, 2.0 ** e, np.float32) * np.linspace(-7.5, 7.5, 32, dtype=np.float32)
+        rows.append(torch.from_numpy(v).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16))
+    arr = np.stack(rows)
+    # pad to a whole number of 128-element macro rows
+    pad = (-len(arr)) % 4
+    arr = np.concatenate([arr, np.zeros((pad, 32), np.uint16)])
+    return arr.reshape(-1, 128)
+
+
+SMALL = {
+    "outlier_act_256x4096": lambda: inputs.outlier_act(),
+    "random_bits_3x160": lambda: inputs.random_bf16_bits((3, 160), seed=5),
+    "random_bits_1x32": lambda: inputs.random_bf16_bits((1, 32), seed=6),
+    "random_bits_5x96": lambda: inputs.random_bf16_bits((5, 96), seed=7),
+    "random_bits_7x384": lambda: inputs.random_bf16_bits((7, 384), seed=8),
+    "random_bits_33x1280": lambda: inputs.random_bf16_bits((33, 1280), seed=9),
+    "heavy_tail_64x4096": lambda: inputs.heavy_tail(rows=64),
+    "moe_4x1536x2048_head": lambda: inputs.moe_w13(experts=2, inter2=48),
+    "special_blocks": lambda: torch.from_numpy(special_blocks().view(np.int16)).view(torch.bfloat16),
+}
+
+
+def usable(name, fmt, m, x):
+    cols = x.shape[-1]
+    return not (m >> 4 and cols % 128)
+
+
+@pytest.mark.parametrize("fm", ALL, ids=ids)
+@pytest.mark.parametrize("name", list(SMALL))
+def test_quantize_parity(mx, oracle_mod, cuda, name, fm):
+    fmt, m = fm
+    x = SMALL[name]()
+    if not usable(name, fmt, m, x):
+        pytest.skip("MBS needs cols % 128 == 0")
+    c, s, mac = mx.quantize(x.to(cuda), fmt, m)
+    torch.cuda.synchronize()
+    oc, os_, omac = oracle_mod.quantize(bits(x), fmt, m)
+    assert np.array_equal(host_u8(s), os_), "scale bytes"
+    assert np.array_equal(host_u8(c), oc), "codes"
+    if m >> 4:
+        assert np.array_equal(host_u8(mac), omac), "macro factors"
+
+
+@pytest.mark.parametrize("fm", ALL, ids=ids)
+@pytest.mark.parametrize("name", ["outlier_act_256x4096", "random_bits_33x1280", "special_blocks",
+                                  "heavy_tail_64x4096"])
+def test_fake_quant_parity(mx, oracle_mod, cuda, name, fm):
+    fmt, m = fm
+    x = SMALL[name]()
+    if not usable(name, fmt, m, x):
+        pytest.skip("MBS needs cols % 128 == 0")
+    xd = x.to(cuda)
+    y, s = mx.fake_quant(xd, fmt, m, return_scales=True)
+    g = inputs.qat_grad(*x.shape, seed=3).to(cuda)
+    gx = mx.fake_quant_bwd(xd, g, fmt, m)
+    torch.cuda.synchronize()
+    oy, os_ = oracle_mod.fake_quant_fwd(bits(x), fmt, m, want_scales=True)
+    assert np.array_equal(bits(y), oy), "fake-quant forward"
+    assert np.array_equal(host_u8(s), os_), "scales_out"
+    ogx = oracle_mod.fake_quant_bwd(bits(x), bits(g), fmt, m)
+    assert np.array_equal(bits(gx), ogx), "straight-through backward"
+
+
+@pytest.mark.parametrize("fm", ALL, ids=ids)
+@pytest.mark.parametrize("name", ["outlier_act_256x4096", "heavy_tail_64x4096", "random_bits_7x384",
+                                  "special_blocks"])
+def test_block_error_parity(mx, oracle_mod, cuda, name, fm):
+    fmt, m = fm
+    x = SMALL[name]()
+    if not usable(name, fmt, m, x):
+        pytest.skip("MBS needs cols % 128 == 0")
+    bs, tot = mx.block_error(x.to(cuda), fmt, m)
+    torch.cuda.synchronize()
+    obs, osd, osx = oracle_mod.block_error(bits(x), fmt, m)
+    # the per-block output is a float: huge blocks overflow it on both sides
+    obs = obs.astype(np.float32).astype(np.float64)
+    gbs = bs.cpu().numpy().astype(np.float64)
+    assert np.array_equal(np.isnan(obs), np.isnan(gbs))
+    assert np.array_equal(np.isinf(obs), np.isinf(gbs))
+    fin = np.isfinite(obs)
+    assert np.allclose(gbs[fin], obs[fin], rtol=REL, atol=0)
+    t = tot.cpu().numpy()
+    for got, want in ((t[0], osd), (t[1], osx)):
+        assert np.isnan(got) == np.isnan(want)
+        if np.isfinite(want):
+            assert np.isclose(got, want, rtol=REL, atol=0)
+
+
+# ------------------------------------------------ exhaustive element values --
+
+def test_every_scaled_value_at_several_exponents(mx, oracle_mod, cuda):
+    """Each block: an anchor fixing E, then every bf16 pattern below it (both signs)."""
+    rows = []
+    allbits = np.arange(1 << 16, dtype=np.uint32)
+    for E in (-127, -126, -90, -7, 0, 3, 64, 125):
+        # anchor 7.9375 * 2^E (max significand below 8) -> FLOOR exponent E
+        anchor_exp = E + 2 + 127
+        if anchor_exp < 1:
+            anchor = 0x0080                  # smallest normal: E clamps to -127
+            lim = 0x0080
+        else:
+            anchor = (anchor_exp << 7) | 0x7F
+            lim = anchor
+        vals = allbits[(allbits & 0x7FFF) <= lim].astype(np.uint16)
+        n = len(vals)
+        per = 31
+        nb = (n + per - 1) // per
+        blk = np.zeros((nb, 32), np.uint16)
+        blk[:, 0] = anchor
+        flat = np.zeros(nb * per, np.uint16)
+        flat[:n] = vals
+        blk[:, 1:] = flat.reshape(nb, per)
+        rows.append(blk)
+    arr = np.concatenate(rows)
+    arr = np.concatenate([arr, np.zeros(((-len(arr)) % 64, 32), np.uint16)]).reshape(-1, 2048)
+    x = torch.from_numpy(arr.view(np.int16)).view(torch.bfloat16)
+    for fmt in (E2M1, E4M3):
+        c, s, _ = mx.quantize(x.to(cuda), fmt, FLOOR)
+        y = mx.fake_quant(x.to(cuda), fmt, FLOOR)
+        torch.cuda.synchronize()
+        oc, os_, _ = oracle_mod.quantize(arr, fmt, FLOOR)
+        assert np.array_equal(host_u8(s), os_)
+        assert np.array_equal(host_u8(c), oc)
+        assert np.array_equal(bits(y), oracle_mod.fake_quant_fwd(arr, fmt, FLOOR))
+
+
+@pytest.mark.parametrize("fmt", [E2M1, E4M3])
+@pytest.mark.parametrize("out_fp32", [0, 1])
+@pytest.mark.parametrize("with_macro", [False, True])
+def test_dequantize_every_code_and_scale(mx, oracle_mod, cuda, fmt, out_fp32, with_macro):
+    if fmt == E4M3 and with_macro:
+        pytest.skip("no MBS for E4M3")
+    rng = np.random.default_rng(23)
+    rows, cols = 256, 512
+    scales = np.tile(np.arange(256, dtype=np.uint8)[:, None], (1, cols // 32))
+    rng.shuffle(scales, axis=1)
+    if fmt == E2M1:
+        codes = rng.integers(0, 256, (rows, cols // 2), dtype=np.uint8)
+        codes[:, :8] = np.arange(0, 256, 17, dtype=np.uint8)[None, :8]
+    else:
+        codes = rng.integers(0, 256, (rows, cols), dtype=np.uint8)
+        codes[0, :256] = np.arange(256, dtype=np.uint8)
+    macro = rng.integers(0, 256, (rows, cols // 128), dtype=np.uint8) if with_macro else None
+    tdev = lambda a: None if a is None else torch.from_numpy(a).to(cuda)
+    out = mx.dequantize(tdev(codes), tdev(scales), tdev(macro), fmt,
+                        torch.float32 if out_fp32 else torch.bfloat16)
+    torch.cuda.synchronize()
+    ref = oracle_mod.dequantize(codes, scales, macro, rows, cols, fmt, out_fp32=bool(out_fp32))
+    got = out.cpu().view(torch.int32 if out_fp32 else torch.int16).numpy()
+    got = got.view(np.uint32 if out_fp32 else np.uint16)
+    assert np.array_equal(got, ref)
+
+
+@pytest.mark.parametrize("fm", ALL, ids=ids)
+def test_dequantize_roundtrip(mx, oracle_mod, cuda, fm):
+    fmt, m = fm
+    x = SMALL["outlier_act_256x4096"]()
+    c, s, mac = mx.quantize(x.to(cuda), fmt, m)
+    y = mx.dequantize(c, s, mac, fmt)
+    yf = mx.dequantize(c, s, mac, fmt, torch.float32)
+    torch.cuda.synchronize()
+    oc, os_, omac = oracle_mod.quantize(bits(x), fmt, m)
+    assert np.array_equal(bits(y), oracle_mod.dequantize(oc, os_, omac, 256, 4096, fmt))
+    assert np.array_equal(yf.cpu().view(torch.int32).numpy().view(np.uint32),
+                          oracle_mod.dequantize(oc, os_, omac, 256, 4096, fmt, out_fp32=True))
+
+
+# -------------------------------------------------- full-size workloads --
+
+def sample_rows(n_rows, k, seed):
+    rng = np.random.default_rng(seed)
+    r = np.sort(rng.choice(n_rows, size=min(k, n_rows), replace=False))
+    r[0], r[-1] = 0, n_rows - 1          # first and last row always
+    return np.unique(r)
+
+
+def test_full_mlp_weight_fp8(mx, oracle_mod, cuda):
+    x = inputs.mlp_weight(device=cuda)
+    c, s, _ = mx.quantize(x, E4M3, FLOOR)
+    torch.cuda.synchronize()
+    r = sample_rows(x.shape[0], 48, 1)
+    xs = bits(x[r])
+    oc, os_, _ = oracle_mod.quantize(xs, E4M3, FLOOR)
+    assert np.array_equal(host_u8(c[r]), oc)
+    assert np.array_equal(host_u8(s[r]), os_)
+    # property over every block: the FLOOR byte from the block amax exponent
+    amax = x.view(-1, 32).abs().amax(dim=1).view(torch.int16).to(torch.int32)
+    want = torch.clamp((amax >> 7) - 8, min=0).to(torch.uint8)
+    assert torch.equal(s.view(-1), want)
+
+
+def test_full_moe_w13_fp4(mx, oracle_mod, cuda):
+    x = inputs.moe_w13(device=cuda).view(-1, 2048)
+    c, s, _ = mx.quantize(x, E2M1, FLOOR)
+    y = mx.dequantize(c, s, None, E2M1)
+    torch.cuda.synchronize()
+    r = sample_rows(x.shape[0], 64, 2)
+    xs = bits(x[r])
+    oc, os_, _ = oracle_mod.quantize(xs, E2M1, FLOOR)
+    assert np.array_equal(host_u8(c[r]), oc)
+    assert np.array_equal(host_u8(s[r]), os_)
+    assert np.array_equal(bits(y[r]), oracle_mod.dequantize(oc, os_, None, len(r), 2048, E2M1))
+    amax = x.view(-1, 32).abs().amax(dim=1).view(torch.int16).to(torch.int32)
+    assert torch.equal(s.view(-1), torch.clamp((amax >> 7) - 2, min=0).to(torch.uint8))
+    # every code decodes to a value no farther from x than half the local grid step
+    err = (y.float() - x.float()).abs()
+    X = torch.pow(2.0, s.float() - 127).repeat_interleave(32, dim=1)
+    assert bool((err <= torch.maximum(X, (x.float().abs() - 6 * X).clamp(min=0))).all())
+
+
+def test_full_qat_tensors(mx, oracle_mod, cuda):
+    for gen, seed in ((inputs.qat_act, 3), (inputs.qat_weight, 4)):
+        x = gen(device=cuda)
+        g = inputs.qat_grad(*x.shape, device=cuda)
+        y = mx.fake_quant(x, E2M1, FLOOR)
+        gx = mx.fake_quant_bwd(x, g, E2M1, FLOOR)
+        torch.cuda.synchronize()
+        r = sample_rows(x.shape[0], 48, seed)
+        assert np.array_equal(bits(y[r]), oracle_mod.fake_quant_fwd(bits(x[r]), E2M1, FLOOR))
+        assert np.array_equal(bits(gx[r]), oracle_mod.fake_quant_bwd(bits(x[r]), bits(g[r]), E2M1, FLOOR))
+
+
+@pytest.mark.parametrize("m", FP4_MODES, ids=lambda m: ids((0, m)))
+def test_full_heavy_tail_modes(mx, oracle_mod, cuda, m):
+    x = inputs.heavy_tail(device=cuda)
+    c, s, mac = mx.quantize(x, E2M1, m)
+    bs, tot = mx.block_error(x, E2M1, m)
+    torch.cuda.synchronize()
+    r = sample_rows(x.shape[0], 12 if m >> 4 == 2 else 32, 5)
+    xs = bits(x[r])
+    oc, os_, omac = oracle_mod.quantize(xs, E2M1, m)
+    assert np.array_equal(host_u8(c[r]), oc)
+    assert np.array_equal(host_u8(s[r]), os_)
+    if m >> 4:
+        assert np.array_equal(host_u8(mac[r]), omac)
+    obs, _, _ = oracle_mod.block_error(xs, E2M1, m)
+    assert np.allclose(bs[r].cpu().numpy(), obs, rtol=REL, atol=0)
+    # totals equal the sum of the per-block values (both from the kernel)
+    assert np.isclose(tot[0].item(), bs.double().sum().item(), rtol=1e-5)
+    assert np.isclose(tot[1].item(), x.double().pow(2).sum().item(), rtol=1e-9)
+
+
+# ------------------------------------------------------ edge behaviour --
+
+def test_guard_bands(mx, cuda):
+    """Outputs never write outside their extent (canary bytes on both sides)."""
+    x = inputs.random_bf16_bits((3, 384), seed=11).to(cuda)
+    for fmt, m in ((E2M1, FLOOR), (E2M1, OAS | MBS_DYNAMIC), (E4M3, CEIL)):
+        ncode = 3 * 384 // (2 if fmt == E2M1 else 1)
+        pad = 256
+        cbuf = torch.full((ncode + 2 * pad,), 0xA5, dtype=torch.uint8, device=cuda)
+        sbuf = torch.full((36 + 2 * pad,), 0x5A, dtype=torch.uint8, device=cuda)
+        mbuf = torch.full((9 + 2 * pad,), 0x3C, dtype=torch.uint8, device=cuda)
+        st = mx.mx_quantize(x.data_ptr(), 3, 384, fmt, m, cbuf[pad:].data_ptr(), sbuf[pad:].data_ptr(),
+                            mbuf[pad:].data_ptr(), torch.cuda.current_stream().cuda_stream)
+        assert st == 0
+        torch.cuda.synchronize()
+        assert bool((cbuf[:pad] == 0xA5).all()) and bool((cbuf[pad + ncode:] == 0xA5).all())
+        assert bool((sbuf[:pad] == 0x5A).all()) and bool((sbuf[pad + 36:] == 0x5A).all())
+        assert bool((mbuf[:pad] == 0x3C).all()) and bool((mbuf[pad + (9 if m >> 4 else 0):] == 0x3C).all())
+    y = torch.full((3 * 384 + 512,), 7, dtype=torch.int16, device=cuda)
+    st = mx.mx_fake_quant_fwd(x.data_ptr(), 3, 384, E2M1, OAS, y[256:].data_ptr(), None,
+                              torch.cuda.current_stream().cuda_stream)
+    torch.cuda.synchronize()
+    assert st == 0 and bool((y[:256] == 7).all()) and bool((y[256 + 3 * 384:] == 7).all())
+
+
+def test_empty_and_zero_rows(mx, cuda):
+    x = torch.empty(0, 64, dtype=torch.bfloat16, device=cuda)
+    c, s, _ = mx.quantize(x)
+    assert c.shape == (0, 32) and s.shape == (0, 2)
+    bs, tot = mx.block_error(x)
+    torch.cuda.synchronize()
+    assert tot.tolist() == [0.0, 0.0]
+
+
+def test_side_stream_and_host_buffers(mx, oracle_mod, cuda):
+    x = inputs.outlier_act()
+    side = torch.cuda.Stream()
+    with torch.cuda.stream(side):
+        c, s, _ = mx.quantize(x.to(cuda, non_blocking=False))
+    side.synchronize()
+    hc, hs, _ = mx.quantize(x.pin_memory())
+    torch.cuda.synchronize()
+    oc, os_, _ = oracle_mod.quantize(bits(x))
+    assert np.array_equal(host_u8(c), oc) and np.array_equal(hc.numpy(), oc)
+    assert np.array_equal(hs.numpy(), os_)
+
+
+def test_autograd_function(mx, oracle_mod, cuda):
+    x = inputs.qat_act(rows=64, cols=256, device=cuda).requires_grad_(True)
+    y = mx.MXFakeQuantize.apply(x, E2M1, FLOOR)
+    g = inputs.qat_grad(64, 256, device=cuda)
+    y.backward(g)
+    torch.cuda.synchronize()
+    xb = bits(x.detach())
+    assert np.array_equal(bits(y.detach()), oracle_mod.fake_quant_fwd(xb))
+    assert np.array_equal(bits(x.grad), oracle_mod.fake_quant_bwd(xb, bits(g)))
