@@ -161,13 +161,19 @@ def quantize(x: torch.Tensor, format: int = E2M1, scaling: int = FLOOR, out=None
     E4M3 bytes); scales uint8 [..., cols/32] (E8M0); macro uint8 [..., cols/128]
     with Macro Block Scaling, else None. ``out`` may supply the three buffers.
     A CPU ``x`` is copied to the current GPU and the outputs come back to the
-    CPU (pinned when ``x`` is pinned).
+    CPU: into ``out`` (host tensors) when given, else into new tensors (pinned
+    when ``x`` is pinned). The copies are enqueued on the current stream.
     """
     if not x.is_cuda:
         dev = torch.device("cuda", torch.cuda.current_device())
         xd = x.to(dev, non_blocking=x.is_pinned())
         res = quantize(xd, format, scaling)
-        return tuple(None if t is None else _to_host(t, x.is_pinned()) for t in res)
+        if out is None:
+            return tuple(None if t is None else _to_host(t, x.is_pinned()) for t in res)
+        for h, d in zip(out, res):
+            if h is not None and d is not None:
+                h.copy_(d, non_blocking=h.is_pinned())
+        return out
     _cuda_bf16(x, "x")
     rows, cols = _rows_cols(x)
     lead = x.shape[:-1]
@@ -200,7 +206,11 @@ def dequantize(codes: torch.Tensor, scales: torch.Tensor, macro=None, format: in
         dev = torch.device("cuda", torch.cuda.current_device())
         pinned = codes.is_pinned()
         args = [None if t is None else t.to(dev, non_blocking=pinned) for t in (codes, scales, macro)]
-        return _to_host(dequantize(*args, format=format, out_dtype=out_dtype), pinned)
+        res = dequantize(*args, format=format, out_dtype=out_dtype)
+        if out is None:
+            return _to_host(res, pinned)
+        out.copy_(res, non_blocking=out.is_pinned())
+        return out
     if codes.dtype != torch.uint8 or scales.dtype != torch.uint8:
         raise ValueError("codes and scales must be uint8")
     cols = codes.shape[-1] * 2 if format == E2M1 else codes.shape[-1]

@@ -190,46 +190,62 @@ __device__ __forceinline__ uint2 nonfinite_e4m3_8(const uint4& x) {
 }
 
 // ------------------------------------------------------- element decoding --
+//
+// Decoding is done with integer operations only. (Feeding the register output
+// of cvt.rn.satfinite.e2m1x2.f32 straight into cvt.rn.f16x2.e2m1x2 gave
+// zeros on sm_100a in this build, while the same decode of codes loaded from
+// memory was right; a table lookup avoids depending on that register path.)
 
-// E2M1 codes (nibble i = element i) -> values in units of the block scale.
+// E2M1 magnitudes 0 .5 1 1.5 2 3 4 6 as bf16 bit patterns, split into their
+// high and low bytes, four entries per 32-bit word (index 0..3, 4..7).
+constexpr uint32_t kE2m1Hi0 = 0x3F3F3F00u, kE2m1Hi1 = 0x40404040u;
+constexpr uint32_t kE2m1Lo0 = 0xC0800000u, kE2m1Lo1 = 0xC0804000u;
+
+// Four E2M1 codes (nibbles 0..3 of c) -> two words of bf16x2 bit patterns.
+__device__ __forceinline__ uint2 e2m1x4_to_bf16(uint32_t c) {
+  const uint32_t sel = c & 0x7777u;                        // magnitude indices
+  const uint32_t hi = __byte_perm(kE2m1Hi0, kE2m1Hi1, sel);
+  const uint32_t lo = __byte_perm(kE2m1Lo0, kE2m1Lo1, sel);
+  uint32_t w0 = __byte_perm(lo, hi, 0x5140);               // elements 0, 1
+  uint32_t w1 = __byte_perm(lo, hi, 0x7362);               // elements 2, 3
+  w0 |= ((c << 12) & 0x8000u) | ((c << 24) & 0x80000000u);  // sign bits 3, 7
+  w1 |= ((c << 4) & 0x8000u) | ((c << 16) & 0x80000000u);   // sign bits 11, 15
+  return make_uint2(w0, w1);
+}
+
+// Eight E2M1 codes (nibble i = element i) -> eight bf16 values (unscaled).
+__device__ __forceinline__ uint4 e2m1x8_to_bf16(uint32_t codes) {
+  const uint2 a = e2m1x4_to_bf16(codes & 0xFFFFu);
+  const uint2 b = e2m1x4_to_bf16(codes >> 16);
+  return make_uint4(a.x, a.y, b.x, b.y);
+}
+
+// E2M1 codes -> unscaled values as floats (exact).
 __device__ __forceinline__ F8 dec_e2m1_8(uint32_t codes) {
-  uint32_t h0, h1, h2, h3;
-  asm("{\n\t.reg .b8 q0, q1, q2, q3;\n\t"
-      "mov.b32 {q0, q1, q2, q3}, %4;\n\t"
-      "cvt.rn.f16x2.e2m1x2 %0, q0;\n\t"
-      "cvt.rn.f16x2.e2m1x2 %1, q1;\n\t"
-      "cvt.rn.f16x2.e2m1x2 %2, q2;\n\t"
-      "cvt.rn.f16x2.e2m1x2 %3, q3;\n\t}"
-      : "=r"(h0), "=r"(h1), "=r"(h2), "=r"(h3)
-      : "r"(codes));
+  const uint4 b = e2m1x8_to_bf16(codes);
   F8 r;
-  const uint32_t h[4] = {h0, h1, h2, h3};
-#pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    r.v[2 * j] = __half2float(__ushort_as_half(static_cast<unsigned short>(h[j] & 0xFFFFu)));
-    r.v[2 * j + 1] = __half2float(__ushort_as_half(static_cast<unsigned short>(h[j] >> 16)));
-  }
+  r.v[0] = bf_lo(b.x); r.v[1] = bf_hi(b.x);
+  r.v[2] = bf_lo(b.y); r.v[3] = bf_hi(b.y);
+  r.v[4] = bf_lo(b.z); r.v[5] = bf_hi(b.z);
+  r.v[6] = bf_lo(b.w); r.v[7] = bf_hi(b.w);
   return r;
 }
 
-// E4M3 bytes (byte i = element i) -> values (NaN codes give NaN).
+// One E4M3fn byte -> float (S.1111.111 -> NaN; subnormals m * 2^-9).
+__device__ __forceinline__ float e4m3_to_f32(uint32_t c) {
+  const uint32_t ef = (c >> 3) & 15u, m = c & 7u;
+  float v = ef ? __uint_as_float(((ef + 120u) << 23) | (m << 20))
+               : static_cast<float>(m) * 0.001953125f;        // m * 2^-9, exact
+  if (ef == 15u && m == 7u) v = __uint_as_float(kNaNf32);
+  return (c & 0x80u) ? -v : v;
+}
+
 __device__ __forceinline__ F8 dec_e4m3_8(uint2 codes) {
-  uint32_t h0, h1, h2, h3;
-  asm("{\n\t.reg .b16 p0, p1, p2, p3;\n\t"
-      "mov.b32 {p0, p1}, %4;\n\t"
-      "mov.b32 {p2, p3}, %5;\n\t"
-      "cvt.rn.f16x2.e4m3x2 %0, p0;\n\t"
-      "cvt.rn.f16x2.e4m3x2 %1, p1;\n\t"
-      "cvt.rn.f16x2.e4m3x2 %2, p2;\n\t"
-      "cvt.rn.f16x2.e4m3x2 %3, p3;\n\t}"
-      : "=r"(h0), "=r"(h1), "=r"(h2), "=r"(h3)
-      : "r"(codes.x), "r"(codes.y));
   F8 r;
-  const uint32_t h[4] = {h0, h1, h2, h3};
 #pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    r.v[2 * j] = __half2float(__ushort_as_half(static_cast<unsigned short>(h[j] & 0xFFFFu)));
-    r.v[2 * j + 1] = __half2float(__ushort_as_half(static_cast<unsigned short>(h[j] >> 16)));
+  for (int i = 0; i < 4; ++i) {
+    r.v[i] = e4m3_to_f32((codes.x >> (8 * i)) & 0xFFu);
+    r.v[4 + i] = e4m3_to_f32((codes.y >> (8 * i)) & 0xFFu);
   }
   return r;
 }
@@ -325,25 +341,26 @@ __device__ __forceinline__ int mbs_floor_byte(uint32_t amax, int k) {
   return max(ex - 2 - ((2 * m7 < k) ? 1 : 0), 0);
 }
 
-// Grid midpoints of E2M1 times (256 + k), for rounding t = 256 |x| 2^-E.
+// Grid midpoints of E2M1 times f = (256 + k) / 256, for rounding the scaled
+// magnitude s = |x| 2^-E (which is below 16, so it never overflows). Each
+// threshold mid * (256 + k) / 256 has at most 12 significant bits: exact.
 struct Thresholds {
   float t[7];
 };
 __device__ __forceinline__ Thresholds mbs_thresholds(int k) {
-  const float fk = static_cast<float>(256 + k);
+  const float f = static_cast<float>(256 + k) * 0.00390625f;   // (256 + k) / 256
   Thresholds T;
-  T.t[0] = 0.25f * fk; T.t[1] = 0.75f * fk; T.t[2] = 1.25f * fk; T.t[3] = 1.75f * fk;
-  T.t[4] = 2.5f * fk;  T.t[5] = 3.5f * fk;  T.t[6] = 5.0f * fk;
+  T.t[0] = 0.25f * f; T.t[1] = 0.75f * f; T.t[2] = 1.25f * f; T.t[3] = 1.75f * f;
+  T.t[4] = 2.5f * f;  T.t[5] = 3.5f * f;  T.t[6] = 5.0f * f;
   return T;
 }
 
-// Magnitude code 0..7 of t = 256 |x| 2^-E under factor (256 + k) / 256. At a
-// midpoint between an even and an odd code the even one wins: strictly above
-// is needed to leave an even code, reaching the midpoint suffices to leave an
-// odd one.
-__device__ __forceinline__ int mbs_round(float t, const Thresholds& T) {
-  return (t > T.t[0]) + (t >= T.t[1]) + (t > T.t[2]) + (t >= T.t[3]) + (t > T.t[4]) +
-         (t >= T.t[5]) + (t > T.t[6]);
+// Magnitude code 0..7 of s = |x| 2^-E under the factor f. At a midpoint
+// between an even and an odd code the even one wins: strictly above is needed
+// to leave an even code, reaching the midpoint suffices to leave an odd one.
+__device__ __forceinline__ int mbs_round(float s, const Thresholds& T) {
+  return (s > T.t[0]) + (s >= T.t[1]) + (s > T.t[2]) + (s >= T.t[3]) + (s > T.t[4]) +
+         (s >= T.t[5]) + (s > T.t[6]);
 }
 
 // E2M1 magnitude (in units of 0.5) of code c: 0 1 2 3 4 6 8 12.
@@ -351,7 +368,7 @@ __device__ __forceinline__ int e2m1_halves(int c) { return (0xC8643210u >> (4 * 
 
 // Eight codes under factor k and exponent byte b (b in [0, 253]).
 __device__ __forceinline__ uint32_t enc_mbs_8(const uint4& x, int b, const Thresholds& T) {
-  const float m = inv_scale_from_byte(b) * 256.0f;   // 256 * 2^-E, exact
+  const float m = inv_scale_from_byte(b);   // 2^-E, exact
   const uint32_t w[4] = {x.x, x.y, x.z, x.w};
   uint32_t r = 0;
 #pragma unroll
@@ -366,8 +383,8 @@ __device__ __forceinline__ uint32_t enc_mbs_8(const uint4& x, int b, const Thres
 }
 
 // Exact OAS comparison of one lane's 8 elements under factor k: candidates
-// E1 (byte b1) and E1 + 1. D = 512 s - 2 q (256 + k) with s = |x| 2^-E1 and q
-// the code magnitude in units of 0.5 (x2 for the coarser candidate): an
+// E1 (byte b1) and E1 + 1. D = 512 s - h (256 + k) with s = |x| 2^-E1 and h
+// the code magnitude in units of 0.5 (doubled for the coarser candidate): an
 // integer below 2^12 for every element that does not round to zero under both.
 __device__ __forceinline__ int oas_delta_mbs8(const uint4& x, int b1, const Thresholds& T,
                                               int k) {
@@ -379,8 +396,8 @@ __device__ __forceinline__ int oas_delta_mbs8(const uint4& x, int b1, const Thre
   for (int j = 0; j < 8; ++j) {
     const uint32_t word = w[j >> 1];
     const float s = fabsf((j & 1) ? bf_hi(word) : bf_lo(word)) * inv1;
-    const int c1 = mbs_round(s * 256.0f, T);
-    const int c2 = mbs_round(s * 128.0f, T);
+    const int c1 = mbs_round(s, T);
+    const int c2 = mbs_round(s * 0.5f, T);
     const float d1 = s * 512.0f - static_cast<float>(e2m1_halves(c1)) * fk;
     const float d2 = s * 512.0f - static_cast<float>(2 * e2m1_halves(c2)) * fk;
     const int i1 = __float2int_rn(d1), i2 = __float2int_rn(d2);

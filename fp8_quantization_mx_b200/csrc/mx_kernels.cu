@@ -170,8 +170,8 @@ __device__ __forceinline__ void process_chunk(const StreamArgs& a, const uint4& 
           ow[j] = (plo ? (gw[j] & 0xFFFFu) : 0u) | (phi ? (gw[j] & 0xFFFF0000u) : 0u);
         }
       } else {
-        const float m = inv_scale_from_byte(s.byte) * 256.0f;
-        const float lim = 6.0f * static_cast<float>(256 + s.k);
+        const float m = inv_scale_from_byte(s.byte);
+        const float lim = 6.0f * static_cast<float>(256 + s.k) * 0.00390625f;   // 6 f, exact
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           const bool plo = fabsf(bf_lo(xw[j])) * m <= lim;
@@ -295,8 +295,8 @@ __device__ __forceinline__ double macro_sse_k(const float* xs, const uint32_t am
 #pragma unroll 4
         for (int i = 0; i < 32; ++i) {
           const float s = xs[32 * b + i] * inv1;
-          const int c1 = mbs_round(s * 256.0f, T);
-          const int c2 = mbs_round(s * 128.0f, T);
+          const int c1 = mbs_round(s, T);
+          const int c2 = mbs_round(s * 0.5f, T);
           const int i1 = __float2int_rn(s * 512.0f - static_cast<float>(e2m1_halves(c1)) * fk);
           const int i2 = __float2int_rn(s * 512.0f - static_cast<float>(2 * e2m1_halves(c2)) * fk);
           acc += i1 * i1 - i2 * i2;
@@ -304,14 +304,15 @@ __device__ __forceinline__ double macro_sse_k(const float* xs, const uint32_t am
         if (acc > 0) byte = b2;
       }
     }
-    const float m = inv_scale_from_byte(byte) * 256.0f;               // 256 * 2^-E
-    const double p = __longlong_as_double(static_cast<long long>(byte - 127 - 8 + 1023) << 52);
+    const float m = inv_scale_from_byte(byte);                          // 2^-E
+    const double p = __longlong_as_double(static_cast<long long>(byte - 127 + 1023) << 52);
 #pragma unroll 8
     for (int i = 0; i < 32; ++i) {
-      const float t = xs[32 * b + i] * m;
-      const int c = mbs_round(t, T);
-      const float dt = t - static_cast<float>(e2m1_halves(c)) * fk * 0.5f;   // exact
-      const double d = static_cast<double>(dt) * p;                             // exact
+      const float s = xs[32 * b + i] * m;
+      const int c = mbs_round(s, T);
+      // s - h (256 + k) / 512 is exact (both sides are multiples of 2^-9 below 2^5)
+      const float ds = s - static_cast<float>(e2m1_halves(c)) * fk * 0.001953125f;
+      const double d = static_cast<double>(ds) * p;                             // exact
       sse = fma(d, d, sse);
     }
   }

@@ -1,0 +1,76 @@
+"""Multi-rank host logic on CPU (gloo, world size 2).
+
+Each rank quantizes its contiguous row shard with the oracle; gathering the
+shards must reproduce the whole-tensor result bit for bit (rows are
+independent, so no exchange is needed), and the timing reduction returns the
+maximum over ranks.
+"""
+
+import os
+import socket
+
+import numpy as np
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+from fp8_quantization_mx_b200.sharding import max_over_ranks, shard_rows
+
+
+def _free_port():
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    p = s.getsockname()[1]
+    s.close()
+    return p
+
+
+def _worker(rank, world, port, x_bits, scaling, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    import oracle
+    r0, r1 = shard_rows(x_bits.shape[0], world, rank)
+    c, s, m = oracle.quantize(np.ascontiguousarray(x_bits[r0:r1]), 0, scaling)
+    parts = [None] * world
+    dist.all_gather_object(parts, (r0, r1, c, s, m))
+    t = max_over_ranks([float(rank + 1), -float(rank)])
+    if rank == 0:
+        out.put((parts, t))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def test_shard_rows_partition():
+    for rows in (0, 1, 7, 196608):
+        for world in (1, 2, 3, 8):
+            spans = [shard_rows(rows, world, r) for r in range(world)]
+            assert spans[0][0] == 0 and spans[-1][1] == rows
+            assert all(a[1] == b[0] for a, b in zip(spans, spans[1:]))
+            sizes = [e - s for s, e in spans]
+            assert max(sizes) - min(sizes) <= 1
+    with pytest.raises(ValueError):
+        shard_rows(10, 2, 2)
+
+
+@pytest.mark.parametrize("scaling", [0, 3, 16])
+def test_two_rank_shards_match_whole_tensor(oracle_mod, scaling):
+    from fp8_quantization_mx_b200 import inputs
+    x = inputs.bf16_bits_numpy(inputs.heavy_tail(rows=37, cols=512, seed=9))
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_worker, args=(r, 2, port, x, scaling, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    parts, t = q.get(timeout=120)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    c_full, s_full, m_full = oracle_mod.quantize(x, 0, scaling)
+    for r0, r1, c, s, m in parts:
+        assert np.array_equal(c, c_full[r0:r1]) and np.array_equal(s, s_full[r0:r1])
+        if m_full is not None:
+            assert np.array_equal(m, m_full[r0:r1])
+    assert sum(p[1] - p[0] for p in parts) == 37
+    assert t == [2.0, 0.0]
