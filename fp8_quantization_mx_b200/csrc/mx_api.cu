@@ -72,7 +72,7 @@ int mx_quantize(const void* x, int64_t rows, int64_t cols, int format, int scali
   const int64_t n = rows * cols;
   if (n == 0) return MX_OK;
   if (!x || !codes || !scales || (mbs && !macro)) return MX_ERR_INVALID_ARG;
-  if (!aligned(x, 16) || !aligned(codes, 16)) return MX_ERR_ALIGN;
+  if (!aligned(x, 32) || !aligned(codes, 16)) return MX_ERR_ALIGN;
   return from_cuda(mxk::launch_quantize(x, n, format, scaling, codes, scales, mbs ? macro : nullptr,
                                         static_cast<cudaStream_t>(stream)));
 }
@@ -87,7 +87,7 @@ int mx_dequantize(const void* codes, const uint8_t* scales, const uint8_t* macro
   const int64_t n = rows * cols;
   if (n == 0) return MX_OK;
   if (!codes || !scales || !out) return MX_ERR_INVALID_ARG;
-  if (!aligned(codes, 16) || !aligned(out, 16)) return MX_ERR_ALIGN;
+  if (!aligned(codes, 16) || !aligned(out, 32)) return MX_ERR_ALIGN;
   return from_cuda(mxk::launch_dequantize(codes, scales, macro, n, format, out_fp32, out,
                                           static_cast<cudaStream_t>(stream)));
 }
@@ -101,7 +101,7 @@ int mx_fake_quant_fwd(const void* x, int64_t rows, int64_t cols, int format, int
   const int64_t n = rows * cols;
   if (n == 0) return MX_OK;
   if (!x || !y) return MX_ERR_INVALID_ARG;
-  if (!aligned(x, 16) || !aligned(y, 16)) return MX_ERR_ALIGN;
+  if (!aligned(x, 32) || !aligned(y, 32)) return MX_ERR_ALIGN;
   return from_cuda(mxk::launch_fake_fwd(x, n, format, scaling, y, scales_out,
                                         static_cast<cudaStream_t>(stream)));
 }
@@ -115,7 +115,7 @@ int mx_fake_quant_bwd(const void* x, const void* grad_y, int64_t rows, int64_t c
   const int64_t n = rows * cols;
   if (n == 0) return MX_OK;
   if (!x || !grad_y || !grad_x) return MX_ERR_INVALID_ARG;
-  if (!aligned(x, 16) || !aligned(grad_y, 16) || !aligned(grad_x, 16)) return MX_ERR_ALIGN;
+  if (!aligned(x, 32) || !aligned(grad_y, 32) || !aligned(grad_x, 32)) return MX_ERR_ALIGN;
   return from_cuda(mxk::launch_fake_bwd(x, grad_y, n, format, scaling, grad_x,
                                         static_cast<cudaStream_t>(stream)));
 }
@@ -131,7 +131,7 @@ int mx_block_error(const void* x, int64_t rows, int64_t cols, int format, int sc
   const int64_t n = rows * cols;
   if (n != 0) {
     if (!x) return MX_ERR_INVALID_ARG;
-    if (!aligned(x, 16) || (block_sse && !aligned(block_sse, 4))) return MX_ERR_ALIGN;
+    if (!aligned(x, 32) || (block_sse && !aligned(block_sse, 4))) return MX_ERR_ALIGN;
   }
   return from_cuda(mxk::launch_block_error(x, n, format, scaling, block_sse, totals,
                                            static_cast<cudaStream_t>(stream)));

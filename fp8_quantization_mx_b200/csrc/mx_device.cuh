@@ -1,33 +1,34 @@
 // Device building blocks of the MX block-32 kernels (sm_100a).
 //
 // Work decomposition shared by every kernel: the bf16 input is viewed as a
-// flat array of 16-byte "chunks" of 8 elements. Because every row length is a
-// multiple of 32 (of 128 with Macro Block Scaling), a 32-element MX block is
-// exactly 4 consecutive chunks and a 128-element macro block 16, in the flat
-// order, whatever the row length. A warp reads 32 consecutive chunks per step
-// (512 contiguous bytes, one 16-byte load per lane), so lanes 4q..4q+3 hold
-// block q of the step and lanes 16h..16h+15 hold macro block h.
+// flat array of 32-byte "slices" of 16 elements, one per lane. Because every
+// row length is a multiple of 32 (of 128 with Macro Block Scaling), a 32-element
+// MX block is exactly 2 consecutive slices and a 128-element macro block 8, in
+// the flat order, whatever the row length. A warp reads 32 consecutive slices
+// per step (1 KiB contiguous, one 32-byte load per lane), so lanes 2q, 2q+1
+// hold block q of the step and lanes 8h..8h+7 hold macro block h.
 //
 // Numerics, per block (OCP Microscaling as restated by "[vLLM] MXFP8/MXFP4"
 // (MX format table) and "Unveiling the Potential of Quantization with MXFP4"
 // (2.A, 2.B)):
-//  * amax is the largest |x| of the block, taken on the bf16 bit patterns with
-//    the sign cleared (an integer compare orders finite values, then Inf, then
-//    NaN, so a non-finite block is one whose amax bits reach 0x7F80);
-//  * the E8M0 byte is computed from the amax exponent field and mantissa bits
-//    with integer arithmetic only;
-//  * x * 2^-E is an exact float product (E is a power of two and the product
-//    never needs more than the 8 significant bits x already has), so the
-//    hardware conversions cvt.rn.satfinite.{e2m1x2,e4m3x2}.f32 see the exact
-//    scaled value and round it to nearest-even with saturation;
-//  * with a macro factor f = (256 + k) / 256 the scaled value x / (f 2^E) is not
-//    exact in float, so it is rounded by comparing 256 |x| 2^-E (exact) with
-//    the grid midpoints times (256 + k) (exact); equality goes to the even code.
+//  * amax is the largest |x| of the block: a max of absolute values on packed
+//    bf16 pairs (NaN-propagating), then the sign cleared; as an integer the
+//    result orders finite values, then Inf, then NaN, so a non-finite block is
+//    one whose amax bits reach 0x7F80;
+//  * the E8M0 byte comes from the amax exponent field and mantissa bits with
+//    integer arithmetic only;
+//  * x * 2^-E is exact in bf16 whenever it is at least 2^-126 (a power-of-two
+//    scaling of an 8-bit significand), and anything smaller rounds to a signed
+//    zero code anyway, so the scaled pairs feed the hardware conversions
+//    cvt.rn.satfinite.{e2m1x2,e4m3x2}.f32 (round to nearest even, saturate);
+//  * with a macro factor f = (256 + k) / 256 the quotient x / (f 2^E) is not
+//    exact, so s = |x| 2^-E (exact, below 16) is compared with the grid
+//    midpoints times f (exact); equality goes to the even code;
+//  * decoding (fake-quant, error, dequantize) is integer only: a byte-permute
+//    table for E2M1 and bit assembly for E4M3, then an exact float product.
 #pragma once
 
 #include <cstdint>
-#include <cuda_bf16.h>
-#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 
 namespace mxk {
@@ -36,24 +37,30 @@ constexpr int kFmtE2M1 = 0;
 constexpr int kFmtE4M3 = 1;
 constexpr int kFloor = 0, kCeil = 1, kOasRule = 2, kOas = 3;
 constexpr int kMbsNone = 0, kMbsStatic = 1, kMbsDynamic = 2;
+constexpr unsigned kFull = 0xFFFFFFFFu;
 
 constexpr uint16_t kNaNbf16 = 0x7FC0;
 constexpr uint32_t kNaNf32 = 0x7FC00000u;
 
+// 16 bf16 values: w[i] holds elements 2i (low half) and 2i+1 (high half).
+struct V16 {
+  uint32_t w[8];
+};
+// 16 floats.
+struct F16 {
+  float v[16];
+};
+
 // ------------------------------------------------------------- memory ops --
 
-// Streaming 16-byte load: read-only path, not kept in L1, 256-byte L2 prefetch.
-__device__ __forceinline__ uint4 ld_stream16(const void* p) {
-  uint4 r;
-  asm volatile("ld.global.nc.L1::no_allocate.L2::256B.v4.u32 {%0, %1, %2, %3}, [%4];"
-               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
-               : "l"(p));
-  return r;
-}
-
-__device__ __forceinline__ uint32_t ld_stream4(const void* p) {
-  uint32_t r;
-  asm volatile("ld.global.nc.L1::no_allocate.u32 %0, [%1];" : "=r"(r) : "l"(p));
+// Streaming 32-byte load: read-only path, not kept in L1, 256-byte L2 prefetch.
+__device__ __forceinline__ V16 ld_stream32(const void* p) {
+  V16 r;
+  asm volatile(
+      "ld.global.nc.L1::no_allocate.L2::256B.v8.u32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+      : "=r"(r.w[0]), "=r"(r.w[1]), "=r"(r.w[2]), "=r"(r.w[3]), "=r"(r.w[4]), "=r"(r.w[5]),
+        "=r"(r.w[6]), "=r"(r.w[7])
+      : "l"(p));
   return r;
 }
 
@@ -65,10 +72,15 @@ __device__ __forceinline__ uint2 ld_stream8(const void* p) {
   return r;
 }
 
-// Streaming (evict-first) stores of outputs nobody re-reads in this kernel.
-__device__ __forceinline__ void st_stream4(void* p, uint32_t v) {
-  asm volatile("st.global.cs.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+__device__ __forceinline__ uint4 ld_stream16(const void* p) {
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+               : "l"(p));
+  return r;
 }
+
+// Streaming (evict-first) stores of outputs nobody re-reads in this kernel.
 __device__ __forceinline__ void st_stream8(void* p, uint2 v) {
   asm volatile("st.global.cs.v2.u32 [%0], {%1, %2};" ::"l"(p), "r"(v.x), "r"(v.y) : "memory");
 }
@@ -77,29 +89,45 @@ __device__ __forceinline__ void st_stream16(void* p, uint4 v) {
                "r"(v.z), "r"(v.w)
                : "memory");
 }
+__device__ __forceinline__ void st_stream32(void* p, const V16& v) {
+  asm volatile("st.global.cs.v8.u32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p),
+               "r"(v.w[0]), "r"(v.w[1]), "r"(v.w[2]), "r"(v.w[3]), "r"(v.w[4]), "r"(v.w[5]),
+               "r"(v.w[6]), "r"(v.w[7])
+               : "memory");
+}
 
 // ------------------------------------------------------------ bf16 / bits --
 
 __device__ __forceinline__ float bf_lo(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
-__device__ __forceinline__ uint32_t max_u16x2(uint32_t a, uint32_t b) {
+// Element i of a V16 as a float (exact).
+__device__ __forceinline__ float elem(const V16& v, int i) {
+  return (i & 1) ? bf_hi(v.w[i >> 1]) : bf_lo(v.w[i >> 1]);
+}
+
+// Per-half max of |a|, |b| (sign of the result = xor of the signs; NaN wins).
+__device__ __forceinline__ uint32_t max_abs_bf16x2(uint32_t a, uint32_t b) {
   uint32_t d;
-  asm("max.u16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  asm("max.NaN.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
   return d;
 }
 
-// Largest |x| bit pattern among 8 bf16 values.
-__device__ __forceinline__ uint32_t amax_bits8(const uint4& v) {
-  const uint32_t m = max_u16x2(max_u16x2(v.x & 0x7FFF7FFFu, v.y & 0x7FFF7FFFu),
-                               max_u16x2(v.z & 0x7FFF7FFFu, v.w & 0x7FFF7FFFu));
+// Largest |x| bit pattern among the 16 bf16 values of a slice.
+__device__ __forceinline__ uint32_t amax_bits16(const V16& v) {
+  const uint32_t a = max_abs_bf16x2(max_abs_bf16x2(v.w[0], v.w[1]), max_abs_bf16x2(v.w[2], v.w[3]));
+  const uint32_t b = max_abs_bf16x2(max_abs_bf16x2(v.w[4], v.w[5]), max_abs_bf16x2(v.w[6], v.w[7]));
+  const uint32_t m = max_abs_bf16x2(a, b) & 0x7FFF7FFFu;
   return max(m & 0xFFFFu, m >> 16);
 }
 
-__device__ __forceinline__ uint32_t quad_max(uint32_t a) {
-  a = max(a, __shfl_xor_sync(0xFFFFFFFFu, a, 1));
-  a = max(a, __shfl_xor_sync(0xFFFFFFFFu, a, 2));
-  return a;
+// Max over the two lanes of a block, and over the eight lanes of a macro block.
+__device__ __forceinline__ uint32_t pair_max(uint32_t a) {
+  return max(a, __shfl_xor_sync(kFull, a, 1));
+}
+__device__ __forceinline__ uint32_t oct_max(uint32_t a) {
+  a = max(a, __shfl_xor_sync(kFull, a, 2));
+  return max(a, __shfl_xor_sync(kFull, a, 4));
 }
 
 // 2^E as a float for E in [-149, 127] (subnormal below -126).
@@ -113,14 +141,24 @@ __device__ __forceinline__ float inv_scale_from_byte(int b) {
   return __uint_as_float(static_cast<uint32_t>(254 - b) << 23);
 }
 
+// 2^-E as a bf16x2 pair for b in [0, 253] (a normal bf16).
+__device__ __forceinline__ uint32_t inv_scale_bf16x2(int b) {
+  return static_cast<uint32_t>(254 - b) * 0x00800080u;
+}
+
+__device__ __forceinline__ uint32_t mul_bf16x2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
 // ------------------------------------------------------- element encoding --
 
-// Eight scaled values -> eight E2M1 codes, element i in nibble i.
-__device__ __forceinline__ uint32_t cvt_e2m1x8(float a0, float a1, float a2, float a3, float a4,
-                                               float a5, float a6, float a7) {
+// Two bf16x2 words (4 scaled values, element order) -> 4 E2M1 codes in the low
+// 16 bits, element i in nibble i. cvt.rn.satfinite.e2m1x2.f32 d, a, b puts a
+// in the upper nibble and b in the lower one.
+__device__ __forceinline__ uint32_t cvt_e2m1x8(const uint32_t s[4]) {
   uint32_t r;
-  // cvt.rn.satfinite.e2m1x2.f32 d, hi, lo: the second operand lands in the
-  // upper nibble, the third in the lower one.
   asm("{\n\t.reg .b8 q0, q1, q2, q3;\n\t"
       "cvt.rn.satfinite.e2m1x2.f32 q0, %2, %1;\n\t"
       "cvt.rn.satfinite.e2m1x2.f32 q1, %4, %3;\n\t"
@@ -128,13 +166,13 @@ __device__ __forceinline__ uint32_t cvt_e2m1x8(float a0, float a1, float a2, flo
       "cvt.rn.satfinite.e2m1x2.f32 q3, %8, %7;\n\t"
       "mov.b32 %0, {q0, q1, q2, q3};\n\t}"
       : "=r"(r)
-      : "f"(a0), "f"(a1), "f"(a2), "f"(a3), "f"(a4), "f"(a5), "f"(a6), "f"(a7));
+      : "f"(bf_lo(s[0])), "f"(bf_hi(s[0])), "f"(bf_lo(s[1])), "f"(bf_hi(s[1])),
+        "f"(bf_lo(s[2])), "f"(bf_hi(s[2])), "f"(bf_lo(s[3])), "f"(bf_hi(s[3])));
   return r;
 }
 
-// Eight scaled values -> eight E4M3 bytes, element i in byte i.
-__device__ __forceinline__ uint2 cvt_e4m3x8(float a0, float a1, float a2, float a3, float a4,
-                                            float a5, float a6, float a7) {
+// Four bf16x2 words -> eight E4M3 bytes, element i in byte i.
+__device__ __forceinline__ uint2 cvt_e4m3x8(const uint32_t s[4]) {
   uint2 r;
   asm("{\n\t.reg .b16 h0, h1, h2, h3;\n\t"
       "cvt.rn.satfinite.e4m3x2.f32 h0, %3, %2;\n\t"
@@ -144,49 +182,51 @@ __device__ __forceinline__ uint2 cvt_e4m3x8(float a0, float a1, float a2, float 
       "mov.b32 %0, {h0, h1};\n\t"
       "mov.b32 %1, {h2, h3};\n\t}"
       : "=r"(r.x), "=r"(r.y)
-      : "f"(a0), "f"(a1), "f"(a2), "f"(a3), "f"(a4), "f"(a5), "f"(a6), "f"(a7));
+      : "f"(bf_lo(s[0])), "f"(bf_hi(s[0])), "f"(bf_lo(s[1])), "f"(bf_hi(s[1])),
+        "f"(bf_lo(s[2])), "f"(bf_hi(s[2])), "f"(bf_lo(s[3])), "f"(bf_hi(s[3])));
   return r;
 }
 
-// The 8 bf16 of a chunk, each multiplied by m (exact for a power of two m).
-struct F8 {
-  float v[8];
-};
-__device__ __forceinline__ F8 scaled8(const uint4& x, float m) {
-  F8 r;
-  r.v[0] = bf_lo(x.x) * m; r.v[1] = bf_hi(x.x) * m;
-  r.v[2] = bf_lo(x.y) * m; r.v[3] = bf_hi(x.y) * m;
-  r.v[4] = bf_lo(x.z) * m; r.v[5] = bf_hi(x.z) * m;
-  r.v[6] = bf_lo(x.w) * m; r.v[7] = bf_hi(x.w) * m;
-  return r;
+// The slice scaled by 2^-E (byte b), as bf16x2 words.
+__device__ __forceinline__ V16 scale_slice(const V16& x, int b) {
+  const uint32_t m = inv_scale_bf16x2(b);
+  V16 s;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) s.w[i] = mul_bf16x2(x.w[i], m);
+  return s;
 }
 
-__device__ __forceinline__ uint32_t enc_e2m1_8(const F8& s) {
-  return cvt_e2m1x8(s.v[0], s.v[1], s.v[2], s.v[3], s.v[4], s.v[5], s.v[6], s.v[7]);
+// 16 E2M1 codes of a scaled slice: nibble i of the result = element i.
+__device__ __forceinline__ uint2 enc_e2m1_16(const V16& s) {
+  return make_uint2(cvt_e2m1x8(&s.w[0]), cvt_e2m1x8(&s.w[4]));
 }
-__device__ __forceinline__ uint2 enc_e4m3_8(const F8& s) {
-  return cvt_e4m3x8(s.v[0], s.v[1], s.v[2], s.v[3], s.v[4], s.v[5], s.v[6], s.v[7]);
+// 16 E4M3 bytes of a scaled slice: byte i = element i.
+__device__ __forceinline__ uint4 enc_e4m3_16(const V16& s) {
+  const uint2 a = cvt_e4m3x8(&s.w[0]);
+  const uint2 b = cvt_e4m3x8(&s.w[4]);
+  return make_uint4(a.x, a.y, b.x, b.y);
 }
 
-// Sign-only codes of a block holding NaN/Inf (E2M1: no NaN exists, so only the
-// sign survives; E4M3: S.1111.111, the NaN code).
-__device__ __forceinline__ uint32_t nonfinite_e2m1_8(const uint4& x) {
-  const uint32_t w[4] = {x.x, x.y, x.z, x.w};
-  uint32_t r = 0;
+// Codes of a block holding NaN/Inf: E2M1 has no NaN, so only the sign
+// survives; E4M3 elements become S.1111.111, the NaN code.
+__device__ __forceinline__ uint2 nonfinite_e2m1_16(const V16& x) {
+  uint32_t r[2] = {0, 0};
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    r[i >> 2] |= ((x.w[i] >> 15) & 1u) << (8 * (i & 3) + 3);
+    r[i >> 2] |= ((x.w[i] >> 31) & 1u) << (8 * (i & 3) + 7);
+  }
+  return make_uint2(r[0], r[1]);
+}
+__device__ __forceinline__ uint4 nonfinite_e4m3_16(const V16& x) {
+  uint32_t r[4];
 #pragma unroll
   for (int j = 0; j < 4; ++j) {
-    r |= ((w[j] >> 15) & 1u) << (8 * j + 3);
-    r |= ((w[j] >> 31) & 1u) << (8 * j + 7);
+    const uint32_t a = x.w[2 * j], b = x.w[2 * j + 1];
+    r[j] = (((a >> 15) & 1u) << 7 | 0x7Fu) | ((((a >> 31) & 1u) << 7 | 0x7Fu) << 8) |
+           ((((b >> 15) & 1u) << 7 | 0x7Fu) << 16) | ((((b >> 31) & 1u) << 7 | 0x7Fu) << 24);
   }
-  return r;
-}
-__device__ __forceinline__ uint2 nonfinite_e4m3_8(const uint4& x) {
-  const uint32_t w[4] = {x.x, x.y, x.z, x.w};
-  uint32_t b[4];
-#pragma unroll
-  for (int j = 0; j < 4; ++j)
-    b[j] = (((w[j] >> 15) & 1u) << 7 | 0x7Fu) | ((((w[j] >> 31) & 1u) << 7 | 0x7Fu) << 8);
-  return make_uint2(b[0] | (b[1] << 16), b[2] | (b[3] << 16));
+  return make_uint4(r[0], r[1], r[2], r[3]);
 }
 
 // ------------------------------------------------------- element decoding --
@@ -213,21 +253,19 @@ __device__ __forceinline__ uint2 e2m1x4_to_bf16(uint32_t c) {
   return make_uint2(w0, w1);
 }
 
-// Eight E2M1 codes (nibble i = element i) -> eight bf16 values (unscaled).
-__device__ __forceinline__ uint4 e2m1x8_to_bf16(uint32_t codes) {
-  const uint2 a = e2m1x4_to_bf16(codes & 0xFFFFu);
-  const uint2 b = e2m1x4_to_bf16(codes >> 16);
-  return make_uint4(a.x, a.y, b.x, b.y);
-}
-
-// E2M1 codes -> unscaled values as floats (exact).
-__device__ __forceinline__ F8 dec_e2m1_8(uint32_t codes) {
-  const uint4 b = e2m1x8_to_bf16(codes);
-  F8 r;
-  r.v[0] = bf_lo(b.x); r.v[1] = bf_hi(b.x);
-  r.v[2] = bf_lo(b.y); r.v[3] = bf_hi(b.y);
-  r.v[4] = bf_lo(b.z); r.v[5] = bf_hi(b.z);
-  r.v[6] = bf_lo(b.w); r.v[7] = bf_hi(b.w);
+// 16 E2M1 codes -> the 16 unscaled values as bf16 bit patterns.
+__device__ __forceinline__ V16 e2m1x16_to_bf16(uint2 codes) {
+  V16 r;
+  const uint32_t c[2] = {codes.x, codes.y};
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const uint2 a = e2m1x4_to_bf16(c[h] & 0xFFFFu);
+    const uint2 b = e2m1x4_to_bf16(c[h] >> 16);
+    r.w[4 * h + 0] = a.x;
+    r.w[4 * h + 1] = a.y;
+    r.w[4 * h + 2] = b.x;
+    r.w[4 * h + 3] = b.y;
+  }
   return r;
 }
 
@@ -240,13 +278,19 @@ __device__ __forceinline__ float e4m3_to_f32(uint32_t c) {
   return (c & 0x80u) ? -v : v;
 }
 
-__device__ __forceinline__ F8 dec_e4m3_8(uint2 codes) {
-  F8 r;
+// Decoded values times p (a power of two): exact floats, overflow to +-inf.
+__device__ __forceinline__ F16 dec_e2m1_16(uint2 codes, float p) {
+  const V16 b = e2m1x16_to_bf16(codes);
+  F16 r;
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    r.v[i] = e4m3_to_f32((codes.x >> (8 * i)) & 0xFFu);
-    r.v[4 + i] = e4m3_to_f32((codes.y >> (8 * i)) & 0xFFu);
-  }
+  for (int i = 0; i < 16; ++i) r.v[i] = elem(b, i) * p;
+  return r;
+}
+__device__ __forceinline__ F16 dec_e4m3_16(uint4 codes, float p) {
+  const uint32_t c[4] = {codes.x, codes.y, codes.z, codes.w};
+  F16 r;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) r.v[i] = e4m3_to_f32((c[i >> 2] >> (8 * (i & 3))) & 0xFFu) * p;
   return r;
 }
 
@@ -287,24 +331,23 @@ __device__ __forceinline__ int rule_byte(uint32_t amax) {
   return max(b, 0);
 }
 
-// Exact OAS comparison for one lane's 8 elements (E2M1, no macro factor):
-// returns sum over the elements of (D1^2 - D2^2) with D = 512 * (s - q), s the
-// value scaled by the finer candidate 2^-E1 and q its dequantized value in the
-// same units under each candidate (E2 = E1 + 1). Elements that quantize to
+// Exact OAS comparison for one lane's 16 elements (E2M1, no macro factor):
+// the sum over the elements of D1^2 - D2^2 with D = 512 (s - q): s the value
+// scaled by the finer candidate 2^-E1 (byte b1) and q its dequantized value in
+// the same units under each candidate (E2 = E1 + 1). Elements that quantize to
 // zero under both have D1 == D2 and cancel; every other D is an integer below
-// 2^11, so the int32 sum over a block is exact.
-__device__ __forceinline__ int oas_delta8(const uint4& x, float inv1) {
-  const F8 s1 = scaled8(x, inv1);
-  F8 s2;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) s2.v[i] = s1.v[i] * 0.5f;
-  const F8 q1 = dec_e2m1_8(enc_e2m1_8(s1));
-  const F8 q2 = dec_e2m1_8(enc_e2m1_8(s2));
+// 2^11 (s then has at least 2^-9 resolution), so the int32 sum is exact.
+__device__ __forceinline__ int oas_delta16(const V16& x, int b1) {
+  const V16 s1 = scale_slice(x, b1);
+  const V16 s2 = scale_slice(x, b1 + 1);
+  const V16 q1 = e2m1x16_to_bf16(enc_e2m1_16(s1));
+  const V16 q2 = e2m1x16_to_bf16(enc_e2m1_16(s2));
   int acc = 0;
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int d1 = __float2int_rn((s1.v[i] - q1.v[i]) * 512.0f);
-    const int d2 = __float2int_rn((s1.v[i] - 2.0f * q2.v[i]) * 512.0f);
+  for (int i = 0; i < 16; ++i) {
+    const float s = elem(s1, i);
+    const int d1 = __float2int_rn((s - elem(q1, i)) * 512.0f);
+    const int d2 = __float2int_rn((s - 2.0f * elem(q2, i)) * 512.0f);
     acc += d1 * d1 - d2 * d2;
   }
   return acc;
@@ -331,14 +374,15 @@ __device__ __forceinline__ int mbs_static_k(uint32_t A) {
   return (c * S + 2) / 3 - 256;
 }
 
-// E8M0 byte of a sub-block under factor k (FLOOR): floor(log2(amax / f)) - 2,
+// E8M0 byte of a sub-block under factor k: floor(log2(amax / f)) - 2 + up,
 // where dividing by f lowers the exponent by one exactly when the amax
-// significand 1 + m7/128 is below f = 1 + k/256, i.e. 2 m7 < k.
-__device__ __forceinline__ int mbs_floor_byte(uint32_t amax, int k) {
+// significand 1 + m7/128 is below f = 1 + k/256, i.e. 2 m7 < k. up = 0 gives
+// the FLOOR byte, up = 1 the next coarser one (the OAS candidate).
+__device__ __forceinline__ int mbs_byte(uint32_t amax, int k, int up) {
   const int ex = static_cast<int>(amax >> 7);
   if (ex == 0) return 0;
   const int m7 = static_cast<int>(amax & 0x7F);
-  return max(ex - 2 - ((2 * m7 < k) ? 1 : 0), 0);
+  return max(ex - 2 + up - ((2 * m7 < k) ? 1 : 0), 0);
 }
 
 // Grid midpoints of E2M1 times f = (256 + k) / 256, for rounding the scaled
@@ -366,36 +410,31 @@ __device__ __forceinline__ int mbs_round(float s, const Thresholds& T) {
 // E2M1 magnitude (in units of 0.5) of code c: 0 1 2 3 4 6 8 12.
 __device__ __forceinline__ int e2m1_halves(int c) { return (0xC8643210u >> (4 * c)) & 0xF; }
 
-// Eight codes under factor k and exponent byte b (b in [0, 253]).
-__device__ __forceinline__ uint32_t enc_mbs_8(const uint4& x, int b, const Thresholds& T) {
+// 16 codes under factor k and exponent byte b (b in [0, 253]).
+__device__ __forceinline__ uint2 enc_mbs_16(const V16& x, int b, const Thresholds& T) {
   const float m = inv_scale_from_byte(b);   // 2^-E, exact
-  const uint32_t w[4] = {x.x, x.y, x.z, x.w};
-  uint32_t r = 0;
+  uint32_t r[2] = {0, 0};
 #pragma unroll
-  for (int j = 0; j < 4; ++j) {
-    const float tlo = fabsf(bf_lo(w[j])) * m;
-    const float thi = fabsf(bf_hi(w[j])) * m;
-    const uint32_t clo = static_cast<uint32_t>(mbs_round(tlo, T)) | (((w[j] >> 15) & 1u) << 3);
-    const uint32_t chi = static_cast<uint32_t>(mbs_round(thi, T)) | (((w[j] >> 31) & 1u) << 3);
-    r |= (clo | (chi << 4)) << (8 * j);
+  for (int i = 0; i < 16; ++i) {
+    const uint32_t sign = (x.w[i >> 1] >> ((i & 1) ? 31 : 15)) & 1u;
+    const uint32_t c = static_cast<uint32_t>(mbs_round(fabsf(elem(x, i)) * m, T)) | (sign << 3);
+    r[i >> 3] |= c << (4 * (i & 7));
   }
-  return r;
+  return make_uint2(r[0], r[1]);
 }
 
-// Exact OAS comparison of one lane's 8 elements under factor k: candidates
+// Exact OAS comparison of one lane's 16 elements under factor k: candidates
 // E1 (byte b1) and E1 + 1. D = 512 s - h (256 + k) with s = |x| 2^-E1 and h
 // the code magnitude in units of 0.5 (doubled for the coarser candidate): an
 // integer below 2^12 for every element that does not round to zero under both.
-__device__ __forceinline__ int oas_delta_mbs8(const uint4& x, int b1, const Thresholds& T,
-                                              int k) {
+__device__ __forceinline__ int oas_delta_mbs16(const V16& x, int b1, const Thresholds& T,
+                                               int k) {
   const float inv1 = inv_scale_from_byte(b1);
   const float fk = static_cast<float>(256 + k);
-  const uint32_t w[4] = {x.x, x.y, x.z, x.w};
   int acc = 0;
 #pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    const uint32_t word = w[j >> 1];
-    const float s = fabsf((j & 1) ? bf_hi(word) : bf_lo(word)) * inv1;
+  for (int i = 0; i < 16; ++i) {
+    const float s = fabsf(elem(x, i)) * inv1;
     const int c1 = mbs_round(s, T);
     const int c2 = mbs_round(s * 0.5f, T);
     const float d1 = s * 512.0f - static_cast<float>(e2m1_halves(c1)) * fk;

@@ -36,8 +36,10 @@
  * flags. All entry points are thread-safe.
  * Empty inputs (rows == 0 or cols == 0) are valid and launch nothing (except
  * that mx_block_error still zeroes its totals).
- * Alignment: x, grad, y, out and codes pointers must be 16-byte aligned;
- * block_sse 4-byte, totals 8-byte; scales and macro have no requirement.
+ * Alignment: x, grad_y, grad_x, y and out must be 32-byte aligned (the
+ * kernels move 32 bytes per lane), codes 16-byte; block_sse 4-byte, totals
+ * 8-byte; scales and macro have no requirement. (torch allocations are
+ * 512-byte aligned; a view that starts mid-buffer may not be.)
  */
 #ifndef MX_H_
 #define MX_H_

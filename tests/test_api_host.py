@@ -16,7 +16,7 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 HEADER = os.path.join(ROOT, "include", "mx.h")
 
 OK, INVALID, SHAPE, ALIGN, UNSUPPORTED, CUDA_ERR = 0, 1, 2, 3, 4, 5
-A = 0x10000          # a 16-byte aligned fake device address (never dereferenced)
+A = 0x10000          # a 256-byte aligned fake device address (never dereferenced)
 
 
 def declared_functions():
@@ -81,7 +81,9 @@ def test_quantize_rejects_shapes_and_pointers(mx):
     assert q(A, 4, 32, 0, 0, A, None, None, 0) == INVALID
     assert q(A, 4, 128, 0, 0x10, A, A, None, 0) == INVALID   # MBS needs macro
     assert q(A + 8, 4, 32, 0, 0, A, A, None, 0) == ALIGN
+    assert q(A + 16, 4, 32, 0, 0, A, A, None, 0) == ALIGN     # x needs 32 bytes
     assert q(A, 4, 32, 0, 0, A + 4, A, None, 0) == ALIGN
+    assert q(A, 4, 32, 0, 0, A + 8, A, None, 0) == ALIGN      # codes need 16
     # scales and macro may sit at any byte address: this one only fails on x
     assert q(A + 2, 4, 128, 0, 0x10, A, A + 1, A + 3, 0) == ALIGN
     # empty inputs are valid and launch nothing (pointers are not needed)
@@ -102,6 +104,8 @@ def test_other_entry_points_validate(mx):
     assert mx.mx_fake_quant_fwd(A, 4, 48, 0, 0, A, None, 0) == SHAPE
     assert mx.mx_fake_quant_fwd(A, 4, 32, 0, 0, None, None, 0) == INVALID
     assert mx.mx_fake_quant_fwd(A, 4, 32, 0, 0, A + 8, None, 0) == ALIGN
+    assert mx.mx_fake_quant_fwd(A, 4, 32, 0, 0, A + 16, None, 0) == ALIGN
+    assert mx.mx_dequantize(A, A, None, 4, 32, 0, 0, A + 16, 0) == ALIGN
     assert mx.mx_fake_quant_bwd(A, A, 4, 32, 0, 0, A + 8, 0) == ALIGN
     assert mx.mx_fake_quant_bwd(A, None, 4, 32, 0, 0, A, 0) == INVALID
     assert mx.mx_fake_quant_bwd(A, A, 4, 64, 0, 0x20, A, 0) == SHAPE
