@@ -24,8 +24,9 @@
 //  * with a macro factor f = (256 + k) / 256 the quotient x / (f 2^E) is not
 //    exact, so s = |x| 2^-E (exact, below 16) is compared with the grid
 //    midpoints times f (exact); equality goes to the even code;
-//  * decoding (fake-quant, error, dequantize) is integer only: a byte-permute
-//    table for E2M1 and bit assembly for E4M3, then an exact float product.
+//  * decoding (fake-quant, error, dequantize): a byte-permute table for E2M1
+//    (integer only) and the hardware cvt.rn.f16x2.e4m3x2 for E4M3 (exact),
+//    then an exact float product with the scale.
 #pragma once
 
 #include <cstdint>
@@ -231,10 +232,11 @@ __device__ __forceinline__ uint4 nonfinite_e4m3_16(const V16& x) {
 
 // ------------------------------------------------------- element decoding --
 //
-// Decoding is done with integer operations only. (Feeding the register output
+// E2M1 is decoded with integer operations only. (Feeding the register output
 // of cvt.rn.satfinite.e2m1x2.f32 straight into cvt.rn.f16x2.e2m1x2 gave
 // zeros on sm_100a in this build, while the same decode of codes loaded from
-// memory was right; a table lookup avoids depending on that register path.)
+// memory was right; a table lookup avoids depending on that register path.
+// The E4M3 pair of conversions showed no such problem in either path.)
 
 // E2M1 magnitudes 0 .5 1 1.5 2 3 4 6 as bf16 bit patterns, split into their
 // high and low bytes, four entries per 32-bit word (index 0..3, 4..7).
@@ -269,13 +271,30 @@ __device__ __forceinline__ V16 e2m1x16_to_bf16(uint2 codes) {
   return r;
 }
 
-// One E4M3fn byte -> float (S.1111.111 -> NaN; subnormals m * 2^-9).
-__device__ __forceinline__ float e4m3_to_f32(uint32_t c) {
-  const uint32_t ef = (c >> 3) & 15u, m = c & 7u;
-  float v = ef ? __uint_as_float(((ef + 120u) << 23) | (m << 20))
-               : static_cast<float>(m) * 0.001953125f;        // m * 2^-9, exact
-  if (ef == 15u && m == 7u) v = __uint_as_float(kNaNf32);
-  return (c & 0x80u) ? -v : v;
+// Eight E4M3fn bytes (byte i = element i) -> four f16x2 words, exact (every
+// E4M3 value is an f16 value; S.1111.111 becomes an f16 NaN). This hardware
+// decode is exact for E4M3 both from memory and from the encoder's registers.
+__device__ __forceinline__ void e4m3x8_to_f16x2(uint32_t lo, uint32_t hi, uint32_t h[4]) {
+  asm("{\n\t.reg .b16 p0, p1, p2, p3;\n\t"
+      "mov.b32 {p0, p1}, %4;\n\t"
+      "mov.b32 {p2, p3}, %5;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %0, p0;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %1, p1;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %2, p2;\n\t"
+      "cvt.rn.f16x2.e4m3x2 %3, p3;\n\t}"
+      : "=r"(h[0]), "=r"(h[1]), "=r"(h[2]), "=r"(h[3])
+      : "r"(lo), "r"(hi));
+}
+
+__device__ __forceinline__ float f16_lo(uint32_t h) {
+  float f;
+  asm("{\n\t.reg .b16 a, b;\n\tmov.b32 {a, b}, %1;\n\tcvt.f32.f16 %0, a;\n\t}" : "=f"(f) : "r"(h));
+  return f;
+}
+__device__ __forceinline__ float f16_hi(uint32_t h) {
+  float f;
+  asm("{\n\t.reg .b16 a, b;\n\tmov.b32 {a, b}, %1;\n\tcvt.f32.f16 %0, b;\n\t}" : "=f"(f) : "r"(h));
+  return f;
 }
 
 // Decoded values times p (a power of two): exact floats, overflow to +-inf.
@@ -287,10 +306,15 @@ __device__ __forceinline__ F16 dec_e2m1_16(uint2 codes, float p) {
   return r;
 }
 __device__ __forceinline__ F16 dec_e4m3_16(uint4 codes, float p) {
-  const uint32_t c[4] = {codes.x, codes.y, codes.z, codes.w};
+  uint32_t h[8];
+  e4m3x8_to_f16x2(codes.x, codes.y, &h[0]);
+  e4m3x8_to_f16x2(codes.z, codes.w, &h[4]);
   F16 r;
 #pragma unroll
-  for (int i = 0; i < 16; ++i) r.v[i] = e4m3_to_f32((c[i >> 2] >> (8 * (i & 3))) & 0xFFu) * p;
+  for (int i = 0; i < 8; ++i) {
+    r.v[2 * i] = f16_lo(h[i]) * p;
+    r.v[2 * i + 1] = f16_hi(h[i]) * p;
+  }
   return r;
 }
 
@@ -331,26 +355,37 @@ __device__ __forceinline__ int rule_byte(uint32_t amax) {
   return max(b, 0);
 }
 
-// Exact OAS comparison for one lane's 16 elements (E2M1, no macro factor):
-// the sum over the elements of D1^2 - D2^2 with D = 512 (s - q): s the value
-// scaled by the finer candidate 2^-E1 (byte b1) and q its dequantized value in
-// the same units under each candidate (E2 = E1 + 1). Elements that quantize to
-// zero under both have D1 == D2 and cancel; every other D is an integer below
-// 2^11 (s then has at least 2^-9 resolution), so the int32 sum is exact.
-__device__ __forceinline__ int oas_delta16(const V16& x, int b1) {
+// OAS evaluation of one lane's 16 elements (E2M1, no macro factor): the codes
+// under both candidates, E1 (byte b1) and E2 = E1 + 1, and the exact
+// difference of their squared errors in units of 2^-10 of the E1 scale,
+//   delta = sum over the elements of (d1^2 - d2^2) = sum (d1 - d2)(d1 + d2),
+// with s = x 2^-E1, d1 = s - q1, d2 = s - 2 q2 (q the code values). Where
+// both codes are zero, d1 == d2 and the term is exactly 0. Elsewhere s has
+// 2^-9 resolution, d1 - d2 = 2 q2 - q1 (a multiple of 1/2, at most 8) and
+// d1 + d2 (a multiple of 2^-9, below 4) multiply exactly, and the running sum
+// of 16 such terms (multiples of 2^-10, each below 4) stays exact in float.
+struct OasEval {
+  uint2 c1, c2;
+  int delta;
+};
+__device__ __forceinline__ OasEval oas_eval16(const V16& x, int b1) {
   const V16 s1 = scale_slice(x, b1);
   const V16 s2 = scale_slice(x, b1 + 1);
-  const V16 q1 = e2m1x16_to_bf16(enc_e2m1_16(s1));
-  const V16 q2 = e2m1x16_to_bf16(enc_e2m1_16(s2));
-  int acc = 0;
+  OasEval r;
+  r.c1 = enc_e2m1_16(s1);
+  r.c2 = enc_e2m1_16(s2);
+  const V16 q1 = e2m1x16_to_bf16(r.c1);
+  const V16 q2 = e2m1x16_to_bf16(r.c2);
+  float acc = 0.0f;
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
     const float s = elem(s1, i);
-    const int d1 = __float2int_rn((s - elem(q1, i)) * 512.0f);
-    const int d2 = __float2int_rn((s - 2.0f * elem(q2, i)) * 512.0f);
-    acc += d1 * d1 - d2 * d2;
+    const float d1 = s - elem(q1, i);
+    const float d2 = fmaf(-2.0f, elem(q2, i), s);
+    acc = fmaf(d1 - d2, d1 + d2, acc);
   }
-  return acc;
+  r.delta = __float2int_rn(acc * 1024.0f);   // an integer below 2^16: exact
+  return r;
 }
 
 // ------------------------------------------------ macro-factor arithmetic --

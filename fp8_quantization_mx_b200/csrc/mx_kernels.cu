@@ -49,9 +49,11 @@ constexpr int kThreads = MX_THREADS;
 
 // Per-block scale state as both lanes of the block see it.
 struct BlockScale {
-  int byte;       // E8M0 byte (255 for a non-finite block)
-  int k;          // macro factor index (0 without MBS)
+  int byte;          // E8M0 byte (255 for a non-finite block)
+  int k;             // macro factor index (0 without MBS)
   bool nonfinite;
+  bool have_codes;   // codes below already hold this lane's E2M1 codes (OAS)
+  uint2 codes;
 };
 
 // Scale decision for the block holding `v`; pa = the block amax bits. Every
@@ -61,6 +63,8 @@ __device__ __forceinline__ BlockScale decide_scale(const V16& v, uint32_t pa, in
   BlockScale s;
   s.nonfinite = pa >= 0x7F80u;
   s.k = k;
+  s.have_codes = false;
+  s.codes = make_uint2(0, 0);
   if (MBS == kMbsNone) {
     s.byte = rule_byte<FMT, RULE>(pa);
     if (RULE == kOas) {
@@ -68,9 +72,12 @@ __device__ __forceinline__ BlockScale decide_scale(const V16& v, uint32_t pa, in
       // for a max significand <= 1.75 the finer grid is element-wise no worse
       const bool need = !s.nonfinite && (pa & 0x7F) > 96 && b2 != s.byte;
       if (__any_sync(kFull, need)) {
-        int d = oas_delta16(v, s.byte);
-        d += __shfl_xor_sync(kFull, d, 1);
-        if (need && d > 0) s.byte = b2;
+        const OasEval e = oas_eval16(v, s.byte);
+        const int d = e.delta + __shfl_xor_sync(kFull, e.delta, 1);
+        const bool up = need && d > 0;
+        if (up) s.byte = b2;
+        s.codes = up ? e.c2 : e.c1;   // the codes of the chosen scale
+        s.have_codes = true;
       }
     }
   } else {
@@ -93,6 +100,7 @@ __device__ __forceinline__ BlockScale decide_scale(const V16& v, uint32_t pa, in
 template <int MBS>
 __device__ __forceinline__ uint2 codes_fp4(const V16& v, const BlockScale& s) {
   if (s.nonfinite) return nonfinite_e2m1_16(v);
+  if (s.have_codes) return s.codes;
   if (MBS == kMbsNone) return enc_e2m1_16(scale_slice(v, s.byte));
   return enc_mbs_16(v, s.byte, mbs_thresholds(s.k));
 }
@@ -450,7 +458,7 @@ int grid_for(K kernel, int64_t tiles, int waves = MX_GRID_WAVES) {
 constexpr int kUnroll = MX_STREAM_UNROLL;
 // Slices per lane in flight in the dequantize kernel.
 #ifndef MX_DEQUANT_UNROLL
-#define MX_DEQUANT_UNROLL 2
+#define MX_DEQUANT_UNROLL 4
 #endif
 
 template <int OP, int FMT, int RULE, int MBS>

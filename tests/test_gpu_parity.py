@@ -71,7 +71,12 @@ def special_blocks():
     # pad to a whole number of 128-element macro rows
     pad = (-len(arr)) % 4
     arr = np.concatenate([arr, np.zeros((pad, 32), np.uint16)])
-    return arr.reshape(-1, 128)
+    # a macro block made only of subnormals (its MBS factor comes from a
+    # subnormal maximum), and one of mixed-sign subnormals and zeros
+    sub = (np.arange(128, dtype=np.uint16) % 127 + 1)
+    mixed = np.where(np.arange(128) % 3 == 0, 0, sub | np.where(np.arange(128) % 2, 0x8000, 0))
+    arr = np.concatenate([arr.reshape(-1, 128), sub[None], mixed.astype(np.uint16)[None]])
+    return arr
 
 
 SMALL = {
