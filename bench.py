@@ -186,7 +186,7 @@ def run_reference(args):
     threads = len(os.sched_getaffinity(0))
     oracle.set_threads(threads)
     # a few experts of the same seeded stack, generated on the host
-    x = inputs.moe_w13(experts=4, device="cpu")
+    x = inputs.moe_w13(experts=16, device="cpu")
     xb = inputs.bf16_bits_numpy(x).reshape(-1, HIDDEN)
     t0 = time.perf_counter()
     oracle.quantize(xb[:512], 0, 0)
@@ -297,6 +297,7 @@ def run_mx(args):
     import fp8_quantization_mx_b200 as mx
     from fp8_quantization_mx_b200 import build as mxbuild
     from fp8_quantization_mx_b200 import inputs
+    from fp8_quantization_mx_b200.sharding import max_over_ranks
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -349,9 +350,7 @@ def run_mx(args):
     total_ms = t_start.elapsed_time(t_end)
     launch_ms = sum(s.elapsed_time(e) for s, e in ev) / len(ev)
     if world > 1:
-        t = torch.tensor([total_ms, launch_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        total_ms, launch_ms = t.tolist()
+        total_ms, launch_ms = max_over_ranks([total_ms, launch_ms], dev)
     ms_per_step = total_ms / args.steps
     value = world * BYTES_STEP / (ms_per_step * 1e-3) / 1e9
 
@@ -372,9 +371,7 @@ def run_mx(args):
     torch.cuda.synchronize()
     e2e_ms = e0.elapsed_time(e1) / e2e_steps
     if world > 1:
-        t = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        e2e_ms = t.item()
+        (e2e_ms,) = max_over_ranks([e2e_ms], dev)
     e2e = {"value": world * BYTES_STEP / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
            "h2d_bytes_per_step": BYTES_IN, "d2h_bytes_per_step": BYTES_CODES + BYTES_SCALES,
            "ms_per_step": e2e_ms}

@@ -22,8 +22,10 @@
 //    zero code anyway, so the scaled pairs feed the hardware conversions
 //    cvt.rn.satfinite.{e2m1x2,e4m3x2}.f32 (round to nearest even, saturate);
 //  * with a macro factor f = (256 + k) / 256 the quotient x / (f 2^E) is not
-//    exact, so s = |x| 2^-E (exact, below 16) is compared with the grid
-//    midpoints times f (exact); equality goes to the even code;
+//    exact in float; it is bracketed by two products with 1/f rounded down
+//    and up, both bounds go through the hardware conversion, and the only way
+//    they can disagree is an exact tie, where the even code wins (see
+//    enc_mbs_cvt_16);
 //  * decoding (fake-quant, error, dequantize): a byte-permute table for E2M1
 //    (integer only) and the hardware cvt.rn.f16x2.e4m3x2 for E4M3 (exact),
 //    then an exact float product with the scale.
@@ -420,64 +422,134 @@ __device__ __forceinline__ int mbs_byte(uint32_t amax, int k, int up) {
   return max(ex - 2 + up - ((2 * m7 < k) ? 1 : 0), 0);
 }
 
-// Grid midpoints of E2M1 times f = (256 + k) / 256, for rounding the scaled
-// magnitude s = |x| 2^-E (which is below 16, so it never overflows). Each
-// threshold mid * (256 + k) / 256 has at most 12 significant bits: exact.
-struct Thresholds {
-  float t[7];
+// Eight floats -> eight E2M1 codes, element i in nibble i.
+__device__ __forceinline__ uint32_t cvt_e2m1_f8(const float* v) {
+  uint32_t r;
+  asm("{\n\t.reg .b8 q0, q1, q2, q3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 q0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 q1, %4, %3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 q2, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 q3, %8, %7;\n\t"
+      "mov.b32 %0, {q0, q1, q2, q3};\n\t}"
+      : "=r"(r)
+      : "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]));
+  return r;
+}
+
+// Bracket of 1/f for f = (256 + k) / 256: L <= 1/f <= H, both within 2^-20.
+struct FactorBracket {
+  float f, L, H;
 };
-__device__ __forceinline__ Thresholds mbs_thresholds(int k) {
-  const float f = static_cast<float>(256 + k) * 0.00390625f;   // (256 + k) / 256
-  Thresholds T;
-  T.t[0] = 0.25f * f; T.t[1] = 0.75f * f; T.t[2] = 1.25f * f; T.t[3] = 1.75f * f;
-  T.t[4] = 2.5f * f;  T.t[5] = 3.5f * f;  T.t[6] = 5.0f * f;
-  return T;
+__device__ __forceinline__ FactorBracket factor_bracket(int k) {
+  FactorBracket r;
+  r.f = static_cast<float>(256 + k) * 0.00390625f;                    // exact
+  const float inv = __fdiv_rn(256.0f, static_cast<float>(256 + k));   // 1/f, rounded
+  r.L = inv * 0.99999904632568359375f;                                // 1 - 2^-20
+  r.H = inv * 1.00000095367431640625f;                                // 1 + 2^-20
+  return r;
 }
 
-// Magnitude code 0..7 of s = |x| 2^-E under the factor f. At a midpoint
-// between an even and an odd code the even one wins: strictly above is needed
-// to leave an even code, reaching the midpoint suffices to leave an odd one.
-__device__ __forceinline__ int mbs_round(float s, const Thresholds& T) {
-  return (s > T.t[0]) + (s >= T.t[1]) + (s > T.t[2]) + (s >= T.t[3]) + (s > T.t[4]) +
-         (s >= T.t[5]) + (s > T.t[6]);
+// Of two nibble-packed code words that agree except where an element's codes
+// are adjacent (c, c+1), keep the even code of each such pair: those bits
+// differ in bit 0, and the odd one of the pair is the one with bit 0 set.
+__device__ __forceinline__ uint32_t even_of_adjacent(uint32_t lo, uint32_t hi) {
+  const uint32_t diff = lo ^ hi;
+  const uint32_t take_hi = (lo & diff & 0x11111111u) * 0xFu;   // nibbles where lo is odd
+  return lo ^ (diff & take_hi);
 }
 
-// E2M1 magnitude (in units of 0.5) of code c: 0 1 2 3 4 6 8 12.
-__device__ __forceinline__ int e2m1_halves(int c) { return (0xC8643210u >> (4 * c)) & 0xF; }
-
-// 16 codes under factor k and exponent byte b (b in [0, 253]).
-__device__ __forceinline__ uint2 enc_mbs_16(const V16& x, int b, const Thresholds& T) {
-  const float m = inv_scale_from_byte(b);   // 2^-E, exact
-  uint32_t r[2] = {0, 0};
+// MBS codes of 16 elements under factor k and exponent byte b, rounded
+// exactly with the hardware converter. The quotient q = s / f (s = x 2^-E
+// exact, f = (256 + k) / 256) is not exact in float, but it is bracketed: with
+// L <= 1/f <= H (within 2^-20 of 1/f, with margin for float rounding),
+// fl(s L) <= |q| <= fl(s H) in magnitude. Rounding to the grid is monotone,
+// so both bounds give the code of q unless the bracket holds a grid midpoint.
+// It can hold one only when q is exactly that midpoint: s has 8 significant
+// bits and mid * f is a multiple of 2^-10, so a q that is not a midpoint lies
+// at least 2^-10 / 10 (relatively) away from every one, far outside the
+// 2^-19 bracket. At a tie the bounds give the two adjacent codes, and the
+// even one is the round-to-nearest-even result.
+__device__ __forceinline__ uint2 enc_mbs_cvt_16(const V16& x, int b, int k) {
+  const FactorBracket fb = factor_bracket(k);
+  const V16 s = scale_slice(x, b);
+  float lo[16], hi[16];
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
-    const uint32_t sign = (x.w[i >> 1] >> ((i & 1) ? 31 : 15)) & 1u;
-    const uint32_t c = static_cast<uint32_t>(mbs_round(fabsf(elem(x, i)) * m, T)) | (sign << 3);
-    r[i >> 3] |= c << (4 * (i & 7));
+    const float e = elem(s, i);
+    lo[i] = e * fb.L;
+    hi[i] = e * fb.H;
   }
-  return make_uint2(r[0], r[1]);
+  return make_uint2(even_of_adjacent(cvt_e2m1_f8(lo), cvt_e2m1_f8(hi)),
+                    even_of_adjacent(cvt_e2m1_f8(lo + 8), cvt_e2m1_f8(hi + 8)));
 }
 
-// Exact OAS comparison of one lane's 16 elements under factor k: candidates
-// E1 (byte b1) and E1 + 1. D = 512 s - h (256 + k) with s = |x| 2^-E1 and h
-// the code magnitude in units of 0.5 (doubled for the coarser candidate): an
-// integer below 2^12 for every element that does not round to zero under both.
-__device__ __forceinline__ int oas_delta_mbs16(const V16& x, int b1, const Thresholds& T,
-                                               int k) {
-  const float inv1 = inv_scale_from_byte(b1);
-  const float fk = static_cast<float>(256 + k);
+// The integer held exactly by a float v with |v| < 2^22 (no conversion unit:
+// adding 1.5 * 2^23 puts v in the low mantissa bits).
+__device__ __forceinline__ int small_int(float v) {
+  return __float_as_int(v + 12582912.0f) - 0x4B400000;
+}
+
+// Codes of 8 non-negative scaled values under the bracket L <= 1/f <= H (see
+// enc_mbs_cvt_16), and their E2M1 magnitudes as floats.
+__device__ __forceinline__ uint32_t mbs_codes8(const float* s8, float L, float H) {
+  float lo[8], hi[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) {
+    lo[j] = s8[j] * L;
+    hi[j] = s8[j] * H;
+  }
+  return even_of_adjacent(cvt_e2m1_f8(lo), cvt_e2m1_f8(hi));
+}
+__device__ __forceinline__ void e2m1x8_values(uint32_t codes, float* v) {
+  const uint2 a = e2m1x4_to_bf16(codes & 0xFFFFu);
+  const uint2 b = e2m1x4_to_bf16(codes >> 16);
+  v[0] = bf_lo(a.x); v[1] = bf_hi(a.x); v[2] = bf_lo(a.y); v[3] = bf_hi(a.y);
+  v[4] = bf_lo(b.x); v[5] = bf_hi(b.x); v[6] = bf_lo(b.y); v[7] = bf_hi(b.y);
+}
+
+// OAS evaluation of one lane's 16 elements under factor k: codes for E1
+// (byte b1) and E2 = E1 + 1 and the exact difference of the squared errors,
+// in units of 2^-18 of the E1 scale: sum of D1^2 - D2^2 with D = 512 d,
+// d1 = s - q1 f and d2 = s - 2 q2 f (s = x 2^-E1, q the code values). Where
+// both codes are zero, d1 == d2 and the term cancels; elsewhere s and q f are
+// multiples of 2^-9, so each d is exact (below 4 in magnitude) and each D an
+// integer below 2^11: the int32 sum is exact.
+__device__ __forceinline__ OasEval oas_eval_mbs16(const V16& x, int b1, int k) {
+  const FactorBracket fb = factor_bracket(k);
+  const V16 s1 = scale_slice(x, b1);
+  float s[16], h[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    s[i] = elem(s1, i);
+    h[i] = s[i] * 0.5f;
+  }
+  OasEval r;
+  {
+    float lo[16], hi[16], lo2[16], hi2[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      lo[i] = s[i] * fb.L;
+      hi[i] = s[i] * fb.H;
+      lo2[i] = h[i] * fb.L;
+      hi2[i] = h[i] * fb.H;
+    }
+    r.c1 = make_uint2(even_of_adjacent(cvt_e2m1_f8(lo), cvt_e2m1_f8(hi)),
+                      even_of_adjacent(cvt_e2m1_f8(lo + 8), cvt_e2m1_f8(hi + 8)));
+    r.c2 = make_uint2(even_of_adjacent(cvt_e2m1_f8(lo2), cvt_e2m1_f8(hi2)),
+                      even_of_adjacent(cvt_e2m1_f8(lo2 + 8), cvt_e2m1_f8(hi2 + 8)));
+  }
+  const V16 q1 = e2m1x16_to_bf16(r.c1);
+  const V16 q2 = e2m1x16_to_bf16(r.c2);
+  const float f2 = fb.f * 2.0f;
   int acc = 0;
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
-    const float s = fabsf(elem(x, i)) * inv1;
-    const int c1 = mbs_round(s, T);
-    const int c2 = mbs_round(s * 0.5f, T);
-    const float d1 = s * 512.0f - static_cast<float>(e2m1_halves(c1)) * fk;
-    const float d2 = s * 512.0f - static_cast<float>(2 * e2m1_halves(c2)) * fk;
-    const int i1 = __float2int_rn(d1), i2 = __float2int_rn(d2);
-    acc += i1 * i1 - i2 * i2;
+    const int D1 = small_int(fmaf(-elem(q1, i), fb.f, s[i]) * 512.0f);
+    const int D2 = small_int(fmaf(-elem(q2, i), f2, s[i]) * 512.0f);
+    acc += D1 * D1 - D2 * D2;
   }
-  return acc;
+  r.delta = acc;
+  return r;
 }
 
 }  // namespace mxk

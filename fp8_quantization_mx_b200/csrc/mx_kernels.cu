@@ -86,9 +86,12 @@ __device__ __forceinline__ BlockScale decide_scale(const V16& v, uint32_t pa, in
       const int b2 = mbs_byte(pa, k, 1);
       const bool need = !s.nonfinite && b2 != s.byte;
       if (__any_sync(kFull, need)) {
-        int d = oas_delta_mbs16(v, s.byte, mbs_thresholds(k), k);
-        d += __shfl_xor_sync(kFull, d, 1);
-        if (need && d > 0) s.byte = b2;
+        const OasEval e = oas_eval_mbs16(v, s.byte, k);
+        const int d = e.delta + __shfl_xor_sync(kFull, e.delta, 1);
+        const bool up = need && d > 0;
+        if (up) s.byte = b2;
+        s.codes = up ? e.c2 : e.c1;   // the codes of the chosen scale
+        s.have_codes = true;
       }
     }
   }
@@ -102,20 +105,31 @@ __device__ __forceinline__ uint2 codes_fp4(const V16& v, const BlockScale& s) {
   if (s.nonfinite) return nonfinite_e2m1_16(v);
   if (s.have_codes) return s.codes;
   if (MBS == kMbsNone) return enc_e2m1_16(scale_slice(v, s.byte));
-  return enc_mbs_16(v, s.byte, mbs_thresholds(s.k));
+  return enc_mbs_cvt_16(v, s.byte, s.k);
 }
 
-// Dequantized values (exact floats, signed) of a finite block's 16 elements.
+// Codes of one lane's 16 elements: E2M1 in .x/.y, E4M3 in all four words.
 template <int FMT, int MBS>
-__device__ __forceinline__ F16 block_values(const V16& v, const BlockScale& s) {
+__device__ __forceinline__ uint4 lane_codes(const V16& v, const BlockScale& s) {
+  if (FMT == kFmtE2M1) {
+    const uint2 c = codes_fp4<MBS>(v, s);
+    return make_uint4(c.x, c.y, 0, 0);
+  }
+  return s.nonfinite ? nonfinite_e4m3_16(v) : enc_e4m3_16(scale_slice(v, s.byte));
+}
+
+// Dequantized values (exact floats, signed) of a finite block's 16 elements
+// from their codes.
+template <int FMT, int MBS>
+__device__ __forceinline__ F16 block_values(const uint4& codes, const BlockScale& s) {
   const int E = s.byte - 127;
   if (FMT == kFmtE2M1) {
     // MBS: value * (256 + k) 2^(E-8) -- the multiplier has 9 significant bits
     // and the product at most 11, both exact in float
     const float p = MBS == kMbsNone ? pow2f(E) : static_cast<float>(256 + s.k) * pow2f(E - 8);
-    return dec_e2m1_16(codes_fp4<MBS>(v, s), p);
+    return dec_e2m1_16(make_uint2(codes.x, codes.y), p);
   }
-  return dec_e4m3_16(enc_e4m3_16(scale_slice(v, s.byte)), pow2f(E));
+  return dec_e4m3_16(codes, pow2f(E));
 }
 
 template <int OP, int FMT, int RULE, int MBS>
@@ -123,13 +137,14 @@ __device__ __forceinline__ void process_slice(const StreamArgs& a, const V16& v,
                                               int64_t c, bool valid, int lane, uint32_t pa, int k,
                                               double& sd, double& sx) {
   const BlockScale s = decide_scale<FMT, RULE, MBS>(v, pa, k);
+  // codes for every lane before any divergent branch (see codes_fp4)
+  uint4 codes = make_uint4(0, 0, 0, 0);
+  if (OP != kOpFakeBwd) codes = lane_codes<FMT, MBS>(v, s);
 
   if (OP == kOpQuant) {
     if (FMT == kFmtE2M1) {
-      const uint2 codes = codes_fp4<MBS>(v, s);
-      if (valid) st_stream8(a.codes + 8 * c, codes);
+      if (valid) st_stream8(a.codes + 8 * c, make_uint2(codes.x, codes.y));
     } else {
-      const uint4 codes = s.nonfinite ? nonfinite_e4m3_16(v) : enc_e4m3_16(scale_slice(v, s.byte));
       if (valid) st_stream16(a.codes + 16 * c, codes);
     }
     if (valid && (lane & 1) == 0) a.scales[c >> 1] = static_cast<uint8_t>(s.byte);
@@ -143,7 +158,7 @@ __device__ __forceinline__ void process_slice(const StreamArgs& a, const V16& v,
 #pragma unroll
       for (int i = 0; i < 8; ++i) o.w[i] = (static_cast<uint32_t>(kNaNbf16) << 16) | kNaNbf16;
     } else {
-      const F16 y = block_values<FMT, MBS>(v, s);
+      const F16 y = block_values<FMT, MBS>(codes, s);
 #pragma unroll
       for (int i = 0; i < 8; ++i) o.w[i] = pack_bf16x2(y.v[2 * i], y.v[2 * i + 1]);
     }
@@ -178,7 +193,7 @@ __device__ __forceinline__ void process_slice(const StreamArgs& a, const V16& v,
         bx = fma(xi, xi, bx);
       }
     } else {
-      const F16 y = block_values<FMT, MBS>(v, s);
+      const F16 y = block_values<FMT, MBS>(codes, s);
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
         const float xf = elem(v, i);
@@ -259,10 +274,10 @@ __global__ void __launch_bounds__(kThreads) stream_kernel(StreamArgs a) {
 // double, in element order: each d is exact in float, d*d exact in double, so
 // the running sum rounds exactly as a sequential double sum does.
 // xs: the 128 magnitudes |x| as floats; amax[4]: sub-block amax bits.
+// Rounding under f uses the bracket of enc_mbs_cvt_16, 8 elements at a time.
 template <int RULE>
 __device__ __forceinline__ double macro_sse_k(const float* xs, const uint32_t amax[4], int k) {
-  const Thresholds T = mbs_thresholds(k);
-  const float fk = static_cast<float>(256 + k);
+  const FactorBracket fb = factor_bracket(k);
   double sse = 0.0;
 #pragma unroll 1
   for (int b = 0; b < 4; ++b) {
@@ -270,30 +285,44 @@ __device__ __forceinline__ double macro_sse_k(const float* xs, const uint32_t am
     if (RULE == kOas) {
       const int b2 = mbs_byte(amax[b], k, 1);
       if (b2 != byte) {
+        // exact SSE difference of the two candidates (see oas_eval_mbs16)
         const float inv1 = inv_scale_from_byte(byte);
+        const float f2 = fb.f * 2.0f;
         int acc = 0;
-#pragma unroll 4
-        for (int i = 0; i < 32; ++i) {
-          const float s = xs[32 * b + i] * inv1;
-          const int c1 = mbs_round(s, T);
-          const int c2 = mbs_round(s * 0.5f, T);
-          const int i1 = __float2int_rn(s * 512.0f - static_cast<float>(e2m1_halves(c1)) * fk);
-          const int i2 = __float2int_rn(s * 512.0f - static_cast<float>(2 * e2m1_halves(c2)) * fk);
-          acc += i1 * i1 - i2 * i2;
+#pragma unroll 1
+        for (int i = 0; i < 32; i += 8) {
+          float s[8], h[8], q1[8], q2[8];
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            s[j] = xs[32 * b + i + j] * inv1;
+            h[j] = s[j] * 0.5f;
+          }
+          e2m1x8_values(mbs_codes8(s, fb.L, fb.H), q1);
+          e2m1x8_values(mbs_codes8(h, fb.L, fb.H), q2);
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            const int D1 = small_int(fmaf(-q1[j], fb.f, s[j]) * 512.0f);
+            const int D2 = small_int(fmaf(-q2[j], f2, s[j]) * 512.0f);
+            acc += D1 * D1 - D2 * D2;
+          }
         }
         if (acc > 0) byte = b2;
       }
     }
     const float m = inv_scale_from_byte(byte);                          // 2^-E
     const double p = __longlong_as_double(static_cast<long long>(byte - 127 + 1023) << 52);
-#pragma unroll 8
-    for (int i = 0; i < 32; ++i) {
-      const float s = xs[32 * b + i] * m;
-      const int c = mbs_round(s, T);
-      // s - h (256 + k) / 512 is exact (both sides are multiples of 2^-9 below 2^5)
-      const float ds = s - static_cast<float>(e2m1_halves(c)) * fk * 0.001953125f;
-      const double d = static_cast<double>(ds) * p;                             // exact
-      sse = fma(d, d, sse);
+#pragma unroll 1
+    for (int i = 0; i < 32; i += 8) {
+      float s[8], q[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) s[j] = xs[32 * b + i + j] * m;
+      e2m1x8_values(mbs_codes8(s, fb.L, fb.H), q);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        // s - q f is exact (both are multiples of 2^-9 below 2^5, or q = 0)
+        const double d = static_cast<double>(fmaf(-q[j], fb.f, s[j])) * p;   // exact
+        sse = fma(d, d, sse);
+      }
     }
   }
   return sse;
@@ -465,7 +494,7 @@ template <int OP, int FMT, int RULE, int MBS>
 cudaError_t launch_stream(const StreamArgs& a, cudaStream_t st) {
   // the error kernel ends with one double atomic per CTA: keep its grid small
   const int waves = OP == kOpError ? 1 : MX_GRID_WAVES;
-  if (MBS == kMbsDynamic) {
+  if constexpr (MBS == kMbsDynamic) {
     auto kern = mbs_dynamic_kernel<OP, RULE>;
     const int grid = grid_for(kern, (a.nslices + 31) / 32, waves);
     kern<<<grid, kThreads, 0, st>>>(a);

@@ -75,7 +75,21 @@ def special_blocks():
     # subnormal maximum), and one of mixed-sign subnormals and zeros
     sub = (np.arange(128, dtype=np.uint16) % 127 + 1)
     mixed = np.where(np.arange(128) % 3 == 0, 0, sub | np.where(np.arange(128) % 2, 0x8000, 0))
-    arr = np.concatenate([arr.reshape(-1, 128), sub[None], mixed.astype(np.uint16)[None]])
+    # macro blocks whose MBS-Static factor is k = 64 (max 7.5) or k = 32 (max
+    # 6.75), filled with the exact grid midpoints times f: every one of them is
+    # a rounding tie under the macro factor
+    ties_rows = []
+    for amax, f in ((7.5, 1.25), (6.75, 1.125)):
+        mids = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0]) * f
+        vals = np.zeros(128, np.float32)
+        for sb in range(4):
+            blk = np.concatenate([[amax], mids, -mids, mids * 0.5, -mids * 0.5, [0.0, -0.0, amax - 0.25]])
+            vals[32 * sb:32 * sb + len(blk)] = blk[:32]
+        b16 = torch.from_numpy(vals).to(torch.bfloat16)
+        assert torch.equal(b16.float(), torch.from_numpy(vals)), "tie values must be bf16-exact"
+        ties_rows.append(b16.view(torch.int16).numpy().view(np.uint16))
+    arr = np.concatenate([arr.reshape(-1, 128), sub[None], mixed.astype(np.uint16)[None],
+                          np.stack(ties_rows)])
     return arr
 
 
