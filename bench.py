@@ -234,6 +234,53 @@ def time_op(fn, reps, flush=None, stream=None):
     return times[len(times) // 2]
 
 
+def stack_ops(mx, x, reps=50):
+    """GB/s of every op on the 403 M-element MoE stack x [rows, 2048]: mean
+    over `reps` back-to-back launches (x is far larger than L2)."""
+    import torch
+    rows, cols = x.shape
+    n = x.numel()
+    dev = x.device
+    c4 = torch.empty(rows, cols // 2, dtype=torch.uint8, device=dev)
+    c8 = torch.empty(rows, cols, dtype=torch.uint8, device=dev)
+    sc = torch.empty(rows, cols // 32, dtype=torch.uint8, device=dev)
+    mac = torch.empty(rows, cols // 128, dtype=torch.uint8, device=dev)
+    y = torch.empty_like(x)
+    g = torch.empty_like(x).normal_()
+    fp4, fp8, fp4m = n * 2.53125, n * 3.03125, n * (2.53125 + 1 / 128)
+    ops = {
+        "fp4_floor_quantize": (lambda: mx.quantize(x, mx.E2M1, mx.FLOOR, out=(c4, sc, None)), fp4),
+        "fp8_floor_quantize": (lambda: mx.quantize(x, mx.E4M3, mx.FLOOR, out=(c8, sc, None)), fp8),
+        "fp4_oas_quantize": (lambda: mx.quantize(x, mx.E2M1, mx.OAS, out=(c4, sc, None)), fp4),
+        "fp4_mbs_static_quantize": (lambda: mx.quantize(x, mx.E2M1, mx.MBS_STATIC, out=(c4, sc, mac)), fp4m),
+        "fp4_oas_mbs_static_quantize": (lambda: mx.quantize(x, mx.E2M1, mx.OAS | mx.MBS_STATIC,
+                                                            out=(c4, sc, mac)), fp4m),
+        "fp4_fake_quant_fwd": (lambda: mx.fake_quant(x, out=y), n * 4),
+        "fp4_fake_quant_bwd": (lambda: mx.fake_quant_bwd(x, g, out=y), n * 6),
+        "fp4_dequantize_bf16": (lambda: mx.dequantize(c4, sc, None, mx.E2M1, out=y), fp4),
+        "fp8_dequantize_bf16": (lambda: mx.dequantize(c8, sc, None, mx.E4M3, out=y), fp8),
+        "fp4_block_error": (lambda: mx.block_error(x, per_block=False), n * 2),
+    }
+    res = {}
+    for name, (fn, nbytes) in ops.items():
+        if name == "fp4_dequantize_bf16":
+            mx.quantize(x, mx.E2M1, mx.FLOOR, out=(c4, sc, None))
+        if name == "fp8_dequantize_bf16":
+            mx.quantize(x, mx.E4M3, mx.FLOOR, out=(c8, sc, None))
+        fn()
+        torch.cuda.synchronize()
+        s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        s.record()
+        for _ in range(reps):
+            fn()
+        e.record()
+        e.synchronize()
+        ms = s.elapsed_time(e) / reps
+        res[name] = {"ms": round(ms, 4), "GB/s": round(nbytes / ms / 1e6, 1)}
+    del c4, c8, sc, mac, y, g
+    return res
+
+
 def other_ops(mx, inputs, dev, reps=10):
     """GB/s of the other ops on their workloads (median of reps; L2 flushed before each)."""
     import torch
@@ -378,8 +425,9 @@ def run_mx(args):
     del hc, hs
 
     ops = None
-    if not args.no_ops and rank == 0:
-        ops = other_ops(mx, inputs, dev)
+    if not args.no_ops and world == 1:
+        ops = {"moe_w13_128x1536x2048": stack_ops(mx, x)}
+        ops.update(other_ops(mx, inputs, dev))
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
