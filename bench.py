@@ -234,9 +234,10 @@ def time_op(fn, reps, flush=None, stream=None):
     return times[len(times) // 2]
 
 
-def stack_ops(mx, x, reps=50):
+def stack_ops(mx, x, reps=50, only=None):
     """GB/s of every op on the 403 M-element MoE stack x [rows, 2048]: mean
-    over `reps` back-to-back launches (x is far larger than L2)."""
+    over `reps` back-to-back launches (x is far larger than L2). `only` names
+    one op to run alone (for profiling)."""
     import torch
     rows, cols = x.shape
     n = x.numel()
@@ -261,6 +262,10 @@ def stack_ops(mx, x, reps=50):
         "fp8_dequantize_bf16": (lambda: mx.dequantize(c8, sc, None, mx.E4M3, out=y), fp8),
         "fp4_block_error": (lambda: mx.block_error(x, per_block=False), n * 2),
     }
+    if only is not None:
+        if only not in ops:
+            raise SystemExit(f"unknown op {only!r}; one of {sorted(ops)}")
+        ops = {only: ops[only]}
     res = {}
     for name, (fn, nbytes) in ops.items():
         if name == "fp4_dequantize_bf16":
@@ -476,12 +481,34 @@ def main():
     ap.add_argument("--impl", choices=["mx", "reference"], default="mx")
     ap.add_argument("--no-ops", action="store_true", help="skip the per-op figures")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--profile-op", default=None,
+                    help="run one op of the MoE-stack table `--steps` times and print its figure "
+                         "(for profilers); no headline line")
+    ap.add_argument("--profile-experts", type=int, default=32,
+                    help="experts of the stack used by --profile-op (32: 201 MB of input, above L2)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
     if args.impl == "reference":
         return run_reference(args)
+    if args.profile_op:
+        return run_profile_op(args)
     return run_mx(args)
+
+
+def run_profile_op(args):
+    """One op of the MoE-stack table, alone (after the stack is generated)."""
+    import torch
+    import fp8_quantization_mx_b200 as mx
+    from fp8_quantization_mx_b200 import build as mxbuild
+    from fp8_quantization_mx_b200 import inputs
+    mxbuild.build()
+    mx.load_library()
+    x = inputs.moe_w13(experts=args.profile_experts, device="cuda").view(-1, HIDDEN)
+    res = stack_ops(mx, x, reps=args.steps, only=args.profile_op)
+    torch.cuda.synchronize()
+    print(json.dumps({"profile_op": args.profile_op, **res[args.profile_op]}), flush=True)
+    return 0
 
 
 if __name__ == "__main__":

@@ -240,16 +240,40 @@ __device__ __forceinline__ uint4 nonfinite_e4m3_16(const V16& x) {
 // memory was right; a table lookup avoids depending on that register path.
 // The E4M3 pair of conversions showed no such problem in either path.)
 
-// E2M1 magnitudes 0 .5 1 1.5 2 3 4 6 as bf16 bit patterns, split into their
-// high and low bytes, four entries per 32-bit word (index 0..3, 4..7).
-constexpr uint32_t kE2m1Hi0 = 0x3F3F3F00u, kE2m1Hi1 = 0x40404040u;
-constexpr uint32_t kE2m1Lo0 = 0xC0800000u, kE2m1Lo1 = 0xC0804000u;
+// A table of the 8 E2M1 magnitudes as bf16 bit patterns, split into their
+// high and low bytes, four entries per 32-bit word (index 0..3, 4..7), for
+// byte-permute lookups.
+struct E2m1Table {
+  uint32_t hi0, hi1, lo0, lo1;
+};
+// Unscaled magnitudes 0 .5 1 1.5 2 3 4 6.
+__device__ __forceinline__ E2m1Table e2m1_unscaled() {
+  return E2m1Table{0x3F3F3F00u, 0x40404040u, 0xC0800000u, 0xC0804000u};
+}
+
+// The magnitudes times 2^E, for E in [-125, 125]: every nonzero product is a
+// normal bf16 whose bit pattern is the unscaled one plus E in the exponent
+// field (E * 128), added to both 16-bit halves of a packed pair at once (no
+// half crosses zero or 0x7F80 in that range); code 0 stays 0.
+__device__ __forceinline__ E2m1Table e2m1_table(int E) {
+  const uint32_t both = static_cast<uint32_t>(E * (128 * 65537));   // E*128 in each half
+  const uint32_t p01 = 0x3F000000u + static_cast<uint32_t>(E * (128 << 16));   // 0, 0.5
+  const uint32_t p23 = 0x3FC03F80u + both;                                   // 1, 1.5
+  const uint32_t p45 = 0x40404000u + both;                                   // 2, 3
+  const uint32_t p67 = 0x40C04080u + both;                                   // 4, 6
+  E2m1Table t;
+  t.hi0 = __byte_perm(p01, p23, 0x7531);
+  t.lo0 = __byte_perm(p01, p23, 0x6420);
+  t.hi1 = __byte_perm(p45, p67, 0x7531);
+  t.lo1 = __byte_perm(p45, p67, 0x6420);
+  return t;
+}
 
 // Four E2M1 codes (nibbles 0..3 of c) -> two words of bf16x2 bit patterns.
-__device__ __forceinline__ uint2 e2m1x4_to_bf16(uint32_t c) {
+__device__ __forceinline__ uint2 e2m1x4_to_bf16(uint32_t c, const E2m1Table& t) {
   const uint32_t sel = c & 0x7777u;                        // magnitude indices
-  const uint32_t hi = __byte_perm(kE2m1Hi0, kE2m1Hi1, sel);
-  const uint32_t lo = __byte_perm(kE2m1Lo0, kE2m1Lo1, sel);
+  const uint32_t hi = __byte_perm(t.hi0, t.hi1, sel);
+  const uint32_t lo = __byte_perm(t.lo0, t.lo1, sel);
   uint32_t w0 = __byte_perm(lo, hi, 0x5140);               // elements 0, 1
   uint32_t w1 = __byte_perm(lo, hi, 0x7362);               // elements 2, 3
   w0 |= ((c << 12) & 0x8000u) | ((c << 24) & 0x80000000u);  // sign bits 3, 7
@@ -257,14 +281,14 @@ __device__ __forceinline__ uint2 e2m1x4_to_bf16(uint32_t c) {
   return make_uint2(w0, w1);
 }
 
-// 16 E2M1 codes -> the 16 unscaled values as bf16 bit patterns.
-__device__ __forceinline__ V16 e2m1x16_to_bf16(uint2 codes) {
+// 16 E2M1 codes -> their values (unscaled, or scaled by the table) as bf16.
+__device__ __forceinline__ V16 e2m1x16_to_bf16(uint2 codes, const E2m1Table& t) {
   V16 r;
   const uint32_t c[2] = {codes.x, codes.y};
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
-    const uint2 a = e2m1x4_to_bf16(c[h] & 0xFFFFu);
-    const uint2 b = e2m1x4_to_bf16(c[h] >> 16);
+    const uint2 a = e2m1x4_to_bf16(c[h] & 0xFFFFu, t);
+    const uint2 b = e2m1x4_to_bf16(c[h] >> 16, t);
     r.w[4 * h + 0] = a.x;
     r.w[4 * h + 1] = a.y;
     r.w[4 * h + 2] = b.x;
@@ -272,6 +296,16 @@ __device__ __forceinline__ V16 e2m1x16_to_bf16(uint2 codes) {
   }
   return r;
 }
+
+__device__ __forceinline__ uint2 e2m1x4_to_bf16(uint32_t c) {
+  return e2m1x4_to_bf16(c, e2m1_unscaled());
+}
+__device__ __forceinline__ V16 e2m1x16_to_bf16(uint2 codes) {
+  return e2m1x16_to_bf16(codes, e2m1_unscaled());
+}
+
+// E8M0 bytes whose E2M1 products are all normal bf16 values: E in [-125, 125].
+__device__ __forceinline__ bool e2m1_table_scale_ok(int b) { return b >= 2 && b <= 252; }
 
 // Eight E4M3fn bytes (byte i = element i) -> four f16x2 words, exact (every
 // E4M3 value is an f16 value; S.1111.111 becomes an f16 NaN). This hardware
@@ -447,6 +481,15 @@ __device__ __forceinline__ FactorBracket factor_bracket(int k) {
   r.L = inv * 0.99999904632568359375f;                                // 1 - 2^-20
   r.H = inv * 1.00000095367431640625f;                                // 1 + 2^-20
   return r;
+}
+
+// OAS under a macro factor: the coarser candidate can only win when the block
+// max, in units of f 2^E1 (byte b1), exceeds 7 -- below that every element's
+// error on the finer grid is no larger (the grids are those of plain OAS
+// scaled by f). amax * 2^-E1 and 7 f are exact floats.
+__device__ __forceinline__ bool mbs_oas_band(uint32_t amax, int b1, int k) {
+  const float s = __uint_as_float(amax << 16) * inv_scale_from_byte(b1);
+  return s > 7.0f * static_cast<float>(256 + k) * 0.00390625f;
 }
 
 // Of two nibble-packed code words that agree except where an element's codes

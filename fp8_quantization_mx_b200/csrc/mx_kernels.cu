@@ -84,7 +84,9 @@ __device__ __forceinline__ BlockScale decide_scale(const V16& v, uint32_t pa, in
     s.byte = mbs_byte(pa, k, 0);
     if (RULE == kOas) {
       const int b2 = mbs_byte(pa, k, 1);
-      const bool need = !s.nonfinite && b2 != s.byte;
+      // as without MBS, the finer candidate is element-wise no worse unless
+      // the scaled block max exceeds 7 f (both sides of the test are exact)
+      const bool need = !s.nonfinite && b2 != s.byte && mbs_oas_band(pa, s.byte, k);
       if (__any_sync(kFull, need)) {
         const OasEval e = oas_eval_mbs16(v, s.byte, k);
         const int d = e.delta + __shfl_xor_sync(kFull, e.delta, 1);
@@ -157,6 +159,9 @@ __device__ __forceinline__ void process_slice(const StreamArgs& a, const V16& v,
     if (s.nonfinite) {
 #pragma unroll
       for (int i = 0; i < 8; ++i) o.w[i] = (static_cast<uint32_t>(kNaNbf16) << 16) | kNaNbf16;
+    } else if (FMT == kFmtE2M1 && MBS == kMbsNone && e2m1_table_scale_ok(s.byte)) {
+      // the products are normal bf16 values: a table of the scaled magnitudes
+      o = e2m1x16_to_bf16(make_uint2(codes.x, codes.y), e2m1_table(s.byte - 127));
     } else {
       const F16 y = block_values<FMT, MBS>(codes, s);
 #pragma unroll
@@ -193,14 +198,30 @@ __device__ __forceinline__ void process_slice(const StreamArgs& a, const V16& v,
         bx = fma(xi, xi, bx);
       }
     } else {
+      // d^2 exactly in double (d is exact in float). x^2 only feeds the tensor
+      // total: in units of the block scale, s = x 2^-E and s^2 are exact
+      // floats unless s^2 underflows (s < 2^-63), which is negligible next to
+      // the block's largest s^2 (at least 4, or, when E is clamped at -127,
+      // no nonzero s is below 2^-6); the 16 are summed pairwise in float
+      // (relative error below 2.4e-7) and scaled by 2^(2E) in double.
       const F16 y = block_values<FMT, MBS>(codes, s);
+      const float inv = inv_scale_from_byte(s.byte);
+      float u[16];
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
         const float xf = elem(v, i);
         const double d = static_cast<double>(xf - y.v[i]);   // exact in float
         bd = fma(d, d, bd);
-        bx = fma(static_cast<double>(xf), static_cast<double>(xf), bx);
+        const float xs = xf * inv;
+        u[i] = xs * xs;
       }
+#pragma unroll
+      for (int w = 8; w >= 1; w >>= 1) {
+#pragma unroll
+        for (int i = 0; i < w; ++i) u[i] += u[i + w];
+      }
+      bx = static_cast<double>(u[0]) *
+           __longlong_as_double(static_cast<long long>(2 * (s.byte - 127) + 1023) << 52);
     }
     const double q = bd + __shfl_xor_sync(kFull, bd, 1);
     if (valid) {
@@ -268,6 +289,96 @@ __global__ void __launch_bounds__(kThreads) stream_kernel(StreamArgs a) {
   if (OP == kOpError) reduce_totals(sd, sx, a.totals);
 }
 
+// ------------------------------------------------------ OAS quantize path --
+
+// MXFP4 OAS quantize (without MBS, or with MBS-Static) in two phases per CTA
+// tile. Phase 1 handles every block whose finer exponent is already the
+// answer (scaled max <= 7, the two candidates equal, or NaN/Inf) exactly as
+// the single-rule kernel does, and appends the other blocks (about a fifth of
+// them for Gaussian data) to a shared-memory list, with their macro factor.
+// Phase 2 evaluates only the listed blocks, two lanes per block and full
+// warps, re-reading their 64 bytes (just loaded, so from L2). Without the
+// split every warp that holds one such block pays for the exact SSE
+// comparison on all of its lanes.
+template <int MBS, int U>
+__global__ void __launch_bounds__(kThreads) oas_quant_kernel(StreamArgs a) {
+  constexpr int kWarps = kThreads / 32;
+  constexpr int kTileSlices = kWarps * 32 * U;
+  // listed blocks: first-slice offset in the low 16 bits, macro k above
+  __shared__ uint32_t list[kTileSlices / 2];
+  __shared__ int count;
+  const int lane = threadIdx.x & 31;
+  const int w = threadIdx.x >> 5;
+  const int64_t tile0 = static_cast<int64_t>(blockIdx.x) * kTileSlices;
+  if (threadIdx.x == 0) count = 0;
+  __syncthreads();
+
+  // phase 1
+  V16 v[U];
+#pragma unroll
+  for (int j = 0; j < U; ++j) {
+    const int64_t c = tile0 + w * 32 * U + 32 * j + lane;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[j].w[i] = 0;
+    if (c < a.nslices) v[j] = ld_stream32(a.x + 32 * c);
+  }
+#pragma unroll
+  for (int j = 0; j < U; ++j) {
+    const int64_t c = tile0 + w * 32 * U + 32 * j + lane;
+    const bool valid = c < a.nslices;
+    const uint32_t pa = pair_max(amax_bits16(v[j]));
+    const bool nonfinite = pa >= 0x7F80u;
+    int k = 0, b1, b2;
+    bool band;
+    if (MBS == kMbsNone) {
+      b1 = rule_byte<kFmtE2M1, kFloor>(pa);
+      b2 = max(static_cast<int>(pa >> 7) - 1, 0);
+      band = (pa & 0x7F) > 96;
+    } else {
+      k = mbs_static_k(oct_max(pa));
+      b1 = mbs_byte(pa, k, 0);
+      b2 = mbs_byte(pa, k, 1);
+      band = mbs_oas_band(pa, b1, k);
+    }
+    const bool need = valid && !nonfinite && band && b2 != b1;
+    if (valid && !need) {
+      uint2 codes;
+      if (nonfinite) codes = nonfinite_e2m1_16(v[j]);
+      else if (MBS == kMbsNone) codes = enc_e2m1_16(scale_slice(v[j], b1));
+      else codes = enc_mbs_cvt_16(v[j], b1, k);
+      st_stream8(a.codes + 8 * c, codes);
+      if ((lane & 1) == 0) a.scales[c >> 1] = static_cast<uint8_t>(nonfinite ? 255 : b1);
+    }
+    if (MBS != kMbsNone && valid && (lane & 7) == 0) a.macro[c >> 3] = static_cast<uint8_t>(k);
+    if (need && (lane & 1) == 0)
+      list[atomicAdd(&count, 1)] = static_cast<uint32_t>(c - tile0) | (static_cast<uint32_t>(k) << 16);
+  }
+  __syncthreads();
+
+  // phase 2: 16 listed blocks per warp step
+  const int n = count;
+  for (int base = w * 16; base < n; base += kWarps * 16) {
+    const int idx = base + (lane >> 1);
+    const bool has = idx < n;
+    const uint32_t entry = has ? list[idx] : 0u;
+    const int64_t c = tile0 + (entry & 0xFFFFu) + (lane & 1);
+    const int k = static_cast<int>(entry >> 16);
+    V16 x;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) x.w[i] = 0;
+    if (has) x = ld_stream32(a.x + 32 * c);
+    const uint32_t pa = pair_max(amax_bits16(x));
+    const int b1 = MBS == kMbsNone ? rule_byte<kFmtE2M1, kFloor>(pa) : mbs_byte(pa, k, 0);
+    const OasEval e = MBS == kMbsNone ? oas_eval16(x, b1) : oas_eval_mbs16(x, b1, k);
+    const int d = e.delta + __shfl_xor_sync(kFull, e.delta, 1);
+    const bool up = d > 0;
+    if (has) {
+      st_stream8(a.codes + 8 * c, up ? e.c2 : e.c1);
+      if ((lane & 1) == 0) a.scales[c >> 1] = static_cast<uint8_t>(up ? b1 + 1 : b1);
+    }
+  }
+}
+
 // ------------------------------------------------------- MBS-Dynamic path --
 
 // Sum of squared errors of one 128-element macro block under factor k, in
@@ -284,7 +395,7 @@ __device__ __forceinline__ double macro_sse_k(const float* xs, const uint32_t am
     int byte = mbs_byte(amax[b], k, 0);
     if (RULE == kOas) {
       const int b2 = mbs_byte(amax[b], k, 1);
-      if (b2 != byte) {
+      if (b2 != byte && mbs_oas_band(amax[b], byte, k)) {
         // exact SSE difference of the two candidates (see oas_eval_mbs16)
         const float inv1 = inv_scale_from_byte(byte);
         const float f2 = fb.f * 2.0f;
@@ -426,6 +537,26 @@ __global__ void __launch_bounds__(kThreads) dequant_kernel(DequantArgs a) {
       const int64_t c = base + 32 * j;
       if (c >= a.nslices) continue;
       const int E = sb[j] - 127;
+      if (FMT == kFmtE2M1 && kk[j] == 0 && e2m1_table_scale_ok(sb[j])) {
+        // common case: the products are normal bf16 values, read straight off
+        // a table of the 8 magnitudes scaled by 2^E (exact)
+        const V16 b = e2m1x16_to_bf16(c4[j], e2m1_table(E));
+        if (OUT32) {
+          V16 o0, o1;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            o0.w[2 * i] = b.w[i] << 16;
+            o0.w[2 * i + 1] = b.w[i] & 0xFFFF0000u;
+            o1.w[2 * i] = b.w[4 + i] << 16;
+            o1.w[2 * i + 1] = b.w[4 + i] & 0xFFFF0000u;
+          }
+          st_stream32(a.out + 64 * c, o0);
+          st_stream32(a.out + 64 * c + 32, o1);
+        } else {
+          st_stream32(a.out + 32 * c, b);
+        }
+        continue;
+      }
       // value * (256 + k) 2^(E-8) (exact); a NaN scale makes every output NaN
       const float p = kk[j] ? static_cast<float>(256 + kk[j]) * pow2f(E - 8) : pow2f(E);
       const F16 y = FMT == kFmtE2M1 ? dec_e2m1_16(c4[j], p) : dec_e4m3_16(c8[j], p);
@@ -498,6 +629,10 @@ cudaError_t launch_stream(const StreamArgs& a, cudaStream_t st) {
     auto kern = mbs_dynamic_kernel<OP, RULE>;
     const int grid = grid_for(kern, (a.nslices + 31) / 32, waves);
     kern<<<grid, kThreads, 0, st>>>(a);
+  } else if constexpr (OP == kOpQuant && FMT == kFmtE2M1 && RULE == kOas) {
+    constexpr int kTile = (kThreads / 32) * 32 * kUnroll;   // slices per CTA
+    const int64_t grid = (a.nslices + kTile - 1) / kTile;
+    oas_quant_kernel<MBS, kUnroll><<<static_cast<int>(grid), kThreads, 0, st>>>(a);
   } else {
     constexpr int U = (MBS == kMbsNone) ? kUnroll : 1;
     auto kern = stream_kernel<OP, FMT, RULE, MBS, U>;
