@@ -154,6 +154,28 @@ __device__ __forceinline__ uint32_t mul_bf16x2(uint32_t a, uint32_t b) {
   asm("mul.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
   return d;
 }
+__device__ __forceinline__ uint32_t sub_bf16x2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("sub.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
+// acc + h * h for the low (high) bf16 half h of w, in f32: the product is
+// exact and the sum rounds once (mixed-precision fma of sm_100).
+__device__ __forceinline__ float sq_acc_lo(uint32_t w, float acc) {
+  float d;
+  asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %1;\n\tfma.rn.f32.bf16 %0, l, l, %2;\n\t}"
+      : "=f"(d)
+      : "r"(w), "f"(acc));
+  return d;
+}
+__device__ __forceinline__ float sq_acc_hi(uint32_t w, float acc) {
+  float d;
+  asm("{\n\t.reg .b16 l, h;\n\tmov.b32 {l, h}, %1;\n\tfma.rn.f32.bf16 %0, h, h, %2;\n\t}"
+      : "=f"(d)
+      : "r"(w), "f"(acc));
+  return d;
+}
 
 // ------------------------------------------------------- element encoding --
 
@@ -279,6 +301,29 @@ __device__ __forceinline__ uint2 e2m1x4_to_bf16(uint32_t c, const E2m1Table& t) 
   w0 |= ((c << 12) & 0x8000u) | ((c << 24) & 0x80000000u);  // sign bits 3, 7
   w1 |= ((c << 4) & 0x8000u) | ((c << 16) & 0x80000000u);   // sign bits 11, 15
   return make_uint2(w0, w1);
+}
+
+// Four E2M1 codes -> the magnitudes of their values (signs dropped).
+__device__ __forceinline__ uint2 e2m1x4_mag_bf16(uint32_t c, const E2m1Table& t) {
+  const uint32_t sel = c & 0x7777u;
+  const uint32_t hi = __byte_perm(t.hi0, t.hi1, sel);
+  const uint32_t lo = __byte_perm(t.lo0, t.lo1, sel);
+  return make_uint2(__byte_perm(lo, hi, 0x5140), __byte_perm(lo, hi, 0x7362));
+}
+__device__ __forceinline__ V16 e2m1x16_mag_bf16(uint2 codes) {
+  const E2m1Table t = e2m1_unscaled();
+  V16 r;
+  const uint32_t c[2] = {codes.x, codes.y};
+#pragma unroll
+  for (int h = 0; h < 2; ++h) {
+    const uint2 a = e2m1x4_mag_bf16(c[h] & 0xFFFFu, t);
+    const uint2 b = e2m1x4_mag_bf16(c[h] >> 16, t);
+    r.w[4 * h + 0] = a.x;
+    r.w[4 * h + 1] = a.y;
+    r.w[4 * h + 2] = b.x;
+    r.w[4 * h + 3] = b.y;
+  }
+  return r;
 }
 
 // 16 E2M1 codes -> their values (unscaled, or scaled by the table) as bf16.
@@ -474,12 +519,17 @@ __device__ __forceinline__ uint32_t cvt_e2m1_f8(const float* v) {
 struct FactorBracket {
   float f, L, H;
 };
+// 1/f from the hardware reciprocal (PTX rcp.approx: at most 1 ulp from 1/f,
+// i.e. within 2^-23 relatively for f in [1, 2)); the 2^-20 margins on either
+// side keep L below and H above 1/f after their own rounding, and both within
+// 2^-19 of it.
 __device__ __forceinline__ FactorBracket factor_bracket(int k) {
   FactorBracket r;
-  r.f = static_cast<float>(256 + k) * 0.00390625f;                    // exact
-  const float inv = __fdiv_rn(256.0f, static_cast<float>(256 + k));   // 1/f, rounded
-  r.L = inv * 0.99999904632568359375f;                                // 1 - 2^-20
-  r.H = inv * 1.00000095367431640625f;                                // 1 + 2^-20
+  r.f = static_cast<float>(256 + k) * 0.00390625f;   // exact
+  float inv;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(inv) : "f"(r.f));
+  r.L = inv * 0.99999904632568359375f;   // 1 - 2^-20
+  r.H = inv * 1.00000095367431640625f;   // 1 + 2^-20
   return r;
 }
 

@@ -189,41 +189,83 @@ __device__ __forceinline__ void process_slice(const StreamArgs& a, const V16& v,
   }
 
   if (OP == kOpError) {
-    double bd = 0.0, bx = 0.0;
+    // In units of the block scale X = 2^E: s = x 2^-E (exact while it is a
+    // normal bf16; below that, errors of at most 2^-134 are negligible by
+    // the bound on Sd below) and the grid value g (code value, times f
+    // under MBS) are exact floats, and so is ds = s - g (s has 8
+    // significant bits, g at most 11, and g != 0 only when |s| is within a
+    // small factor of |g|). ds^2 and s^2 are summed in
+    // float, four fma chains of four per lane and then pairwise, so the
+    // block's sum of the 32 ds^2 carries a relative error of at most 7 u
+    // (u = 2^-24; all terms are non-negative) and the result, Sd 2^(2E)
+    // rounded to float, at most 8 u. Terms that underflow in float
+    // (ds < 2^-63) add absolute errors below 2^-144 in these units, so this
+    // holds while Sd >= 2^-90; the final rounding is relative only while
+    // the result is a normal float. Blocks outside those bounds (and those
+    // whose dequantized values pass the float range) take the exact path:
+    // d = x - y in float, d^2 summed in double.
+    const int bs = s.nonfinite ? 127 : s.byte;
+    const int E = bs - 127;
+    const double p2 = __longlong_as_double(static_cast<long long>(2 * E + 1023) << 52);
+    const V16 sl = scale_slice(v, bs);
+    float ad[4] = {0.0f, 0.0f, 0.0f, 0.0f}, ax[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+    if (FMT == kFmtE2M1 && MBS == kMbsNone) {
+      // |s| - |g| (the code keeps the sign of s) is exact in bf16 too: for s
+      // in [2^e, 2^(e+1)) the grid step is 2^(e-1), so |d| <= 2^(e-2) (or
+      // below 2 when s saturates to 6) and d is a multiple of 2^(e-7)
+      const V16 g = e2m1x16_mag_bf16(make_uint2(codes.x, codes.y));
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {
+        const uint32_t d = sub_bf16x2(sl.w[i] & 0x7FFF7FFFu, g.w[i]);
+        ad[(2 * i) & 3] = sq_acc_lo(d, ad[(2 * i) & 3]);
+        ad[(2 * i + 1) & 3] = sq_acc_hi(d, ad[(2 * i + 1) & 3]);
+        ax[(2 * i) & 3] = sq_acc_lo(sl.w[i], ax[(2 * i) & 3]);
+        ax[(2 * i + 1) & 3] = sq_acc_hi(sl.w[i], ax[(2 * i + 1) & 3]);
+      }
+    } else {
+      const F16 g = FMT == kFmtE2M1
+                        ? dec_e2m1_16(make_uint2(codes.x, codes.y),
+                                      static_cast<float>(256 + s.k) * 0.00390625f)
+                        : dec_e4m3_16(codes, 1.0f);
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const float si = elem(sl, i);
+        const float di = si - g.v[i];
+        ad[i & 3] = fmaf(di, di, ad[i & 3]);
+        ax[i & 3] = fmaf(si, si, ax[i & 3]);
+      }
+    }
+    const float ld = (ad[0] + ad[1]) + (ad[2] + ad[3]);
+    const float lx = (ax[0] + ax[1]) + (ax[2] + ax[3]);
+    const float Sd = ld + __shfl_xor_sync(kFull, ld, 1);
+    double q = static_cast<double>(Sd) * p2;
+    double bd = static_cast<double>(ld) * p2;
+    double bx = static_cast<double>(lx) * p2;
+    const bool exact = !s.nonfinite && pa != 0 && !(Sd >= 0x1p-90f && q >= 0x1p-120 && q < 0x1p120);
+    if (__any_sync(kFull, exact)) {
+      const F16 y = block_values<FMT, MBS>(codes, s);
+      double ed = 0.0;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        const double d = static_cast<double>(elem(v, i) - y.v[i]);   // exact in float
+        ed = fma(d, d, ed);
+      }
+      const double eq = ed + __shfl_xor_sync(kFull, ed, 1);
+      if (exact) {
+        bd = ed;
+        q = eq;
+      }
+    }
     if (s.nonfinite) {
-      bd = __int_as_float(0x7FC00000);
+      // the dequantized block is NaN; x^2 (possibly inf) still feeds the total
+      bd = q = __int_as_float(0x7FC00000);
+      bx = 0.0;
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
         const double xi = elem(v, i);
         bx = fma(xi, xi, bx);
       }
-    } else {
-      // d^2 exactly in double (d is exact in float). x^2 only feeds the tensor
-      // total: in units of the block scale, s = x 2^-E and s^2 are exact
-      // floats unless s^2 underflows (s < 2^-63), which is negligible next to
-      // the block's largest s^2 (at least 4, or, when E is clamped at -127,
-      // no nonzero s is below 2^-6); the 16 are summed pairwise in float
-      // (relative error below 2.4e-7) and scaled by 2^(2E) in double.
-      const F16 y = block_values<FMT, MBS>(codes, s);
-      const float inv = inv_scale_from_byte(s.byte);
-      float u[16];
-#pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        const float xf = elem(v, i);
-        const double d = static_cast<double>(xf - y.v[i]);   // exact in float
-        bd = fma(d, d, bd);
-        const float xs = xf * inv;
-        u[i] = xs * xs;
-      }
-#pragma unroll
-      for (int w = 8; w >= 1; w >>= 1) {
-#pragma unroll
-        for (int i = 0; i < w; ++i) u[i] += u[i + w];
-      }
-      bx = static_cast<double>(u[0]) *
-           __longlong_as_double(static_cast<long long>(2 * (s.byte - 127) + 1023) << 52);
     }
-    const double q = bd + __shfl_xor_sync(kFull, bd, 1);
     if (valid) {
       if (a.block_sse && (lane & 1) == 0) a.block_sse[c >> 1] = static_cast<float>(q);
       sd += bd;
