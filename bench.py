@@ -261,7 +261,13 @@ def stack_ops(mx, x, reps=50, only=None):
         "fp4_dequantize_bf16": (lambda: mx.dequantize(c4, sc, None, mx.E2M1, out=y), fp4),
         "fp8_dequantize_bf16": (lambda: mx.dequantize(c8, sc, None, mx.E4M3, out=y), fp8),
         "fp4_block_error": (lambda: mx.block_error(x, per_block=False), n * 2),
+        "fp4_mbs_dynamic_quantize": (lambda: mx.quantize(x, mx.E2M1, mx.MBS_DYNAMIC, out=(c4, sc, mac)),
+                                     fp4m),
+        "fp4_oas_mbs_dynamic_quantize": (lambda: mx.quantize(x, mx.E2M1, mx.OAS | mx.MBS_DYNAMIC,
+                                                             out=(c4, sc, mac)), fp4m),
     }
+    # the OAS + MBS-Dynamic search is ~100x slower than a stream: fewer launches
+    op_reps = {"fp4_oas_mbs_dynamic_quantize": 3}
     if only is not None:
         if only not in ops:
             raise SystemExit(f"unknown op {only!r}; one of {sorted(ops)}")
@@ -274,13 +280,14 @@ def stack_ops(mx, x, reps=50, only=None):
             mx.quantize(x, mx.E4M3, mx.FLOOR, out=(c8, sc, None))
         fn()
         torch.cuda.synchronize()
+        n_reps = min(reps, op_reps.get(name, reps))
         s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         s.record()
-        for _ in range(reps):
+        for _ in range(n_reps):
             fn()
         e.record()
         e.synchronize()
-        ms = s.elapsed_time(e) / reps
+        ms = s.elapsed_time(e) / n_reps
         res[name] = {"ms": round(ms, 4), "GB/s": round(nbytes / ms / 1e6, 1)}
     del c4, c8, sc, mac, y, g
     return res

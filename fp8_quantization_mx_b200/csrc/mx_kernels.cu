@@ -8,8 +8,9 @@
 // grid has one warp per tile and the block scheduler refills the SMs (measured
 // faster on B200 than a persistent grid); the error kernel keeps a persistent
 // grid so that its per-CTA atomics stay few.
-// Nothing is staged through shared memory except the 128 magnitudes of a
-// macro block during the MBS-Dynamic search; no kernel waits on a flag.
+// Shared memory holds only the block lists of the two-phase OAS quantize
+// kernel and the magnitudes and per-k sums of the MBS-Dynamic sweep; no
+// kernel waits on a flag.
 //
 // Sources restated: "[vLLM] MXFP8/MXFP4: microscaling format quantization"
 // (MX format table; MXFP8 block-32 scaling; MXFP4 packing), "[Axolotl] MXFP4
@@ -274,10 +275,11 @@ __device__ __forceinline__ void process_slice(const StreamArgs& a, const V16& v,
   }
 }
 
-// Sum of the per-lane error partials into totals: warp, then CTA, then one
-// double atomic per CTA.
+// Sum of the per-lane error partials into totals: warp, then CTA (NW warps),
+// then one double atomic per CTA.
+template <int NW = kThreads / 32>
 __device__ __forceinline__ void reduce_totals(double sd, double sx, double* totals) {
-  __shared__ double red[2][kThreads / 32];
+  __shared__ double red[2][NW];
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) {
     sd += __shfl_xor_sync(kFull, sd, o);
@@ -291,7 +293,7 @@ __device__ __forceinline__ void reduce_totals(double sd, double sx, double* tota
   __syncthreads();
   if (threadIdx.x == 0) {
     double td = 0.0, tx = 0.0;
-    for (int i = 0; i < kThreads / 32; ++i) {
+    for (int i = 0; i < NW; ++i) {
       td += red[0][i];
       tx += red[1][i];
     }
@@ -481,22 +483,308 @@ __device__ __forceinline__ double macro_sse_k(const float* xs, const uint32_t am
   return sse;
 }
 
+// ----------------------------------------------------- MBS-Dynamic sweep --
+//
+// The definition evaluates all 256 factors element by element (macro_sse_k
+// above does exactly that for one k). The same argmin follows from an exact
+// sweep over k:
+//
+// For sub-block i with amax exponent field ex and mantissa m7, the byte is
+// B0 = max(ex - 2, 0) while k <= 2 m7 (regime 0) and B1 = max(ex - 3, 0)
+// above (regime 1). Within a regime the scale 2^E is fixed, and with
+// t = |x| 2^-E, F = 256 + k and the code value q = Q / 2 (Q in
+// {0,1,2,3,4,6,8,12}), the error is d = (T - Q F) 2^(E-9) with T = 512 t. T is
+// an integer whenever t > 1/4 ("big"; t has 8 significant bits). Smaller
+// elements round to 0 for every k and contribute x^2.
+//
+// The code of a big element is the number of midpoints mu it lies above:
+// t / f > mu, or t / f == mu with the even neighbour above. With M = 4 mu in
+// {1,3,5,7,10,14,20} that is an integer test of 2T against M F. So the code
+// drops by one at the integer breakpoint F_m of each midpoint m, at most twice
+// over F in [256, 511]. Per sub-block and regime,
+//   SSE(k) = 2^(2E-18) (C - 2 F A(k) + F^2 B(k)) + X,
+// with C = sum of T^2, A = sum of T Q, B = sum of Q^2 over the big elements,
+// and X = sum of x^2 over the others. A and B are step functions of k, built
+// from per-k event deltas in shared memory and a prefix scan. Every term of
+// the bracket is an integer below 2^34, exact in double.
+//
+// Under OAS each sub-block takes, for every k, the smaller SSE of its byte
+// and the coarser candidate max(ex - 1 - r, 0) (an exact comparison in the
+// definition, the finer one on a tie): a second level of the same sums.
+//
+// The argmin must match the element-order double sums of the definition.
+// These sums are within 127 u of the exact SSE, and the sweep's doubles
+// within about 16 u (u = 2^-53). So any k whose swept value exceeds the
+// minimum by more than a factor 1 + 2^-40 cannot be the argmin or tie with
+// it. The remaining candidates (usually one) are re-evaluated in element
+// order by macro_sse_k. A minimum of exactly 0 means the exact SSE is 0 for
+// those k, so their double sums are 0 too and the smallest wins.
+
+constexpr int kSweepThreads = 128;
+constexpr int kSweepWarps = kSweepThreads / 32;
+
+// Rows of per-k deltas are padded by 4 words every 32 entries, so that the
+// scan's 16-byte loads (8 consecutive k per lane) hit distinct banks.
+constexpr int kSweepRow = 256 + 32;
+__device__ __forceinline__ int sweep_slot(int k) { return k + ((k >> 5) << 2); }
+
+// Levels of sub-block scale per regime: FLOOR has one (B_r); OAS two
+// (B_r and the coarser max(ex - 1 - r, 0)), of which the smaller SSE counts.
+template <int RULE>
+struct SweepShared {
+  static constexpr int kLevels = RULE == kOas ? 2 : 1;
+  float xs[4][128 + 1];                  // magnitudes of the warp's 4 macro blocks
+  int d[2 * 2 * kLevels][kSweepRow];     // per-k deltas of A and B for each (regime, level)
+  uint8_t cand[256];                     // candidate k for the element-order re-evaluation
+};
+
+// Q = 2 x the E2M1 magnitude of code c (0..7).
+__device__ __forceinline__ int code_q2(int c) {
+  return c <= 4 ? c : (c == 5 ? 6 : (c == 6 ? 8 : 12));
+}
+
+// Prefix sums of row[0..255] at this lane's 8 consecutive k (8 lane + j),
+// then the lane's entries cleared for the next use.
+__device__ __forceinline__ void scan_row8(int* row, int lane, int out[8]) {
+  int4* p = reinterpret_cast<int4*>(row + sweep_slot(8 * lane));
+  const int4 u = p[0], w = p[1];
+  out[0] = u.x;
+  out[1] = out[0] + u.y;
+  out[2] = out[1] + u.z;
+  out[3] = out[2] + u.w;
+  out[4] = out[3] + w.x;
+  out[5] = out[4] + w.y;
+  out[6] = out[5] + w.z;
+  out[7] = out[6] + w.w;
+  int incl = out[7];
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int t = __shfl_up_sync(kFull, incl, o);
+    if (lane >= o) incl += t;
+  }
+  const int excl = incl - out[7];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) out[j] += excl;
+  p[0] = make_int4(0, 0, 0, 0);
+  p[1] = make_int4(0, 0, 0, 0);
+}
+
+__device__ __forceinline__ double warp_sum_f64(double v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(kFull, v, o);
+  return v;
+}
+
+// The MBS-Dynamic factor of macro block g of this warp (warp-collective).
+// am: the 4 sub-block amax bits (0 for a macro block holding NaN/Inf, whose
+// staged magnitudes are zeros).
+template <int RULE>
+__device__ __forceinline__ int sweep_macro(SweepShared<RULE>& sh, int g, const uint32_t am[4],
+                                           int lane) {
+  constexpr int NL = SweepShared<RULE>::kLevels;
+  double tot[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) tot[j] = 0.0;
+  const float* xs = sh.xs[g];
+#pragma unroll 1
+  for (int i = 0; i < 4; ++i) {
+    const int ex = static_cast<int>(am[i] >> 7);
+    const int K = 2 * static_cast<int>(am[i] & 0x7F);   // regime 0 for k <= K
+    const float xf = xs[32 * i + lane];
+    const uint32_t xb = __float_as_uint(xf) >> 16;       // |x| as bf16 bits
+    const int exx = static_cast<int>(xb >> 7);
+    const int sig = exx ? static_cast<int>(128 | (xb & 0x7F)) : static_cast<int>(xb & 0x7F);
+    const double x2 = static_cast<double>(xf) * static_cast<double>(xf);   // exact
+    // per (regime r, level u), index q = 2 r + u ... flattened as r * NL + u
+    int a0[2 * NL], b0[2 * NL];
+    unsigned cc[2 * NL];
+    double xt[2 * NL], scl[2 * NL];
+#pragma unroll
+    for (int q = 0; q < 2 * NL; ++q) {
+      const int r = q / NL, u = q % NL;
+      const int Bl = max(ex - 2 + u - r, 0);   // the sub-block byte (MBS rule, OAS candidate u)
+      // T = 512 |x| 2^(127 - Bl) = sig 2^sh (sh <= 5 whenever T > 128)
+      const int sh_ = (exx ? exx : 1) + 2 - Bl;
+      const bool big = sh_ > 0 || (sh_ == 0 && sig > 128);
+      const int T = big ? (sig << sh_) : 0;
+      const int T2 = 2 * T;
+      // F_m: the first F at which the element is no longer above midpoint m
+      int Fm[7];
+      Fm[0] = T2;                 // 1/4, even below: above iff 2T > F
+      Fm[1] = T2 / 3 + 1;         // 3/4, even above: above iff 2T >= 3F
+      Fm[2] = (T2 + 4) / 5;       // 5/4
+      Fm[3] = T2 / 7 + 1;         // 7/4
+      Fm[4] = (T2 + 9) / 10;      // 5/2
+      Fm[5] = T2 / 14 + 1;        // 7/2
+      Fm[6] = (T2 + 19) / 20;     // 5
+      int c0 = 0;
+#pragma unroll
+      for (int m = 0; m < 7; ++m) c0 += Fm[m] > 256 ? 1 : 0;
+      // Q[m] - Q[m+1] and Q[m]^2 - Q[m+1]^2 when the code drops from m+1 to m
+      constexpr int kDq[7] = {-1, -1, -1, -1, -2, -2, -4};
+      constexpr int kDq2[7] = {-1, -3, -5, -7, -20, -28, -80};
+#pragma unroll
+      for (int m = 0; m < 7; ++m) {
+        const int km = Fm[m] - 256;
+        if (km >= 1 && km <= 255) {
+          atomicAdd(&sh.d[2 * q][sweep_slot(km)], T * kDq[m]);
+          atomicAdd(&sh.d[2 * q + 1][sweep_slot(km)], kDq2[m]);
+        }
+      }
+      const int q0 = code_q2(c0);
+      a0[q] = __reduce_add_sync(kFull, T * q0);
+      b0[q] = __reduce_add_sync(kFull, q0 * q0);
+      cc[q] = __reduce_add_sync(kFull, static_cast<unsigned>(T * T));
+      xt[q] = warp_sum_f64(big ? 0.0 : x2);
+      scl[q] = __longlong_as_double(static_cast<long long>(2 * (Bl - 127) - 18 + 1023) << 52);
+    }
+    __syncwarp();
+    // A(k), B(k) per level, of the regime each of this lane's k falls in
+    int sa[NL][8], sb[NL][8];
+#pragma unroll
+    for (int u = 0; u < NL; ++u) {
+      int pa[8], pb[8];
+      scan_row8(sh.d[2 * u], lane, pa);
+      scan_row8(sh.d[2 * u + 1], lane, pb);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        sa[u][j] = a0[u] + pa[j];
+        sb[u][j] = b0[u] + pb[j];
+      }
+      scan_row8(sh.d[2 * (NL + u)], lane, pa);
+      scan_row8(sh.d[2 * (NL + u) + 1], lane, pb);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        if (8 * lane + j > K) {
+          sa[u][j] = a0[NL + u] + pa[j];
+          sb[u][j] = b0[NL + u] + pb[j];
+        }
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      const int k = 8 * lane + j;
+      const int r0 = k > K ? NL : 0;
+      const int F = 256 + k;
+      double best = 0.0;
+#pragma unroll
+      for (int u = 0; u < NL; ++u) {
+        // S = C - 2 F A + F^2 B = C + F (F B - 2 A): F B - 2 A fits in 25
+        // bits, the product and the (non-negative) sum in 34
+        const int inner = F * sb[u][j] - 2 * sa[u][j];
+        const long long S = static_cast<long long>(r0 ? cc[NL + u] : cc[u]) +
+                            static_cast<long long>(F) * inner;
+        const double v = fma(static_cast<double>(S), r0 ? scl[NL + u] : scl[u],
+                             r0 ? xt[NL + u] : xt[u]);
+        best = u == 0 ? v : fmin(best, v);   // OAS: the smaller of the two scales
+      }
+      tot[j] += best;
+    }
+    __syncwarp();   // every lane cleared its entries before the next scatter
+  }
+
+  double mn = tot[0];
+#pragma unroll
+  for (int j = 1; j < 8; ++j) mn = fmin(mn, tot[j]);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mn = fmin(mn, __shfl_xor_sync(kFull, mn, o));
+  const double thr = mn * (1.0 + 0x1p-40);
+  unsigned m8 = 0;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) m8 |= (tot[j] <= thr ? 1u : 0u) << j;
+  const int cnt = static_cast<int>(__reduce_add_sync(kFull, static_cast<unsigned>(__popc(m8))));
+  if (cnt == 1 || mn == 0.0) {
+    const unsigned mine = m8 ? 8u * lane + __ffs(m8) - 1 : 256u;
+    return static_cast<int>(__reduce_min_sync(kFull, mine));
+  }
+  // near-ties: the element-order double sums decide
+  int pos = __popc(m8);
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int t = __shfl_up_sync(kFull, pos, o);
+    if (lane >= o) pos += t;
+  }
+  pos -= __popc(m8);
+#pragma unroll
+  for (int j = 0; j < 8; ++j)
+    if ((m8 >> j) & 1u) sh.cand[pos++] = static_cast<uint8_t>(8 * lane + j);
+  __syncwarp();
+  double best = 0.0;
+  int bk = 256;
+#pragma unroll 1
+  for (int o = 0; o < cnt; o += 32) {
+    const int idx = o + lane;
+    if (idx < cnt) {
+      const int kc = sh.cand[idx];
+      const double s = macro_sse_k<RULE>(xs, am, kc);
+      if (bk == 256 || s < best || (s == best && kc < bk)) {
+        best = s;
+        bk = kc;
+      }
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const double ob = __shfl_xor_sync(kFull, best, o);
+    const int ok = __shfl_xor_sync(kFull, bk, o);
+    if (ok != 256 && (bk == 256 || ob < best || (ob == best && ok < bk))) {
+      best = ob;
+      bk = ok;
+    }
+  }
+  __syncwarp();   // cand is free again
+  return bk;
+}
+
 template <int OP, int RULE>
-__global__ void __launch_bounds__(kThreads) mbs_dynamic_kernel(StreamArgs a) {
-  // four macro blocks per warp step, 8 lanes each; the +1 pad puts the four
-  // groups' broadcast reads of one step in four different banks
-  __shared__ float stage[kThreads / 32][4][128 + 1];
+__global__ void __launch_bounds__(kSweepThreads, 4) mbs_sweep_kernel(StreamArgs a) {
+  __shared__ __align__(16) SweepShared<RULE> shared[kSweepWarps];
+  SweepShared<RULE>& sh = shared[threadIdx.x >> 5];
   const int lane = threadIdx.x & 31;
   const int grp = lane >> 3;
   const int l8 = lane & 7;
-  const int w = threadIdx.x >> 5;
   const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
   double sd = 0.0, sx = 0.0;
-  float* xs = stage[w][grp];
+#pragma unroll
+  for (int q = 0; q < 4 * SweepShared<RULE>::kLevels; ++q) {
+    int4* p = reinterpret_cast<int4*>(&sh.d[q][sweep_slot(8 * lane)]);
+    p[0] = make_int4(0, 0, 0, 0);
+    p[1] = make_int4(0, 0, 0, 0);
+  }
   for (int64_t tile = warp; tile * 32 < a.nslices; tile += nwarps) {
     const int64_t c = tile * 32 + lane;
     const bool valid = c < a.nslices;
+    uint32_t pa, A;
+    bool finite;
+    {
+      V16 v;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v.w[i] = 0;
+      if (valid) v = ld_stream32(a.x + 32 * c);
+      pa = pair_max(amax_bits16(v));
+      A = oct_max(pa);
+      finite = A < 0x7F80u;
+      __syncwarp();   // the previous tile's reads of xs are done
+#pragma unroll
+      for (int i = 0; i < 16; ++i) sh.xs[grp][16 * l8 + i] = finite ? fabsf(elem(v, i)) : 0.0f;
+      __syncwarp();
+    }
+    int k = 0;
+#pragma unroll 1
+    for (int gg = 0; gg < 4; ++gg) {
+      const bool fin_g = __shfl_sync(kFull, A, gg << 3) < 0x7F80u;
+      uint32_t am[4];
+#pragma unroll
+      for (int b = 0; b < 4; ++b) {
+        const uint32_t ab = __shfl_sync(kFull, pa, (gg << 3) + 2 * b);
+        am[b] = fin_g ? ab : 0u;
+      }
+      const int kg = sweep_macro<RULE>(sh, gg, am, lane);
+      if (gg == grp) k = kg;
+    }
+    if (!finite) k = 0;
+    // the slice again (from L2) rather than held in registers through the sweep
     V16 v, g;
 #pragma unroll
     for (int i = 0; i < 8; ++i) v.w[i] = g.w[i] = 0;
@@ -504,45 +792,9 @@ __global__ void __launch_bounds__(kThreads) mbs_dynamic_kernel(StreamArgs a) {
       v = ld_stream32(a.x + 32 * c);
       if (OP == kOpFakeBwd) g = ld_stream32(a.gy + 32 * c);
     }
-    const uint32_t pa = pair_max(amax_bits16(v));
-    const uint32_t A = oct_max(pa);
-    const bool finite = A < 0x7F80u;
-    uint32_t amax[4];
-#pragma unroll
-    for (int b = 0; b < 4; ++b) {
-      const uint32_t ab = __shfl_sync(kFull, pa, (grp << 3) + 2 * b);
-      amax[b] = finite ? ab : 0u;
-    }
-    // Every lane runs the same search so the shuffles stay converged; a macro
-    // block holding NaN/Inf searches zeros and then uses k = 0.
-    __syncwarp();
-#pragma unroll
-    for (int i = 0; i < 16; ++i) xs[16 * l8 + i] = finite ? fabsf(elem(v, i)) : 0.0f;
-    __syncwarp();
-    double best = 0.0;
-    int best_k = -1;
-#pragma unroll 1
-    for (int j = 0; j < 32; ++j) {
-      const int kk = l8 + 8 * j;
-      const double s = macro_sse_k<RULE>(xs, amax, kk);
-      if (best_k < 0 || s < best) {
-        best = s;
-        best_k = kk;
-      }
-    }
-#pragma unroll
-    for (int o = 1; o < 8; o <<= 1) {
-      const double ob = __shfl_xor_sync(kFull, best, o);
-      const int ok = __shfl_xor_sync(kFull, best_k, o);
-      if (ob < best || (ob == best && ok < best_k)) {
-        best = ob;
-        best_k = ok;
-      }
-    }
-    const int k = finite ? best_k : 0;
     process_slice<OP, kFmtE2M1, RULE, kMbsDynamic>(a, v, g, c, valid, lane, pa, k, sd, sx);
   }
-  if (OP == kOpError) reduce_totals(sd, sx, a.totals);
+  if (OP == kOpError) reduce_totals<kSweepWarps>(sd, sx, a.totals);
 }
 
 // ------------------------------------------------------------- dequantize --
@@ -668,9 +920,16 @@ cudaError_t launch_stream(const StreamArgs& a, cudaStream_t st) {
   // the error kernel ends with one double atomic per CTA: keep its grid small
   const int waves = OP == kOpError ? 1 : MX_GRID_WAVES;
   if constexpr (MBS == kMbsDynamic) {
-    auto kern = mbs_dynamic_kernel<OP, RULE>;
-    const int grid = grid_for(kern, (a.nslices + 31) / 32, waves);
-    kern<<<grid, kThreads, 0, st>>>(a);
+    auto kern = mbs_sweep_kernel<OP, RULE>;
+    const int64_t tiles = (a.nslices + 31) / 32;
+    int64_t grid = (tiles + kSweepWarps - 1) / kSweepWarps;
+    if (OP == kOpError) {
+      int per_sm = 0;
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kSweepThreads, 0);
+      const int64_t cap = static_cast<int64_t>(sm_count()) * (per_sm > 0 ? per_sm : 1);
+      if (grid > cap) grid = cap;
+    }
+    kern<<<static_cast<int>(grid > 0 ? grid : 1), kSweepThreads, 0, st>>>(a);
   } else if constexpr (OP == kOpQuant && FMT == kFmtE2M1 && RULE == kOas) {
     constexpr int kTile = (kThreads / 32) * 32 * kUnroll;   // slices per CTA
     const int64_t grid = (a.nslices + kTile - 1) / kTile;

@@ -93,6 +93,27 @@ def special_blocks():
     return arr
 
 
+def sweep_tie_blocks():
+    """Macro blocks whose MBS-Dynamic SSE is smallest, with the same nonzero
+    value, at two factors: constants exact on the grid under both k = 0 and
+    k = 128 (6 -> 6 or 4; 3 -> 6 or 4 one binade down) or k = 64 and k = 224
+    (7.5 -> 6 or 4), plus tiny elements that round to 0 under every factor.
+    The smaller k must win; the search must not stop at the first of them."""
+    rows = []
+    for c, tiny in ((6.0, 2.0 ** -9), (3.0, -2.0 ** -10), (7.5, 2.0 ** -8), (-7.5, 2.0 ** -20),
+                    (5.0, 2.0 ** -9)):
+        v = np.full(128, c, np.float32)
+        v[37], v[100] = tiny, -tiny
+        rows.append(v)
+    v = np.concatenate([np.full(32, 6.0), np.full(32, -3.0), np.full(32, 0.75),
+                        np.full(32, 6.0 * 2 ** -10)]).astype(np.float32)
+    v[5] = 2.0 ** -12
+    rows.append(v)
+    t = torch.from_numpy(np.stack(rows)).to(torch.bfloat16)
+    assert torch.equal(t.float(), torch.from_numpy(np.stack(rows)))
+    return t
+
+
 SMALL = {
     "outlier_act_256x4096": lambda: inputs.outlier_act(),
     "random_bits_3x160": lambda: inputs.random_bf16_bits((3, 160), seed=5),
@@ -103,6 +124,7 @@ SMALL = {
     "heavy_tail_64x4096": lambda: inputs.heavy_tail(rows=64),
     "moe_4x1536x2048_head": lambda: inputs.moe_w13(experts=2, inter2=48),
     "special_blocks": lambda: torch.from_numpy(special_blocks().view(np.int16)).view(torch.bfloat16),
+    "sweep_tie_blocks": sweep_tie_blocks,
 }
 
 
@@ -129,7 +151,7 @@ def test_quantize_parity(mx, oracle_mod, cuda, name, fm):
 
 @pytest.mark.parametrize("fm", ALL, ids=ids)
 @pytest.mark.parametrize("name", ["outlier_act_256x4096", "random_bits_33x1280", "special_blocks",
-                                  "heavy_tail_64x4096"])
+                                  "heavy_tail_64x4096", "sweep_tie_blocks"])
 def test_fake_quant_parity(mx, oracle_mod, cuda, name, fm):
     fmt, m = fm
     x = SMALL[name]()
@@ -149,7 +171,7 @@ def test_fake_quant_parity(mx, oracle_mod, cuda, name, fm):
 
 @pytest.mark.parametrize("fm", ALL, ids=ids)
 @pytest.mark.parametrize("name", ["outlier_act_256x4096", "heavy_tail_64x4096", "random_bits_7x384",
-                                  "special_blocks"])
+                                  "special_blocks", "sweep_tie_blocks"])
 def test_block_error_parity(mx, oracle_mod, cuda, name, fm):
     fmt, m = fm
     x = SMALL[name]()
