@@ -19,8 +19,7 @@ import numpy as np
 
 from .build import build_oracle, oracle_library_path
 
-E2M1 = 0
-E4M3 = 1
+E2M1, E4M3, E5M2, E3M2, E2M3, INT8 = 0, 1, 2, 3, 4, 5
 FLOOR, CEIL, OAS_RULE, OAS = 0, 1, 2, 3
 MBS_STATIC, MBS_DYNAMIC = 1 << 4, 2 << 4
 
@@ -49,6 +48,8 @@ def _load():
     for name in ("oracle_decode_e2m1", "oracle_decode_e4m3", "oracle_decode_e8m0"):
         getattr(lib, name).argtypes = [c_int]
         getattr(lib, name).restype = ctypes.c_double
+    lib.oracle_decode_element.argtypes = [c_int, c_int]
+    lib.oracle_decode_element.restype = ctypes.c_double
     lib.oracle_round_element.argtypes = [ctypes.c_double, ctypes.c_double, c_int]
     lib.oracle_round_element.restype = c_int
     lib.oracle_round_array.argtypes = [dp, i64, ctypes.c_double, c_int,
@@ -101,6 +102,10 @@ def decode_e2m1(code: int) -> float:
 
 def decode_e4m3(code: int) -> float:
     return _load().oracle_decode_e4m3(int(code))
+
+
+def decode_element(code: int, fmt: int) -> float:
+    return _load().oracle_decode_element(int(code), int(fmt))
 
 
 def decode_e8m0(b: int) -> float:

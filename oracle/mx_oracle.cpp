@@ -56,6 +56,10 @@ namespace {
 
 constexpr int kFmtE2M1 = 0;
 constexpr int kFmtE4M3 = 1;
+constexpr int kFmtE5M2 = 2;
+constexpr int kFmtE3M2 = 3;
+constexpr int kFmtE2M3 = 4;
+constexpr int kFmtInt8 = 5;
 
 constexpr int kScaleFloor = 0;
 constexpr int kScaleCeil = 1;
@@ -148,6 +152,47 @@ double decode_e4m3(int code) {
   return sign ? -v : v;
 }
 
+// E5M2: 1 sign, 5 exponent (bias 15), 2 mantissa, IEEE-style: exponent 31
+// is Inf (mantissa 0) or NaN ([VL] MX table, MXFP8 elements E4M3/E5M2).
+double decode_e5m2(int code) {
+  const int sign = (code >> 7) & 1;
+  const int ef = (code >> 2) & 31;
+  const int mf = code & 3;
+  double v;
+  if (ef == 31) v = mf ? std::numeric_limits<double>::quiet_NaN() : std::numeric_limits<double>::infinity();
+  else if (ef == 0) v = std::ldexp(mf / 4.0, -14);
+  else v = std::ldexp(1.0 + mf / 4.0, ef - 15);
+  return sign ? -v : v;
+}
+
+// FP6 elements of MXFP6 ([VL] MX table: E3M2 / E2M3), no Inf/NaN: 1 sign bit
+// (bit 5), then the exponent and mantissa fields.
+// E3M2: 3 exponent (bias 3), 2 mantissa.
+double decode_e3m2(int code) {
+  const int sign = (code >> 5) & 1;
+  const int ef = (code >> 2) & 7;
+  const int mf = code & 3;
+  const double v = ef == 0 ? std::ldexp(mf / 4.0, -2) : std::ldexp(1.0 + mf / 4.0, ef - 3);
+  return sign ? -v : v;
+}
+// E2M3: 2 exponent (bias 1), 3 mantissa.
+double decode_e2m3(int code) {
+  const int sign = (code >> 5) & 1;
+  const int ef = (code >> 3) & 3;
+  const int mf = code & 7;
+  const double v = ef == 0 ? mf / 8.0 : std::ldexp(1.0 + mf / 8.0, ef - 1);
+  return sign ? -v : v;
+}
+
+// MXINT8 elements ([VL] MX table: INT8): an 8-bit two's complement integer i
+// read as i * 2^-6, so that the largest power of two it holds is 2^0 as for
+// the float elements; magnitudes up to 127/64 (the code -128 is never
+// produced: saturation is symmetric).
+double decode_int8(int code) {
+  const int i = code >= 128 ? code - 256 : code;
+  return std::ldexp(static_cast<double>(i), -6);
+}
+
 // E8M0: an unsigned biased exponent, the value 2^(b-127); 0xFF is NaN
 // ([VL] table; [UP] section 1: scale factors are powers of two only).
 double decode_e8m0(int b) {
@@ -155,10 +200,47 @@ double decode_e8m0(int b) {
   return std::ldexp(1.0, b - 127);
 }
 
-int num_magnitude_codes(int fmt) { return fmt == kFmtE2M1 ? 8 : 127; }
-int sign_bit(int fmt) { return fmt == kFmtE2M1 ? 0x8 : 0x80; }
-double magnitude(int fmt, int c) { return fmt == kFmtE2M1 ? decode_e2m1(c) : decode_e4m3(c); }
+double element_value(int code, int fmt) {
+  switch (fmt) {
+    case kFmtE2M1: return decode_e2m1(code);
+    case kFmtE4M3: return decode_e4m3(code);
+    case kFmtE5M2: return decode_e5m2(code);
+    case kFmtE3M2: return decode_e3m2(code);
+    case kFmtE2M3: return decode_e2m3(code);
+    default: return decode_int8(code);
+  }
+}
+
+// Non-negative magnitudes are the codes 0 .. n-1 in increasing order (E4M3
+// stops before its NaN, E5M2 before Inf).
+int num_magnitude_codes(int fmt) {
+  switch (fmt) {
+    case kFmtE2M1: return 8;
+    case kFmtE4M3: return 127;
+    case kFmtE5M2: return 124;
+    case kFmtE3M2:
+    case kFmtE2M3: return 32;
+    default: return 128;
+  }
+}
+int sign_bit(int fmt) {
+  switch (fmt) {
+    case kFmtE2M1: return 0x8;
+    case kFmtE3M2:
+    case kFmtE2M3: return 0x20;
+    default: return 0x80;
+  }
+}
+// Code of the magnitude index c with the sign of v (INT8: two's complement,
+// which has no negative zero).
+int signed_code(int c, bool negative, int fmt) {
+  if (fmt == kFmtInt8) return negative ? ((256 - c) & 0xFF) : c;
+  return negative ? (c | sign_bit(fmt)) : c;
+}
+double magnitude(int fmt, int c) { return element_value(c, fmt); }
 double max_value(int fmt) { return magnitude(fmt, num_magnitude_codes(fmt) - 1); }
+// The smallest nonzero magnitude.
+double min_magnitude(int fmt) { return magnitude(fmt, 1); }
 
 // floor(log2 a) for finite a > 0.
 int floor_log2(double a) {
@@ -183,7 +265,7 @@ int clamp_exp(int E) { return std::min(127, std::max(-127, E)); }
 int round_element(double v, double X, int fmt) {
   const double a = std::fabs(v);
   const int top = num_magnitude_codes(fmt) - 1;
-  if (a >= X * magnitude(fmt, top)) return std::signbit(v) ? (top | sign_bit(fmt)) : top;
+  if (a >= X * magnitude(fmt, top)) return signed_code(top, std::signbit(v), fmt);
   int best = 0;
   double best_d = std::fabs(a - X * magnitude(fmt, 0));
   for (int c = 1; c < num_magnitude_codes(fmt); ++c) {
@@ -193,11 +275,7 @@ int round_element(double v, double X, int fmt) {
       best_d = d;
     }
   }
-  return std::signbit(v) ? (best | sign_bit(fmt)) : best;
-}
-
-double element_value(int code, int fmt) {
-  return fmt == kFmtE2M1 ? decode_e2m1(code) : decode_e4m3(code);
+  return signed_code(best, std::signbit(v), fmt);
 }
 
 bool block_has_nonfinite(const double* x, int n) {
@@ -221,23 +299,28 @@ int floor_log2_over(double a, double f) {
   return e;
 }
 
-// Exact comparison of the two candidate SSEs of an OAS decision. Elements whose
-// dequantized value is the same under both scales add the same term to both
-// sums and drop out; every remaining term is a square of an exact difference,
-// a multiple of one common unit and below 2^26 of it, so the double sum of at
-// most 32 such terms is exact. Returns true when the coarser scale X2 has the
-// strictly smaller SSE.
+// Exact comparison of the two candidate SSEs of an OAS decision: the real
+// sums compared, not their rounded values. Elements whose dequantized value
+// is the same under both scales add the same term to both sums and drop out.
+// Every remaining element has |x| of at least half the smallest nonzero
+// magnitude times X1, so x (8 significant bits), y1 and y2 are all integer
+// multiples of U = min_magnitude * 2^(E1 - 9), where 2^E1 is the power of
+// two in X1 = f * 2^E1 (y carries f = F / 256 with F an integer). Each
+// difference is then an exact integer D below 2^44 units, and the sum of
+// D1^2 - D2^2 is accumulated exactly in 128-bit integers. Returns true when
+// the coarser scale X2 has the strictly smaller SSE.
 bool coarser_scale_wins(const double* x, int n, double X1, double X2, int fmt) {
-  double delta = 0.0;   // SSE(X1) - SSE(X2) over the differing elements
+  const double U = std::ldexp(min_magnitude(fmt), floor_log2(X1) - 9);
+  __int128 delta = 0;   // (SSE(X1) - SSE(X2)) / U^2 over the differing elements
   for (int i = 0; i < n; ++i) {
     const double y1 = element_value(round_element(x[i], X1, fmt), fmt) * X1;
     const double y2 = element_value(round_element(x[i], X2, fmt), fmt) * X2;
     if (y1 == y2) continue;
-    const double d1 = x[i] - y1;
-    const double d2 = x[i] - y2;
-    delta += d1 * d1 - d2 * d2;
+    const auto D1 = static_cast<int64_t>((x[i] - y1) / U);   // exact integers
+    const auto D2 = static_cast<int64_t>((x[i] - y2) / U);
+    delta += static_cast<__int128>(D1) * D1 - static_cast<__int128>(D2) * D2;
   }
-  return delta > 0.0;
+  return delta > 0;
 }
 
 // Scale exponent of one finite 32-element block for the base rules, with the
@@ -319,9 +402,12 @@ BlockResult quantize_block(const double* x, int fmt, int rule, double f) {
     r.X = std::numeric_limits<double>::quiet_NaN();
     for (int i = 0; i < kBlock; ++i) {
       const int s = std::signbit(x[i]) ? sign_bit(fmt) : 0;
-      // E4M3 elements of a NaN-scale block are NaN (S.1111.111); E2M1 has no
-      // NaN, so only the sign is kept.
-      r.codes[i] = fmt == kFmtE2M1 ? s : (s | 0x7F);
+      // The FP8 elements of a NaN-scale block are NaN (E4M3 S.1111.111, E5M2
+      // S.11111.11); E2M1 and FP6 have no NaN, so only the sign is kept;
+      // INT8 has neither NaN nor -0: 0.
+      if (fmt == kFmtE4M3 || fmt == kFmtE5M2) r.codes[i] = s | 0x7F;
+      else if (fmt == kFmtInt8) r.codes[i] = 0;
+      else r.codes[i] = s;
     }
     return r;
   }
@@ -455,6 +541,7 @@ uint16_t oracle_encode_bf16_rne(double v) { return encode_bf16_rne(v); }
 double oracle_decode_e2m1(int code) { return decode_e2m1(code); }
 double oracle_decode_e4m3(int code) { return decode_e4m3(code); }
 double oracle_decode_e8m0(int b) { return decode_e8m0(b); }
+double oracle_decode_element(int code, int fmt) { return element_value(code, fmt); }
 int oracle_round_element(double v, double X, int fmt) { return round_element(v, X, fmt); }
 
 // round_element over an array (one X for all), for exhaustive checks.
@@ -476,8 +563,9 @@ int oracle_macro_k(const uint16_t* x128, int fmt, int scaling) {
   return macro_k(x, fmt, scaling & 0xF, scaling >> 4);
 }
 
-// Codes (FP4: two per byte, even element in the low nibble; FP8: one per
-// byte), E8M0 scale bytes [rows, cols/32], and MBS factor bytes [rows, cols/128].
+// Codes (FP4: two per byte, even element in the low nibble; FP8, FP6 and
+// INT8: one per byte, FP6 in the low 6 bits), E8M0 scale bytes
+// [rows, cols/32], and MBS factor bytes [rows, cols/128].
 void oracle_quantize(const uint16_t* x, int64_t rows, int64_t cols, int fmt, int scaling,
                      uint8_t* codes, uint8_t* scales, uint8_t* macro) {
   parallel_rows(rows, [&](int64_t r0, int64_t r1) {

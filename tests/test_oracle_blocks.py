@@ -18,7 +18,7 @@ with open(os.path.join(HERE, "golden", "hand_blocks.json")) as f:
     GOLDEN = json.load(f)
 
 MODES = {"FLOOR": 0, "CEIL": 1, "OAS_RULE": 2, "OAS": 3, "MBS_STATIC": 1 << 4}
-FMTS = {"E2M1": 0, "E4M3": 1}
+FMTS = {"E2M1": 0, "E4M3": 1, "E5M2": 2, "E3M2": 3, "E2M3": 4, "INT8": 5}
 
 
 def _block(values, n=32):

@@ -1,0 +1,234 @@
+"""Pins of the oracle's MXFP8-E5M2, MXFP6 (E3M2, E2M3) and MXINT8 elements.
+
+"[vLLM] MXFP8/MXFP4: microscaling format quantization" lists these element
+types beside E4M3 and E2M1, each with block 32 and an E8M0 scale (MX format
+table). The pages do not spell out the encodings, so the oracle uses the
+standard minifloat fields and the tests compare it with libraries that share
+no code with it:
+* E5M2 with torch.float8_e5m2 and ml_dtypes.float8_e5m2 (IEEE-style, with
+  Inf/NaN at exponent 31);
+* E3M2 and E2M3 with ml_dtypes.float6_e3m2fn and float6_e2m3fn (no Inf/NaN;
+  ml_dtypes saturates on overflow);
+* INT8 with numpy's int8 reading of the byte times 2^-6, rounded by np.rint
+  (round half to even) and clipped to +-127.
+
+Scale bytes follow the written-out FLOOR and CEIL rules with each format's
+emax (the exponent of its largest power of two: 15, 4, 2, 0). OAS is checked
+as the exact argmin of the block SSE over {e - emax, e - emax + 1}, with
+exact rational SSEs from library codes; E4M3 is included, as OAS now applies
+to it too.
+"""
+
+from fractions import Fraction
+
+import ml_dtypes
+import numpy as np
+import pytest
+import torch
+
+E4M3, E5M2, E3M2, E2M3, INT8 = 1, 2, 3, 4, 5
+FLOOR, CEIL, OAS = 0, 1, 3
+EMAX = {E4M3: 8, E5M2: 15, E3M2: 4, E2M3: 2, INT8: 0}
+MAXV = {E4M3: 448.0, E5M2: 57344.0, E3M2: 28.0, E2M3: 7.5, INT8: 127 / 64}
+
+
+def lib_codes(q, fmt):
+    """Codes of the scaled values q (float64) from the libraries: round to
+    nearest even with saturation, sign kept (INT8: two's complement)."""
+    q = np.asarray(q, np.float64)
+    if fmt == E4M3:
+        q32 = np.clip(q, -448.0, 448.0).astype(np.float32)
+        return torch.from_numpy(q32).to(torch.float8_e4m3fn).view(torch.uint8).numpy().astype(np.int32)
+    if fmt == E5M2:
+        q32 = np.clip(q, -57344.0, 57344.0).astype(np.float32)
+        return torch.from_numpy(q32).to(torch.float8_e5m2).view(torch.uint8).numpy().astype(np.int32)
+    if fmt in (E3M2, E2M3):
+        t = ml_dtypes.float6_e3m2fn if fmt == E3M2 else ml_dtypes.float6_e2m3fn
+        with np.errstate(over="ignore"):
+            return q.astype(np.float32).astype(t).view(np.uint8).astype(np.int32)
+    i = np.clip(np.rint(q * 64.0), -127, 127).astype(np.int64)
+    return (i & 0xFF).astype(np.int32)
+
+
+def lib_values(codes, fmt):
+    codes = np.asarray(codes, np.uint8)
+    if fmt == E4M3:
+        return torch.from_numpy(codes).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    if fmt == E5M2:
+        return torch.from_numpy(codes).view(torch.float8_e5m2).to(torch.float64).numpy()
+    if fmt == E3M2:
+        return codes.view(ml_dtypes.float6_e3m2fn).astype(np.float64)
+    if fmt == E2M3:
+        return codes.view(ml_dtypes.float6_e2m3fn).astype(np.float64)
+    return codes.view(np.int8).astype(np.float64) / 64.0
+
+
+# ------------------------------------------------------------- value sets --
+
+def test_e5m2_all_bytes(oracle_mod):
+    got = np.array([oracle_mod.decode_element(b, E5M2) for b in range(256)])
+    for ref in (torch.arange(256, dtype=torch.uint8).view(torch.float8_e5m2).to(torch.float64).numpy(),
+                np.arange(256, dtype=np.uint8).view(ml_dtypes.float8_e5m2).astype(np.float64)):
+        nan = np.isnan(ref)
+        assert np.array_equal(nan, np.isnan(got))
+        assert np.array_equal(got[~nan], ref[~nan])
+    assert np.nanmax(got[np.isfinite(got)]) == 57344.0
+    assert set(np.nonzero(np.isinf(got))[0]) == {0x7C, 0xFC}
+
+
+@pytest.mark.parametrize("fmt,t", [(E3M2, ml_dtypes.float6_e3m2fn), (E2M3, ml_dtypes.float6_e2m3fn)])
+def test_fp6_all_codes(oracle_mod, fmt, t):
+    got = np.array([oracle_mod.decode_element(c, fmt) for c in range(64)])
+    ref = np.arange(64, dtype=np.uint8).view(t).astype(np.float64)
+    assert np.array_equal(got, ref)
+    assert np.array_equal(np.signbit(got), np.signbit(ref))   # bit 5 is the sign, 32 is -0
+    assert got.max() == MAXV[fmt]
+
+
+def test_int8_all_bytes(oracle_mod):
+    got = np.array([oracle_mod.decode_element(b, INT8) for b in range(256)])
+    assert np.array_equal(got, np.arange(256, dtype=np.uint8).view(np.int8) / 64.0)
+
+
+def test_emax_is_the_largest_power_of_two(oracle_mod):
+    for fmt, emax in EMAX.items():
+        n = 256 if fmt != E3M2 and fmt != E2M3 else 64
+        vals = np.array([oracle_mod.decode_element(c, fmt) for c in range(n)])
+        vmax = vals[np.isfinite(vals)].max()
+        assert vmax == MAXV[fmt] and 2.0 ** emax <= vmax < 2.0 ** (emax + 1)
+
+
+# --------------------------------------------------------------- rounding --
+
+def _finite_bf16_values():
+    bits = np.arange(1 << 16, dtype=np.uint16)
+    v = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(torch.float64).numpy()
+    return v[np.isfinite(v)]
+
+
+VALUES = _finite_bf16_values()
+
+
+@pytest.mark.parametrize("fmt", [E5M2, E3M2, E2M3, INT8])
+@pytest.mark.parametrize("E", [-127, -126, -100, -40, -17, -9, -3, 0, 2, 5, 30, 90, 125, 127])
+def test_rounding_every_bf16(oracle_mod, fmt, E):
+    X = 2.0 ** E
+    got = oracle_mod.round_array(VALUES, X, fmt)
+    # INT8 has no -0: a negative that rounds to 0 is code 0, as numpy gives
+    assert np.array_equal(got, lib_codes(VALUES / X, fmt))
+
+
+def test_ties_go_to_even_codes(oracle_mod):
+    # E2M3 grid step 0.5 in [4, 8): 4.25 -> 4.0 (mantissa 000), 4.75 -> 5.0 (010)
+    assert oracle_mod.round_element(4.25, 1.0, E2M3) == 0x18
+    assert oracle_mod.round_element(4.75, 1.0, E2M3) == 0x1A
+    # E3M2 subnormal step 1/16: 1/32 -> 0, 3/32 -> 1/8 (code 2)
+    assert oracle_mod.round_element(1 / 32, 1.0, E3M2) == 0
+    assert oracle_mod.round_element(3 / 32, 1.0, E3M2) == 2
+    # INT8: 0.5 / 64 -> 0, 1.5 / 64 -> 2 / 64, -2.5 / 64 -> -2 / 64
+    assert oracle_mod.round_element(0.5 / 64, 1.0, INT8) == 0
+    assert oracle_mod.round_element(1.5 / 64, 1.0, INT8) == 2
+    assert oracle_mod.round_element(-2.5 / 64, 1.0, INT8) == 254
+
+
+def test_saturation_and_signs(oracle_mod):
+    assert oracle_mod.round_element(1e30, 1.0, E5M2) == 0x7B
+    assert oracle_mod.round_element(-1e30, 1.0, E5M2) == 0xFB
+    assert oracle_mod.round_element(61440.0, 1.0, E5M2) == 0x7B   # a tie past the top
+    assert oracle_mod.round_element(-1e30, 1.0, E3M2) == 0x3F
+    assert oracle_mod.round_element(-0.001, 1.0, E2M3) == 0x20    # -0 kept
+    assert oracle_mod.round_element(1e30, 1.0, INT8) == 0x7F
+    assert oracle_mod.round_element(-1e30, 1.0, INT8) == 0x81     # -127, never -128
+    assert oracle_mod.round_element(-0.001, 1.0, INT8) == 0
+
+
+# ------------------------------------------------------------ scale rules --
+
+def _to_bf16_bits(x):
+    return torch.from_numpy(np.ascontiguousarray(x, np.float32)).to(torch.bfloat16) \
+        .view(torch.int16).numpy().view(np.uint16)
+
+
+def _bits_to_f64(b):
+    return torch.from_numpy(b.view(np.int16)).view(torch.bfloat16).to(torch.float64).numpy()
+
+
+def blocks(n, seed):
+    """Seeded blocks: Gaussian and Student-t at scales 2^-30 .. 2^30, some with
+    the max significand near the top of its binade (where CEIL and OAS act)."""
+    rng = np.random.default_rng(seed)
+    scale = 2.0 ** rng.integers(-30, 30, (n, 1))
+    x = np.where(rng.random((n, 1)) < 0.5, rng.standard_normal((n, 32)), rng.standard_t(2, (n, 32)))
+    x = x * scale
+    top = rng.random(n) < 0.4
+    x[top, 0] = np.sign(x[top, 0] + 1e-300) * (1.75 + 0.25 * rng.random(top.sum())) * \
+        np.abs(x[top]).max(axis=1) * 1.01
+    return _to_bf16_bits(x)
+
+
+@pytest.mark.parametrize("fmt", [E4M3, E5M2, E3M2, E2M3, INT8])
+def test_floor_and_ceil_bytes_by_definition(oracle_mod, fmt):
+    bits = blocks(3000, 40 + fmt)
+    xf = _bits_to_f64(bits)
+    amax = np.abs(xf).max(axis=1)
+    e = np.frexp(amax)[1] - 1
+    nz = amax > 0
+    _, s, _ = oracle_mod.quantize(bits, fmt, FLOOR)
+    assert np.array_equal(s[:, 0], np.where(nz, np.clip(e - EMAX[fmt], -127, 127) + 127, 0))
+    _, s, _ = oracle_mod.quantize(bits, fmt, CEIL)
+    E = np.where(amax <= MAXV[fmt] * 2.0 ** (e - EMAX[fmt]), e - EMAX[fmt], e - EMAX[fmt] + 1)
+    assert np.array_equal(s[:, 0], np.where(nz, np.clip(E, -127, 127) + 127, 0))
+
+
+def exact_sse(x, y):
+    return sum((Fraction(float(a)) - Fraction(float(b))) ** 2 for a, b in zip(x, y))
+
+
+@pytest.mark.parametrize("fmt", [E4M3, E5M2, E3M2, E2M3])
+def test_oas_is_the_exact_argmin(oracle_mod, fmt):
+    bits = blocks(1500, 60 + fmt)
+    xf = _bits_to_f64(bits)
+    _, s, _ = oracle_mod.quantize(bits, fmt, OAS)
+    amax = np.abs(xf).max(axis=1)
+    e = np.frexp(amax)[1] - 1
+    coarser = 0
+    for i in range(len(xf)):
+        if amax[i] == 0:
+            continue
+        E1 = int(np.clip(e[i] - EMAX[fmt], -127, 127))
+        E2 = int(np.clip(e[i] - EMAX[fmt] + 1, -127, 127))
+        if E1 == E2:
+            assert int(s[i, 0]) == E1 + 127
+            continue
+        y1 = lib_values(lib_codes(xf[i] / 2.0 ** E1, fmt), fmt) * 2.0 ** E1
+        y2 = lib_values(lib_codes(xf[i] / 2.0 ** E2, fmt), fmt) * 2.0 ** E2
+        s1, s2 = exact_sse(xf[i], y1), exact_sse(xf[i], y2)
+        want = E2 if s2 < s1 else E1
+        coarser += want == E2
+        assert int(s[i, 0]) == want + 127, (i, s1, s2)
+    assert coarser > 0   # the seeded blocks do exercise the coarser choice
+
+
+@pytest.mark.parametrize("fmt", [E5M2, E3M2, E2M3, INT8])
+def test_fake_quant_idempotent_and_bwd_mask(oracle_mod, fmt):
+    bits = blocks(500, 80 + fmt)
+    y = oracle_mod.fake_quant_fwd(bits, fmt, FLOOR)
+    y2 = oracle_mod.fake_quant_fwd(y, fmt, FLOOR)
+    assert np.array_equal(y, y2)
+    # the straight-through mask passes exactly the elements within maxv * X
+    g = _to_bf16_bits(np.ones_like(_bits_to_f64(bits)))
+    gx = _bits_to_f64(oracle_mod.fake_quant_bwd(bits, g, fmt, FLOOR))
+    xf = _bits_to_f64(bits)
+    _, s, _ = oracle_mod.quantize(bits, fmt, FLOOR)
+    X = 2.0 ** (s[:, :1].astype(np.float64) - 127)
+    assert np.array_equal(gx == 1.0, np.abs(xf) <= MAXV[fmt] * X)
+
+
+def test_nonfinite_block_codes(oracle_mod):
+    b = np.zeros((1, 32), np.uint16)
+    b[0, 0] = 0x7FC0          # NaN
+    b[0, 1] = 0xBF80          # -1.0
+    for fmt, neg in ((E5M2, 0xFF), (E3M2, 0x20), (E2M3, 0x20), (INT8, 0)):
+        c, s, _ = oracle_mod.quantize(b, fmt, FLOOR)
+        assert int(s[0, 0]) == 255
+        assert int(c[0, 1]) == neg
