@@ -261,6 +261,14 @@ def stack_ops(mx, x, reps=50, only=None):
         "fp4_dequantize_bf16": (lambda: mx.dequantize(c4, sc, None, mx.E2M1, out=y), fp4),
         "fp8_dequantize_bf16": (lambda: mx.dequantize(c8, sc, None, mx.E4M3, out=y), fp8),
         "fp4_block_error": (lambda: mx.block_error(x, per_block=False), n * 2),
+        "e5m2_floor_quantize": (lambda: mx.quantize(x, mx.E5M2, mx.FLOOR, out=(c8, sc, None)), fp8),
+        "e3m2_floor_quantize": (lambda: mx.quantize(x, mx.E3M2, mx.FLOOR, out=(c8, sc, None)), fp8),
+        "e2m3_floor_quantize": (lambda: mx.quantize(x, mx.E2M3, mx.FLOOR, out=(c8, sc, None)), fp8),
+        "int8_floor_quantize": (lambda: mx.quantize(x, mx.INT8, mx.FLOOR, out=(c8, sc, None)), fp8),
+        "e4m3_oas_quantize": (lambda: mx.quantize(x, mx.E4M3, mx.OAS, out=(c8, sc, None)), fp8),
+        "e5m2_oas_quantize": (lambda: mx.quantize(x, mx.E5M2, mx.OAS, out=(c8, sc, None)), fp8),
+        "e2m3_oas_quantize": (lambda: mx.quantize(x, mx.E2M3, mx.OAS, out=(c8, sc, None)), fp8),
+        "int8_dequantize_bf16": (lambda: mx.dequantize(c8, sc, None, mx.INT8, out=y), fp8),
         "fp4_mbs_dynamic_quantize": (lambda: mx.quantize(x, mx.E2M1, mx.MBS_DYNAMIC, out=(c4, sc, mac)),
                                      fp4m),
         "fp4_oas_mbs_dynamic_quantize": (lambda: mx.quantize(x, mx.E2M1, mx.OAS | mx.MBS_DYNAMIC,
@@ -278,6 +286,8 @@ def stack_ops(mx, x, reps=50, only=None):
             mx.quantize(x, mx.E2M1, mx.FLOOR, out=(c4, sc, None))
         if name == "fp8_dequantize_bf16":
             mx.quantize(x, mx.E4M3, mx.FLOOR, out=(c8, sc, None))
+        if name == "int8_dequantize_bf16":
+            mx.quantize(x, mx.INT8, mx.FLOOR, out=(c8, sc, None))
         fn()
         torch.cuda.synchronize()
         n_reps = min(reps, op_reps.get(name, reps))

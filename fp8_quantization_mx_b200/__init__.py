@@ -31,7 +31,7 @@ import os
 import torch
 
 __all__ = [
-    "E2M1", "E4M3", "FLOOR", "CEIL", "OAS_RULE", "OAS", "MBS_STATIC", "MBS_DYNAMIC",
+    "E2M1", "E4M3", "E5M2", "E3M2", "E2M3", "INT8", "FLOOR", "CEIL", "OAS_RULE", "OAS", "MBS_STATIC", "MBS_DYNAMIC",
     "MXError", "library_path", "load_library",
     "mx_quantize", "mx_dequantize", "mx_fake_quant_fwd", "mx_fake_quant_bwd",
     "mx_block_error", "mx_status_string", "mx_version",
@@ -40,8 +40,12 @@ __all__ = [
 ]
 
 # formats (mx_format_t)
-E2M1 = 0
-E4M3 = 1
+E2M1 = 0   # MXFP4
+E4M3 = 1   # MXFP8
+E5M2 = 2   # MXFP8
+E3M2 = 3   # MXFP6 (one code per byte, low 6 bits)
+E2M3 = 4   # MXFP6
+INT8 = 5   # MXINT8 (i * 2^-6)
 MXFP4_FORMAT = E2M1
 MXFP8_FORMAT = E4M3
 # scaling (mx_scaling_t)
@@ -157,8 +161,8 @@ def quantize(x: torch.Tensor, format: int = E2M1, scaling: int = FLOOR, out=None
     """MX-quantizes bf16 ``x`` [..., cols] along its last dimension.
 
     Returns ``(codes, scales, macro)``: codes uint8 [..., cols/2] (MXFP4, two
-    codes per byte, even element in the low nibble) or [..., cols] (MXFP8,
-    E4M3 bytes); scales uint8 [..., cols/32] (E8M0); macro uint8 [..., cols/128]
+    codes per byte, even element in the low nibble) or [..., cols] (every other
+    format, one code per byte); scales uint8 [..., cols/32] (E8M0); macro uint8 [..., cols/128]
     with Macro Block Scaling, else None. ``out`` may supply the three buffers.
     A CPU ``x`` is copied to the current GPU and the outputs come back to the
     CPU: into ``out`` (host tensors) when given, else into new tensors (pinned

@@ -30,14 +30,19 @@ int check_shape(int64_t rows, int64_t cols, bool mbs) {
 }
 
 // Format and scaling combinations the kernels implement.
+bool known_format(int format) { return format >= MX_FMT_E2M1 && format <= MX_FMT_INT8; }
+
 int check_mode(int format, int scaling) {
-  if (format != MX_FMT_E2M1 && format != MX_FMT_E4M3) return MX_ERR_UNSUPPORTED;
+  if (!known_format(format)) return MX_ERR_UNSUPPORTED;
   if (scaling < 0 || (scaling & ~0x3F) != 0) return MX_ERR_UNSUPPORTED;
   const int rule = scaling & 0xF;
   const int mbs = scaling >> 4;
   if (rule > MX_SCALE_OAS || mbs > 2) return MX_ERR_UNSUPPORTED;
-  if (format == MX_FMT_E4M3 && (rule == MX_SCALE_OAS_RULE || rule == MX_SCALE_OAS || mbs != 0))
-    return MX_ERR_UNSUPPORTED;
+  if (format != MX_FMT_E2M1) {
+    // one-byte formats: FLOOR, CEIL, and OAS for the float elements
+    if (mbs != 0 || rule == MX_SCALE_OAS_RULE) return MX_ERR_UNSUPPORTED;
+    if (format == MX_FMT_INT8 && rule == MX_SCALE_OAS) return MX_ERR_UNSUPPORTED;
+  }
   if (mbs != 0 && rule != MX_SCALE_FLOOR && rule != MX_SCALE_OAS) return MX_ERR_UNSUPPORTED;
   return MX_OK;
 }
@@ -79,8 +84,8 @@ int mx_quantize(const void* x, int64_t rows, int64_t cols, int format, int scali
 
 int mx_dequantize(const void* codes, const uint8_t* scales, const uint8_t* macro, int64_t rows,
                   int64_t cols, int format, int out_fp32, void* out, void* stream) {
-  if (format != MX_FMT_E2M1 && format != MX_FMT_E4M3) return MX_ERR_UNSUPPORTED;
-  if (format == MX_FMT_E4M3 && macro) return MX_ERR_UNSUPPORTED;
+  if (!known_format(format)) return MX_ERR_UNSUPPORTED;
+  if (format != MX_FMT_E2M1 && macro) return MX_ERR_UNSUPPORTED;
   if (out_fp32 != 0 && out_fp32 != 1) return MX_ERR_INVALID_ARG;
   int st = check_shape(rows, cols, macro != nullptr);
   if (st != MX_OK) return st;

@@ -20,15 +20,17 @@
 //  * x * 2^-E is exact in bf16 whenever it is at least 2^-126 (a power-of-two
 //    scaling of an 8-bit significand), and anything smaller rounds to a signed
 //    zero code anyway, so the scaled pairs feed the hardware conversions
-//    cvt.rn.satfinite.{e2m1x2,e4m3x2}.f32 (round to nearest even, saturate);
+//    cvt.rn.satfinite.{e2m1x2,e4m3x2,e5m2x2,e3m2x2,e2m3x2}.f32 (round to
+//    nearest even, saturate) or, for INT8, an fma-based integer rounding;
 //  * with a macro factor f = (256 + k) / 256 the quotient x / (f 2^E) is not
 //    exact in float; it is bracketed by two products with 1/f rounded down
 //    and up, both bounds go through the hardware conversion, and the only way
 //    they can disagree is an exact tie, where the even code wins (see
 //    enc_mbs_cvt_16);
 //  * decoding (fake-quant, error, dequantize): a byte-permute table for E2M1
-//    (integer only) and the hardware cvt.rn.f16x2.e4m3x2 for E4M3 (exact),
-//    then an exact float product with the scale.
+//    (integer only), the hardware cvt.rn.f16x2.{e4m3x2,e5m2x2,e3m2x2,e2m3x2}
+//    for the other float elements and an integer-to-float step for INT8 (all
+//    exact), then an exact float product with the scale.
 #pragma once
 
 #include <cstdint>
@@ -38,6 +40,10 @@ namespace mxk {
 
 constexpr int kFmtE2M1 = 0;
 constexpr int kFmtE4M3 = 1;
+constexpr int kFmtE5M2 = 2;
+constexpr int kFmtE3M2 = 3;
+constexpr int kFmtE2M3 = 4;
+constexpr int kFmtInt8 = 5;
 constexpr int kFloor = 0, kCeil = 1, kOasRule = 2, kOas = 3;
 constexpr int kMbsNone = 0, kMbsStatic = 1, kMbsDynamic = 2;
 constexpr unsigned kFull = 0xFFFFFFFFu;
@@ -139,14 +145,15 @@ __device__ __forceinline__ float pow2f(int E) {
                    : __uint_as_float(1u << (E + 149));
 }
 
-// 2^-E for an E8M0 byte b = E + 127 in [0, 253]: always a normal float.
+// 2^-E for an E8M0 byte b = E + 127 in [0, 254]: a normal float, except
+// 2^-127 (b = 254, reached only by INT8, whose emax is 0), a subnormal.
 __device__ __forceinline__ float inv_scale_from_byte(int b) {
-  return __uint_as_float(static_cast<uint32_t>(254 - b) << 23);
+  return b <= 253 ? __uint_as_float(static_cast<uint32_t>(254 - b) << 23) : __uint_as_float(0x00400000u);
 }
 
-// 2^-E as a bf16x2 pair for b in [0, 253] (a normal bf16).
+// 2^-E as a bf16x2 pair for b in [0, 254] (2^-127 is the bf16 subnormal 0x0040).
 __device__ __forceinline__ uint32_t inv_scale_bf16x2(int b) {
-  return static_cast<uint32_t>(254 - b) * 0x00800080u;
+  return b <= 253 ? static_cast<uint32_t>(254 - b) * 0x00800080u : 0x00400040u;
 }
 
 __device__ __forceinline__ uint32_t mul_bf16x2(uint32_t a, uint32_t b) {
@@ -406,6 +413,143 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return r;
 }
 
+// ------------------------------------------------------- one-byte formats --
+//
+// E4M3, E5M2, E3M2 and E2M3 codes come from the hardware converters
+// cvt.rn.satfinite.{e4m3x2,e5m2x2,e3m2x2,e2m3x2}.f32 (round to nearest even,
+// saturating, sign kept; an FP6 code sits in the low 6 bits of its byte) and
+// decode through cvt.rn.f16x2.{...}x2 (every such value is an f16 value). An
+// INT8 code is RNE(64 s) of the scaled value s clamped to +-127/64, two's
+// complement, so that the element reads i * 2^-6.
+
+#define MXK_CVT_BYTES_X8(NAME, TYPE)                                                 \
+  __device__ __forceinline__ uint2 NAME(const uint32_t s[4]) {                     \
+    uint2 r;                                                                        \
+    asm("{\n\t.reg .b16 h0, h1, h2, h3;\n\t"                                       \
+        "cvt.rn.satfinite." TYPE ".f32 h0, %3, %2;\n\t"                             \
+        "cvt.rn.satfinite." TYPE ".f32 h1, %5, %4;\n\t"                             \
+        "cvt.rn.satfinite." TYPE ".f32 h2, %7, %6;\n\t"                             \
+        "cvt.rn.satfinite." TYPE ".f32 h3, %9, %8;\n\t"                             \
+        "mov.b32 %0, {h0, h1};\n\t"                                                 \
+        "mov.b32 %1, {h2, h3};\n\t}"                                                \
+        : "=r"(r.x), "=r"(r.y)                                                      \
+        : "f"(bf_lo(s[0])), "f"(bf_hi(s[0])), "f"(bf_lo(s[1])), "f"(bf_hi(s[1])),   \
+          "f"(bf_lo(s[2])), "f"(bf_hi(s[2])), "f"(bf_lo(s[3])), "f"(bf_hi(s[3])));  \
+    return r;                                                                       \
+  }
+MXK_CVT_BYTES_X8(cvt_e5m2x8, "e5m2x2")
+MXK_CVT_BYTES_X8(cvt_e3m2x8, "e3m2x2")
+MXK_CVT_BYTES_X8(cvt_e2m3x8, "e2m3x2")
+#undef MXK_CVT_BYTES_X8
+
+// INT8 codes of four bf16x2 words of scaled values: 64 s (exact) clamped to
+// +-127, plus 1.5 * 2^23 in one fma, leaves RNE(64 s) in the low mantissa
+// bits, so the low byte is the two's complement code.
+__device__ __forceinline__ uint2 cvt_int8x8(const uint32_t s[4]) {
+  uint32_t t[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const float v = (i & 1) ? bf_hi(s[i >> 1]) : bf_lo(s[i >> 1]);
+    const float c = fminf(fmaxf(v, -1.984375f), 1.984375f);
+    t[i] = __float_as_uint(fmaf(c, 64.0f, 12582912.0f));
+  }
+  return make_uint2(__byte_perm(__byte_perm(t[0], t[1], 0x0040), __byte_perm(t[2], t[3], 0x0040), 0x5410),
+                    __byte_perm(__byte_perm(t[4], t[5], 0x0040), __byte_perm(t[6], t[7], 0x0040), 0x5410));
+}
+
+template <int FMT>
+__device__ __forceinline__ uint2 cvt_bytes_x8(const uint32_t s[4]) {
+  if constexpr (FMT == kFmtE4M3) return cvt_e4m3x8(s);
+  else if constexpr (FMT == kFmtE5M2) return cvt_e5m2x8(s);
+  else if constexpr (FMT == kFmtE3M2) return cvt_e3m2x8(s);
+  else if constexpr (FMT == kFmtE2M3) return cvt_e2m3x8(s);
+  else return cvt_int8x8(s);
+}
+
+// 16 one-byte codes of a scaled slice: byte i = element i.
+template <int FMT>
+__device__ __forceinline__ uint4 enc_bytes_16(const V16& s) {
+  const uint2 a = cvt_bytes_x8<FMT>(&s.w[0]);
+  const uint2 b = cvt_bytes_x8<FMT>(&s.w[4]);
+  return make_uint4(a.x, a.y, b.x, b.y);
+}
+
+// Codes of a block holding NaN/Inf: the FP8 NaN S.1111.111 / S.11111.11
+// (0x7F with the sign); FP6 has no NaN, so only the sign (bit 5); INT8 has
+// neither NaN nor -0: 0.
+template <int FMT>
+__device__ __forceinline__ uint4 nonfinite_bytes_16(const V16& x) {
+  if constexpr (FMT == kFmtE4M3 || FMT == kFmtE5M2) {
+    return nonfinite_e4m3_16(x);
+  } else if constexpr (FMT == kFmtInt8) {
+    return make_uint4(0, 0, 0, 0);
+  } else {
+    uint32_t r[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint32_t a = x.w[2 * j], b = x.w[2 * j + 1];
+      r[j] = (((a >> 15) & 1u) << 5) | (((a >> 31) & 1u) << 13) | (((b >> 15) & 1u) << 21) |
+             (((b >> 31) & 1u) << 29);
+    }
+    return make_uint4(r[0], r[1], r[2], r[3]);
+  }
+}
+
+#define MXK_BYTES_TO_F16X2(NAME, TYPE)                                         \
+  __device__ __forceinline__ void NAME(uint32_t lo, uint32_t hi, uint32_t h[4]) { \
+    asm("{\n\t.reg .b16 p0, p1, p2, p3;\n\t"                                   \
+        "mov.b32 {p0, p1}, %4;\n\t"                                            \
+        "mov.b32 {p2, p3}, %5;\n\t"                                            \
+        "cvt.rn.f16x2." TYPE " %0, p0;\n\t"                                    \
+        "cvt.rn.f16x2." TYPE " %1, p1;\n\t"                                    \
+        "cvt.rn.f16x2." TYPE " %2, p2;\n\t"                                    \
+        "cvt.rn.f16x2." TYPE " %3, p3;\n\t}"                                   \
+        : "=r"(h[0]), "=r"(h[1]), "=r"(h[2]), "=r"(h[3])                       \
+        : "r"(lo), "r"(hi));                                                   \
+  }
+MXK_BYTES_TO_F16X2(e5m2x8_to_f16x2, "e5m2x2")
+MXK_BYTES_TO_F16X2(e3m2x8_to_f16x2, "e3m2x2")
+MXK_BYTES_TO_F16X2(e2m3x8_to_f16x2, "e2m3x2")
+#undef MXK_BYTES_TO_F16X2
+
+// Decoded values of 16 one-byte codes times p (a power of two): exact floats
+// (INT8: i * 2^-6 * p, exact down to 2^-149), overflow to +-inf, NaN codes NaN.
+template <int FMT>
+__device__ __forceinline__ F16 dec_bytes_16(uint4 codes, float p) {
+  if constexpr (FMT == kFmtE4M3) {
+    return dec_e4m3_16(codes, p);
+  } else if constexpr (FMT == kFmtInt8) {
+    F16 r;
+    const uint32_t w[4] = {codes.x, codes.y, codes.z, codes.w};
+    const float q = p * 0.015625f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const int v = static_cast<int>(w[i >> 2] << (24 - 8 * (i & 3))) >> 24;   // sign-extended
+      r.v[i] = (__int_as_float(0x4B400000 + v) - 12582912.0f) * q;
+    }
+    return r;
+  } else {
+    F16 r;
+    uint32_t h[8];
+    if constexpr (FMT == kFmtE5M2) {
+      e5m2x8_to_f16x2(codes.x, codes.y, &h[0]);
+      e5m2x8_to_f16x2(codes.z, codes.w, &h[4]);
+    } else if constexpr (FMT == kFmtE3M2) {
+      e3m2x8_to_f16x2(codes.x, codes.y, &h[0]);
+      e3m2x8_to_f16x2(codes.z, codes.w, &h[4]);
+    } else {
+      e2m3x8_to_f16x2(codes.x, codes.y, &h[0]);
+      e2m3x8_to_f16x2(codes.z, codes.w, &h[4]);
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      r.v[2 * i] = f16_lo(h[i]) * p;
+      r.v[2 * i + 1] = f16_hi(h[i]) * p;
+    }
+    return r;
+  }
+}
+
 // -------------------------------------------------------- scale selection --
 
 template <int FMT>
@@ -415,25 +559,60 @@ struct Elem<kFmtE2M1> {
   static constexpr int emax = 2;          // 6 = 1.5 * 2^2
   static constexpr float maxv = 6.0f;
   static constexpr int ceil_m7 = 64;      // significand above 1.5 overflows 4m <= 6
+  static constexpr int min_log2 = -1;     // smallest magnitude 1/2
 };
 template <>
 struct Elem<kFmtE4M3> {
   static constexpr int emax = 8;          // 448 = 1.75 * 2^8
   static constexpr float maxv = 448.0f;
   static constexpr int ceil_m7 = 96;      // significand above 1.75 overflows 256m <= 448
+  static constexpr int min_log2 = -9;     // smallest magnitude 2^-9
+};
+template <>
+struct Elem<kFmtE5M2> {
+  static constexpr int emax = 15;         // 57344 = 1.75 * 2^15
+  static constexpr float maxv = 57344.0f;
+  static constexpr int ceil_m7 = 96;
+  static constexpr int min_log2 = -16;
+};
+template <>
+struct Elem<kFmtE3M2> {
+  static constexpr int emax = 4;          // 28 = 1.75 * 2^4
+  static constexpr float maxv = 28.0f;
+  static constexpr int ceil_m7 = 96;
+  static constexpr int min_log2 = -4;
+};
+template <>
+struct Elem<kFmtE2M3> {
+  static constexpr int emax = 2;          // 7.5 = 1.875 * 2^2
+  static constexpr float maxv = 7.5f;
+  static constexpr int ceil_m7 = 112;     // significand above 1.875 overflows
+  static constexpr int min_log2 = -3;
+};
+template <>
+struct Elem<kFmtInt8> {
+  static constexpr int emax = 0;          // i * 2^-6, |i| <= 127: 127/64 < 2
+  static constexpr float maxv = 1.984375f;
+  static constexpr int ceil_m7 = 126;     // significand 1 + 127/128 overflows 127/64
+  static constexpr int min_log2 = -6;
 };
 
 // E8M0 byte of a finite block from its amax bits for the rules decided by the
 // amax alone (FLOOR, CEIL, OAS_RULE); OAS starts from FLOOR. A subnormal or
-// zero amax has exponent field 0 and always clamps to byte 0 (E = -127).
+// zero amax has exponent field 0 and always clamps to byte 0 (E = -127); the
+// top clamp (E = 127, byte 254) is reachable only with emax 0 (INT8).
 template <int FMT, int RULE>
 __device__ __forceinline__ int rule_byte(uint32_t amax) {
   const int ex = static_cast<int>(amax >> 7);
+  // a subnormal amax is below 2^-126: E = -127 under every rule (and its
+  // mantissa bits are not a normalised significand, so the tests below would
+  // misread them when emax is 0)
+  if (ex == 0) return 0;
   const int m7 = static_cast<int>(amax & 0x7F);
   int b = ex - Elem<FMT>::emax;
   if (RULE == kCeil) b += (m7 > Elem<FMT>::ceil_m7) ? 1 : 0;
   if (RULE == kOasRule) b += (m7 > 96) ? 1 : 0;
-  return max(b, 0);
+  return min(max(b, 0), 254);
 }
 
 // OAS evaluation of one lane's 16 elements (E2M1, no macro factor): the codes
@@ -467,6 +646,52 @@ __device__ __forceinline__ OasEval oas_eval16(const V16& x, int b1) {
   }
   r.delta = __float2int_rn(acc * 1024.0f);   // an integer below 2^16: exact
   return r;
+}
+
+// OAS evaluation of one lane's 16 elements for a one-byte float format
+// (E4M3, E5M2, E3M2, E2M3): the codes under both candidates, E1 (byte b1) and
+// E2 = E1 + 1, and the exact difference of their squared errors,
+//   delta = sum (d1^2 - d2^2) = sum (D1 - D2)(D1 + D2)   in units of U^2,
+// with s = x 2^-E1, d1 = s - q1, d2 = s - 2 q2 (q the code values) and
+// D = d / U, U = 2^(min_log2 - 9) (in units of the E1 scale). An element that
+// rounds differently under the two candidates has |s| of at least half the
+// smallest magnitude, so s (8 significant bits) and both grid values are
+// multiples of U and D1, D2 are exact integers below 2^41; an element that
+// rounds to the same value gives D1 == D2 whatever its size. The products
+// reach 2^82 for E5M2, so the sum is kept in 128-bit integers.
+struct OasEvalBytes {
+  uint4 c1, c2;
+  __int128 delta;
+};
+template <int FMT>
+__device__ __forceinline__ OasEvalBytes oas_eval_bytes16(const V16& x, int b1) {
+  const V16 s1 = scale_slice(x, b1);
+  const V16 s2 = scale_slice(x, b1 + 1);
+  OasEvalBytes r;
+  r.c1 = enc_bytes_16<FMT>(s1);
+  r.c2 = enc_bytes_16<FMT>(s2);
+  const F16 q1 = dec_bytes_16<FMT>(r.c1, 1.0f);
+  const F16 q2 = dec_bytes_16<FMT>(r.c2, 2.0f);   // E2 values in units of the E1 scale
+  const float unit = pow2f(9 - Elem<FMT>::min_log2);
+  __int128 acc = 0;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const float si = elem(s1, i);
+    const long long D1 = __float2ll_rn((si - q1.v[i]) * unit);
+    const long long D2 = __float2ll_rn((si - q2.v[i]) * unit);
+    acc += static_cast<__int128>(D1 - D2) * static_cast<__int128>(D1 + D2);
+  }
+  r.delta = acc;
+  return r;
+}
+
+// The sum of a 128-bit value over a lane pair.
+__device__ __forceinline__ __int128 pair_sum_i128(__int128 v) {
+  const unsigned long long lo = static_cast<unsigned long long>(v);
+  const long long hi = static_cast<long long>(v >> 64);
+  const unsigned long long olo = __shfl_xor_sync(kFull, lo, 1);
+  const long long ohi = __shfl_xor_sync(kFull, hi, 1);
+  return v + ((static_cast<__int128>(ohi) << 64) | static_cast<__int128>(olo));
 }
 
 // ------------------------------------------------ macro-factor arithmetic --

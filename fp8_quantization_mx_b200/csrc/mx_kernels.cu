@@ -53,8 +53,8 @@ struct BlockScale {
   int byte;          // E8M0 byte (255 for a non-finite block)
   int k;             // macro factor index (0 without MBS)
   bool nonfinite;
-  bool have_codes;   // codes below already hold this lane's E2M1 codes (OAS)
-  uint2 codes;
+  bool have_codes;   // codes below already hold this lane's codes (OAS)
+  uint4 codes;       // E2M1 in .x/.y, one-byte formats in all four words
 };
 
 // Scale decision for the block holding `v`; pa = the block amax bits. Every
@@ -65,10 +65,10 @@ __device__ __forceinline__ BlockScale decide_scale(const V16& v, uint32_t pa, in
   s.nonfinite = pa >= 0x7F80u;
   s.k = k;
   s.have_codes = false;
-  s.codes = make_uint2(0, 0);
+  s.codes = make_uint4(0, 0, 0, 0);
   if (MBS == kMbsNone) {
     s.byte = rule_byte<FMT, RULE>(pa);
-    if (RULE == kOas) {
+    if constexpr (RULE == kOas && FMT == kFmtE2M1) {
       const int b2 = max(static_cast<int>(pa >> 7) - 1, 0);
       // for a max significand <= 1.75 the finer grid is element-wise no worse
       const bool need = !s.nonfinite && (pa & 0x7F) > 96 && b2 != s.byte;
@@ -77,7 +77,23 @@ __device__ __forceinline__ BlockScale decide_scale(const V16& v, uint32_t pa, in
         const int d = e.delta + __shfl_xor_sync(kFull, e.delta, 1);
         const bool up = need && d > 0;
         if (up) s.byte = b2;
-        s.codes = up ? e.c2 : e.c1;   // the codes of the chosen scale
+        const uint2 c = up ? e.c2 : e.c1;   // the codes of the chosen scale
+        s.codes = make_uint4(c.x, c.y, 0, 0);
+        s.have_codes = true;
+      }
+    } else if constexpr (RULE == kOas) {
+      // One-byte float formats: every element within maxv of the finer scale
+      // is no worse there (the coarser grid, doubled, is a subset of the finer
+      // one up to maxv), so only a scaled max above maxv -- the CEIL
+      // threshold on the amax significand -- needs the exact comparison.
+      const int b2 = max(static_cast<int>(pa >> 7) - Elem<FMT>::emax + 1, 0);
+      const bool need = !s.nonfinite && (pa & 0x7F) > Elem<FMT>::ceil_m7 && b2 != s.byte;
+      if (__any_sync(kFull, need)) {
+        const OasEvalBytes e = oas_eval_bytes16<FMT>(v, s.byte);
+        const __int128 d = pair_sum_i128(e.delta);
+        const bool up = need && d > 0;
+        if (up) s.byte = b2;
+        s.codes = up ? e.c2 : e.c1;
         s.have_codes = true;
       }
     }
@@ -93,7 +109,8 @@ __device__ __forceinline__ BlockScale decide_scale(const V16& v, uint32_t pa, in
         const int d = e.delta + __shfl_xor_sync(kFull, e.delta, 1);
         const bool up = need && d > 0;
         if (up) s.byte = b2;
-        s.codes = up ? e.c2 : e.c1;   // the codes of the chosen scale
+        const uint2 c = up ? e.c2 : e.c1;   // the codes of the chosen scale
+        s.codes = make_uint4(c.x, c.y, 0, 0);
         s.have_codes = true;
       }
     }
@@ -106,19 +123,23 @@ __device__ __forceinline__ BlockScale decide_scale(const V16& v, uint32_t pa, in
 template <int MBS>
 __device__ __forceinline__ uint2 codes_fp4(const V16& v, const BlockScale& s) {
   if (s.nonfinite) return nonfinite_e2m1_16(v);
-  if (s.have_codes) return s.codes;
+  if (s.have_codes) return make_uint2(s.codes.x, s.codes.y);
   if (MBS == kMbsNone) return enc_e2m1_16(scale_slice(v, s.byte));
   return enc_mbs_cvt_16(v, s.byte, s.k);
 }
 
-// Codes of one lane's 16 elements: E2M1 in .x/.y, E4M3 in all four words.
+// Codes of one lane's 16 elements: E2M1 in .x/.y, one-byte formats in all
+// four words.
 template <int FMT, int MBS>
 __device__ __forceinline__ uint4 lane_codes(const V16& v, const BlockScale& s) {
-  if (FMT == kFmtE2M1) {
+  if constexpr (FMT == kFmtE2M1) {
     const uint2 c = codes_fp4<MBS>(v, s);
     return make_uint4(c.x, c.y, 0, 0);
+  } else {
+    if (s.nonfinite) return nonfinite_bytes_16<FMT>(v);
+    if (s.have_codes) return s.codes;
+    return enc_bytes_16<FMT>(scale_slice(v, s.byte));
   }
-  return s.nonfinite ? nonfinite_e4m3_16(v) : enc_e4m3_16(scale_slice(v, s.byte));
 }
 
 // Dequantized values (exact floats, signed) of a finite block's 16 elements
@@ -132,7 +153,7 @@ __device__ __forceinline__ F16 block_values(const uint4& codes, const BlockScale
     const float p = MBS == kMbsNone ? pow2f(E) : static_cast<float>(256 + s.k) * pow2f(E - 8);
     return dec_e2m1_16(make_uint2(codes.x, codes.y), p);
   }
-  return dec_e4m3_16(codes, pow2f(E));
+  return dec_bytes_16<FMT>(codes, pow2f(E));
 }
 
 template <int OP, int FMT, int RULE, int MBS>
@@ -227,7 +248,7 @@ __device__ __forceinline__ void process_slice(const StreamArgs& a, const V16& v,
       const F16 g = FMT == kFmtE2M1
                         ? dec_e2m1_16(make_uint2(codes.x, codes.y),
                                       static_cast<float>(256 + s.k) * 0.00390625f)
-                        : dec_e4m3_16(codes, 1.0f);
+                        : dec_bytes_16<FMT>(codes, 1.0f);
 #pragma unroll
       for (int i = 0; i < 16; ++i) {
         const float si = elem(sl, i);
@@ -853,7 +874,9 @@ __global__ void __launch_bounds__(kThreads) dequant_kernel(DequantArgs a) {
       }
       // value * (256 + k) 2^(E-8) (exact); a NaN scale makes every output NaN
       const float p = kk[j] ? static_cast<float>(256 + kk[j]) * pow2f(E - 8) : pow2f(E);
-      const F16 y = FMT == kFmtE2M1 ? dec_e2m1_16(c4[j], p) : dec_e4m3_16(c8[j], p);
+      F16 y;
+      if constexpr (FMT == kFmtE2M1) y = dec_e2m1_16(c4[j], p);
+      else y = dec_bytes_16<FMT>(c8[j], p);
       const bool nan_scale = sb[j] == 255;
       if (OUT32) {
         V16 o0, o1;
@@ -943,13 +966,27 @@ cudaError_t launch_stream(const StreamArgs& a, cudaStream_t st) {
   return cudaGetLastError();
 }
 
+// One-byte formats: FLOOR, CEIL and (float elements) OAS; no macro factor.
+template <int OP, int FMT>
+cudaError_t dispatch_bytes(const StreamArgs& a, int rule, cudaStream_t st) {
+  if (rule == kFloor) return launch_stream<OP, FMT, kFloor, kMbsNone>(a, st);
+  if constexpr (FMT != kFmtInt8) {
+    if (rule == kOas) return launch_stream<OP, FMT, kOas, kMbsNone>(a, st);
+  }
+  return launch_stream<OP, FMT, kCeil, kMbsNone>(a, st);
+}
+
 template <int OP>
 cudaError_t dispatch_stream(const StreamArgs& a, int fmt, int scaling, cudaStream_t st) {
   const int rule = scaling & 0xF;
   const int mbs = scaling >> 4;
-  if (fmt == kFmtE4M3) {
-    if (rule == kFloor) return launch_stream<OP, kFmtE4M3, kFloor, kMbsNone>(a, st);
-    return launch_stream<OP, kFmtE4M3, kCeil, kMbsNone>(a, st);
+  switch (fmt) {
+    case kFmtE4M3: return dispatch_bytes<OP, kFmtE4M3>(a, rule, st);
+    case kFmtE5M2: return dispatch_bytes<OP, kFmtE5M2>(a, rule, st);
+    case kFmtE3M2: return dispatch_bytes<OP, kFmtE3M2>(a, rule, st);
+    case kFmtE2M3: return dispatch_bytes<OP, kFmtE2M3>(a, rule, st);
+    case kFmtInt8: return dispatch_bytes<OP, kFmtInt8>(a, rule, st);
+    default: break;
   }
   if (mbs == kMbsNone) {
     switch (rule) {
@@ -1012,6 +1049,17 @@ cudaError_t launch_block_error(const void* x, int64_t n, int fmt, int scaling, f
   return dispatch_stream<kOpError>(a, fmt, scaling, st);
 }
 
+template <int FMT, int U>
+void launch_dequant_bytes(const DequantArgs& a, int64_t tiles, int out_fp32, cudaStream_t st) {
+  if (out_fp32) {
+    auto k = dequant_kernel<FMT, 1, U>;
+    k<<<grid_for(k, tiles), kThreads, 0, st>>>(a);
+  } else {
+    auto k = dequant_kernel<FMT, 0, U>;
+    k<<<grid_for(k, tiles), kThreads, 0, st>>>(a);
+  }
+}
+
 cudaError_t launch_dequantize(const void* codes, const uint8_t* scales, const uint8_t* macro,
                               int64_t n, int fmt, int out_fp32, void* out, cudaStream_t st) {
   DequantArgs a{};
@@ -1031,12 +1079,12 @@ cudaError_t launch_dequantize(const void* codes, const uint8_t* scales, const ui
       k<<<grid_for(k, tiles), kThreads, 0, st>>>(a);
     }
   } else {
-    if (out_fp32) {
-      auto k = dequant_kernel<kFmtE4M3, 1, U>;
-      k<<<grid_for(k, tiles), kThreads, 0, st>>>(a);
-    } else {
-      auto k = dequant_kernel<kFmtE4M3, 0, U>;
-      k<<<grid_for(k, tiles), kThreads, 0, st>>>(a);
+    switch (fmt) {
+      case kFmtE4M3: launch_dequant_bytes<kFmtE4M3, U>(a, tiles, out_fp32, st); break;
+      case kFmtE5M2: launch_dequant_bytes<kFmtE5M2, U>(a, tiles, out_fp32, st); break;
+      case kFmtE3M2: launch_dequant_bytes<kFmtE3M2, U>(a, tiles, out_fp32, st); break;
+      case kFmtE2M3: launch_dequant_bytes<kFmtE2M3, U>(a, tiles, out_fp32, st); break;
+      default: launch_dequant_bytes<kFmtInt8, U>(a, tiles, out_fp32, st); break;
     }
   }
   return cudaGetLastError();

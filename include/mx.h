@@ -9,18 +9,21 @@
  *  [VL] "[vLLM] MXFP8/MXFP4: microscaling format quantization" [MXFP8: block-32
  *       scaling: contiguous weight -> (fp8 elements, uint8 scales), dynamic
  *       scheme only] [MXFP4: uint8 storage, two FP4 values per byte, last dim
- *       halved] [MX format table: E2M1 / E4M3 elements, E8M0 scale, block 32,
- *       one scale byte per 32 elements].
+ *       halved] [MX format table: E4M3/E5M2, E3M2/E2M3, E2M1 and INT8
+ *       elements, E8M0 scale, block 32, one scale byte per 32 elements].
  *  [UP] "Unveiling the Potential of Quantization with MXFP4: Strategies for
  *       Quantization Error Reduction" [technical summary 1: E8M0 = 2^k only]
- *       [2.A Overflow-Aware Scaling] [2.B Macro Block Scaling] [3-4: QSNR].
+ *       [2.A Overflow-Aware Scaling] [2.B Macro Block Scaling] [3-4: QSNR]
+ *       [5: OAS and MBS generalize to MXFP6 and MXFP8].
  *
  * Layout (every call): x is row-major contiguous [rows, cols] bf16, cols a
  * multiple of 32; block b of row r is elements [32b, 32b+32) of that row.
  * A 3-D tensor [E, R, C] is passed as rows = E*R, cols = C.
  *   codes  MXFP4: uint8 [rows, cols/2], element 2j in the low nibble and 2j+1
  *                 in the high nibble of byte j; bit 3 of a nibble is the sign.
- *          MXFP8: uint8 [rows, cols], one E4M3 ("fn": no Inf, S.1111.111 = NaN).
+ *          other formats: uint8 [rows, cols], one code per element (E4M3,
+ *                 E5M2, INT8: the whole byte; E3M2 / E2M3: the low 6 bits,
+ *                 bit 5 the sign, bits 6-7 zero).
  *   scales uint8 [rows, cols/32], E8M0: byte s means 2^(s-127); 255 is NaN.
  *   macro  uint8 [rows, cols/128] (MBS only): k, the macro factor f = 1 + k/256
  *          of the 128-element macro block [128m, 128m+128) of the row.
@@ -50,30 +53,40 @@
 extern "C" {
 #endif
 
-/* Element formats ([VL] MX format table). */
+/* Element formats ([VL] MX format table: MXFP8 E4M3/E5M2, MXFP6 E3M2/E2M3,
+ * MXFP4 E2M1, MXINT8 INT8; block 32 and an E8M0 scale for all). emax is the
+ * exponent of the largest power of two the element holds. */
 typedef enum {
-  MX_FMT_E2M1 = 0, /* MXFP4: magnitudes {0, .5, 1, 1.5, 2, 3, 4, 6} ([UP] 2.A: max 6.0) */
-  MX_FMT_E4M3 = 1  /* MXFP8: E4M3fn, max 448 */
+  MX_FMT_E2M1 = 0, /* MXFP4: magnitudes {0, .5, 1, 1.5, 2, 3, 4, 6} ([UP] 2.A: max 6.0), emax 2 */
+  MX_FMT_E4M3 = 1, /* MXFP8: E4M3fn (bias 7, no Inf, S.1111.111 = NaN), max 448, emax 8 */
+  MX_FMT_E5M2 = 2, /* MXFP8: E5M2 (bias 15, IEEE Inf/NaN at exponent 31), max 57344, emax 15 */
+  MX_FMT_E3M2 = 3, /* MXFP6: E3M2 (bias 3, no Inf/NaN), max 28, emax 4 */
+  MX_FMT_E2M3 = 4, /* MXFP6: E2M3 (bias 1, no Inf/NaN), max 7.5, emax 2 */
+  MX_FMT_INT8 = 5  /* MXINT8: two's complement i read as i * 2^-6, |i| <= 127, emax 0 */
 } mx_format_t;
 
 /* Scale selection. Low 4 bits: the base rule; bits 4-5: Macro Block Scaling.
- * emax is the exponent of the element's largest value (2 for E2M1, 8 for E4M3)
+ * emax is the exponent of the element's largest power of two (mx_format_t)
  * and e = floor(log2 amax) of the block. Every rule clamps E to [-127, 127];
  * an all-zero block gets E = -127 (byte 0); a block holding NaN or Inf gets
- * byte 255 and element codes that keep only the sign (E4M3: S.1111.111). */
+ * byte 255 and element codes NaN for FP8 (S.1111.111, S.11111.11), only the
+ * sign for FP4 and FP6, and 0 for INT8. */
 typedef enum {
-  /* OCP rule 2^(e - emax): amax lands in [4, 8) (E2M1) or [256, 512) (E4M3);
-   * values above the largest element saturate. FP4 and FP8. */
+  /* OCP rule 2^(e - emax): amax lands in [2^emax, 2^(emax+1)), e.g. [4, 8)
+   * for E2M1 or [256, 512) for E4M3; values above the largest element
+   * saturate. Every format. */
   MX_SCALE_FLOOR = 0,
   /* [UP] 2.A's "existing" scale: the smallest 2^E with amax <= maxv * 2^E
-   * (no element saturates). FP4 and FP8. */
+   * (no element saturates, within the E8M0 range). Every format. */
   MX_SCALE_CEIL = 1,
   /* [UP] 2.A as a rule on the mantissa bits: under the no-overflow scale a
    * block max in (3.0, 3.5] of the 6.0 range is mapped to (6.0, 7.0] instead,
    * i.e. E = e - 2 when the amax significand is at most 1.75, else e - 1. FP4. */
   MX_SCALE_OAS_RULE = 2,
   /* Overflow-Aware Scaling as a per-block minimum-SSE choice between the
-   * FLOOR exponent and FLOOR + 1 (exact comparison; a tie keeps FLOOR). FP4. */
+   * FLOOR exponent and FLOOR + 1 (exact comparison; a tie keeps FLOOR). The
+   * float elements: FP4, and ([UP] 5: OAS generalizes to MXFP6/MXFP8) E4M3,
+   * E5M2, E3M2, E2M3; not INT8. */
   MX_SCALE_OAS = 3,
   /* [UP] 2.B Macro Block Scaling, OR-able with MX_SCALE_FLOOR or MX_SCALE_OAS;
    * FP4 only; cols must be a multiple of 128. Each 128-element macro block
@@ -96,8 +109,8 @@ typedef enum {
 } mx_status_t;
 
 /* Quantize ([VL] MXFP8/MXFP4 sections; [UP] 2.A/2.B for the scaling modes).
- * x: device bf16 [rows, cols]. codes: device, FP4 rows*cols/2 bytes or FP8
- * rows*cols bytes. scales: device uint8 [rows, cols/32]. macro: device uint8
+ * x: device bf16 [rows, cols]. codes: device, FP4 rows*cols/2 bytes, every
+ * other format rows*cols bytes (FP6 codes in the low 6 bits, bits 6-7 zero). scales: device uint8 [rows, cols/32]. macro: device uint8
  * [rows, cols/128] when scaling has an MBS bit (required then), else ignored
  * and may be NULL. Elements: round to nearest, ties to the even code, values
  * past the largest magnitude saturate, the sign is kept (small negatives -> -0). */
@@ -105,9 +118,10 @@ int mx_quantize(const void* x, int64_t rows, int64_t cols, int format, int scali
                 void* codes, uint8_t* scales, uint8_t* macro, void* stream);
 
 /* Dequantize: out = value(code) * f * 2^(scale - 127), f = 1 + k/256 from
- * `macro` (NULL means f = 1). out_fp32 = 0: bf16 (rounded to nearest even;
- * exact for FP4 without MBS); 1: float (exact). A scale byte of 255 or an
- * E4M3 NaN code gives the canonical NaN (0x7FC0 / 0x7FC00000). */
+ * `macro` (NULL means f = 1; FP4 only). out_fp32 = 0: bf16 (rounded to
+ * nearest even; exact for FP4 without MBS); 1: float (exact). A scale byte of
+ * 255 or an FP8 NaN code gives the canonical NaN (0x7FC0 / 0x7FC00000); an
+ * E5M2 Inf code gives +-Inf. */
 int mx_dequantize(const void* codes, const uint8_t* scales, const uint8_t* macro,
                   int64_t rows, int64_t cols, int format, int out_fp32, void* out,
                   void* stream);

@@ -61,9 +61,12 @@ def test_product_does_not_use_the_oracle():
 
 
 @pytest.mark.parametrize("fmt,scaling,status", [
-    (2, 0, UNSUPPORTED), (0, 4, UNSUPPORTED), (0, 0x30, UNSUPPORTED), (0, 0x40, UNSUPPORTED),
-    (1, 2, UNSUPPORTED), (1, 3, UNSUPPORTED), (1, 0x10, UNSUPPORTED), (0, 0x11, UNSUPPORTED),
+    (6, 0, UNSUPPORTED), (0, 4, UNSUPPORTED), (0, 0x30, UNSUPPORTED), (0, 0x40, UNSUPPORTED),
+    (1, 2, UNSUPPORTED), (1, 0x10, UNSUPPORTED), (0, 0x11, UNSUPPORTED),
     (0, 0x12, UNSUPPORTED), (-1, 0, UNSUPPORTED), (0, -1, UNSUPPORTED),
+    # one-byte formats: no OAS_RULE, no macro blocks; INT8 has no OAS
+    (2, 2, UNSUPPORTED), (3, 0x20, UNSUPPORTED), (4, 0x13, UNSUPPORTED), (5, 3, UNSUPPORTED),
+    (5, 2, UNSUPPORTED), (2, 0x10, UNSUPPORTED),
 ])
 def test_quantize_rejects_modes(mx, fmt, scaling, status):
     assert mx.mx_quantize(A, 4, 128, fmt, scaling, A, A, A, 0) == status
@@ -96,11 +99,12 @@ def test_other_entry_points_validate(mx):
     assert mx.mx_dequantize(A, A, A, 4, 96, 0, 0, A, 0) == SHAPE
     assert mx.mx_dequantize(A, A, A, 4, 128, 1, 0, A, 0) == UNSUPPORTED   # FP8 has no MBS
     assert mx.mx_dequantize(A, A, None, 4, 32, 0, 2, A, 0) == INVALID
-    assert mx.mx_dequantize(A, A, None, 4, 32, 3, 0, A, 0) == UNSUPPORTED
+    assert mx.mx_dequantize(A, A, None, 4, 32, 6, 0, A, 0) == UNSUPPORTED
+    assert mx.mx_dequantize(A, A, A, 4, 128, 5, 0, A, 0) == UNSUPPORTED   # only FP4 has MBS
     assert mx.mx_dequantize(A + 8, A, None, 4, 32, 0, 0, A, 0) == ALIGN
     assert mx.mx_dequantize(A, None, None, 4, 32, 0, 0, A, 0) == INVALID
     assert mx.mx_dequantize(None, None, None, 0, 32, 0, 0, None, 0) == OK
-    assert mx.mx_fake_quant_fwd(A, 4, 32, 1, 3, A, None, 0) == UNSUPPORTED
+    assert mx.mx_fake_quant_fwd(A, 4, 32, 5, 3, A, None, 0) == UNSUPPORTED
     assert mx.mx_fake_quant_fwd(A, 4, 48, 0, 0, A, None, 0) == SHAPE
     assert mx.mx_fake_quant_fwd(A, 4, 32, 0, 0, None, None, 0) == INVALID
     assert mx.mx_fake_quant_fwd(A, 4, 32, 0, 0, A + 8, None, 0) == ALIGN

@@ -16,12 +16,16 @@ from fp8_quantization_mx_b200 import inputs
 
 pytestmark = pytest.mark.gpu
 
-E2M1, E4M3 = 0, 1
+E2M1, E4M3, E5M2, E3M2, E2M3, INT8 = 0, 1, 2, 3, 4, 5
 FLOOR, CEIL, OAS_RULE, OAS = 0, 1, 2, 3
 MBS_STATIC, MBS_DYNAMIC = 16, 32
 FP4_MODES = [FLOOR, CEIL, OAS_RULE, OAS, MBS_STATIC, MBS_DYNAMIC, OAS | MBS_STATIC, OAS | MBS_DYNAMIC]
-FP8_MODES = [FLOOR, CEIL]
-ALL = [(E2M1, m) for m in FP4_MODES] + [(E4M3, m) for m in FP8_MODES]
+BYTE_FMTS = [E4M3, E5M2, E3M2, E2M3, INT8]
+BYTE_MODES = {E4M3: [FLOOR, CEIL, OAS], E5M2: [FLOOR, CEIL, OAS], E3M2: [FLOOR, CEIL, OAS],
+              E2M3: [FLOOR, CEIL, OAS], INT8: [FLOOR, CEIL]}
+ALL = [(E2M1, m) for m in FP4_MODES] + [(f, m) for f in BYTE_FMTS for m in BYTE_MODES[f]]
+EMAX = {E2M1: 2, E4M3: 8, E5M2: 15, E3M2: 4, E2M3: 2, INT8: 0}
+FMT_NAMES = {E2M1: "fp4", E4M3: "e4m3", E5M2: "e5m2", E3M2: "e3m2", E2M3: "e2m3", INT8: "int8"}
 REL = 1e-6
 
 
@@ -31,7 +35,7 @@ def ids(fm):
     s = names[m & 15]
     if m >> 4:
         s += "+MBS_" + ("STATIC" if m >> 4 == 1 else "DYNAMIC")
-    return ("fp4-" if fmt == 0 else "fp8-") + s
+    return FMT_NAMES[fmt] + "-" + s
 
 
 def bits(t):
@@ -222,7 +226,7 @@ def test_every_scaled_value_at_several_exponents(mx, oracle_mod, cuda):
     arr = np.concatenate(rows)
     arr = np.concatenate([arr, np.zeros(((-len(arr)) % 64, 32), np.uint16)]).reshape(-1, 2048)
     x = torch.from_numpy(arr.view(np.int16)).view(torch.bfloat16)
-    for fmt in (E2M1, E4M3):
+    for fmt in [E2M1] + BYTE_FMTS:
         c, s, _ = mx.quantize(x.to(cuda), fmt, FLOOR)
         y = mx.fake_quant(x.to(cuda), fmt, FLOOR)
         torch.cuda.synchronize()
@@ -232,12 +236,12 @@ def test_every_scaled_value_at_several_exponents(mx, oracle_mod, cuda):
         assert np.array_equal(bits(y), oracle_mod.fake_quant_fwd(arr, fmt, FLOOR))
 
 
-@pytest.mark.parametrize("fmt", [E2M1, E4M3])
+@pytest.mark.parametrize("fmt", [E2M1] + BYTE_FMTS)
 @pytest.mark.parametrize("out_fp32", [0, 1])
 @pytest.mark.parametrize("with_macro", [False, True])
 def test_dequantize_every_code_and_scale(mx, oracle_mod, cuda, fmt, out_fp32, with_macro):
-    if fmt == E4M3 and with_macro:
-        pytest.skip("no MBS for E4M3")
+    if fmt != E2M1 and with_macro:
+        pytest.skip("macro factors are FP4 only")
     rng = np.random.default_rng(23)
     rows, cols = 256, 512
     scales = np.tile(np.arange(256, dtype=np.uint8)[:, None], (1, cols // 32))
@@ -248,6 +252,8 @@ def test_dequantize_every_code_and_scale(mx, oracle_mod, cuda, fmt, out_fp32, wi
     else:
         codes = rng.integers(0, 256, (rows, cols), dtype=np.uint8)
         codes[0, :256] = np.arange(256, dtype=np.uint8)
+        if fmt in (E3M2, E2M3):
+            codes &= 0x3F          # an FP6 code occupies the low 6 bits of its byte
     macro = rng.integers(0, 256, (rows, cols // 128), dtype=np.uint8) if with_macro else None
     tdev = lambda a: None if a is None else torch.from_numpy(a).to(cuda)
     out = mx.dequantize(tdev(codes), tdev(scales), tdev(macro), fmt,
@@ -282,18 +288,19 @@ def sample_rows(n_rows, k, seed):
     return np.unique(r)
 
 
-def test_full_mlp_weight_fp8(mx, oracle_mod, cuda):
+@pytest.mark.parametrize("fmt", BYTE_FMTS, ids=lambda f: FMT_NAMES[f])
+def test_full_mlp_weight_bytes(mx, oracle_mod, cuda, fmt):
     x = inputs.mlp_weight(device=cuda)
-    c, s, _ = mx.quantize(x, E4M3, FLOOR)
+    c, s, _ = mx.quantize(x, fmt, FLOOR)
     torch.cuda.synchronize()
     r = sample_rows(x.shape[0], 48, 1)
     xs = bits(x[r])
-    oc, os_, _ = oracle_mod.quantize(xs, E4M3, FLOOR)
+    oc, os_, _ = oracle_mod.quantize(xs, fmt, FLOOR)
     assert np.array_equal(host_u8(c[r]), oc)
     assert np.array_equal(host_u8(s[r]), os_)
     # property over every block: the FLOOR byte from the block amax exponent
     amax = x.view(-1, 32).abs().amax(dim=1).view(torch.int16).to(torch.int32)
-    want = torch.clamp((amax >> 7) - 8, min=0).to(torch.uint8)
+    want = torch.clamp((amax >> 7) - EMAX[fmt], min=0).to(torch.uint8)
     assert torch.equal(s.view(-1), want)
 
 
@@ -353,7 +360,8 @@ def test_full_heavy_tail_modes(mx, oracle_mod, cuda, m):
 def test_guard_bands(mx, cuda):
     """Outputs never write outside their extent (canary bytes on both sides)."""
     x = inputs.random_bf16_bits((3, 384), seed=11).to(cuda)
-    for fmt, m in ((E2M1, FLOOR), (E2M1, OAS | MBS_DYNAMIC), (E4M3, CEIL)):
+    for fmt, m in ((E2M1, FLOOR), (E2M1, OAS | MBS_DYNAMIC), (E4M3, CEIL), (E5M2, OAS),
+                   (E2M3, OAS), (INT8, FLOOR)):
         ncode = 3 * 384 // (2 if fmt == E2M1 else 1)
         pad = 256
         cbuf = torch.full((ncode + 2 * pad,), 0xA5, dtype=torch.uint8, device=cuda)
