@@ -552,6 +552,13 @@ __device__ __forceinline__ F16 dec_bytes_16(uint4 codes, float p) {
 
 // -------------------------------------------------------- scale selection --
 
+// oas_m7: OAS can prefer the coarser exponent E1 + 1 only when the block max,
+// scaled by 2^-E1, exceeds the midpoint between maxv and the first value of
+// the coarser grid above it, 2 * (the element after maxv / 2): below that
+// every element rounds to a value at least as close on the finer grid
+// (maxv / 2 is an element, so maxv is on both grids, and the coarser grid
+// below maxv is a subset of the finer one). In significand terms: M7 above
+// oas_m7.
 template <int FMT>
 struct Elem;
 template <>
@@ -559,6 +566,7 @@ struct Elem<kFmtE2M1> {
   static constexpr int emax = 2;          // 6 = 1.5 * 2^2
   static constexpr float maxv = 6.0f;
   static constexpr int ceil_m7 = 64;      // significand above 1.5 overflows 4m <= 6
+  static constexpr int oas_m7 = 96;       // OAS band: scaled max above 7 (see below)
   static constexpr int min_log2 = -1;     // smallest magnitude 1/2
 };
 template <>
@@ -566,6 +574,7 @@ struct Elem<kFmtE4M3> {
   static constexpr int emax = 8;          // 448 = 1.75 * 2^8
   static constexpr float maxv = 448.0f;
   static constexpr int ceil_m7 = 96;      // significand above 1.75 overflows 256m <= 448
+  static constexpr int oas_m7 = 104;      // scaled max above 464
   static constexpr int min_log2 = -9;     // smallest magnitude 2^-9
 };
 template <>
@@ -573,6 +582,7 @@ struct Elem<kFmtE5M2> {
   static constexpr int emax = 15;         // 57344 = 1.75 * 2^15
   static constexpr float maxv = 57344.0f;
   static constexpr int ceil_m7 = 96;
+  static constexpr int oas_m7 = 112;      // scaled max above 61440
   static constexpr int min_log2 = -16;
 };
 template <>
@@ -580,6 +590,7 @@ struct Elem<kFmtE3M2> {
   static constexpr int emax = 4;          // 28 = 1.75 * 2^4
   static constexpr float maxv = 28.0f;
   static constexpr int ceil_m7 = 96;
+  static constexpr int oas_m7 = 112;      // scaled max above 30
   static constexpr int min_log2 = -4;
 };
 template <>
@@ -587,6 +598,7 @@ struct Elem<kFmtE2M3> {
   static constexpr int emax = 2;          // 7.5 = 1.875 * 2^2
   static constexpr float maxv = 7.5f;
   static constexpr int ceil_m7 = 112;     // significand above 1.875 overflows
+  static constexpr int oas_m7 = 120;      // scaled max above 7.75
   static constexpr int min_log2 = -3;
 };
 template <>
@@ -594,6 +606,7 @@ struct Elem<kFmtInt8> {
   static constexpr int emax = 0;          // i * 2^-6, |i| <= 127: 127/64 < 2
   static constexpr float maxv = 1.984375f;
   static constexpr int ceil_m7 = 126;     // significand 1 + 127/128 overflows 127/64
+  static constexpr int oas_m7 = 127;      // (no OAS for INT8)
   static constexpr int min_log2 = -6;
 };
 

@@ -82,12 +82,10 @@ __device__ __forceinline__ BlockScale decide_scale(const V16& v, uint32_t pa, in
         s.have_codes = true;
       }
     } else if constexpr (RULE == kOas) {
-      // One-byte float formats: every element within maxv of the finer scale
-      // is no worse there (the coarser grid, doubled, is a subset of the finer
-      // one up to maxv), so only a scaled max above maxv -- the CEIL
-      // threshold on the amax significand -- needs the exact comparison.
+      // One-byte float formats: only a block max past the band (oas_m7) can
+      // prefer the coarser scale.
       const int b2 = max(static_cast<int>(pa >> 7) - Elem<FMT>::emax + 1, 0);
-      const bool need = !s.nonfinite && (pa & 0x7F) > Elem<FMT>::ceil_m7 && b2 != s.byte;
+      const bool need = !s.nonfinite && (pa & 0x7F) > Elem<FMT>::oas_m7 && b2 != s.byte;
       if (__any_sync(kFull, need)) {
         const OasEvalBytes e = oas_eval_bytes16<FMT>(v, s.byte);
         const __int128 d = pair_sum_i128(e.delta);
@@ -356,16 +354,17 @@ __global__ void __launch_bounds__(kThreads) stream_kernel(StreamArgs a) {
 
 // ------------------------------------------------------ OAS quantize path --
 
-// MXFP4 OAS quantize (without MBS, or with MBS-Static) in two phases per CTA
-// tile. Phase 1 handles every block whose finer exponent is already the
-// answer (scaled max <= 7, the two candidates equal, or NaN/Inf) exactly as
-// the single-rule kernel does, and appends the other blocks (about a fifth of
-// them for Gaussian data) to a shared-memory list, with their macro factor.
-// Phase 2 evaluates only the listed blocks, two lanes per block and full
-// warps, re-reading their 64 bytes (just loaded, so from L2). Without the
-// split every warp that holds one such block pays for the exact SSE
-// comparison on all of its lanes.
-template <int MBS, int U>
+// OAS quantize in two phases per CTA tile: MXFP4 without MBS or with
+// MBS-Static, and the one-byte float formats. Phase 1 handles every block
+// whose finer exponent is already the answer (scaled max inside the band of
+// Elem<FMT>::oas_m7 -- under MBS: at most 7f --, the two candidates equal, or
+// NaN/Inf) exactly as the single-rule kernel does, and appends the other
+// blocks (a fifth or fewer for Gaussian data) to a shared-memory list, with
+// their macro factor. Phase 2 evaluates only the listed blocks, two lanes per
+// block and full warps, re-reading their 64 bytes (just loaded, so from L2).
+// Without the split every warp that holds one such block pays for the exact
+// SSE comparison on all of its lanes.
+template <int FMT, int MBS, int U>
 __global__ void __launch_bounds__(kThreads) oas_quant_kernel(StreamArgs a) {
   constexpr int kWarps = kThreads / 32;
   constexpr int kTileSlices = kWarps * 32 * U;
@@ -396,9 +395,9 @@ __global__ void __launch_bounds__(kThreads) oas_quant_kernel(StreamArgs a) {
     int k = 0, b1, b2;
     bool band;
     if (MBS == kMbsNone) {
-      b1 = rule_byte<kFmtE2M1, kFloor>(pa);
-      b2 = max(static_cast<int>(pa >> 7) - 1, 0);
-      band = (pa & 0x7F) > 96;
+      b1 = rule_byte<FMT, kFloor>(pa);
+      b2 = max(static_cast<int>(pa >> 7) - Elem<FMT>::emax + 1, 0);
+      band = (pa & 0x7F) > Elem<FMT>::oas_m7;
     } else {
       k = mbs_static_k(oct_max(pa));
       b1 = mbs_byte(pa, k, 0);
@@ -407,11 +406,16 @@ __global__ void __launch_bounds__(kThreads) oas_quant_kernel(StreamArgs a) {
     }
     const bool need = valid && !nonfinite && band && b2 != b1;
     if (valid && !need) {
-      uint2 codes;
-      if (nonfinite) codes = nonfinite_e2m1_16(v[j]);
-      else if (MBS == kMbsNone) codes = enc_e2m1_16(scale_slice(v[j], b1));
-      else codes = enc_mbs_cvt_16(v[j], b1, k);
-      st_stream8(a.codes + 8 * c, codes);
+      if constexpr (FMT == kFmtE2M1) {
+        uint2 codes;
+        if (nonfinite) codes = nonfinite_e2m1_16(v[j]);
+        else if (MBS == kMbsNone) codes = enc_e2m1_16(scale_slice(v[j], b1));
+        else codes = enc_mbs_cvt_16(v[j], b1, k);
+        st_stream8(a.codes + 8 * c, codes);
+      } else {
+        st_stream16(a.codes + 16 * c, nonfinite ? nonfinite_bytes_16<FMT>(v[j])
+                                                : enc_bytes_16<FMT>(scale_slice(v[j], b1)));
+      }
       if ((lane & 1) == 0) a.scales[c >> 1] = static_cast<uint8_t>(nonfinite ? 255 : b1);
     }
     if (MBS != kMbsNone && valid && (lane & 7) == 0) a.macro[c >> 3] = static_cast<uint8_t>(k);
@@ -433,13 +437,18 @@ __global__ void __launch_bounds__(kThreads) oas_quant_kernel(StreamArgs a) {
     for (int i = 0; i < 8; ++i) x.w[i] = 0;
     if (has) x = ld_stream32(a.x + 32 * c);
     const uint32_t pa = pair_max(amax_bits16(x));
-    const int b1 = MBS == kMbsNone ? rule_byte<kFmtE2M1, kFloor>(pa) : mbs_byte(pa, k, 0);
-    const OasEval e = MBS == kMbsNone ? oas_eval16(x, b1) : oas_eval_mbs16(x, b1, k);
-    const int d = e.delta + __shfl_xor_sync(kFull, e.delta, 1);
-    const bool up = d > 0;
-    if (has) {
-      st_stream8(a.codes + 8 * c, up ? e.c2 : e.c1);
-      if ((lane & 1) == 0) a.scales[c >> 1] = static_cast<uint8_t>(up ? b1 + 1 : b1);
+    const int b1 = MBS == kMbsNone ? rule_byte<FMT, kFloor>(pa) : mbs_byte(pa, k, 0);
+    if constexpr (FMT == kFmtE2M1) {
+      const OasEval e = MBS == kMbsNone ? oas_eval16(x, b1) : oas_eval_mbs16(x, b1, k);
+      const int d = e.delta + __shfl_xor_sync(kFull, e.delta, 1);
+      const bool up = d > 0;
+      if (has) st_stream8(a.codes + 8 * c, up ? e.c2 : e.c1);
+      if (has && (lane & 1) == 0) a.scales[c >> 1] = static_cast<uint8_t>(up ? b1 + 1 : b1);
+    } else {
+      const OasEvalBytes e = oas_eval_bytes16<FMT>(x, b1);
+      const bool up = pair_sum_i128(e.delta) > 0;
+      if (has) st_stream16(a.codes + 16 * c, up ? e.c2 : e.c1);
+      if (has && (lane & 1) == 0) a.scales[c >> 1] = static_cast<uint8_t>(up ? b1 + 1 : b1);
     }
   }
 }
@@ -953,10 +962,10 @@ cudaError_t launch_stream(const StreamArgs& a, cudaStream_t st) {
       if (grid > cap) grid = cap;
     }
     kern<<<static_cast<int>(grid > 0 ? grid : 1), kSweepThreads, 0, st>>>(a);
-  } else if constexpr (OP == kOpQuant && FMT == kFmtE2M1 && RULE == kOas) {
+  } else if constexpr (OP == kOpQuant && RULE == kOas) {
     constexpr int kTile = (kThreads / 32) * 32 * kUnroll;   // slices per CTA
     const int64_t grid = (a.nslices + kTile - 1) / kTile;
-    oas_quant_kernel<MBS, kUnroll><<<static_cast<int>(grid), kThreads, 0, st>>>(a);
+    oas_quant_kernel<FMT, MBS, kUnroll><<<static_cast<int>(grid), kThreads, 0, st>>>(a);
   } else {
     constexpr int U = (MBS == kMbsNone) ? kUnroll : 1;
     auto kern = stream_kernel<OP, FMT, RULE, MBS, U>;

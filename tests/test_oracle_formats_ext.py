@@ -232,3 +232,32 @@ def test_nonfinite_block_codes(oracle_mod):
         c, s, _ = oracle_mod.quantize(b, fmt, FLOOR)
         assert int(s[0, 0]) == 255
         assert int(c[0, 1]) == neg
+
+
+# The OAS comparison is only needed above the midpoint between maxv and the
+# first coarser-grid value past it, 2 * (the element after maxv / 2): below
+# that every element's error on the finer grid is no larger. The kernels skip
+# the comparison there; the oracle never does, so this pins the shortcut.
+OAS_MID = {E4M3: (448 + 480) / 2, E5M2: (57344 + 65536) / 2, E3M2: (28 + 32) / 2,
+           E2M3: (7.5 + 8) / 2}
+
+
+@pytest.mark.parametrize("fmt", [E4M3, E5M2, E3M2, E2M3])
+def test_oas_keeps_floor_below_the_band(oracle_mod, fmt):
+    rng = np.random.default_rng(90 + fmt)
+    n = 4000
+    x = rng.standard_normal((n, 32)) * 2.0 ** rng.integers(-20, 20, (n, 1))
+    # put many block maxima just below and just above the band edge
+    e = np.floor(np.log2(np.abs(x).max(axis=1)))
+    edge = OAS_MID[fmt] / 2.0 ** EMAX[fmt]          # significand at the band edge
+    m = edge + rng.choice([-1, 1], n) * rng.random(n) * (2 - edge)
+    x[:, 0] = m * 2.0 ** e
+    bits = _to_bf16_bits(x)
+    xf = _bits_to_f64(bits)
+    _, s_f, _ = oracle_mod.quantize(bits, fmt, FLOOR)
+    _, s_o, _ = oracle_mod.quantize(bits, fmt, OAS)
+    amax = np.abs(xf).max(axis=1)
+    scaled = amax / 2.0 ** (s_f[:, 0].astype(np.float64) - 127)
+    below = scaled <= OAS_MID[fmt]
+    assert np.array_equal(s_o[below, 0], s_f[below, 0])
+    assert (s_o[~below, 0] != s_f[~below, 0]).any()   # above the edge the coarser scale does win
