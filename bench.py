@@ -246,6 +246,7 @@ def stack_ops(mx, x, reps=50, only=None):
     c8 = torch.empty(rows, cols, dtype=torch.uint8, device=dev)
     sc = torch.empty(rows, cols // 32, dtype=torch.uint8, device=dev)
     mac = torch.empty(rows, cols // 128, dtype=torch.uint8, device=dev)
+    sc_mma = torch.empty(mx.mx_scale_bytes(rows, cols, mx.MMA_SCALES), dtype=torch.uint8, device=dev)
     y = torch.empty_like(x)
     g = torch.empty_like(x).normal_()
     fp4, fp8, fp4m = n * 2.53125, n * 3.03125, n * (2.53125 + 1 / 128)
@@ -261,6 +262,8 @@ def stack_ops(mx, x, reps=50, only=None):
         "fp4_dequantize_bf16": (lambda: mx.dequantize(c4, sc, None, mx.E2M1, out=y), fp4),
         "fp8_dequantize_bf16": (lambda: mx.dequantize(c8, sc, None, mx.E4M3, out=y), fp8),
         "fp4_block_error": (lambda: mx.block_error(x, per_block=False), n * 2),
+        "fp4_floor_quantize_mma_scales": (lambda: mx.quantize(x, mx.E2M1, mx.FLOOR | mx.MMA_SCALES,
+                                                              out=(c4, sc_mma, None)), fp4),
         "e5m2_floor_quantize": (lambda: mx.quantize(x, mx.E5M2, mx.FLOOR, out=(c8, sc, None)), fp8),
         "e3m2_floor_quantize": (lambda: mx.quantize(x, mx.E3M2, mx.FLOOR, out=(c8, sc, None)), fp8),
         "e2m3_floor_quantize": (lambda: mx.quantize(x, mx.E2M3, mx.FLOOR, out=(c8, sc, None)), fp8),
@@ -299,7 +302,7 @@ def stack_ops(mx, x, reps=50, only=None):
         e.synchronize()
         ms = s.elapsed_time(e) / n_reps
         res[name] = {"ms": round(ms, 4), "GB/s": round(nbytes / ms / 1e6, 1)}
-    del c4, c8, sc, mac, y, g
+    del c4, c8, sc, mac, sc_mma, y, g
     return res
 
 

@@ -34,7 +34,7 @@ __all__ = [
     "E2M1", "E4M3", "E5M2", "E3M2", "E2M3", "INT8", "FLOOR", "CEIL", "OAS_RULE", "OAS", "MBS_STATIC", "MBS_DYNAMIC",
     "MXError", "library_path", "load_library",
     "mx_quantize", "mx_dequantize", "mx_fake_quant_fwd", "mx_fake_quant_bwd",
-    "mx_block_error", "mx_status_string", "mx_version",
+    "mx_block_error", "mx_status_string", "mx_version", "mx_scale_bytes", "MMA_SCALES",
     "quantize", "dequantize", "fake_quant", "fake_quant_bwd", "block_error", "MXFakeQuantize",
     "MXFP4_FORMAT", "MXFP8_FORMAT",
 ]
@@ -46,6 +46,9 @@ E5M2 = 2   # MXFP8
 E3M2 = 3   # MXFP6 (one code per byte, low 6 bits)
 E2M3 = 4   # MXFP6
 INT8 = 5   # MXINT8 (i * 2^-6)
+# OR into `scaling`: scale bytes in the tiled layout of block-scaled tensor-core
+# GEMMs (a flat uint8 buffer of mx_scale_bytes(rows, cols, scaling) bytes)
+MMA_SCALES = 1 << 8
 MXFP4_FORMAT = E2M1
 MXFP8_FORMAT = E4M3
 # scaling (mx_scaling_t)
@@ -90,6 +93,8 @@ def load_library():
     lib.mx_status_string.argtypes = [c_int]
     lib.mx_status_string.restype = ctypes.c_char_p
     lib.mx_version.restype = c_int
+    lib.mx_scale_bytes.argtypes = [i64, i64, c_int]
+    lib.mx_scale_bytes.restype = i64
     _lib = lib
     return lib
 
@@ -123,6 +128,10 @@ def mx_status_string(status: int) -> str:
 
 def mx_version() -> int:
     return load_library().mx_version()
+
+
+def mx_scale_bytes(rows, cols, scaling) -> int:
+    return load_library().mx_scale_bytes(rows, cols, scaling)
 
 
 # ----------------------------------------------------------- tensor layer --
@@ -181,11 +190,11 @@ def quantize(x: torch.Tensor, format: int = E2M1, scaling: int = FLOOR, out=None
     _cuda_bf16(x, "x")
     rows, cols = _rows_cols(x)
     lead = x.shape[:-1]
-    mbs = (scaling >> 4) != 0
+    mbs = ((scaling >> 4) & 3) != 0
     if out is None:
         ccols = cols // 2 if format == E2M1 else cols
         codes = torch.empty(*lead, ccols, dtype=torch.uint8, device=x.device)
-        scales = torch.empty(*lead, cols // 32, dtype=torch.uint8, device=x.device)
+        scales = _scales_buffer(lead, rows, cols, scaling, x.device)
         macro = torch.empty(*lead, cols // 128, dtype=torch.uint8, device=x.device) if mbs else None
     else:
         codes, scales, macro = out
@@ -203,14 +212,21 @@ def _to_host(t: torch.Tensor, pinned: bool) -> torch.Tensor:
     return t.cpu()
 
 
+def _scales_buffer(lead, rows, cols, scaling, device):
+    if scaling & MMA_SCALES:
+        return torch.empty(mx_scale_bytes(rows, cols, scaling), dtype=torch.uint8, device=device)
+    return torch.empty(*lead, cols // 32, dtype=torch.uint8, device=device)
+
+
 def dequantize(codes: torch.Tensor, scales: torch.Tensor, macro=None, format: int = E2M1,
-               out_dtype=torch.bfloat16, out=None):
-    """Inverse of ``quantize``: value(code) * f * 2^(scale - 127) as bf16 or fp32."""
+               out_dtype=torch.bfloat16, out=None, mma_scales: bool = False):
+    """Inverse of ``quantize``: value(code) * f * 2^(scale - 127) as bf16 or fp32.
+    ``mma_scales``: ``scales`` is in the MMA_SCALES layout."""
     if not codes.is_cuda:
         dev = torch.device("cuda", torch.cuda.current_device())
         pinned = codes.is_pinned()
         args = [None if t is None else t.to(dev, non_blocking=pinned) for t in (codes, scales, macro)]
-        res = dequantize(*args, format=format, out_dtype=out_dtype)
+        res = dequantize(*args, format=format, out_dtype=out_dtype, mma_scales=mma_scales)
         if out is None:
             return _to_host(res, pinned)
         out.copy_(res, non_blocking=out.is_pinned())
@@ -224,8 +240,9 @@ def dequantize(codes: torch.Tensor, scales: torch.Tensor, macro=None, format: in
     if out is None:
         out = torch.empty(*codes.shape[:-1], cols, dtype=out_dtype, device=codes.device)
     with torch.cuda.device(codes.device):
+        flags = int(out_dtype == torch.float32) | (MMA_SCALES if mma_scales else 0)
         _check(mx_dequantize(_ptr(codes), _ptr(scales), _ptr(macro), rows, cols, format,
-                             int(out_dtype == torch.float32), _ptr(out), _stream(codes.device)),
+                             flags, _ptr(out), _stream(codes.device)),
                "mx_dequantize")
     return out
 
@@ -236,8 +253,7 @@ def fake_quant(x: torch.Tensor, format: int = E2M1, scaling: int = FLOOR, out=No
     _cuda_bf16(x, "x")
     rows, cols = _rows_cols(x)
     y = torch.empty_like(x) if out is None else out
-    scales = (torch.empty(*x.shape[:-1], cols // 32, dtype=torch.uint8, device=x.device)
-              if return_scales else None)
+    scales = _scales_buffer(x.shape[:-1], rows, cols, scaling, x.device) if return_scales else None
     with torch.cuda.device(x.device):
         _check(mx_fake_quant_fwd(_ptr(x), rows, cols, format, scaling, _ptr(y), _ptr(scales),
                                  _stream(x.device)), "mx_fake_quant_fwd")

@@ -49,6 +49,32 @@ int check_mode(int format, int scaling) {
 
 int from_cuda(cudaError_t e) { return e == cudaSuccess ? MX_OK : MX_ERR_CUDA; }
 
+// The scale map of a call; flags holds MX_SCALES_MMA or not.
+mxk::ScaleMap scale_map(int64_t cols, int flags) {
+  mxk::ScaleMap m{0, 0, 0.0};
+  if (flags & MX_SCALES_MMA) {
+    m.bpr = cols / 32;
+    m.nct = (m.bpr + 3) / 4;
+    m.inv = 1.0 / static_cast<double>(m.bpr);
+  }
+  return m;
+}
+
+int64_t scale_bytes(int64_t rows, int64_t cols, int flags) {
+  if (!(flags & MX_SCALES_MMA)) return rows * (cols / 32);
+  return (rows + 127) / 128 * 128 * ((cols / 32 + 3) / 4 * 4);
+}
+
+// The tiled layout pads rows to 128 and block columns to 4; the padding must
+// read as zero bytes, so it is cleared on the stream before the kernel writes
+// the real scales.
+cudaError_t clear_padding(uint8_t* scales, int64_t rows, int64_t cols, int flags,
+                          cudaStream_t st) {
+  if (!(flags & MX_SCALES_MMA) || !scales) return cudaSuccess;
+  if (rows % 128 == 0 && (cols / 32) % 4 == 0) return cudaSuccess;
+  return cudaMemsetAsync(scales, 0, static_cast<size_t>(scale_bytes(rows, cols, flags)), st);
+}
+
 }  // namespace
 
 extern "C" {
@@ -67,8 +93,16 @@ const char* mx_status_string(int status) {
   }
 }
 
+int64_t mx_scale_bytes(int64_t rows, int64_t cols, int scaling) {
+  if (rows < 0 || cols < 0 || cols % 32 != 0) return -1;
+  if (rows > 0 && cols > 0 && rows > kMaxElems / cols) return -1;
+  return scale_bytes(rows, cols, scaling & MX_SCALES_MMA);
+}
+
 int mx_quantize(const void* x, int64_t rows, int64_t cols, int format, int scaling, void* codes,
                 uint8_t* scales, uint8_t* macro, void* stream) {
+  const int layout = scaling & MX_SCALES_MMA;
+  scaling &= ~MX_SCALES_MMA;
   int st = check_mode(format, scaling);
   if (st != MX_OK) return st;
   const bool mbs = (scaling >> 4) != 0;
@@ -78,15 +112,19 @@ int mx_quantize(const void* x, int64_t rows, int64_t cols, int format, int scali
   if (n == 0) return MX_OK;
   if (!x || !codes || !scales || (mbs && !macro)) return MX_ERR_INVALID_ARG;
   if (!aligned(x, 32) || !aligned(codes, 16)) return MX_ERR_ALIGN;
+  const auto cs = static_cast<cudaStream_t>(stream);
+  if (clear_padding(scales, rows, cols, layout, cs) != cudaSuccess) return MX_ERR_CUDA;
   return from_cuda(mxk::launch_quantize(x, n, format, scaling, codes, scales, mbs ? macro : nullptr,
-                                        static_cast<cudaStream_t>(stream)));
+                                        scale_map(cols, layout), cs));
 }
 
 int mx_dequantize(const void* codes, const uint8_t* scales, const uint8_t* macro, int64_t rows,
                   int64_t cols, int format, int out_fp32, void* out, void* stream) {
   if (!known_format(format)) return MX_ERR_UNSUPPORTED;
   if (format != MX_FMT_E2M1 && macro) return MX_ERR_UNSUPPORTED;
-  if (out_fp32 != 0 && out_fp32 != 1) return MX_ERR_INVALID_ARG;
+  if ((out_fp32 & ~(1 | MX_SCALES_MMA)) != 0) return MX_ERR_INVALID_ARG;
+  const int layout = out_fp32 & MX_SCALES_MMA;
+  out_fp32 &= 1;
   int st = check_shape(rows, cols, macro != nullptr);
   if (st != MX_OK) return st;
   const int64_t n = rows * cols;
@@ -94,11 +132,14 @@ int mx_dequantize(const void* codes, const uint8_t* scales, const uint8_t* macro
   if (!codes || !scales || !out) return MX_ERR_INVALID_ARG;
   if (!aligned(codes, 16) || !aligned(out, 32)) return MX_ERR_ALIGN;
   return from_cuda(mxk::launch_dequantize(codes, scales, macro, n, format, out_fp32, out,
+                                          scale_map(cols, layout),
                                           static_cast<cudaStream_t>(stream)));
 }
 
 int mx_fake_quant_fwd(const void* x, int64_t rows, int64_t cols, int format, int scaling, void* y,
                       uint8_t* scales_out, void* stream) {
+  const int layout = scaling & MX_SCALES_MMA;
+  scaling &= ~MX_SCALES_MMA;
   int st = check_mode(format, scaling);
   if (st != MX_OK) return st;
   st = check_shape(rows, cols, (scaling >> 4) != 0);
@@ -107,8 +148,10 @@ int mx_fake_quant_fwd(const void* x, int64_t rows, int64_t cols, int format, int
   if (n == 0) return MX_OK;
   if (!x || !y) return MX_ERR_INVALID_ARG;
   if (!aligned(x, 32) || !aligned(y, 32)) return MX_ERR_ALIGN;
+  const auto cs = static_cast<cudaStream_t>(stream);
+  if (clear_padding(scales_out, rows, cols, layout, cs) != cudaSuccess) return MX_ERR_CUDA;
   return from_cuda(mxk::launch_fake_fwd(x, n, format, scaling, y, scales_out,
-                                        static_cast<cudaStream_t>(stream)));
+                                        scale_map(cols, layout), cs));
 }
 
 int mx_fake_quant_bwd(const void* x, const void* grad_y, int64_t rows, int64_t cols, int format,

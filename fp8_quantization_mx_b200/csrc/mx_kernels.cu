@@ -33,7 +33,26 @@ struct StreamArgs {
   uint8_t* out;       // bf16 y (forward) or grad_x (backward), 32 bytes per slice
   float* block_sse;   // one float per block (error)
   double* totals;     // {sum d^2, sum x^2} (error)
+  ScaleMap smap;      // where each block's scale byte goes
 };
+
+// Byte offset of block b's scale under the map (see ScaleMap). The row index
+// r = b / bpr comes from the rounded reciprocal: b < 2^35 and both roundings
+// are relative 2^-53, so the estimate is off by at most one, which the
+// remainder test corrects.
+__device__ __forceinline__ int64_t scale_offset(const ScaleMap& m, int64_t b) {
+  if (m.bpr == 0) return b;
+  int64_t r = __double2ll_rz(static_cast<double>(b) * m.inv);
+  int64_t j = b - r * m.bpr;
+  if (j < 0) {
+    --r;
+    j += m.bpr;
+  } else if (j >= m.bpr) {
+    ++r;
+    j -= m.bpr;
+  }
+  return ((r >> 7) * m.nct + (j >> 2)) * 512 + (r & 31) * 16 + ((r >> 5) & 3) * 4 + (j & 3);
+}
 
 constexpr int kOpQuant = 0, kOpFakeFwd = 1, kOpFakeBwd = 2, kOpError = 3;
 
@@ -169,7 +188,7 @@ __device__ __forceinline__ void process_slice(const StreamArgs& a, const V16& v,
     } else {
       if (valid) st_stream16(a.codes + 16 * c, codes);
     }
-    if (valid && (lane & 1) == 0) a.scales[c >> 1] = static_cast<uint8_t>(s.byte);
+    if (valid && (lane & 1) == 0) a.scales[scale_offset(a.smap, c >> 1)] = static_cast<uint8_t>(s.byte);
     if (MBS != kMbsNone && valid && (lane & 7) == 0) a.macro[c >> 3] = static_cast<uint8_t>(s.k);
     return;
   }
@@ -188,7 +207,7 @@ __device__ __forceinline__ void process_slice(const StreamArgs& a, const V16& v,
       for (int i = 0; i < 8; ++i) o.w[i] = pack_bf16x2(y.v[2 * i], y.v[2 * i + 1]);
     }
     if (valid) st_stream32(a.out + 32 * c, o);
-    if (a.scales && valid && (lane & 1) == 0) a.scales[c >> 1] = static_cast<uint8_t>(s.byte);
+    if (a.scales && valid && (lane & 1) == 0) a.scales[scale_offset(a.smap, c >> 1)] = static_cast<uint8_t>(s.byte);
     return;
   }
 
@@ -416,7 +435,7 @@ __global__ void __launch_bounds__(kThreads) oas_quant_kernel(StreamArgs a) {
         st_stream16(a.codes + 16 * c, nonfinite ? nonfinite_bytes_16<FMT>(v[j])
                                                 : enc_bytes_16<FMT>(scale_slice(v[j], b1)));
       }
-      if ((lane & 1) == 0) a.scales[c >> 1] = static_cast<uint8_t>(nonfinite ? 255 : b1);
+      if ((lane & 1) == 0) a.scales[scale_offset(a.smap, c >> 1)] = static_cast<uint8_t>(nonfinite ? 255 : b1);
     }
     if (MBS != kMbsNone && valid && (lane & 7) == 0) a.macro[c >> 3] = static_cast<uint8_t>(k);
     if (need && (lane & 1) == 0)
@@ -443,12 +462,12 @@ __global__ void __launch_bounds__(kThreads) oas_quant_kernel(StreamArgs a) {
       const int d = e.delta + __shfl_xor_sync(kFull, e.delta, 1);
       const bool up = d > 0;
       if (has) st_stream8(a.codes + 8 * c, up ? e.c2 : e.c1);
-      if (has && (lane & 1) == 0) a.scales[c >> 1] = static_cast<uint8_t>(up ? b1 + 1 : b1);
+      if (has && (lane & 1) == 0) a.scales[scale_offset(a.smap, c >> 1)] = static_cast<uint8_t>(up ? b1 + 1 : b1);
     } else {
       const OasEvalBytes e = oas_eval_bytes16<FMT>(x, b1);
       const bool up = pair_sum_i128(e.delta) > 0;
       if (has) st_stream16(a.codes + 16 * c, up ? e.c2 : e.c1);
-      if (has && (lane & 1) == 0) a.scales[c >> 1] = static_cast<uint8_t>(up ? b1 + 1 : b1);
+      if (has && (lane & 1) == 0) a.scales[scale_offset(a.smap, c >> 1)] = static_cast<uint8_t>(up ? b1 + 1 : b1);
     }
   }
 }
@@ -835,6 +854,7 @@ struct DequantArgs {
   const uint8_t* macro;   // may be null
   int64_t nslices;
   uint8_t* out;           // bf16 (32 bytes per slice) or float (64 bytes per slice)
+  ScaleMap smap;
 };
 
 template <int FMT, int OUT32, int U>
@@ -853,7 +873,7 @@ __global__ void __launch_bounds__(kThreads) dequant_kernel(DequantArgs a) {
       const bool valid = c < a.nslices;
       if (FMT == kFmtE2M1) c4[j] = valid ? ld_stream8(a.codes + 8 * c) : make_uint2(0, 0);
       else c8[j] = valid ? ld_stream16(a.codes + 16 * c) : make_uint4(0, 0, 0, 0);
-      sb[j] = valid ? a.scales[c >> 1] : 0;
+      sb[j] = valid ? a.scales[scale_offset(a.smap, c >> 1)] : 0;
       kk[j] = (valid && a.macro) ? a.macro[c >> 3] : 0;
     }
 #pragma unroll
@@ -1023,8 +1043,9 @@ StreamArgs stream_args(const void* x, int64_t n) {
 }  // namespace
 
 cudaError_t launch_quantize(const void* x, int64_t n, int fmt, int scaling, void* codes,
-                            uint8_t* scales, uint8_t* macro, cudaStream_t st) {
+                            uint8_t* scales, uint8_t* macro, ScaleMap sm, cudaStream_t st) {
   StreamArgs a = stream_args(x, n);
+  a.smap = sm;
   a.codes = static_cast<uint8_t*>(codes);
   a.scales = scales;
   a.macro = macro;
@@ -1032,8 +1053,9 @@ cudaError_t launch_quantize(const void* x, int64_t n, int fmt, int scaling, void
 }
 
 cudaError_t launch_fake_fwd(const void* x, int64_t n, int fmt, int scaling, void* y,
-                            uint8_t* scales_out, cudaStream_t st) {
+                            uint8_t* scales_out, ScaleMap sm, cudaStream_t st) {
   StreamArgs a = stream_args(x, n);
+  a.smap = sm;
   a.out = static_cast<uint8_t*>(y);
   a.scales = scales_out;
   return dispatch_stream<kOpFakeFwd>(a, fmt, scaling, st);
@@ -1070,8 +1092,10 @@ void launch_dequant_bytes(const DequantArgs& a, int64_t tiles, int out_fp32, cud
 }
 
 cudaError_t launch_dequantize(const void* codes, const uint8_t* scales, const uint8_t* macro,
-                              int64_t n, int fmt, int out_fp32, void* out, cudaStream_t st) {
+                              int64_t n, int fmt, int out_fp32, void* out, ScaleMap sm,
+                              cudaStream_t st) {
   DequantArgs a{};
+  a.smap = sm;
   a.codes = static_cast<const uint8_t*>(codes);
   a.scales = scales;
   a.macro = macro;

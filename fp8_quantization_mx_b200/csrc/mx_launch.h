@@ -7,12 +7,24 @@
 
 namespace mxk {
 
+// Where the E8M0 byte of block b (row-major block index) lives: bpr == 0 is
+// the plain [rows, cols/32] array; otherwise the tiled layout of block-scaled
+// tensor-core operands (128 rows x 4 block columns per 512-byte tile, tiles
+// row-major with nct tiles per tile row, inside a tile the byte
+// (r % 32) * 16 + (r / 32) * 4 + (j % 4)).
+struct ScaleMap {
+  int64_t bpr;   // blocks per row (cols / 32), or 0 for the plain layout
+  int64_t nct;   // tiles per tile row: ceil(bpr / 4)
+  double inv;    // 1 / bpr, rounded (for the row index of a block)
+};
+
 cudaError_t launch_quantize(const void* x, int64_t n, int fmt, int scaling, void* codes,
-                            uint8_t* scales, uint8_t* macro, cudaStream_t st);
+                            uint8_t* scales, uint8_t* macro, ScaleMap sm, cudaStream_t st);
 cudaError_t launch_dequantize(const void* codes, const uint8_t* scales, const uint8_t* macro,
-                              int64_t n, int fmt, int out_fp32, void* out, cudaStream_t st);
+                              int64_t n, int fmt, int out_fp32, void* out, ScaleMap sm,
+                              cudaStream_t st);
 cudaError_t launch_fake_fwd(const void* x, int64_t n, int fmt, int scaling, void* y,
-                            uint8_t* scales_out, cudaStream_t st);
+                            uint8_t* scales_out, ScaleMap sm, cudaStream_t st);
 cudaError_t launch_fake_bwd(const void* x, const void* gy, int64_t n, int fmt, int scaling,
                             void* gx, cudaStream_t st);
 cudaError_t launch_block_error(const void* x, int64_t n, int fmt, int scaling, float* block_sse,

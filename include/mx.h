@@ -96,7 +96,17 @@ typedef enum {
    * at most 6. DYNAMIC: the k in 0..255 with the smallest macro-block SSE
    * (double, summed in element order; a tie keeps the smaller k). */
   MX_MBS_STATIC = 1 << 4,
-  MX_MBS_DYNAMIC = 2 << 4
+  MX_MBS_DYNAMIC = 2 << 4,
+  /* Layout flag, OR-able with any of the above for mx_quantize and
+   * mx_fake_quant_fwd (and in mx_dequantize's flags): the E8M0 bytes are
+   * written (read) in the tiled layout that block-scaled tensor-core GEMMs
+   * on sm_100 consume (the one cuBLASLt's 1-D block-scaling-factor layout
+   * documents) instead of plain [rows, cols/32]. Rows are padded to 128 and
+   * block columns to 4; the scale of row r, block column j sits at byte
+   *   ((r / 128) * T + j / 4) * 512 + (r % 32) * 16 + ((r / 32) % 4) * 4 + j % 4,
+   * T = ceil(cols / 128) tiles per 128-row band. Padding bytes are zero.
+   * mx_scale_bytes gives the buffer size. Macro factors keep their layout. */
+  MX_SCALES_MMA = 1 << 8
 } mx_scaling_t;
 
 typedef enum {
@@ -117,9 +127,15 @@ typedef enum {
 int mx_quantize(const void* x, int64_t rows, int64_t cols, int format, int scaling,
                 void* codes, uint8_t* scales, uint8_t* macro, void* stream);
 
+/* Bytes of the scale buffer of a [rows, cols] tensor: rows * cols / 32, or
+ * the padded size of the MX_SCALES_MMA layout when `scaling` has that flag.
+ * -1 for an invalid shape. Host only; no device work. */
+int64_t mx_scale_bytes(int64_t rows, int64_t cols, int scaling);
+
 /* Dequantize: out = value(code) * f * 2^(scale - 127), f = 1 + k/256 from
- * `macro` (NULL means f = 1; FP4 only). out_fp32 = 0: bf16 (rounded to
- * nearest even; exact for FP4 without MBS); 1: float (exact). A scale byte of
+ * `macro` (NULL means f = 1; FP4 only). out_fp32 (flags): bit 0 clear: bf16
+ * (rounded to nearest even; exact for FP4 without MBS); set: float (exact);
+ * MX_SCALES_MMA: `scales` is in the tiled layout (see mx_scaling_t). A scale byte of
  * 255 or an FP8 NaN code gives the canonical NaN (0x7FC0 / 0x7FC00000); an
  * E5M2 Inf code gives +-Inf. */
 int mx_dequantize(const void* codes, const uint8_t* scales, const uint8_t* macro,

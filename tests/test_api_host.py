@@ -126,3 +126,22 @@ def test_binding_refuses_cpu_tensors_for_device_only_calls(mx):
         mx.fake_quant(x)
     with pytest.raises(ValueError):
         mx.block_error(x)
+
+
+def test_scale_bytes_and_mma_layout_flag(mx):
+    sb = mx.mx_scale_bytes
+    MMA = 1 << 8
+    assert sb(4, 128, 0) == 16
+    assert sb(4, 128, MMA) == 128 * 4                  # one 128 x 4 tile
+    assert sb(300, 224, MMA) == 384 * 8                # rows -> 384, 7 block columns -> 8
+    assert sb(256, 512, MMA | 3) == 256 * 16
+    assert sb(0, 64, MMA) == 0
+    assert sb(4, 33, MMA) == -1 and sb(-1, 32, 0) == -1
+    # the flag is accepted by quantize / fake-quant (checked before any launch) ...
+    assert mx.mx_quantize(A, 4, 33, 0, MMA, A, A, None, 0) == SHAPE
+    assert mx.mx_quantize(None, 0, 32, 1, MMA | 1, None, None, None, 0) == OK
+    assert mx.mx_quantize(A, 4, 128, 0, MMA | 0x200, A, A, A, 0) == UNSUPPORTED
+    # ... and by dequantize as a flags bit; block error has no scale output
+    assert mx.mx_dequantize(A, A, None, 4, 33, 0, MMA | 1, A, 0) == SHAPE
+    assert mx.mx_dequantize(A, A, None, 4, 32, 0, MMA | 2, A, 0) == INVALID
+    assert mx.mx_block_error(A, 4, 32, 0, MMA, None, A, 0) == UNSUPPORTED
