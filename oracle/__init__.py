@@ -20,6 +20,15 @@ import numpy as np
 from .build import build_oracle, oracle_library_path
 
 E2M1, E4M3, E5M2, E3M2, E2M3, INT8 = 0, 1, 2, 3, 4, 5
+E2M1_B16, NVFP4 = 6, 7   # block-16 comparison formats (E8M0 / E4M3 scales)
+
+
+def block_size(fmt: int) -> int:
+    return 16 if fmt in (E2M1_B16, NVFP4) else 32
+
+
+def packed_fp4(fmt: int) -> bool:
+    return fmt in (E2M1, E2M1_B16, NVFP4)
 FLOOR, CEIL, OAS_RULE, OAS = 0, 1, 2, 3
 MBS_STATIC, MBS_DYNAMIC = 1 << 4, 2 << 4
 
@@ -136,9 +145,9 @@ def macro_k(x128, fmt: int, scaling: int) -> int:
     return _load().oracle_macro_k(_ptr(x128, ctypes.c_uint16), fmt, scaling)
 
 
-def _shape(x, scaling=0):
+def _shape(x, scaling=0, fmt=E2M1):
     rows, cols = (1, x.shape[0]) if x.ndim == 1 else (int(np.prod(x.shape[:-1])), x.shape[-1])
-    assert cols % 32 == 0, "rows must hold whole 32-element blocks"
+    assert cols % block_size(fmt) == 0, "rows must hold whole blocks"
     assert not (scaling >> 4) or cols % 128 == 0, "MBS needs whole 128-element macro blocks"
     return rows, cols
 
@@ -146,17 +155,18 @@ def _shape(x, scaling=0):
 def quantize(x, fmt: int = E2M1, scaling: int = FLOOR):
     """Returns (codes, scales, macro); macro is None without MBS."""
     x = _bf16(x)
-    rows, cols = _shape(x, scaling)
-    ncode = rows * cols // 2 if fmt == E2M1 else rows * cols
+    rows, cols = _shape(x, scaling, fmt)
+    bs = block_size(fmt)
+    ncode = rows * cols // 2 if packed_fp4(fmt) else rows * cols
     codes = np.zeros(ncode, np.uint8)
-    scales = np.zeros(rows * cols // 32, np.uint8)
+    scales = np.zeros(rows * cols // bs, np.uint8)
     macro = np.zeros(rows * cols // 128, np.uint8) if scaling >> 4 else None
     _load().oracle_quantize(_ptr(x, ctypes.c_uint16), rows, cols, fmt, scaling,
                             _ptr(codes, ctypes.c_uint8), _ptr(scales, ctypes.c_uint8),
                             _ptr(macro, ctypes.c_uint8))
-    ccols = cols // 2 if fmt == E2M1 else cols
+    ccols = cols // 2 if packed_fp4(fmt) else cols
     codes = codes.reshape(*x.shape[:-1], ccols)
-    scales = scales.reshape(*x.shape[:-1], cols // 32)
+    scales = scales.reshape(*x.shape[:-1], cols // bs)
     if macro is not None:
         macro = macro.reshape(*x.shape[:-1], cols // 128)
     return codes, scales, macro
@@ -177,14 +187,14 @@ def dequantize(codes, scales, macro, rows: int, cols: int, fmt: int = E2M1, out_
 
 def fake_quant_fwd(x, fmt: int = E2M1, scaling: int = FLOOR, want_scales: bool = False):
     x = _bf16(x)
-    rows, cols = _shape(x, scaling)
+    rows, cols = _shape(x, scaling, fmt)
     y = np.zeros(rows * cols, np.uint16)
-    scales = np.zeros(rows * cols // 32, np.uint8) if want_scales else None
+    scales = np.zeros(rows * cols // block_size(fmt), np.uint8) if want_scales else None
     _load().oracle_fake_quant_fwd(_ptr(x, ctypes.c_uint16), rows, cols, fmt, scaling,
                                   _ptr(y, ctypes.c_uint16), _ptr(scales, ctypes.c_uint8))
     y = y.reshape(x.shape)
     if want_scales:
-        return y, scales.reshape(*x.shape[:-1], cols // 32)
+        return y, scales.reshape(*x.shape[:-1], cols // block_size(fmt))
     return y
 
 
@@ -192,7 +202,7 @@ def fake_quant_bwd(x, gy, fmt: int = E2M1, scaling: int = FLOOR):
     x = _bf16(x)
     gy = _bf16(gy)
     assert gy.shape == x.shape
-    rows, cols = _shape(x, scaling)
+    rows, cols = _shape(x, scaling, fmt)
     gx = np.zeros(rows * cols, np.uint16)
     _load().oracle_fake_quant_bwd(_ptr(x, ctypes.c_uint16), _ptr(gy, ctypes.c_uint16), rows, cols,
                                   fmt, scaling, _ptr(gx, ctypes.c_uint16))
@@ -202,11 +212,11 @@ def fake_quant_bwd(x, gy, fmt: int = E2M1, scaling: int = FLOOR):
 def block_error(x, fmt: int = E2M1, scaling: int = FLOOR, want_blocks: bool = True):
     """Returns (block_sse [rows, cols/32] float64 or None, sum_d2, sum_x2)."""
     x = _bf16(x)
-    rows, cols = _shape(x, scaling)
-    bs = np.zeros(rows * cols // 32, np.float64) if want_blocks else None
+    rows, cols = _shape(x, scaling, fmt)
+    bs = np.zeros(rows * cols // block_size(fmt), np.float64) if want_blocks else None
     totals = np.zeros(2, np.float64)
     _load().oracle_block_error(_ptr(x, ctypes.c_uint16), rows, cols, fmt, scaling,
                                _ptr(bs, ctypes.c_double), _ptr(totals, ctypes.c_double))
     if bs is not None:
-        bs = bs.reshape(*x.shape[:-1], cols // 32)
+        bs = bs.reshape(*x.shape[:-1], cols // block_size(fmt))
     return bs, float(totals[0]), float(totals[1])

@@ -60,6 +60,11 @@ constexpr int kFmtE5M2 = 2;
 constexpr int kFmtE3M2 = 3;
 constexpr int kFmtE2M3 = 4;
 constexpr int kFmtInt8 = 5;
+// The comparison formats of [UP] section 1's gap analysis: E2M1 elements in
+// 16-element blocks, with an E8M0 scale (MXFP4 at block 16) or an E4M3 scale
+// (NVFP4).
+constexpr int kFmtE2M1B16 = 6;
+constexpr int kFmtNvfp4 = 7;
 
 constexpr int kScaleFloor = 0;
 constexpr int kScaleCeil = 1;
@@ -238,6 +243,11 @@ int signed_code(int c, bool negative, int fmt) {
   return negative ? (c | sign_bit(fmt)) : c;
 }
 double magnitude(int fmt, int c) { return element_value(c, fmt); }
+
+// The element format, block size and code packing of an API format.
+int elem_fmt(int fmt) { return (fmt == kFmtE2M1B16 || fmt == kFmtNvfp4) ? kFmtE2M1 : fmt; }
+int block_size(int fmt) { return (fmt == kFmtE2M1B16 || fmt == kFmtNvfp4) ? 16 : kBlock; }
+bool packed_fp4(int fmt) { return elem_fmt(fmt) == kFmtE2M1; }
 double max_value(int fmt) { return magnitude(fmt, num_magnitude_codes(fmt) - 1); }
 // The smallest nonzero magnitude.
 double min_magnitude(int fmt) { return magnitude(fmt, 1); }
@@ -390,17 +400,46 @@ int mbs_static_k(const double* x, int n, int fmt) {
 
 struct BlockResult {
   int scale_byte;
-  double X;            // effective scale f * 2^E (NaN for a non-finite block)
+  double X;            // effective scale f * 2^E, or the NVFP4 scale (NaN for a non-finite block)
   int codes[kBlock];
 };
 
-// Quantize one 32-element block with base rule `rule` under macro factor f.
-BlockResult quantize_block(const double* x, int fmt, int rule, double f) {
+// NVFP4 block ([UP] section 1: E4M3 scale factors with mantissa bits, block
+// 16): the scale is amax / 6 rounded to the nearest E4M3 value (ties to
+// even, saturating at 448) and the elements are x / s rounded onto the E2M1
+// grid. amax / 6 is exact in double wherever it sits on an E4M3 midpoint and
+// at least 2^-12 (relatively) away from every midpoint otherwise, so its one
+// double rounding cannot move the E4M3 choice. A scale of 0 (amax below
+// 2^-10 * 6 / 2) leaves only the signs.
+BlockResult quantize_block_nvfp4(const double* x) {
   BlockResult r{};
-  if (block_has_nonfinite(x, kBlock)) {
+  const int n = 16;
+  if (block_has_nonfinite(x, n)) {
+    r.scale_byte = 0x7F;   // the E4M3 NaN
+    r.X = std::numeric_limits<double>::quiet_NaN();
+    for (int i = 0; i < n; ++i) r.codes[i] = std::signbit(x[i]) ? sign_bit(kFmtE2M1) : 0;
+    return r;
+  }
+  r.scale_byte = round_element(block_amax(x, n) / 6.0, 1.0, kFmtE4M3);
+  r.X = decode_e4m3(r.scale_byte);
+  for (int i = 0; i < n; ++i) {
+    if (r.X == 0.0) r.codes[i] = std::signbit(x[i]) ? sign_bit(kFmtE2M1) : 0;
+    else r.codes[i] = round_element(x[i], r.X, kFmtE2M1);
+  }
+  return r;
+}
+
+// Quantize one block (32 elements, 16 for the block-16 formats) with base
+// rule `rule` under macro factor f.
+BlockResult quantize_block(const double* x, int api_fmt, int rule, double f) {
+  if (api_fmt == kFmtNvfp4) return quantize_block_nvfp4(x);
+  const int fmt = elem_fmt(api_fmt);
+  const int n = block_size(api_fmt);
+  BlockResult r{};
+  if (block_has_nonfinite(x, n)) {
     r.scale_byte = 0xFF;
     r.X = std::numeric_limits<double>::quiet_NaN();
-    for (int i = 0; i < kBlock; ++i) {
+    for (int i = 0; i < n; ++i) {
       const int s = std::signbit(x[i]) ? sign_bit(fmt) : 0;
       // The FP8 elements of a NaN-scale block are NaN (E4M3 S.1111.111, E5M2
       // S.11111.11); E2M1 and FP6 have no NaN, so only the sign is kept;
@@ -411,10 +450,10 @@ BlockResult quantize_block(const double* x, int fmt, int rule, double f) {
     }
     return r;
   }
-  const int E = block_exponent(x, kBlock, fmt, rule, f);
+  const int E = block_exponent(x, n, fmt, rule, f);
   r.scale_byte = E + 127;
   r.X = f * std::ldexp(1.0, E);
-  for (int i = 0; i < kBlock; ++i) r.codes[i] = round_element(x[i], r.X, fmt);
+  for (int i = 0; i < n; ++i) r.codes[i] = round_element(x[i], r.X, fmt);
   return r;
 }
 
@@ -492,22 +531,23 @@ struct RowQuant {
 RowQuant quantize_row(const double* x, int64_t cols, int fmt, int scaling) {
   const int rule = scaling & 0xF;
   const int mbs = scaling >> 4;
+  const int bs = block_size(fmt);
   RowQuant q;
   q.codes.resize(cols);
-  q.scale_bytes.resize(cols / kBlock);
-  q.X.resize(cols / kBlock);
+  q.scale_bytes.resize(cols / bs);
+  q.X.resize(cols / bs);
   if (mbs) q.ks.resize(cols / kMacro);
-  for (int64_t b = 0; b < cols / kBlock; ++b) {
+  for (int64_t b = 0; b < cols / bs; ++b) {
     double f = 1.0;
     if (mbs) {
-      const int64_t m = b / (kMacro / kBlock);
-      if (b % (kMacro / kBlock) == 0) q.ks[m] = macro_k(x + m * kMacro, fmt, rule, mbs);
+      const int64_t m = b / (kMacro / bs);
+      if (b % (kMacro / bs) == 0) q.ks[m] = macro_k(x + m * kMacro, fmt, rule, mbs);
       f = macro_factor(q.ks[m]);
     }
-    const BlockResult r = quantize_block(x + b * kBlock, fmt, rule, f);
+    const BlockResult r = quantize_block(x + b * bs, fmt, rule, f);
     q.scale_bytes[b] = r.scale_byte;
     q.X[b] = r.X;
-    for (int i = 0; i < kBlock; ++i) q.codes[b * kBlock + i] = r.codes[i];
+    for (int i = 0; i < bs; ++i) q.codes[b * bs + i] = r.codes[i];
   }
   return q;
 }
@@ -515,8 +555,10 @@ RowQuant quantize_row(const double* x, int64_t cols, int fmt, int scaling) {
 // Dequantized value of one element as an exact double (NaN for a NaN scale or
 // a NaN element).
 double dequant_value(int code, int scale_byte, int k, int fmt) {
+  // NVFP4: the scale byte is an E4M3 value (NaN for S.1111.111)
+  if (fmt == kFmtNvfp4) return element_value(code, kFmtE2M1) * decode_e4m3(scale_byte);
   if (scale_byte == 0xFF) return std::numeric_limits<double>::quiet_NaN();
-  return element_value(code, fmt) * macro_factor(k) * decode_e8m0(scale_byte);
+  return element_value(code, elem_fmt(fmt)) * macro_factor(k) * decode_e8m0(scale_byte);
 }
 
 uint32_t float_bits(float v) {
@@ -573,12 +615,12 @@ void oracle_quantize(const uint16_t* x, int64_t rows, int64_t cols, int fmt, int
     for (int64_t r = r0; r < r1; ++r) {
       decode_row(x + r * cols, cols, row.data());
       const RowQuant q = quantize_row(row.data(), cols, fmt, scaling);
-      for (int64_t b = 0; b < cols / kBlock; ++b)
-        scales[r * (cols / kBlock) + b] = static_cast<uint8_t>(q.scale_bytes[b]);
+      const int64_t nb = cols / block_size(fmt);
+      for (int64_t b = 0; b < nb; ++b) scales[r * nb + b] = static_cast<uint8_t>(q.scale_bytes[b]);
       if (macro && (scaling >> 4))
         for (int64_t m = 0; m < cols / kMacro; ++m)
           macro[r * (cols / kMacro) + m] = static_cast<uint8_t>(q.ks[m]);
-      if (fmt == kFmtE2M1) {
+      if (packed_fp4(fmt)) {
         for (int64_t c = 0; c < cols; c += 2)
           codes[r * (cols / 2) + c / 2] =
               static_cast<uint8_t>(q.codes[c] | (q.codes[c + 1] << 4));
@@ -597,13 +639,14 @@ void oracle_dequantize(const uint8_t* codes, const uint8_t* scales, const uint8_
     for (int64_t r = r0; r < r1; ++r) {
       for (int64_t c = 0; c < cols; ++c) {
         int code;
-        if (fmt == kFmtE2M1) {
+        if (packed_fp4(fmt)) {
           const uint8_t byte = codes[r * (cols / 2) + c / 2];
           code = (c % 2 == 0) ? (byte & 0xF) : (byte >> 4);
         } else {
           code = codes[r * cols + c];
         }
-        const int sb = scales[r * (cols / kBlock) + c / kBlock];
+        const int bs = block_size(fmt);
+        const int sb = scales[r * (cols / bs) + c / bs];
         const int k = macro ? macro[r * (cols / kMacro) + c / kMacro] : 0;
         const double v = dequant_value(code, sb, k, fmt);
         if (out_fp32) {
@@ -625,15 +668,16 @@ void oracle_fake_quant_fwd(const uint16_t* x, int64_t rows, int64_t cols, int fm
     for (int64_t r = r0; r < r1; ++r) {
       decode_row(x + r * cols, cols, row.data());
       const RowQuant q = quantize_row(row.data(), cols, fmt, scaling);
+      const int bs = block_size(fmt);
       for (int64_t c = 0; c < cols; ++c) {
-        const int64_t b = c / kBlock;
+        const int64_t b = c / bs;
         const int k = (scaling >> 4) ? q.ks[c / kMacro] : 0;
         const double v = dequant_value(q.codes[c], q.scale_bytes[b], k, fmt);
         y[r * cols + c] = std::isnan(v) ? kNaNbf16 : encode_bf16_rne(v);
       }
       if (scales_out)
-        for (int64_t b = 0; b < cols / kBlock; ++b)
-          scales_out[r * (cols / kBlock) + b] = static_cast<uint8_t>(q.scale_bytes[b]);
+        for (int64_t b = 0; b < cols / bs; ++b)
+          scales_out[r * (cols / bs) + b] = static_cast<uint8_t>(q.scale_bytes[b]);
     }
   });
 }
@@ -642,14 +686,14 @@ void oracle_fake_quant_fwd(const uint16_t* x, int64_t rows, int64_t cols, int fm
 // block's effective scale, as in the forward), else +0; NaN x gives +0.
 void oracle_fake_quant_bwd(const uint16_t* x, const uint16_t* gy, int64_t rows, int64_t cols,
                            int fmt, int scaling, uint16_t* gx) {
-  const double maxv = max_value(fmt);
+  const double maxv = max_value(elem_fmt(fmt));
   parallel_rows(rows, [&](int64_t r0, int64_t r1) {
     std::vector<double> row(cols);
     for (int64_t r = r0; r < r1; ++r) {
       decode_row(x + r * cols, cols, row.data());
       const RowQuant q = quantize_row(row.data(), cols, fmt, scaling);
       for (int64_t c = 0; c < cols; ++c) {
-        const double X = q.X[c / kBlock];   // NaN for a non-finite block
+        const double X = q.X[c / block_size(fmt)];   // NaN for a non-finite block
         const bool pass = std::fabs(row[c]) <= maxv * X;
         gx[r * cols + c] = pass ? gy[r * cols + c] : 0;
       }
@@ -672,10 +716,11 @@ void oracle_block_error(const uint16_t* x, int64_t rows, int64_t cols, int fmt, 
     for (int64_t r = r0; r < r1; ++r) {
       decode_row(x + r * cols, cols, row.data());
       const RowQuant q = quantize_row(row.data(), cols, fmt, scaling);
-      for (int64_t b = 0; b < cols / kBlock; ++b) {
+      const int bsz = block_size(fmt);
+      for (int64_t b = 0; b < cols / bsz; ++b) {
         double bs = 0.0;
-        for (int i = 0; i < kBlock; ++i) {
-          const int64_t c = b * kBlock + i;
+        for (int i = 0; i < bsz; ++i) {
+          const int64_t c = b * bsz + i;
           const int k = (scaling >> 4) ? q.ks[c / kMacro] : 0;
           // ŷ as a float: exact, except that a value past the float range is
           // infinite (only reachable for amax in the top binade of bf16)
@@ -685,7 +730,7 @@ void oracle_block_error(const uint16_t* x, int64_t rows, int64_t cols, int fmt, 
           sx += row[c] * row[c];
         }
         sd += bs;
-        if (block_sse) block_sse[r * (cols / kBlock) + b] = bs;
+        if (block_sse) block_sse[r * (cols / bsz) + b] = bs;
       }
     }
     part_d[t] = sd;
