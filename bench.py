@@ -245,8 +245,10 @@ def stack_ops(mx, x, reps=50, only=None):
     c4 = torch.empty(rows, cols // 2, dtype=torch.uint8, device=dev)
     c8 = torch.empty(rows, cols, dtype=torch.uint8, device=dev)
     sc = torch.empty(rows, cols // 32, dtype=torch.uint8, device=dev)
+    sc16 = torch.empty(rows, cols // 16, dtype=torch.uint8, device=dev)
     mac = torch.empty(rows, cols // 128, dtype=torch.uint8, device=dev)
-    sc_mma = torch.empty(mx.mx_scale_bytes(rows, cols, mx.MMA_SCALES), dtype=torch.uint8, device=dev)
+    sc_mma = torch.empty(mx.mx_scale_bytes(rows, cols, mx.E2M1, mx.MMA_SCALES), dtype=torch.uint8,
+                         device=dev)
     y = torch.empty_like(x)
     g = torch.empty_like(x).normal_()
     fp4, fp8, fp4m = n * 2.53125, n * 3.03125, n * (2.53125 + 1 / 128)
@@ -264,6 +266,10 @@ def stack_ops(mx, x, reps=50, only=None):
         "fp4_block_error": (lambda: mx.block_error(x, per_block=False), n * 2),
         "fp4_floor_quantize_mma_scales": (lambda: mx.quantize(x, mx.E2M1, mx.FLOOR | mx.MMA_SCALES,
                                                               out=(c4, sc_mma, None)), fp4),
+        "nvfp4_quantize": (lambda: mx.quantize(x, mx.NVFP4, mx.FLOOR, out=(c4, sc16, None)),
+                           n * (2.5 + 1 / 16)),
+        "fp4b16_floor_quantize": (lambda: mx.quantize(x, mx.E2M1_B16, mx.FLOOR, out=(c4, sc16, None)),
+                                  n * (2.5 + 1 / 16)),
         "e5m2_floor_quantize": (lambda: mx.quantize(x, mx.E5M2, mx.FLOOR, out=(c8, sc, None)), fp8),
         "e3m2_floor_quantize": (lambda: mx.quantize(x, mx.E3M2, mx.FLOOR, out=(c8, sc, None)), fp8),
         "e2m3_floor_quantize": (lambda: mx.quantize(x, mx.E2M3, mx.FLOOR, out=(c8, sc, None)), fp8),
@@ -302,7 +308,7 @@ def stack_ops(mx, x, reps=50, only=None):
         e.synchronize()
         ms = s.elapsed_time(e) / n_reps
         res[name] = {"ms": round(ms, 4), "GB/s": round(nbytes / ms / 1e6, 1)}
-    del c4, c8, sc, mac, sc_mma, y, g
+    del c4, c8, sc, sc16, mac, sc_mma, y, g
     return res
 
 
@@ -345,18 +351,25 @@ def other_ops(mx, inputs, dev, reps=10):
         del x3, g3, y3
     x4 = inputs.heavy_tail(device=dev)
     n4 = x4.numel()
-    modes = [("FLOOR", 0), ("CEIL", 1), ("OAS_RULE", 2), ("OAS", 3), ("MBS_STATIC", 16),
-             ("MBS_DYNAMIC", 32), ("OAS+MBS_STATIC", 19), ("OAS+MBS_DYNAMIC", 35)]
-    for mname, m in modes:
-        bufs = mx.quantize(x4, mx.E2M1, m)
+    # the eight MXFP4 modes, then the block-16 comparison formats of the
+    # MXFP4 / NVFP4 gap analysis (MSE and SQNR on the same tensor)
+    modes = [("fp4", mx.E2M1, "FLOOR", 0), ("fp4", mx.E2M1, "CEIL", 1),
+             ("fp4", mx.E2M1, "OAS_RULE", 2), ("fp4", mx.E2M1, "OAS", 3),
+             ("fp4", mx.E2M1, "MBS_STATIC", 16), ("fp4", mx.E2M1, "MBS_DYNAMIC", 32),
+             ("fp4", mx.E2M1, "OAS+MBS_STATIC", 19), ("fp4", mx.E2M1, "OAS+MBS_DYNAMIC", 35),
+             ("fp4b16", mx.E2M1_B16, "FLOOR", 0), ("fp4b16", mx.E2M1_B16, "OAS", 3),
+             ("nvfp4", mx.NVFP4, "FLOOR", 0)]
+    for fname, fmt, mname, m in modes:
+        bufs = mx.quantize(x4, fmt, m)
         extra = n4 // 128 if m >> 4 else 0
-        rec(f"heavy_tail_8192x4096/fp4_{mname}_quantize", 2 * n4 + n4 // 2 + n4 // 32 + extra,
-            lambda: mx.quantize(x4, mx.E2M1, m, out=bufs))
-        _, tot = mx.block_error(x4, mx.E2M1, m, per_block=False)
-        rec(f"heavy_tail_8192x4096/fp4_{mname}_block_error", 2 * n4,
-            lambda: mx.block_error(x4, mx.E2M1, m, per_block=False))
+        rec(f"heavy_tail_8192x4096/{fname}_{mname}_quantize",
+            2 * n4 + n4 // 2 + n4 // mx.block_size(fmt) + extra,
+            lambda: mx.quantize(x4, fmt, m, out=bufs))
+        _, tot = mx.block_error(x4, fmt, m, per_block=False)
+        rec(f"heavy_tail_8192x4096/{fname}_{mname}_block_error", 2 * n4,
+            lambda: mx.block_error(x4, fmt, m, per_block=False))
         t = tot.cpu().tolist()
-        res[f"heavy_tail_8192x4096/fp4_{mname}_block_error"].update(
+        res[f"heavy_tail_8192x4096/{fname}_{mname}_block_error"].update(
             {"mse": t[0] / n4, "sqnr_db": (10 * __import__("math").log10(t[1] / t[0])) if t[0] > 0 else None})
     del x4
     return res

@@ -35,6 +35,7 @@ __all__ = [
     "MXError", "library_path", "load_library",
     "mx_quantize", "mx_dequantize", "mx_fake_quant_fwd", "mx_fake_quant_bwd",
     "mx_block_error", "mx_status_string", "mx_version", "mx_scale_bytes", "MMA_SCALES",
+    "E2M1_B16", "NVFP4", "block_size",
     "quantize", "dequantize", "fake_quant", "fake_quant_bwd", "block_error", "MXFakeQuantize",
     "MXFP4_FORMAT", "MXFP8_FORMAT",
 ]
@@ -47,8 +48,16 @@ E3M2 = 3   # MXFP6 (one code per byte, low 6 bits)
 E2M3 = 4   # MXFP6
 INT8 = 5   # MXINT8 (i * 2^-6)
 # OR into `scaling`: scale bytes in the tiled layout of block-scaled tensor-core
-# GEMMs (a flat uint8 buffer of mx_scale_bytes(rows, cols, scaling) bytes)
+# GEMMs (a flat uint8 buffer of mx_scale_bytes(rows, cols, format, scaling) bytes)
 MMA_SCALES = 1 << 8
+E2M1_B16 = 6  # MXFP4 at block 16 (E8M0 scales [..., cols/16])
+NVFP4 = 7     # E2M1 at block 16 with E4M3 scales amax/6 (FLOOR only)
+_PACKED = (E2M1, E2M1_B16, NVFP4)
+
+
+def block_size(format: int) -> int:
+    """Elements per scale byte: 16 for the block-16 formats, else 32."""
+    return 16 if format in (E2M1_B16, NVFP4) else 32
 MXFP4_FORMAT = E2M1
 MXFP8_FORMAT = E4M3
 # scaling (mx_scaling_t)
@@ -93,7 +102,7 @@ def load_library():
     lib.mx_status_string.argtypes = [c_int]
     lib.mx_status_string.restype = ctypes.c_char_p
     lib.mx_version.restype = c_int
-    lib.mx_scale_bytes.argtypes = [i64, i64, c_int]
+    lib.mx_scale_bytes.argtypes = [i64, i64, c_int, c_int]
     lib.mx_scale_bytes.restype = i64
     _lib = lib
     return lib
@@ -130,8 +139,8 @@ def mx_version() -> int:
     return load_library().mx_version()
 
 
-def mx_scale_bytes(rows, cols, scaling) -> int:
-    return load_library().mx_scale_bytes(rows, cols, scaling)
+def mx_scale_bytes(rows, cols, format, scaling) -> int:
+    return load_library().mx_scale_bytes(rows, cols, format, scaling)
 
 
 # ----------------------------------------------------------- tensor layer --
@@ -192,9 +201,9 @@ def quantize(x: torch.Tensor, format: int = E2M1, scaling: int = FLOOR, out=None
     lead = x.shape[:-1]
     mbs = ((scaling >> 4) & 3) != 0
     if out is None:
-        ccols = cols // 2 if format == E2M1 else cols
+        ccols = cols // 2 if format in _PACKED else cols
         codes = torch.empty(*lead, ccols, dtype=torch.uint8, device=x.device)
-        scales = _scales_buffer(lead, rows, cols, scaling, x.device)
+        scales = _scales_buffer(lead, rows, cols, format, scaling, x.device)
         macro = torch.empty(*lead, cols // 128, dtype=torch.uint8, device=x.device) if mbs else None
     else:
         codes, scales, macro = out
@@ -212,10 +221,11 @@ def _to_host(t: torch.Tensor, pinned: bool) -> torch.Tensor:
     return t.cpu()
 
 
-def _scales_buffer(lead, rows, cols, scaling, device):
+def _scales_buffer(lead, rows, cols, format, scaling, device):
     if scaling & MMA_SCALES:
-        return torch.empty(mx_scale_bytes(rows, cols, scaling), dtype=torch.uint8, device=device)
-    return torch.empty(*lead, cols // 32, dtype=torch.uint8, device=device)
+        return torch.empty(mx_scale_bytes(rows, cols, format, scaling), dtype=torch.uint8,
+                           device=device)
+    return torch.empty(*lead, cols // block_size(format), dtype=torch.uint8, device=device)
 
 
 def dequantize(codes: torch.Tensor, scales: torch.Tensor, macro=None, format: int = E2M1,
@@ -233,8 +243,8 @@ def dequantize(codes: torch.Tensor, scales: torch.Tensor, macro=None, format: in
         return out
     if codes.dtype != torch.uint8 or scales.dtype != torch.uint8:
         raise ValueError("codes and scales must be uint8")
-    cols = codes.shape[-1] * 2 if format == E2M1 else codes.shape[-1]
-    rows = codes.numel() * (2 if format == E2M1 else 1) // cols if cols else 0
+    cols = codes.shape[-1] * 2 if format in _PACKED else codes.shape[-1]
+    rows = codes.numel() * (2 if format in _PACKED else 1) // cols if cols else 0
     if out_dtype not in (torch.bfloat16, torch.float32):
         raise ValueError("out_dtype must be bfloat16 or float32")
     if out is None:
@@ -253,7 +263,7 @@ def fake_quant(x: torch.Tensor, format: int = E2M1, scaling: int = FLOOR, out=No
     _cuda_bf16(x, "x")
     rows, cols = _rows_cols(x)
     y = torch.empty_like(x) if out is None else out
-    scales = _scales_buffer(x.shape[:-1], rows, cols, scaling, x.device) if return_scales else None
+    scales = _scales_buffer(x.shape[:-1], rows, cols, format, scaling, x.device) if return_scales else None
     with torch.cuda.device(x.device):
         _check(mx_fake_quant_fwd(_ptr(x), rows, cols, format, scaling, _ptr(y), _ptr(scales),
                                  _stream(x.device)), "mx_fake_quant_fwd")
@@ -284,7 +294,7 @@ def block_error(x: torch.Tensor, format: int = E2M1, scaling: int = FLOOR,
     """
     _cuda_bf16(x, "x")
     rows, cols = _rows_cols(x)
-    bs = (torch.empty(*x.shape[:-1], cols // 32, dtype=torch.float32, device=x.device)
+    bs = (torch.empty(*x.shape[:-1], cols // block_size(format), dtype=torch.float32, device=x.device)
           if per_block else None)
     totals = torch.empty(2, dtype=torch.float64, device=x.device)
     with torch.cuda.device(x.device):

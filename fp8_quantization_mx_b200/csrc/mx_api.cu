@@ -21,16 +21,19 @@ constexpr int64_t kMaxElems = int64_t(1) << 40;
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
 
-int check_shape(int64_t rows, int64_t cols, bool mbs) {
+// Elements per scale: 16 for the block-16 formats, else 32.
+int block_of(int format) { return (format == MX_FMT_E2M1_B16 || format == MX_FMT_NVFP4) ? 16 : 32; }
+
+int check_shape(int64_t rows, int64_t cols, bool mbs, int block = 32) {
   if (rows < 0 || cols < 0) return MX_ERR_INVALID_ARG;
-  if (cols % 32 != 0) return MX_ERR_SHAPE;
+  if (cols % block != 0) return MX_ERR_SHAPE;
   if (mbs && cols % 128 != 0) return MX_ERR_SHAPE;
   if (rows > 0 && cols > 0 && rows > kMaxElems / cols) return MX_ERR_INVALID_ARG;
   return MX_OK;
 }
 
 // Format and scaling combinations the kernels implement.
-bool known_format(int format) { return format >= MX_FMT_E2M1 && format <= MX_FMT_INT8; }
+bool known_format(int format) { return format >= MX_FMT_E2M1 && format <= MX_FMT_NVFP4; }
 
 int check_mode(int format, int scaling) {
   if (!known_format(format)) return MX_ERR_UNSUPPORTED;
@@ -38,6 +41,8 @@ int check_mode(int format, int scaling) {
   const int rule = scaling & 0xF;
   const int mbs = scaling >> 4;
   if (rule > MX_SCALE_OAS || mbs > 2) return MX_ERR_UNSUPPORTED;
+  if (format == MX_FMT_NVFP4) return scaling == MX_SCALE_FLOOR ? MX_OK : MX_ERR_UNSUPPORTED;
+  if (format == MX_FMT_E2M1_B16) return mbs == 0 ? MX_OK : MX_ERR_UNSUPPORTED;
   if (format != MX_FMT_E2M1) {
     // one-byte formats: FLOOR, CEIL, and OAS for the float elements
     if (mbs != 0 || rule == MX_SCALE_OAS_RULE) return MX_ERR_UNSUPPORTED;
@@ -50,29 +55,29 @@ int check_mode(int format, int scaling) {
 int from_cuda(cudaError_t e) { return e == cudaSuccess ? MX_OK : MX_ERR_CUDA; }
 
 // The scale map of a call; flags holds MX_SCALES_MMA or not.
-mxk::ScaleMap scale_map(int64_t cols, int flags) {
+mxk::ScaleMap scale_map(int64_t cols, int flags, int block) {
   mxk::ScaleMap m{0, 0, 0.0};
   if (flags & MX_SCALES_MMA) {
-    m.bpr = cols / 32;
+    m.bpr = cols / block;
     m.nct = (m.bpr + 3) / 4;
     m.inv = 1.0 / static_cast<double>(m.bpr);
   }
   return m;
 }
 
-int64_t scale_bytes(int64_t rows, int64_t cols, int flags) {
-  if (!(flags & MX_SCALES_MMA)) return rows * (cols / 32);
-  return (rows + 127) / 128 * 128 * ((cols / 32 + 3) / 4 * 4);
+int64_t scale_bytes(int64_t rows, int64_t cols, int flags, int block) {
+  if (!(flags & MX_SCALES_MMA)) return rows * (cols / block);
+  return (rows + 127) / 128 * 128 * ((cols / block + 3) / 4 * 4);
 }
 
 // The tiled layout pads rows to 128 and block columns to 4; the padding must
 // read as zero bytes, so it is cleared on the stream before the kernel writes
 // the real scales.
-cudaError_t clear_padding(uint8_t* scales, int64_t rows, int64_t cols, int flags,
+cudaError_t clear_padding(uint8_t* scales, int64_t rows, int64_t cols, int flags, int block,
                           cudaStream_t st) {
   if (!(flags & MX_SCALES_MMA) || !scales) return cudaSuccess;
-  if (rows % 128 == 0 && (cols / 32) % 4 == 0) return cudaSuccess;
-  return cudaMemsetAsync(scales, 0, static_cast<size_t>(scale_bytes(rows, cols, flags)), st);
+  if (rows % 128 == 0 && (cols / block) % 4 == 0) return cudaSuccess;
+  return cudaMemsetAsync(scales, 0, static_cast<size_t>(scale_bytes(rows, cols, flags, block)), st);
 }
 
 }  // namespace
@@ -93,10 +98,12 @@ const char* mx_status_string(int status) {
   }
 }
 
-int64_t mx_scale_bytes(int64_t rows, int64_t cols, int scaling) {
-  if (rows < 0 || cols < 0 || cols % 32 != 0) return -1;
+int64_t mx_scale_bytes(int64_t rows, int64_t cols, int format, int scaling) {
+  if (!known_format(format)) return -1;
+  const int block = block_of(format);
+  if (rows < 0 || cols < 0 || cols % block != 0) return -1;
   if (rows > 0 && cols > 0 && rows > kMaxElems / cols) return -1;
-  return scale_bytes(rows, cols, scaling & MX_SCALES_MMA);
+  return scale_bytes(rows, cols, scaling & MX_SCALES_MMA, block);
 }
 
 int mx_quantize(const void* x, int64_t rows, int64_t cols, int format, int scaling, void* codes,
@@ -106,16 +113,16 @@ int mx_quantize(const void* x, int64_t rows, int64_t cols, int format, int scali
   int st = check_mode(format, scaling);
   if (st != MX_OK) return st;
   const bool mbs = (scaling >> 4) != 0;
-  st = check_shape(rows, cols, mbs);
+  st = check_shape(rows, cols, mbs, block_of(format));
   if (st != MX_OK) return st;
   const int64_t n = rows * cols;
   if (n == 0) return MX_OK;
   if (!x || !codes || !scales || (mbs && !macro)) return MX_ERR_INVALID_ARG;
   if (!aligned(x, 32) || !aligned(codes, 16)) return MX_ERR_ALIGN;
   const auto cs = static_cast<cudaStream_t>(stream);
-  if (clear_padding(scales, rows, cols, layout, cs) != cudaSuccess) return MX_ERR_CUDA;
+  if (clear_padding(scales, rows, cols, layout, block_of(format), cs) != cudaSuccess) return MX_ERR_CUDA;
   return from_cuda(mxk::launch_quantize(x, n, format, scaling, codes, scales, mbs ? macro : nullptr,
-                                        scale_map(cols, layout), cs));
+                                        scale_map(cols, layout, block_of(format)), cs));
 }
 
 int mx_dequantize(const void* codes, const uint8_t* scales, const uint8_t* macro, int64_t rows,
@@ -125,14 +132,14 @@ int mx_dequantize(const void* codes, const uint8_t* scales, const uint8_t* macro
   if ((out_fp32 & ~(1 | MX_SCALES_MMA)) != 0) return MX_ERR_INVALID_ARG;
   const int layout = out_fp32 & MX_SCALES_MMA;
   out_fp32 &= 1;
-  int st = check_shape(rows, cols, macro != nullptr);
+  int st = check_shape(rows, cols, macro != nullptr, block_of(format));
   if (st != MX_OK) return st;
   const int64_t n = rows * cols;
   if (n == 0) return MX_OK;
   if (!codes || !scales || !out) return MX_ERR_INVALID_ARG;
   if (!aligned(codes, 16) || !aligned(out, 32)) return MX_ERR_ALIGN;
   return from_cuda(mxk::launch_dequantize(codes, scales, macro, n, format, out_fp32, out,
-                                          scale_map(cols, layout),
+                                          scale_map(cols, layout, block_of(format)),
                                           static_cast<cudaStream_t>(stream)));
 }
 
@@ -142,23 +149,23 @@ int mx_fake_quant_fwd(const void* x, int64_t rows, int64_t cols, int format, int
   scaling &= ~MX_SCALES_MMA;
   int st = check_mode(format, scaling);
   if (st != MX_OK) return st;
-  st = check_shape(rows, cols, (scaling >> 4) != 0);
+  st = check_shape(rows, cols, (scaling >> 4) != 0, block_of(format));
   if (st != MX_OK) return st;
   const int64_t n = rows * cols;
   if (n == 0) return MX_OK;
   if (!x || !y) return MX_ERR_INVALID_ARG;
   if (!aligned(x, 32) || !aligned(y, 32)) return MX_ERR_ALIGN;
   const auto cs = static_cast<cudaStream_t>(stream);
-  if (clear_padding(scales_out, rows, cols, layout, cs) != cudaSuccess) return MX_ERR_CUDA;
+  if (clear_padding(scales_out, rows, cols, layout, block_of(format), cs) != cudaSuccess) return MX_ERR_CUDA;
   return from_cuda(mxk::launch_fake_fwd(x, n, format, scaling, y, scales_out,
-                                        scale_map(cols, layout), cs));
+                                        scale_map(cols, layout, block_of(format)), cs));
 }
 
 int mx_fake_quant_bwd(const void* x, const void* grad_y, int64_t rows, int64_t cols, int format,
                       int scaling, void* grad_x, void* stream) {
   int st = check_mode(format, scaling);
   if (st != MX_OK) return st;
-  st = check_shape(rows, cols, (scaling >> 4) != 0);
+  st = check_shape(rows, cols, (scaling >> 4) != 0, block_of(format));
   if (st != MX_OK) return st;
   const int64_t n = rows * cols;
   if (n == 0) return MX_OK;
@@ -172,7 +179,7 @@ int mx_block_error(const void* x, int64_t rows, int64_t cols, int format, int sc
                    float* block_sse, double* totals, void* stream) {
   int st = check_mode(format, scaling);
   if (st != MX_OK) return st;
-  st = check_shape(rows, cols, (scaling >> 4) != 0);
+  st = check_shape(rows, cols, (scaling >> 4) != 0, block_of(format));
   if (st != MX_OK) return st;
   if (!totals) return MX_ERR_INVALID_ARG;
   if (!aligned(totals, 8)) return MX_ERR_ALIGN;

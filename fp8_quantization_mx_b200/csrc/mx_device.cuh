@@ -44,6 +44,10 @@ constexpr int kFmtE5M2 = 2;
 constexpr int kFmtE3M2 = 3;
 constexpr int kFmtE2M3 = 4;
 constexpr int kFmtInt8 = 5;
+// 16-element blocks, E2M1 elements: MXFP4 at block 16 (E8M0 scale) and
+// NVFP4 (E4M3 scale), the comparison formats of the MXFP4/NVFP4 gap analysis.
+constexpr int kFmtE2M1B16 = 6;
+constexpr int kFmtNvfp4 = 7;
 constexpr int kFloor = 0, kCeil = 1, kOasRule = 2, kOas = 3;
 constexpr int kMbsNone = 0, kMbsStatic = 1, kMbsDynamic = 2;
 constexpr unsigned kFull = 0xFFFFFFFFu;
@@ -831,6 +835,51 @@ __device__ __forceinline__ uint32_t mbs_codes8(const float* s8, float L, float H
   }
   return even_of_adjacent(cvt_e2m1_f8(lo), cvt_e2m1_f8(hi));
 }
+// ---------------------------------------------------------------- NVFP4 --
+//
+// The block scale is amax / 6 rounded to E4M3 (ties to even, saturating):
+// the IEEE quotient amax / 6 in float lies exactly on an E4M3 midpoint when
+// the real one does (then it is a short dyadic number) and otherwise at least
+// 2^-12 (relatively) from every midpoint, far beyond its 2^-24 rounding, so
+// the hardware E4M3 conversion of it is the correctly rounded scale. Returns
+// the E4M3 byte; the NaN byte 0x7F for a non-finite block.
+__device__ __forceinline__ int nvfp4_scale_byte(uint32_t amax) {
+  if (amax >= 0x7F80u) return 0x7F;
+  const float q = __fdiv_rn(__uint_as_float(amax << 16), 6.0f);
+  uint16_t h;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(h) : "f"(0.0f), "f"(q));
+  return h & 0xFF;
+}
+// The value of an E4M3 byte as a float (exact; NaN for S.1111.111).
+__device__ __forceinline__ float e4m3_value(int byte) {
+  uint32_t h;
+  const uint16_t b = static_cast<uint16_t>(byte);
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"(b));
+  return f16_lo(h);
+}
+
+// E2M1 codes of x / s for a positive E4M3 scale value s: as with the macro
+// factor, x / s is bracketed by two products with 1/s moved 2^-20 down and up
+// (1/s from the hardware reciprocal, within 1 ulp) and both bounds are
+// converted. x (8 significant bits) and mid * s (a midpoint of the grid times
+// a 4-bit s) differ, unless equal, by at least 2^-8 of x, so the bounds
+// disagree only at an exact tie, where the even code is kept.
+__device__ __forceinline__ uint2 enc_e2m1_div_16(const V16& x, float s) {
+  float inv;
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(inv) : "f"(s));
+  const float L = inv * 0.99999904632568359375f;   // 1 - 2^-20
+  const float H = inv * 1.00000095367431640625f;   // 1 + 2^-20
+  float lo[16], hi[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const float e = elem(x, i);
+    lo[i] = e * L;
+    hi[i] = e * H;
+  }
+  return make_uint2(even_of_adjacent(cvt_e2m1_f8(lo), cvt_e2m1_f8(hi)),
+                    even_of_adjacent(cvt_e2m1_f8(lo + 8), cvt_e2m1_f8(hi + 8)));
+}
+
 __device__ __forceinline__ void e2m1x8_values(uint32_t codes, float* v) {
   const uint2 a = e2m1x4_to_bf16(codes & 0xFFFFu);
   const uint2 b = e2m1x4_to_bf16(codes >> 16);

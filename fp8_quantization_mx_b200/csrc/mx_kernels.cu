@@ -313,6 +313,96 @@ __device__ __forceinline__ void process_slice(const StreamArgs& a, const V16& v,
   }
 }
 
+// The 16-element-block formats (MXFP4 at block 16, NVFP4): a lane's slice
+// is one whole block, so nothing is exchanged between lanes and the block
+// index is the slice index.
+template <int OP, int FMT, int RULE>
+__device__ __forceinline__ void process_slice16(const StreamArgs& a, const V16& v, const V16& g,
+                                                int64_t c, bool valid, double& sd, double& sx) {
+  const uint32_t am = amax_bits16(v);
+  const bool nonfinite = am >= 0x7F80u;
+  int byte;
+  float scale;   // the block's scale value (0 leaves only the signs)
+  uint2 codes = make_uint2(0, 0);
+  if constexpr (FMT == kFmtNvfp4) {
+    byte = nvfp4_scale_byte(am);
+    scale = nonfinite ? 0.0f : e4m3_value(byte);
+    if (OP != kOpFakeBwd)
+      codes = (nonfinite || scale == 0.0f) ? nonfinite_e2m1_16(v) : enc_e2m1_div_16(v, scale);
+  } else {
+    byte = rule_byte<kFmtE2M1, RULE>(am);
+    bool have = false;
+    if constexpr (RULE == kOas) {
+      const int b2 = max(static_cast<int>(am >> 7) - 1, 0);
+      const bool need = !nonfinite && (am & 0x7F) > Elem<kFmtE2M1>::oas_m7 && b2 != byte;
+      if (__any_sync(kFull, need)) {
+        const OasEval e = oas_eval16(v, byte);
+        const bool up = need && e.delta > 0;   // the lane holds the whole block
+        if (up) byte = b2;
+        codes = up ? e.c2 : e.c1;
+        have = true;
+      }
+    }
+    if (nonfinite) byte = 255;
+    scale = pow2f(byte - 127);
+    if (OP != kOpFakeBwd && !have) codes = nonfinite ? nonfinite_e2m1_16(v) : enc_e2m1_16(scale_slice(v, byte));
+    if (OP != kOpFakeBwd && have && nonfinite) codes = nonfinite_e2m1_16(v);
+  }
+
+  if (OP == kOpQuant) {
+    if (valid) {
+      st_stream8(a.codes + 8 * c, codes);
+      a.scales[scale_offset(a.smap, c)] = static_cast<uint8_t>(byte);
+    }
+    return;
+  }
+  if (OP == kOpFakeBwd) {
+    // |x| <= 6 s (exact in float); nothing passes in a NaN/Inf block
+    const float lim = 6.0f * scale;
+    V16 o;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const bool plo = !nonfinite && fabsf(bf_lo(v.w[i])) <= lim;
+      const bool phi = !nonfinite && fabsf(bf_hi(v.w[i])) <= lim;
+      o.w[i] = (plo ? (g.w[i] & 0xFFFFu) : 0u) | (phi ? (g.w[i] & 0xFFFF0000u) : 0u);
+    }
+    if (valid) st_stream32(a.out + 32 * c, o);
+    return;
+  }
+  // values q * s: exact floats (at most 2 + 4 significant bits)
+  const F16 y = dec_e2m1_16(codes, scale);
+  if (OP == kOpFakeFwd) {
+    V16 o;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      o.w[i] = nonfinite ? ((static_cast<uint32_t>(kNaNbf16) << 16) | kNaNbf16)
+                         : pack_bf16x2(y.v[2 * i], y.v[2 * i + 1]);
+    }
+    if (valid) {
+      st_stream32(a.out + 32 * c, o);
+      if (a.scales) a.scales[scale_offset(a.smap, c)] = static_cast<uint8_t>(byte);
+    }
+    return;
+  }
+  if (OP == kOpError) {
+    // d = x - y exact in float; d^2 summed in double (one lane, one block)
+    double bd = 0.0, bx = 0.0;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const float xf = elem(v, i);
+      const double d = static_cast<double>(xf - y.v[i]);
+      bd = fma(d, d, bd);
+      bx = fma(static_cast<double>(xf), static_cast<double>(xf), bx);
+    }
+    if (nonfinite) bd = __int_as_float(0x7FC00000);
+    if (valid) {
+      if (a.block_sse) a.block_sse[c] = static_cast<float>(bd);
+      sd += bd;
+      sx += bx;
+    }
+  }
+}
+
 // Sum of the per-lane error partials into totals: warp, then CTA (NW warps),
 // then one double atomic per CTA.
 template <int NW = kThreads / 32>
@@ -362,10 +452,14 @@ __global__ void __launch_bounds__(kThreads) stream_kernel(StreamArgs a) {
 #pragma unroll
     for (int j = 0; j < U; ++j) {
       const int64_t c = base + 32 * j;
-      const uint32_t pa = pair_max(amax_bits16(v[j]));
-      int k = 0;
-      if (MBS == kMbsStatic) k = mbs_static_k(oct_max(pa));
-      process_slice<OP, FMT, RULE, MBS>(a, v[j], g[j], c, c < a.nslices, lane, pa, k, sd, sx);
+      if constexpr (FMT == kFmtE2M1B16 || FMT == kFmtNvfp4) {
+        process_slice16<OP, FMT, RULE>(a, v[j], g[j], c, c < a.nslices, sd, sx);
+      } else {
+        const uint32_t pa = pair_max(amax_bits16(v[j]));
+        int k = 0;
+        if (MBS == kMbsStatic) k = mbs_static_k(oct_max(pa));
+        process_slice<OP, FMT, RULE, MBS>(a, v[j], g[j], c, c < a.nslices, lane, pa, k, sd, sx);
+      }
     }
   }
   if (OP == kOpError) reduce_totals(sd, sx, a.totals);
@@ -862,6 +956,9 @@ __global__ void __launch_bounds__(kThreads) dequant_kernel(DequantArgs a) {
   const int lane = threadIdx.x & 31;
   const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+  // E2M1 elements (two per byte), and blocks of 16 (one scale per slice)
+  constexpr bool kPacked = FMT == kFmtE2M1 || FMT == kFmtE2M1B16 || FMT == kFmtNvfp4;
+  constexpr int kSliceShift = (FMT == kFmtE2M1B16 || FMT == kFmtNvfp4) ? 0 : 1;
   for (int64_t tile = warp; tile * 32 * U < a.nslices; tile += nwarps) {
     const int64_t base = tile * 32 * U + lane;
     uint2 c4[U];
@@ -871,9 +968,9 @@ __global__ void __launch_bounds__(kThreads) dequant_kernel(DequantArgs a) {
     for (int j = 0; j < U; ++j) {
       const int64_t c = base + 32 * j;
       const bool valid = c < a.nslices;
-      if (FMT == kFmtE2M1) c4[j] = valid ? ld_stream8(a.codes + 8 * c) : make_uint2(0, 0);
+      if (kPacked) c4[j] = valid ? ld_stream8(a.codes + 8 * c) : make_uint2(0, 0);
       else c8[j] = valid ? ld_stream16(a.codes + 16 * c) : make_uint4(0, 0, 0, 0);
-      sb[j] = valid ? a.scales[scale_offset(a.smap, c >> 1)] : 0;
+      sb[j] = valid ? a.scales[scale_offset(a.smap, c >> kSliceShift)] : 0;
       kk[j] = (valid && a.macro) ? a.macro[c >> 3] : 0;
     }
 #pragma unroll
@@ -881,7 +978,7 @@ __global__ void __launch_bounds__(kThreads) dequant_kernel(DequantArgs a) {
       const int64_t c = base + 32 * j;
       if (c >= a.nslices) continue;
       const int E = sb[j] - 127;
-      if (FMT == kFmtE2M1 && kk[j] == 0 && e2m1_table_scale_ok(sb[j])) {
+      if ((FMT == kFmtE2M1 || FMT == kFmtE2M1B16) && kk[j] == 0 && e2m1_table_scale_ok(sb[j])) {
         // common case: the products are normal bf16 values, read straight off
         // a table of the 8 magnitudes scaled by 2^E (exact)
         const V16 b = e2m1x16_to_bf16(c4[j], e2m1_table(E));
@@ -901,12 +998,20 @@ __global__ void __launch_bounds__(kThreads) dequant_kernel(DequantArgs a) {
         }
         continue;
       }
-      // value * (256 + k) 2^(E-8) (exact); a NaN scale makes every output NaN
-      const float p = kk[j] ? static_cast<float>(256 + kk[j]) * pow2f(E - 8) : pow2f(E);
+      // value * (256 + k) 2^(E-8), or value * s for an NVFP4 scale s (exact);
+      // a NaN scale makes every output NaN
+      float p;
+      bool nan_scale;
+      if constexpr (FMT == kFmtNvfp4) {
+        p = e4m3_value(sb[j]);
+        nan_scale = isnan(p);
+      } else {
+        p = kk[j] ? static_cast<float>(256 + kk[j]) * pow2f(E - 8) : pow2f(E);
+        nan_scale = sb[j] == 255;
+      }
       F16 y;
-      if constexpr (FMT == kFmtE2M1) y = dec_e2m1_16(c4[j], p);
+      if constexpr (kPacked) y = dec_e2m1_16(c4[j], p);
       else y = dec_bytes_16<FMT>(c8[j], p);
-      const bool nan_scale = sb[j] == 255;
       if (OUT32) {
         V16 o0, o1;
 #pragma unroll
@@ -982,7 +1087,7 @@ cudaError_t launch_stream(const StreamArgs& a, cudaStream_t st) {
       if (grid > cap) grid = cap;
     }
     kern<<<static_cast<int>(grid > 0 ? grid : 1), kSweepThreads, 0, st>>>(a);
-  } else if constexpr (OP == kOpQuant && RULE == kOas) {
+  } else if constexpr (OP == kOpQuant && RULE == kOas && FMT != kFmtE2M1B16) {
     constexpr int kTile = (kThreads / 32) * 32 * kUnroll;   // slices per CTA
     const int64_t grid = (a.nslices + kTile - 1) / kTile;
     oas_quant_kernel<FMT, MBS, kUnroll><<<static_cast<int>(grid), kThreads, 0, st>>>(a);
@@ -1009,6 +1114,15 @@ template <int OP>
 cudaError_t dispatch_stream(const StreamArgs& a, int fmt, int scaling, cudaStream_t st) {
   const int rule = scaling & 0xF;
   const int mbs = scaling >> 4;
+  if (fmt == kFmtNvfp4) return launch_stream<OP, kFmtNvfp4, kFloor, kMbsNone>(a, st);
+  if (fmt == kFmtE2M1B16) {
+    switch (rule) {
+      case kFloor: return launch_stream<OP, kFmtE2M1B16, kFloor, kMbsNone>(a, st);
+      case kCeil: return launch_stream<OP, kFmtE2M1B16, kCeil, kMbsNone>(a, st);
+      case kOasRule: return launch_stream<OP, kFmtE2M1B16, kOasRule, kMbsNone>(a, st);
+      default: return launch_stream<OP, kFmtE2M1B16, kOas, kMbsNone>(a, st);
+    }
+  }
   switch (fmt) {
     case kFmtE4M3: return dispatch_bytes<OP, kFmtE4M3>(a, rule, st);
     case kFmtE5M2: return dispatch_bytes<OP, kFmtE5M2>(a, rule, st);
@@ -1113,6 +1227,8 @@ cudaError_t launch_dequantize(const void* codes, const uint8_t* scales, const ui
     }
   } else {
     switch (fmt) {
+      case kFmtE2M1B16: launch_dequant_bytes<kFmtE2M1B16, U>(a, tiles, out_fp32, st); break;
+      case kFmtNvfp4: launch_dequant_bytes<kFmtNvfp4, U>(a, tiles, out_fp32, st); break;
       case kFmtE4M3: launch_dequant_bytes<kFmtE4M3, U>(a, tiles, out_fp32, st); break;
       case kFmtE5M2: launch_dequant_bytes<kFmtE5M2, U>(a, tiles, out_fp32, st); break;
       case kFmtE3M2: launch_dequant_bytes<kFmtE3M2, U>(a, tiles, out_fp32, st); break;

@@ -17,9 +17,10 @@
  *       [5: OAS and MBS generalize to MXFP6 and MXFP8].
  *
  * Layout (every call): x is row-major contiguous [rows, cols] bf16, cols a
- * multiple of 32; block b of row r is elements [32b, 32b+32) of that row.
+ * multiple of 32 (16 for the block-16 formats); block b of row r is elements
+ * [32b, 32b+32) of that row ([16b, 16b+16) for the block-16 formats).
  * A 3-D tensor [E, R, C] is passed as rows = E*R, cols = C.
- *   codes  MXFP4: uint8 [rows, cols/2], element 2j in the low nibble and 2j+1
+ *   codes  MXFP4 (and the block-16 formats): uint8 [rows, cols/2], element 2j in the low nibble and 2j+1
  *                 in the high nibble of byte j; bit 3 of a nibble is the sign.
  *          other formats: uint8 [rows, cols], one code per element (E4M3,
  *                 E5M2, INT8: the whole byte; E3M2 / E2M3: the low 6 bits,
@@ -54,15 +55,24 @@ extern "C" {
 #endif
 
 /* Element formats ([VL] MX format table: MXFP8 E4M3/E5M2, MXFP6 E3M2/E2M3,
- * MXFP4 E2M1, MXINT8 INT8; block 32 and an E8M0 scale for all). emax is the
- * exponent of the largest power of two the element holds. */
+ * MXFP4 E2M1, MXINT8 INT8; block 32 and an E8M0 scale for all), and two
+ * block-16 comparison formats. emax is the exponent of the largest power of
+ * two the element holds. */
 typedef enum {
   MX_FMT_E2M1 = 0, /* MXFP4: magnitudes {0, .5, 1, 1.5, 2, 3, 4, 6} ([UP] 2.A: max 6.0), emax 2 */
   MX_FMT_E4M3 = 1, /* MXFP8: E4M3fn (bias 7, no Inf, S.1111.111 = NaN), max 448, emax 8 */
   MX_FMT_E5M2 = 2, /* MXFP8: E5M2 (bias 15, IEEE Inf/NaN at exponent 31), max 57344, emax 15 */
   MX_FMT_E3M2 = 3, /* MXFP6: E3M2 (bias 3, no Inf/NaN), max 28, emax 4 */
   MX_FMT_E2M3 = 4, /* MXFP6: E2M3 (bias 1, no Inf/NaN), max 7.5, emax 2 */
-  MX_FMT_INT8 = 5  /* MXINT8: two's complement i read as i * 2^-6, |i| <= 127, emax 0 */
+  MX_FMT_INT8 = 5, /* MXINT8: two's complement i read as i * 2^-6, |i| <= 127, emax 0 */
+  /* The two comparison formats of [UP] 1's MXFP4/NVFP4 gap analysis: E2M1
+   * elements in 16-element blocks (cols a multiple of 16; scales
+   * [rows, cols/16]). */
+  MX_FMT_E2M1_B16 = 6, /* MXFP4 at block 16: E8M0 scales, every base rule, no MBS */
+  MX_FMT_NVFP4 = 7     /* E4M3 scale s = amax / 6 rounded to nearest even and saturated
+                        * (no tensor-level scale), elements RNE_sat(x / s); scaling
+                        * MX_SCALE_FLOOR only (the one rule); a zero scale keeps only
+                        * the signs; a NaN/Inf block gets the E4M3 NaN byte 0x7F */
 } mx_format_t;
 
 /* Scale selection. Low 4 bits: the base rule; bits 4-5: Macro Block Scaling.
@@ -101,10 +111,10 @@ typedef enum {
    * mx_fake_quant_fwd (and in mx_dequantize's flags): the E8M0 bytes are
    * written (read) in the tiled layout that block-scaled tensor-core GEMMs
    * on sm_100 consume (the one cuBLASLt's 1-D block-scaling-factor layout
-   * documents) instead of plain [rows, cols/32]. Rows are padded to 128 and
-   * block columns to 4; the scale of row r, block column j sits at byte
+   * documents) instead of plain [rows, cols/block]. Rows are padded to 128
+   * and block columns to 4; the scale of row r, block column j sits at byte
    *   ((r / 128) * T + j / 4) * 512 + (r % 32) * 16 + ((r / 32) % 4) * 4 + j % 4,
-   * T = ceil(cols / 128) tiles per 128-row band. Padding bytes are zero.
+   * T = ceil(cols / (4 * block)) tiles per 128-row band. Padding bytes are zero.
    * mx_scale_bytes gives the buffer size. Macro factors keep their layout. */
   MX_SCALES_MMA = 1 << 8
 } mx_scaling_t;
@@ -127,10 +137,10 @@ typedef enum {
 int mx_quantize(const void* x, int64_t rows, int64_t cols, int format, int scaling,
                 void* codes, uint8_t* scales, uint8_t* macro, void* stream);
 
-/* Bytes of the scale buffer of a [rows, cols] tensor: rows * cols / 32, or
- * the padded size of the MX_SCALES_MMA layout when `scaling` has that flag.
- * -1 for an invalid shape. Host only; no device work. */
-int64_t mx_scale_bytes(int64_t rows, int64_t cols, int scaling);
+/* Bytes of the scale buffer of a [rows, cols] tensor in `format`: rows *
+ * cols / block, or the padded size of the MX_SCALES_MMA layout when `scaling`
+ * has that flag. -1 for an invalid format or shape. Host only. */
+int64_t mx_scale_bytes(int64_t rows, int64_t cols, int format, int scaling);
 
 /* Dequantize: out = value(code) * f * 2^(scale - 127), f = 1 + k/256 from
  * `macro` (NULL means f = 1; FP4 only). out_fp32 (flags): bit 0 clear: bf16

@@ -61,7 +61,9 @@ def test_product_does_not_use_the_oracle():
 
 
 @pytest.mark.parametrize("fmt,scaling,status", [
-    (6, 0, UNSUPPORTED), (0, 4, UNSUPPORTED), (0, 0x30, UNSUPPORTED), (0, 0x40, UNSUPPORTED),
+    (8, 0, UNSUPPORTED), (0, 4, UNSUPPORTED), (0, 0x30, UNSUPPORTED), (0, 0x40, UNSUPPORTED),
+    # block-16 formats: MXFP4-B16 has no MBS, NVFP4 has its one rule
+    (6, 0x10, UNSUPPORTED), (7, 1, UNSUPPORTED), (7, 3, UNSUPPORTED), (7, 0x10, UNSUPPORTED),
     (1, 2, UNSUPPORTED), (1, 0x10, UNSUPPORTED), (0, 0x11, UNSUPPORTED),
     (0, 0x12, UNSUPPORTED), (-1, 0, UNSUPPORTED), (0, -1, UNSUPPORTED),
     # one-byte formats: no OAS_RULE, no macro blocks; INT8 has no OAS
@@ -99,7 +101,9 @@ def test_other_entry_points_validate(mx):
     assert mx.mx_dequantize(A, A, A, 4, 96, 0, 0, A, 0) == SHAPE
     assert mx.mx_dequantize(A, A, A, 4, 128, 1, 0, A, 0) == UNSUPPORTED   # FP8 has no MBS
     assert mx.mx_dequantize(A, A, None, 4, 32, 0, 2, A, 0) == INVALID
-    assert mx.mx_dequantize(A, A, None, 4, 32, 6, 0, A, 0) == UNSUPPORTED
+    assert mx.mx_dequantize(A, A, None, 4, 32, 8, 0, A, 0) == UNSUPPORTED
+    assert mx.mx_dequantize(A, A, None, 4, 24, 7, 0, A, 0) == SHAPE       # NVFP4: cols % 16
+    assert mx.mx_quantize(A, 4, 24, 6, 0, A, A, None, 0) == SHAPE
     assert mx.mx_dequantize(A, A, A, 4, 128, 5, 0, A, 0) == UNSUPPORTED   # only FP4 has MBS
     assert mx.mx_dequantize(A + 8, A, None, 4, 32, 0, 0, A, 0) == ALIGN
     assert mx.mx_dequantize(A, None, None, 4, 32, 0, 0, A, 0) == INVALID
@@ -129,14 +133,16 @@ def test_binding_refuses_cpu_tensors_for_device_only_calls(mx):
 
 
 def test_scale_bytes_and_mma_layout_flag(mx):
-    sb = mx.mx_scale_bytes
     MMA = 1 << 8
+    sb = lambda r, c, s, f=0: mx.mx_scale_bytes(r, c, f, s)
     assert sb(4, 128, 0) == 16
     assert sb(4, 128, MMA) == 128 * 4                  # one 128 x 4 tile
     assert sb(300, 224, MMA) == 384 * 8                # rows -> 384, 7 block columns -> 8
     assert sb(256, 512, MMA | 3) == 256 * 16
     assert sb(0, 64, MMA) == 0
     assert sb(4, 33, MMA) == -1 and sb(-1, 32, 0) == -1
+    assert sb(4, 48, 0, 7) == 12 and sb(4, 48, 0, 1) == -1   # block 16 (NVFP4) vs 32
+    assert sb(4, 48, MMA, 6) == 128 * 4 and sb(4, 32, 0, 8) == -1
     # the flag is accepted by quantize / fake-quant (checked before any launch) ...
     assert mx.mx_quantize(A, 4, 33, 0, MMA, A, A, None, 0) == SHAPE
     assert mx.mx_quantize(None, 0, 32, 1, MMA | 1, None, None, None, 0) == OK

@@ -46,7 +46,7 @@ def test_tiled_scales_are_the_plain_ones_moved(mx, oracle_mod, cuda, shape, fm):
     if (m >> 4) and cols % 128:
         pytest.skip("MBS needs cols % 128 == 0")
     x = inputs.random_bf16_bits((rows, cols), seed=rows + cols).to(cuda)
-    n = mx.mx_scale_bytes(rows, cols, MMA)
+    n = mx.mx_scale_bytes(rows, cols, fmt, MMA)
     # canary-filled buffer: the padding must come back as zeros
     sbuf = torch.full((n,), 0xA5, dtype=torch.uint8, device=cuda)
     codes = torch.empty(rows, cols // 2 if fmt == E2M1 else cols, dtype=torch.uint8, device=cuda)
@@ -107,6 +107,35 @@ def test_mxfp4_tiled_scales_drive_a_block_scaled_gemm(mx, cuda):
                              sa.view(torch.float8_e8m0fnu), sb.view(torch.float8_e8m0fnu))
     ya = mx.dequantize(ca, sa, None, E2M1, torch.float32, mma_scales=True)
     yb = mx.dequantize(cb, sb, None, E2M1, torch.float32, mma_scales=True)
+    torch.cuda.synchronize()
+    ref = ya.double().cpu() @ yb.double().cpu().t()
+    got = out.double().cpu()
+    assert (got - ref).abs().max().item() <= 1e-2 * ref.abs().max().item()
+    assert (got - ref).abs().mean().item() <= 1e-2 * ref.abs().mean().item()
+
+
+def test_nvfp4_tiled_scales_drive_a_block_scaled_gemm(mx, cuda):
+    """NVFP4 (E2M1, block 16, E4M3 scales) through the library's single-level
+    1x16 block-scaled GEMM: checks the encoding and the layout at block 16."""
+    NVFP4 = 7
+    M, N, K = 256, 128, 512
+    a = inputs.normal_weight(M, K, seed=11, device=cuda, std=1.0)
+    b = inputs.normal_weight(N, K, seed=12, device=cuda, std=1.0)
+    ca, sa, _ = mx.quantize(a, NVFP4, FLOOR | MMA)
+    cb, sb, _ = mx.quantize(b, NVFP4, FLOOR | MMA)
+    if not hasattr(torch, "float4_e2m1fn_x2"):
+        pytest.skip("no packed FP4 dtype in this torch")
+    F = torch.nn.functional
+    try:
+        out = F.scaled_mm(ca.view(torch.float4_e2m1fn_x2), cb.view(torch.float4_e2m1fn_x2).t(),
+                          sa.view(torch.float8_e4m3fn), F.ScalingType.BlockWise1x16,
+                          sb.view(torch.float8_e4m3fn), F.ScalingType.BlockWise1x16,
+                          swizzle_a=F.SwizzleType.SWIZZLE_32_4_4,
+                          swizzle_b=F.SwizzleType.SWIZZLE_32_4_4, output_dtype=torch.bfloat16)
+    except (RuntimeError, NotImplementedError, TypeError) as e:
+        pytest.skip(f"NVFP4 scaled_mm unavailable here: {str(e).splitlines()[0][:160]}")
+    ya = mx.dequantize(ca, sa, None, NVFP4, torch.float32, mma_scales=True)
+    yb = mx.dequantize(cb, sb, None, NVFP4, torch.float32, mma_scales=True)
     torch.cuda.synchronize()
     ref = ya.double().cpu() @ yb.double().cpu().t()
     got = out.double().cpu()

@@ -16,16 +16,21 @@ from fp8_quantization_mx_b200 import inputs
 
 pytestmark = pytest.mark.gpu
 
-E2M1, E4M3, E5M2, E3M2, E2M3, INT8 = 0, 1, 2, 3, 4, 5
+E2M1, E4M3, E5M2, E3M2, E2M3, INT8, E2M1_B16, NVFP4 = 0, 1, 2, 3, 4, 5, 6, 7
 FLOOR, CEIL, OAS_RULE, OAS = 0, 1, 2, 3
 MBS_STATIC, MBS_DYNAMIC = 16, 32
 FP4_MODES = [FLOOR, CEIL, OAS_RULE, OAS, MBS_STATIC, MBS_DYNAMIC, OAS | MBS_STATIC, OAS | MBS_DYNAMIC]
 BYTE_FMTS = [E4M3, E5M2, E3M2, E2M3, INT8]
 BYTE_MODES = {E4M3: [FLOOR, CEIL, OAS], E5M2: [FLOOR, CEIL, OAS], E3M2: [FLOOR, CEIL, OAS],
               E2M3: [FLOOR, CEIL, OAS], INT8: [FLOOR, CEIL]}
-ALL = [(E2M1, m) for m in FP4_MODES] + [(f, m) for f in BYTE_FMTS for m in BYTE_MODES[f]]
+B16_MODES = [(E2M1_B16, FLOOR), (E2M1_B16, CEIL), (E2M1_B16, OAS_RULE), (E2M1_B16, OAS), (NVFP4, FLOOR)]
+ALL = ([(E2M1, m) for m in FP4_MODES] + [(f, m) for f in BYTE_FMTS for m in BYTE_MODES[f]] +
+       B16_MODES)
+PACKED = (E2M1, E2M1_B16, NVFP4)
+BLOCK = {f: (16 if f in (E2M1_B16, NVFP4) else 32) for f in range(8)}
 EMAX = {E2M1: 2, E4M3: 8, E5M2: 15, E3M2: 4, E2M3: 2, INT8: 0}
-FMT_NAMES = {E2M1: "fp4", E4M3: "e4m3", E5M2: "e5m2", E3M2: "e3m2", E2M3: "e2m3", INT8: "int8"}
+FMT_NAMES = {E2M1: "fp4", E4M3: "e4m3", E5M2: "e5m2", E3M2: "e3m2", E2M3: "e2m3", INT8: "int8",
+             E2M1_B16: "fp4b16", NVFP4: "nvfp4"}
 REL = 1e-6
 
 
@@ -226,7 +231,7 @@ def test_every_scaled_value_at_several_exponents(mx, oracle_mod, cuda):
     arr = np.concatenate(rows)
     arr = np.concatenate([arr, np.zeros(((-len(arr)) % 64, 32), np.uint16)]).reshape(-1, 2048)
     x = torch.from_numpy(arr.view(np.int16)).view(torch.bfloat16)
-    for fmt in [E2M1] + BYTE_FMTS:
+    for fmt in [E2M1] + BYTE_FMTS + [E2M1_B16, NVFP4]:
         c, s, _ = mx.quantize(x.to(cuda), fmt, FLOOR)
         y = mx.fake_quant(x.to(cuda), fmt, FLOOR)
         torch.cuda.synchronize()
@@ -236,7 +241,7 @@ def test_every_scaled_value_at_several_exponents(mx, oracle_mod, cuda):
         assert np.array_equal(bits(y), oracle_mod.fake_quant_fwd(arr, fmt, FLOOR))
 
 
-@pytest.mark.parametrize("fmt", [E2M1] + BYTE_FMTS)
+@pytest.mark.parametrize("fmt", [E2M1] + BYTE_FMTS + [E2M1_B16, NVFP4])
 @pytest.mark.parametrize("out_fp32", [0, 1])
 @pytest.mark.parametrize("with_macro", [False, True])
 def test_dequantize_every_code_and_scale(mx, oracle_mod, cuda, fmt, out_fp32, with_macro):
@@ -244,9 +249,10 @@ def test_dequantize_every_code_and_scale(mx, oracle_mod, cuda, fmt, out_fp32, wi
         pytest.skip("macro factors are FP4 only")
     rng = np.random.default_rng(23)
     rows, cols = 256, 512
-    scales = np.tile(np.arange(256, dtype=np.uint8)[:, None], (1, cols // 32))
+    # every scale byte in every row (NVFP4: every E4M3 byte, NaN and negative included)
+    scales = np.tile(np.arange(256, dtype=np.uint8)[:, None], (1, cols // BLOCK[fmt]))
     rng.shuffle(scales, axis=1)
-    if fmt == E2M1:
+    if fmt in PACKED:
         codes = rng.integers(0, 256, (rows, cols // 2), dtype=np.uint8)
         codes[:, :8] = np.arange(0, 256, 17, dtype=np.uint8)[None, :8]
     else:
@@ -361,18 +367,19 @@ def test_guard_bands(mx, cuda):
     """Outputs never write outside their extent (canary bytes on both sides)."""
     x = inputs.random_bf16_bits((3, 384), seed=11).to(cuda)
     for fmt, m in ((E2M1, FLOOR), (E2M1, OAS | MBS_DYNAMIC), (E4M3, CEIL), (E5M2, OAS),
-                   (E2M3, OAS), (INT8, FLOOR)):
-        ncode = 3 * 384 // (2 if fmt == E2M1 else 1)
+                   (E2M3, OAS), (INT8, FLOOR), (E2M1_B16, OAS), (NVFP4, FLOOR)):
+        ncode = 3 * 384 // (2 if fmt in PACKED else 1)
+        nsc = 3 * 384 // BLOCK[fmt]
         pad = 256
         cbuf = torch.full((ncode + 2 * pad,), 0xA5, dtype=torch.uint8, device=cuda)
-        sbuf = torch.full((36 + 2 * pad,), 0x5A, dtype=torch.uint8, device=cuda)
+        sbuf = torch.full((nsc + 2 * pad,), 0x5A, dtype=torch.uint8, device=cuda)
         mbuf = torch.full((9 + 2 * pad,), 0x3C, dtype=torch.uint8, device=cuda)
         st = mx.mx_quantize(x.data_ptr(), 3, 384, fmt, m, cbuf[pad:].data_ptr(), sbuf[pad:].data_ptr(),
                             mbuf[pad:].data_ptr(), torch.cuda.current_stream().cuda_stream)
         assert st == 0
         torch.cuda.synchronize()
         assert bool((cbuf[:pad] == 0xA5).all()) and bool((cbuf[pad + ncode:] == 0xA5).all())
-        assert bool((sbuf[:pad] == 0x5A).all()) and bool((sbuf[pad + 36:] == 0x5A).all())
+        assert bool((sbuf[:pad] == 0x5A).all()) and bool((sbuf[pad + nsc:] == 0x5A).all())
         assert bool((mbuf[:pad] == 0x3C).all()) and bool((mbuf[pad + (9 if m >> 4 else 0):] == 0x3C).all())
     y = torch.full((3 * 384 + 512,), 7, dtype=torch.int16, device=cuda)
     st = mx.mx_fake_quant_fwd(x.data_ptr(), 3, 384, E2M1, OAS, y[256:].data_ptr(), None,
@@ -412,3 +419,19 @@ def test_autograd_function(mx, oracle_mod, cuda):
     xb = bits(x.detach())
     assert np.array_equal(bits(y.detach()), oracle_mod.fake_quant_fwd(xb))
     assert np.array_equal(bits(x.grad), oracle_mod.fake_quant_bwd(xb, bits(g)))
+
+
+@pytest.mark.parametrize("fm", [(E2M1_B16, OAS), (NVFP4, FLOOR)], ids=ids)
+def test_full_qat_act_block16(mx, oracle_mod, cuda, fm):
+    fmt, m = fm
+    x = inputs.qat_act(device=cuda)
+    c, s, _ = mx.quantize(x, fmt, m)
+    bs, tot = mx.block_error(x, fmt, m)
+    torch.cuda.synchronize()
+    r = sample_rows(x.shape[0], 32, 5)
+    xs = bits(x[r])
+    oc, os_, _ = oracle_mod.quantize(xs, fmt, m)
+    assert np.array_equal(host_u8(c[r]), oc)
+    assert np.array_equal(host_u8(s[r]), os_)
+    obs, _, _ = oracle_mod.block_error(xs, fmt, m)
+    assert np.allclose(bs[r].cpu().numpy(), obs, rtol=REL, atol=0)
