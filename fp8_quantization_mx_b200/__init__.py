@@ -184,10 +184,15 @@ def quantize(x: torch.Tensor, format: int = E2M1, scaling: int = FLOOR, out=None
     with Macro Block Scaling, else None. ``out`` may supply the three buffers.
     A CPU ``x`` is copied to the current GPU and the outputs come back to the
     CPU: into ``out`` (host tensors) when given, else into new tensors (pinned
-    when ``x`` is pinned). The copies are enqueued on the current stream.
+    when ``x`` is pinned). A pinned ``x`` is moved in row chunks so that its
+    upload, the kernels and the download of earlier chunks overlap (PCIe is
+    full duplex); the current stream waits for all of it, so the call orders
+    like a single kernel on the current stream.
     """
     if not x.is_cuda:
         dev = torch.device("cuda", torch.cuda.current_device())
+        if x.is_pinned() and x.numel() * 2 >= 2 * _CHUNK_BYTES:
+            return _quantize_host_pipelined(x, format, scaling, out, dev)
         xd = x.to(dev, non_blocking=x.is_pinned())
         res = quantize(xd, format, scaling)
         if out is None:
@@ -211,6 +216,73 @@ def quantize(x: torch.Tensor, format: int = E2M1, scaling: int = FLOOR, out=None
         _check(mx_quantize(_ptr(x), rows, cols, format, scaling, _ptr(codes), _ptr(scales),
                            _ptr(macro), _stream(x.device)), "mx_quantize")
     return codes, scales, macro
+
+
+# host <-> device pipelining of quantize on pinned host tensors
+_CHUNK_BYTES = 64 << 20
+_SIDE_STREAMS = {}
+
+
+def _side_streams(dev):
+    if dev.index not in _SIDE_STREAMS:
+        with torch.cuda.device(dev):
+            _SIDE_STREAMS[dev.index] = (torch.cuda.Stream(dev), torch.cuda.Stream(dev))
+    return _SIDE_STREAMS[dev.index]
+
+
+def _quantize_host_pipelined(x, format, scaling, out, dev):
+    rows, cols = _rows_cols(x)
+    lead = x.shape[:-1]
+    mbs = ((scaling >> 4) & 3) != 0
+    mma = (scaling & MMA_SCALES) != 0
+    ccols = cols // 2 if format in _PACKED else cols
+    bs = block_size(format)
+    if out is None:
+        hc = torch.empty(*lead, ccols, dtype=torch.uint8, pin_memory=True)
+        hs = (torch.empty(mx_scale_bytes(rows, cols, format, scaling), dtype=torch.uint8,
+                          pin_memory=True) if mma else
+              torch.empty(*lead, cols // bs, dtype=torch.uint8, pin_memory=True))
+        hm = torch.empty(*lead, cols // 128, dtype=torch.uint8, pin_memory=True) if mbs else None
+    else:
+        hc, hs, hm = out
+    # chunks of whole 128-row bands (tiled scales then stay contiguous per chunk)
+    chunk = max(128, (_CHUNK_BYTES // max(1, cols * 2)) // 128 * 128)
+    with torch.cuda.device(dev):
+        cur = torch.cuda.current_stream(dev)
+        s_in, s_out = _side_streams(dev)
+        xd = torch.empty(rows, cols, dtype=torch.bfloat16, device=dev)
+        cd = torch.empty(rows, ccols, dtype=torch.uint8, device=dev)
+        sd = torch.empty(hs.numel(), dtype=torch.uint8, device=dev)
+        md = torch.empty(rows, cols // 128, dtype=torch.uint8, device=dev) if mbs else None
+        x2, hc2, hs1 = x.reshape(rows, cols), hc.reshape(rows, ccols), hs.reshape(-1)
+        hm2 = hm.reshape(rows, cols // 128) if mbs else None
+        nct = (cols // bs + 3) // 4
+        s_in.wait_stream(cur)
+        s_out.wait_stream(cur)
+        for r0 in range(0, rows, chunk):
+            r1 = min(rows, r0 + chunk)
+            with torch.cuda.stream(s_in):
+                xd[r0:r1].copy_(x2[r0:r1], non_blocking=True)
+            cur.wait_stream(s_in)
+            # scale bytes of rows [r0, r1): a contiguous range in either layout
+            s0 = (r0 // 128) * nct * 512 if mma else r0 * (cols // bs)
+            s1 = s0 + mx_scale_bytes(r1 - r0, cols, format, scaling)
+            _check(mx_quantize(_ptr(xd[r0:r1]), r1 - r0, cols, format, scaling, _ptr(cd[r0:r1]),
+                               _ptr(sd[s0:s1]), _ptr(md[r0:r1]) if mbs else None, cur.cuda_stream),
+                   "mx_quantize")
+            s_out.wait_stream(cur)
+            with torch.cuda.stream(s_out):
+                hc2[r0:r1].copy_(cd[r0:r1], non_blocking=True)
+                hs1[s0:s1].copy_(sd[s0:s1], non_blocking=True)
+                if mbs:
+                    hm2[r0:r1].copy_(md[r0:r1], non_blocking=True)
+        # The device buffers were allocated on the current stream, which now
+        # waits for everything the side streams did with them (and waited for
+        # every upload before the kernels): any later reuse of their memory on
+        # the current stream is ordered after that work, so they need no
+        # record_stream (which would keep the allocator from reusing them).
+        cur.wait_stream(s_out)
+    return hc, hs, hm
 
 
 def _to_host(t: torch.Tensor, pinned: bool) -> torch.Tensor:

@@ -435,3 +435,22 @@ def test_full_qat_act_block16(mx, oracle_mod, cuda, fm):
     assert np.array_equal(host_u8(s[r]), os_)
     obs, _, _ = oracle_mod.block_error(xs, fmt, m)
     assert np.allclose(bs[r].cpu().numpy(), obs, rtol=REL, atol=0)
+
+
+@pytest.mark.parametrize("fm", [(E2M1, FLOOR), (E2M1, OAS | MBS_STATIC), (NVFP4, FLOOR | (1 << 8))],
+                         ids=["fp4-FLOOR", "fp4-OAS+MBS_STATIC", "nvfp4-mma-scales"])
+def test_pinned_host_quantize_is_pipelined_and_identical(mx, cuda, fm):
+    """A pinned host tensor above two chunks goes through the chunked
+    upload / kernel / download pipeline (chunks of 512 and 488 rows here);
+    the result must equal the all-device call bit for bit."""
+    fmt, m = fm
+    x = inputs.random_bf16_bits((1000, 65536), seed=31)
+    xh = x.pin_memory()
+    hc, hs, hm = mx.quantize(xh, fmt, m)
+    torch.cuda.synchronize()
+    dc, ds, dm = mx.quantize(x.to(cuda), fmt, m)
+    torch.cuda.synchronize()
+    assert hc.is_pinned() and hs.is_pinned()
+    assert torch.equal(hc, dc.cpu()) and torch.equal(hs, ds.cpu())
+    if dm is not None:
+        assert torch.equal(hm, dm.cpu())
