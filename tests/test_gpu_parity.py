@@ -454,3 +454,29 @@ def test_pinned_host_quantize_is_pipelined_and_identical(mx, cuda, fm):
     assert torch.equal(hc, dc.cpu()) and torch.equal(hs, ds.cpu())
     if dm is not None:
         assert torch.equal(hm, dm.cpu())
+
+
+def test_more_than_2_31_elements(mx, oracle_mod, cuda):
+    """A tensor past 2^31 elements (4.3 GB of bf16): slice, block and scale
+    indices must not wrap. Rows around element 2^31 and the last rows are
+    checked against the oracle; every block's FLOOR byte against its amax."""
+    rows, cols = 1049088, 2048                       # 2,148,532,224 elements
+    g = torch.Generator(device=cuda).manual_seed(77)
+    x = torch.empty(rows, cols, dtype=torch.bfloat16, device=cuda)
+    x.normal_(generator=g)
+    c, s, _ = mx.quantize(x, E2M1, FLOOR)
+    torch.cuda.synchronize()
+    edge = (1 << 31) // cols                          # the row holding element 2^31
+    r = np.array([0, edge - 1, edge, edge + 1, rows - 2, rows - 1])
+    xs = bits(x[r])
+    oc, os_, _ = oracle_mod.quantize(xs, E2M1, FLOOR)
+    assert np.array_equal(host_u8(c[r]), oc)
+    assert np.array_equal(host_u8(s[r]), os_)
+    amax = x.view(-1, 32).abs().amax(dim=1).view(torch.int16).to(torch.int32)
+    want = torch.clamp((amax >> 7) - 2, min=0).to(torch.uint8)
+    assert torch.equal(s.view(-1), want)
+    del amax, want
+    y = mx.dequantize(c[-4:], s[-4:], None, E2M1)
+    torch.cuda.synchronize()
+    assert np.array_equal(bits(y), oracle_mod.dequantize(host_u8(c[-4:]), host_u8(s[-4:]), None,
+                                                         4, cols, E2M1))
