@@ -462,12 +462,13 @@ BlockResult quantize_block(const double* x, int api_fmt, int rule, double f) {
 // running sum rounds in this fixed order).
 double macro_sse(const double* x, int fmt, int rule, int k) {
   const double f = macro_factor(k);
+  const int bs = block_size(fmt);   // 32, or 16 for MXFP4 at block 16
   double sse = 0.0;
-  for (int b = 0; b < kMacro / kBlock; ++b) {
-    const BlockResult r = quantize_block(x + b * kBlock, fmt, rule, f);
-    for (int i = 0; i < kBlock; ++i) {
-      const double y = element_value(r.codes[i], fmt) * r.X;
-      const double d = x[b * kBlock + i] - y;
+  for (int b = 0; b < kMacro / bs; ++b) {
+    const BlockResult r = quantize_block(x + b * bs, fmt, rule, f);
+    for (int i = 0; i < bs; ++i) {
+      const double y = element_value(r.codes[i], elem_fmt(fmt)) * r.X;
+      const double d = x[b * bs + i] - y;
       sse = sse + d * d;
     }
   }
@@ -494,7 +495,7 @@ int mbs_dynamic_k(const double* x, int fmt, int rule) {
 int macro_k(const double* x, int fmt, int rule, int mbs) {
   if (mbs == 0) return 0;
   if (block_has_nonfinite(x, kMacro)) return 0;
-  return mbs == kMbsStatic ? mbs_static_k(x, kMacro, fmt) : mbs_dynamic_k(x, fmt, rule);
+  return mbs == kMbsStatic ? mbs_static_k(x, kMacro, elem_fmt(fmt)) : mbs_dynamic_k(x, fmt, rule);
 }
 
 // Decoded row of bf16 values.

@@ -175,7 +175,8 @@ def _macro_sse_f64(x, y):
 
 
 @pytest.mark.parametrize("rule", [FLOOR, OAS])
-def test_mbs_dynamic_no_worse_than_static_and_plain(oracle_mod, rule):
+@pytest.mark.parametrize("fmt", [0, 6], ids=["block32", "block16"])
+def test_mbs_dynamic_no_worse_than_static_and_plain(oracle_mod, rule, fmt):
     rng = np.random.default_rng(16)
     x = rng.standard_normal((6, 128 * 8)) * 2.0 ** rng.integers(-10, 10, (6, 1))
     x[:, rng.integers(0, 1024, 12)] *= 30
@@ -183,8 +184,8 @@ def test_mbs_dynamic_no_worse_than_static_and_plain(oracle_mod, rule):
     xf = _bits_to_f64(bits)
     ys = {}
     for m in (rule, rule | MBS_STATIC, rule | MBS_DYNAMIC):
-        c, s, mac = oracle_mod.quantize(bits, 0, m)
-        ys[m] = oracle_mod.dequantize(c, s, mac, 6, 1024, 0, out_fp32=True).view(np.float32).astype(np.float64)
+        c, s, mac = oracle_mod.quantize(bits, fmt, m)
+        ys[m] = oracle_mod.dequantize(c, s, mac, 6, 1024, fmt, out_fp32=True).view(np.float32).astype(np.float64)
     for r in range(6):
         for mb in range(8):
             sl = slice(128 * mb, 128 * mb + 128)
@@ -213,27 +214,30 @@ def _np_floor_log2_over(a, f):
     return np.where(f * 2.0 ** e > a, e - 1, e)
 
 
-def _np_mbs(xm, k):
-    """FLOOR sub-block bytes and the element-order SSE of a macro block for factor k."""
+def _np_mbs(xm, k, bs=32):
+    """FLOOR sub-block bytes and the element-order SSE of a macro block for
+    factor k, with sub-blocks of bs elements (32, or 16 for MXFP4 at block 16)."""
     f = 1 + k / 256
-    blocks = np.abs(xm).reshape(4, 32)
+    blocks = np.abs(xm).reshape(128 // bs, bs)
     amax = blocks.max(axis=1)
     ep = np.where(amax > 0, _np_floor_log2_over(np.where(amax > 0, amax, 1), f), -200)
     E = np.clip(ep - 2, -127, 127)
     X = f * 2.0 ** E
-    codes = _np_round_e2m1(blocks, np.repeat(X[:, None], 32, 1))
+    codes = _np_round_e2m1(blocks, np.repeat(X[:, None], bs, 1))
     y = GRID[codes] * X[:, None]
     return E + 127, _macro_sse_f64(blocks.ravel(), y.ravel())
 
 
-def test_mbs_factors_vs_numpy_restatement(oracle_mod):
+@pytest.mark.parametrize("fmt,bs", [(0, 32), (6, 16)], ids=["block32", "block16"])
+def test_mbs_factors_vs_numpy_restatement(oracle_mod, fmt, bs):
     rng = np.random.default_rng(17)
     x = rng.standard_normal((4, 128 * 6)) * 2.0 ** rng.integers(-6, 6, (4, 1))
     x[:, rng.integers(0, 768, 10)] *= 25
     bits = _to_bf16_bits(x)
     xf = _bits_to_f64(bits)
-    _, s_st, k_st = oracle_mod.quantize(bits, 0, MBS_STATIC)
-    _, s_dy, k_dy = oracle_mod.quantize(bits, 0, MBS_DYNAMIC)
+    nb = 128 // bs
+    _, s_st, k_st = oracle_mod.quantize(bits, fmt, MBS_STATIC)
+    _, s_dy, k_dy = oracle_mod.quantize(bits, fmt, MBS_DYNAMIC)
     for r in range(4):
         for mb in range(6):
             xm = xf[r, 128 * mb:128 * mb + 128]
@@ -246,13 +250,13 @@ def test_mbs_factors_vs_numpy_restatement(oracle_mod):
                 p += 1
             k = next((k for k in range(256) if 6 * (256 + k) * 2.0 ** p >= 256 * A), 0)
             assert int(k_st[r, mb]) == k
-            bytes_st, _ = _np_mbs(xm, k)
-            assert np.array_equal(s_st[r, 4 * mb:4 * mb + 4].astype(int), bytes_st)
+            bytes_st, _ = _np_mbs(xm, k, bs)
+            assert np.array_equal(s_st[r, nb * mb:nb * mb + nb].astype(int), bytes_st)
             # dynamic: argmin over all 256 factors of the element-order SSE
-            sses = [_np_mbs(xm, kk)[1] for kk in range(256)]
+            sses = [_np_mbs(xm, kk, bs)[1] for kk in range(256)]
             kd = int(np.argmin(sses))                  # first minimum = smallest k
             assert int(k_dy[r, mb]) == kd
-            assert np.array_equal(s_dy[r, 4 * mb:4 * mb + 4].astype(int), _np_mbs(xm, kd)[0])
+            assert np.array_equal(s_dy[r, nb * mb:nb * mb + nb].astype(int), _np_mbs(xm, kd, bs)[0])
 
 
 @pytest.mark.parametrize("fmt,rule", [(0, FLOOR), (1, FLOOR), (0, CEIL), (1, CEIL)])
