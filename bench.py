@@ -358,6 +358,8 @@ def other_ops(mx, inputs, dev, reps=10):
              ("fp4", mx.E2M1, "MBS_STATIC", 16), ("fp4", mx.E2M1, "MBS_DYNAMIC", 32),
              ("fp4", mx.E2M1, "OAS+MBS_STATIC", 19), ("fp4", mx.E2M1, "OAS+MBS_DYNAMIC", 35),
              ("fp4b16", mx.E2M1_B16, "FLOOR", 0), ("fp4b16", mx.E2M1_B16, "OAS", 3),
+             ("fp4b16", mx.E2M1_B16, "MBS_STATIC", 16), ("fp4b16", mx.E2M1_B16, "MBS_DYNAMIC", 32),
+             ("fp4b16", mx.E2M1_B16, "OAS+MBS_DYNAMIC", 35),
              ("nvfp4", mx.NVFP4, "FLOOR", 0)]
     for fname, fmt, mname, m in modes:
         bufs = mx.quantize(x4, fmt, m)

@@ -42,7 +42,8 @@ int check_mode(int format, int scaling) {
   const int mbs = scaling >> 4;
   if (rule > MX_SCALE_OAS || mbs > 2) return MX_ERR_UNSUPPORTED;
   if (format == MX_FMT_NVFP4) return scaling == MX_SCALE_FLOOR ? MX_OK : MX_ERR_UNSUPPORTED;
-  if (format == MX_FMT_E2M1_B16) return mbs == 0 ? MX_OK : MX_ERR_UNSUPPORTED;
+  if (format == MX_FMT_E2M1_B16)   // MBS as for MXFP4: over FLOOR or OAS
+    return (mbs == 0 || rule == MX_SCALE_FLOOR || rule == MX_SCALE_OAS) ? MX_OK : MX_ERR_UNSUPPORTED;
   if (format != MX_FMT_E2M1) {
     // one-byte formats: FLOOR, CEIL, and OAS for the float elements
     if (mbs != 0 || rule == MX_SCALE_OAS_RULE) return MX_ERR_UNSUPPORTED;
@@ -128,7 +129,7 @@ int mx_quantize(const void* x, int64_t rows, int64_t cols, int format, int scali
 int mx_dequantize(const void* codes, const uint8_t* scales, const uint8_t* macro, int64_t rows,
                   int64_t cols, int format, int out_fp32, void* out, void* stream) {
   if (!known_format(format)) return MX_ERR_UNSUPPORTED;
-  if (format != MX_FMT_E2M1 && macro) return MX_ERR_UNSUPPORTED;
+  if (format != MX_FMT_E2M1 && format != MX_FMT_E2M1_B16 && macro) return MX_ERR_UNSUPPORTED;
   if ((out_fp32 & ~(1 | MX_SCALES_MMA)) != 0) return MX_ERR_INVALID_ARG;
   const int layout = out_fp32 & MX_SCALES_MMA;
   out_fp32 &= 1;

@@ -316,13 +316,14 @@ __device__ __forceinline__ void process_slice(const StreamArgs& a, const V16& v,
 // The 16-element-block formats (MXFP4 at block 16, NVFP4): a lane's slice
 // is one whole block, so nothing is exchanged between lanes and the block
 // index is the slice index.
-template <int OP, int FMT, int RULE>
+template <int OP, int FMT, int RULE, int MBS>
 __device__ __forceinline__ void process_slice16(const StreamArgs& a, const V16& v, const V16& g,
-                                                int64_t c, bool valid, double& sd, double& sx) {
+                                                int64_t c, bool valid, int lane, int k,
+                                                double& sd, double& sx) {
   const uint32_t am = amax_bits16(v);
   const bool nonfinite = am >= 0x7F80u;
   int byte;
-  float scale;   // the block's scale value (0 leaves only the signs)
+  float scale;   // the block's scale value, f 2^E under MBS (0 leaves only the signs)
   uint2 codes = make_uint2(0, 0);
   if constexpr (FMT == kFmtNvfp4) {
     byte = nvfp4_scale_byte(am);
@@ -330,13 +331,17 @@ __device__ __forceinline__ void process_slice16(const StreamArgs& a, const V16& 
     if (OP != kOpFakeBwd)
       codes = (nonfinite || scale == 0.0f) ? nonfinite_e2m1_16(v) : enc_e2m1_div_16(v, scale);
   } else {
-    byte = rule_byte<kFmtE2M1, RULE>(am);
+    // MXFP4 at block 16: the base rules, or under a macro factor k the
+    // exponent of amax / f (and OAS on x / f), exactly as at block 32
+    byte = MBS == kMbsNone ? rule_byte<kFmtE2M1, RULE>(am) : mbs_byte(am, k, 0);
     bool have = false;
     if constexpr (RULE == kOas) {
-      const int b2 = max(static_cast<int>(am >> 7) - 1, 0);
-      const bool need = !nonfinite && (am & 0x7F) > Elem<kFmtE2M1>::oas_m7 && b2 != byte;
+      const int b2 = MBS == kMbsNone ? max(static_cast<int>(am >> 7) - 1, 0) : mbs_byte(am, k, 1);
+      const bool band = MBS == kMbsNone ? (am & 0x7F) > Elem<kFmtE2M1>::oas_m7
+                                        : mbs_oas_band(am, byte, k);
+      const bool need = !nonfinite && band && b2 != byte;
       if (__any_sync(kFull, need)) {
-        const OasEval e = oas_eval16(v, byte);
+        const OasEval e = MBS == kMbsNone ? oas_eval16(v, byte) : oas_eval_mbs16(v, byte, k);
         const bool up = need && e.delta > 0;   // the lane holds the whole block
         if (up) byte = b2;
         codes = up ? e.c2 : e.c1;
@@ -344,8 +349,12 @@ __device__ __forceinline__ void process_slice16(const StreamArgs& a, const V16& 
       }
     }
     if (nonfinite) byte = 255;
-    scale = pow2f(byte - 127);
-    if (OP != kOpFakeBwd && !have) codes = nonfinite ? nonfinite_e2m1_16(v) : enc_e2m1_16(scale_slice(v, byte));
+    scale = MBS == kMbsNone ? pow2f(byte - 127) : static_cast<float>(256 + k) * pow2f(byte - 127 - 8);
+    if (OP != kOpFakeBwd && !have) {
+      if (nonfinite) codes = nonfinite_e2m1_16(v);
+      else if (MBS == kMbsNone) codes = enc_e2m1_16(scale_slice(v, byte));
+      else codes = enc_mbs_cvt_16(v, byte, k);
+    }
     if (OP != kOpFakeBwd && have && nonfinite) codes = nonfinite_e2m1_16(v);
   }
 
@@ -353,6 +362,7 @@ __device__ __forceinline__ void process_slice16(const StreamArgs& a, const V16& 
     if (valid) {
       st_stream8(a.codes + 8 * c, codes);
       a.scales[scale_offset(a.smap, c)] = static_cast<uint8_t>(byte);
+      if (MBS != kMbsNone && (lane & 7) == 0) a.macro[c >> 3] = static_cast<uint8_t>(k);
     }
     return;
   }
@@ -453,7 +463,10 @@ __global__ void __launch_bounds__(kThreads) stream_kernel(StreamArgs a) {
     for (int j = 0; j < U; ++j) {
       const int64_t c = base + 32 * j;
       if constexpr (FMT == kFmtE2M1B16 || FMT == kFmtNvfp4) {
-        process_slice16<OP, FMT, RULE>(a, v[j], g[j], c, c < a.nslices, sd, sx);
+        int k = 0;
+        // the macro max: over the lane pair, then over the 8 lanes
+        if (MBS == kMbsStatic) k = mbs_static_k(oct_max(pair_max(amax_bits16(v[j]))));
+        process_slice16<OP, FMT, RULE, MBS>(a, v[j], g[j], c, c < a.nslices, lane, k, sd, sx);
       } else {
         const uint32_t pa = pair_max(amax_bits16(v[j]));
         int k = 0;
@@ -571,14 +584,15 @@ __global__ void __launch_bounds__(kThreads) oas_quant_kernel(StreamArgs a) {
 // Sum of squared errors of one 128-element macro block under factor k, in
 // double, in element order: each d is exact in float, d*d exact in double, so
 // the running sum rounds exactly as a sequential double sum does.
-// xs: the 128 magnitudes |x| as floats; amax[4]: sub-block amax bits.
+// xs: the 128 magnitudes |x| as floats; amax[128 / BS]: sub-block amax bits
+// (sub-blocks of BS = 32 elements, or 16 for MXFP4 at block 16).
 // Rounding under f uses the bracket of enc_mbs_cvt_16, 8 elements at a time.
-template <int RULE>
-__device__ __forceinline__ double macro_sse_k(const float* xs, const uint32_t amax[4], int k) {
+template <int RULE, int BS>
+__device__ __forceinline__ double macro_sse_k(const float* xs, const uint32_t* amax, int k) {
   const FactorBracket fb = factor_bracket(k);
   double sse = 0.0;
 #pragma unroll 1
-  for (int b = 0; b < 4; ++b) {
+  for (int b = 0; b < 128 / BS; ++b) {
     int byte = mbs_byte(amax[b], k, 0);
     if (RULE == kOas) {
       const int b2 = mbs_byte(amax[b], k, 1);
@@ -588,11 +602,11 @@ __device__ __forceinline__ double macro_sse_k(const float* xs, const uint32_t am
         const float f2 = fb.f * 2.0f;
         int acc = 0;
 #pragma unroll 1
-        for (int i = 0; i < 32; i += 8) {
+        for (int i = 0; i < BS; i += 8) {
           float s[8], h[8], q1[8], q2[8];
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
-            s[j] = xs[32 * b + i + j] * inv1;
+            s[j] = xs[BS * b + i + j] * inv1;
             h[j] = s[j] * 0.5f;
           }
           e2m1x8_values(mbs_codes8(s, fb.L, fb.H), q1);
@@ -610,10 +624,10 @@ __device__ __forceinline__ double macro_sse_k(const float* xs, const uint32_t am
     const float m = inv_scale_from_byte(byte);                          // 2^-E
     const double p = __longlong_as_double(static_cast<long long>(byte - 127 + 1023) << 52);
 #pragma unroll 1
-    for (int i = 0; i < 32; i += 8) {
+    for (int i = 0; i < BS; i += 8) {
       float s[8], q[8];
 #pragma unroll
-      for (int j = 0; j < 8; ++j) s[j] = xs[32 * b + i + j] * m;
+      for (int j = 0; j < 8; ++j) s[j] = xs[BS * b + i + j] * m;
       e2m1x8_values(mbs_codes8(s, fb.L, fb.H), q);
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
@@ -721,8 +735,8 @@ __device__ __forceinline__ double warp_sum_f64(double v) {
 // The MBS-Dynamic factor of macro block g of this warp (warp-collective).
 // am: the 4 sub-block amax bits (0 for a macro block holding NaN/Inf, whose
 // staged magnitudes are zeros).
-template <int RULE>
-__device__ __forceinline__ int sweep_macro(SweepShared<RULE>& sh, int g, const uint32_t am[4],
+template <int RULE, int BS>
+__device__ __forceinline__ int sweep_macro(SweepShared<RULE>& sh, int g, const uint32_t* am,
                                            int lane) {
   constexpr int NL = SweepShared<RULE>::kLevels;
   double tot[8];
@@ -730,10 +744,11 @@ __device__ __forceinline__ int sweep_macro(SweepShared<RULE>& sh, int g, const u
   for (int j = 0; j < 8; ++j) tot[j] = 0.0;
   const float* xs = sh.xs[g];
 #pragma unroll 1
-  for (int i = 0; i < 4; ++i) {
+  for (int i = 0; i < 128 / BS; ++i) {
     const int ex = static_cast<int>(am[i] >> 7);
     const int K = 2 * static_cast<int>(am[i] & 0x7F);   // regime 0 for k <= K
-    const float xf = xs[32 * i + lane];
+    // one element per lane (16-element sub-blocks: lanes 16..31 add nothing)
+    const float xf = (BS == 32 || lane < 16) ? xs[BS * i + lane] : 0.0f;
     const uint32_t xb = __float_as_uint(xf) >> 16;       // |x| as bf16 bits
     const int exx = static_cast<int>(xb >> 7);
     const int sig = exx ? static_cast<int>(128 | (xb & 0x7F)) : static_cast<int>(xb & 0x7F);
@@ -859,7 +874,7 @@ __device__ __forceinline__ int sweep_macro(SweepShared<RULE>& sh, int g, const u
     const int idx = o + lane;
     if (idx < cnt) {
       const int kc = sh.cand[idx];
-      const double s = macro_sse_k<RULE>(xs, am, kc);
+      const double s = macro_sse_k<RULE, BS>(xs, am, kc);
       if (bk == 256 || s < best || (s == best && kc < bk)) {
         best = s;
         bk = kc;
@@ -879,8 +894,9 @@ __device__ __forceinline__ int sweep_macro(SweepShared<RULE>& sh, int g, const u
   return bk;
 }
 
-template <int OP, int RULE>
+template <int OP, int RULE, int FMT>
 __global__ void __launch_bounds__(kSweepThreads, 4) mbs_sweep_kernel(StreamArgs a) {
+  constexpr int BS = FMT == kFmtE2M1B16 ? 16 : 32;   // sub-block size
   __shared__ __align__(16) SweepShared<RULE> shared[kSweepWarps];
   SweepShared<RULE>& sh = shared[threadIdx.x >> 5];
   const int lane = threadIdx.x & 31;
@@ -898,14 +914,15 @@ __global__ void __launch_bounds__(kSweepThreads, 4) mbs_sweep_kernel(StreamArgs 
   for (int64_t tile = warp; tile * 32 < a.nslices; tile += nwarps) {
     const int64_t c = tile * 32 + lane;
     const bool valid = c < a.nslices;
-    uint32_t pa, A;
+    uint32_t a16, pa, A;
     bool finite;
     {
       V16 v;
 #pragma unroll
       for (int i = 0; i < 8; ++i) v.w[i] = 0;
       if (valid) v = ld_stream32(a.x + 32 * c);
-      pa = pair_max(amax_bits16(v));
+      a16 = amax_bits16(v);
+      pa = pair_max(a16);
       A = oct_max(pa);
       finite = A < 0x7F80u;
       __syncwarp();   // the previous tile's reads of xs are done
@@ -917,13 +934,14 @@ __global__ void __launch_bounds__(kSweepThreads, 4) mbs_sweep_kernel(StreamArgs 
 #pragma unroll 1
     for (int gg = 0; gg < 4; ++gg) {
       const bool fin_g = __shfl_sync(kFull, A, gg << 3) < 0x7F80u;
-      uint32_t am[4];
+      uint32_t am[128 / BS];
 #pragma unroll
-      for (int b = 0; b < 4; ++b) {
-        const uint32_t ab = __shfl_sync(kFull, pa, (gg << 3) + 2 * b);
+      for (int b = 0; b < 128 / BS; ++b) {
+        const uint32_t ab = BS == 32 ? __shfl_sync(kFull, pa, (gg << 3) + 2 * b)
+                                     : __shfl_sync(kFull, a16, (gg << 3) + b);
         am[b] = fin_g ? ab : 0u;
       }
-      const int kg = sweep_macro<RULE>(sh, gg, am, lane);
+      const int kg = sweep_macro<RULE, BS>(sh, gg, am, lane);
       if (gg == grp) k = kg;
     }
     if (!finite) k = 0;
@@ -935,7 +953,10 @@ __global__ void __launch_bounds__(kSweepThreads, 4) mbs_sweep_kernel(StreamArgs 
       v = ld_stream32(a.x + 32 * c);
       if (OP == kOpFakeBwd) g = ld_stream32(a.gy + 32 * c);
     }
-    process_slice<OP, kFmtE2M1, RULE, kMbsDynamic>(a, v, g, c, valid, lane, pa, k, sd, sx);
+    if constexpr (BS == 32)
+      process_slice<OP, kFmtE2M1, RULE, kMbsDynamic>(a, v, g, c, valid, lane, pa, k, sd, sx);
+    else
+      process_slice16<OP, kFmtE2M1B16, RULE, kMbsDynamic>(a, v, g, c, valid, lane, k, sd, sx);
   }
   if (OP == kOpError) reduce_totals<kSweepWarps>(sd, sx, a.totals);
 }
@@ -1077,7 +1098,7 @@ cudaError_t launch_stream(const StreamArgs& a, cudaStream_t st) {
   // the error kernel ends with one double atomic per CTA: keep its grid small
   const int waves = OP == kOpError ? 1 : MX_GRID_WAVES;
   if constexpr (MBS == kMbsDynamic) {
-    auto kern = mbs_sweep_kernel<OP, RULE>;
+    auto kern = mbs_sweep_kernel<OP, RULE, FMT>;
     const int64_t tiles = (a.nslices + 31) / 32;
     int64_t grid = (tiles + kSweepWarps - 1) / kSweepWarps;
     if (OP == kOpError) {
@@ -1116,6 +1137,15 @@ cudaError_t dispatch_stream(const StreamArgs& a, int fmt, int scaling, cudaStrea
   const int mbs = scaling >> 4;
   if (fmt == kFmtNvfp4) return launch_stream<OP, kFmtNvfp4, kFloor, kMbsNone>(a, st);
   if (fmt == kFmtE2M1B16) {
+    const int mbs = scaling >> 4;
+    if (mbs == kMbsStatic) {
+      if (rule == kFloor) return launch_stream<OP, kFmtE2M1B16, kFloor, kMbsStatic>(a, st);
+      return launch_stream<OP, kFmtE2M1B16, kOas, kMbsStatic>(a, st);
+    }
+    if (mbs == kMbsDynamic) {
+      if (rule == kFloor) return launch_stream<OP, kFmtE2M1B16, kFloor, kMbsDynamic>(a, st);
+      return launch_stream<OP, kFmtE2M1B16, kOas, kMbsDynamic>(a, st);
+    }
     switch (rule) {
       case kFloor: return launch_stream<OP, kFmtE2M1B16, kFloor, kMbsNone>(a, st);
       case kCeil: return launch_stream<OP, kFmtE2M1B16, kCeil, kMbsNone>(a, st);

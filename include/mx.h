@@ -68,7 +68,9 @@ typedef enum {
   /* The two comparison formats of [UP] 1's MXFP4/NVFP4 gap analysis: E2M1
    * elements in 16-element blocks (cols a multiple of 16; scales
    * [rows, cols/16]). */
-  MX_FMT_E2M1_B16 = 6, /* MXFP4 at block 16: E8M0 scales, every base rule, no MBS */
+  MX_FMT_E2M1_B16 = 6, /* MXFP4 at block 16: E8M0 scales, every base rule; MBS over the eight
+                        * 16-element sub-blocks of each 128-element macro block ([UP] 2.B's
+                        * 1x16 base blocks) */
   MX_FMT_NVFP4 = 7     /* E4M3 scale s = amax / 6 rounded to nearest even and saturated
                         * (no tensor-level scale), elements RNE_sat(x / s); scaling
                         * MX_SCALE_FLOOR only (the one rule); a zero scale keeps only

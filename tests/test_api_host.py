@@ -63,7 +63,8 @@ def test_product_does_not_use_the_oracle():
 @pytest.mark.parametrize("fmt,scaling,status", [
     (8, 0, UNSUPPORTED), (0, 4, UNSUPPORTED), (0, 0x30, UNSUPPORTED), (0, 0x40, UNSUPPORTED),
     # block-16 formats: MXFP4-B16 has no MBS, NVFP4 has its one rule
-    (6, 0x10, UNSUPPORTED), (7, 1, UNSUPPORTED), (7, 3, UNSUPPORTED), (7, 0x10, UNSUPPORTED),
+    (6, 0x11, UNSUPPORTED), (6, 0x12, UNSUPPORTED), (7, 1, UNSUPPORTED), (7, 3, UNSUPPORTED),
+    (7, 0x10, UNSUPPORTED),
     (1, 2, UNSUPPORTED), (1, 0x10, UNSUPPORTED), (0, 0x11, UNSUPPORTED),
     (0, 0x12, UNSUPPORTED), (-1, 0, UNSUPPORTED), (0, -1, UNSUPPORTED),
     # one-byte formats: no OAS_RULE, no macro blocks; INT8 has no OAS

@@ -23,7 +23,9 @@ FP4_MODES = [FLOOR, CEIL, OAS_RULE, OAS, MBS_STATIC, MBS_DYNAMIC, OAS | MBS_STAT
 BYTE_FMTS = [E4M3, E5M2, E3M2, E2M3, INT8]
 BYTE_MODES = {E4M3: [FLOOR, CEIL, OAS], E5M2: [FLOOR, CEIL, OAS], E3M2: [FLOOR, CEIL, OAS],
               E2M3: [FLOOR, CEIL, OAS], INT8: [FLOOR, CEIL]}
-B16_MODES = [(E2M1_B16, FLOOR), (E2M1_B16, CEIL), (E2M1_B16, OAS_RULE), (E2M1_B16, OAS), (NVFP4, FLOOR)]
+B16_MODES = [(E2M1_B16, FLOOR), (E2M1_B16, CEIL), (E2M1_B16, OAS_RULE), (E2M1_B16, OAS),
+             (E2M1_B16, MBS_STATIC), (E2M1_B16, MBS_DYNAMIC), (E2M1_B16, OAS | MBS_STATIC),
+             (E2M1_B16, OAS | MBS_DYNAMIC), (NVFP4, FLOOR)]
 ALL = ([(E2M1, m) for m in FP4_MODES] + [(f, m) for f in BYTE_FMTS for m in BYTE_MODES[f]] +
        B16_MODES)
 PACKED = (E2M1, E2M1_B16, NVFP4)
@@ -245,8 +247,8 @@ def test_every_scaled_value_at_several_exponents(mx, oracle_mod, cuda):
 @pytest.mark.parametrize("out_fp32", [0, 1])
 @pytest.mark.parametrize("with_macro", [False, True])
 def test_dequantize_every_code_and_scale(mx, oracle_mod, cuda, fmt, out_fp32, with_macro):
-    if fmt != E2M1 and with_macro:
-        pytest.skip("macro factors are FP4 only")
+    if fmt not in (E2M1, E2M1_B16) and with_macro:
+        pytest.skip("macro factors are MXFP4 only")
     rng = np.random.default_rng(23)
     rows, cols = 256, 512
     # every scale byte in every row (NVFP4: every E4M3 byte, NaN and negative included)
