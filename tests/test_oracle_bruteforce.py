@@ -314,3 +314,56 @@ def test_block_error_consistent_with_dequantize(oracle_mod):
         d2 = ((xf - y) ** 2).reshape(25, 32, 32).sum(-1)
         assert np.allclose(bs, d2, rtol=1e-12, atol=0)
         assert np.isclose(sd, d2.sum(), rtol=1e-12) and np.isclose(sx, (xf ** 2).sum(), rtol=1e-12)
+
+
+# ------------------------------------------------ 10^5 blocks, vectorised --
+
+def _sse_at(xf, E):
+    """Per-block SSE with codes from ml_dtypes at per-block exponents E (float64;
+    each d and d^2 is exact, the 32-term sums round at most slightly)."""
+    X = 2.0 ** E[:, None]
+    with np.errstate(over="ignore"):
+        q = (xf / X).astype(np.float32).astype(ml_dtypes.float4_e2m1fn).astype(np.float64)
+    return ((xf - q * X) ** 2).sum(axis=1)
+
+
+def test_bruteforce_1e5_blocks(oracle_mod):
+    """10^5 seeded blocks (Gaussian, heavy-tailed, amax on powers of two, on
+    grid points and midpoints, in the OAS band): FLOOR/CEIL/OAS_RULE bytes by
+    their closed forms; OAS is the exact argmin over {e-2, e-1}; exponents
+    >= e never beat e-1; OAS <= OAS_RULE <= CEIL and OAS <= FLOOR. Exact
+    rationals settle every comparison closer than 1e-9."""
+    bits = random_blocks(100_000, 31)
+    xf = _bits_to_f64(bits)
+    amax = np.abs(xf).max(axis=1)
+    e = np.frexp(amax)[1] - 1
+    ok = (amax > 0) & (e - 2 >= -126) & (e + 3 <= 127)
+    xf, bits, e, amax = xf[ok], bits[ok], e[ok], amax[ok]
+    assert len(xf) > 90_000
+    s = {m: oracle_mod.quantize(bits, 0, m)[1][:, 0].astype(int) - 127
+         for m in (FLOOR, CEIL, OAS_RULE, OAS)}
+    assert np.array_equal(s[FLOOR], e - 2)
+    Ec = np.where(amax <= 6 * 2.0 ** (e - 2), e - 2, e - 1)
+    assert np.array_equal(s[CEIL], Ec)
+    nrm = amax / 2.0 ** Ec
+    assert np.array_equal(s[OAS_RULE], np.where((nrm > 3) & (nrm <= 3.5), Ec - 1, Ec))
+
+    s1, s2 = _sse_at(xf, e - 2), _sse_at(xf, e - 1)
+    close = np.abs(s1 - s2) <= 1e-9 * np.maximum(s1, s2)
+    want = np.where(s2 < s1, e - 1, e - 2)
+    for i in np.nonzero(close)[0]:        # near ties: decide exactly
+        a = exact_sse(xf[i], e2m1_values_lib(xf[i], e[i] - 2))
+        b = exact_sse(xf[i], e2m1_values_lib(xf[i], e[i] - 1))
+        want[i] = e[i] - 1 if b < a else e[i] - 2
+    assert np.array_equal(s[OAS], want)
+
+    for d in range(1, 6):                 # exponents e .. e+4 never beat e-1
+        sd = _sse_at(xf, e - 1 + d)
+        worse = sd < s2 * (1 - 1e-9)
+        assert not worse.any()
+
+    sse = {m: _sse_at(xf, s[m]) for m in s}
+    tol = 1e-9 * sse[CEIL]
+    assert np.all(sse[OAS] <= sse[OAS_RULE] + tol)
+    assert np.all(sse[OAS_RULE] <= sse[CEIL] + tol)
+    assert np.all(sse[OAS] <= sse[FLOOR] + tol)
