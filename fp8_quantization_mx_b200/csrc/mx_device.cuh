@@ -236,12 +236,6 @@ __device__ __forceinline__ V16 scale_slice(const V16& x, int b) {
 __device__ __forceinline__ uint2 enc_e2m1_16(const V16& s) {
   return make_uint2(cvt_e2m1x8(&s.w[0]), cvt_e2m1x8(&s.w[4]));
 }
-// 16 E4M3 bytes of a scaled slice: byte i = element i.
-__device__ __forceinline__ uint4 enc_e4m3_16(const V16& s) {
-  const uint2 a = cvt_e4m3x8(&s.w[0]);
-  const uint2 b = cvt_e4m3x8(&s.w[4]);
-  return make_uint4(a.x, a.y, b.x, b.y);
-}
 
 // Codes of a block holding NaN/Inf: E2M1 has no NaN, so only the sign
 // survives; E4M3 elements become S.1111.111, the NaN code.

@@ -74,3 +74,38 @@ def test_two_rank_shards_match_whole_tensor(oracle_mod, scaling):
             assert np.array_equal(m, m_full[r0:r1])
     assert sum(p[1] - p[0] for p in parts) == 37
     assert t == [2.0, 0.0]
+
+
+def _err_worker(rank, world, port, x_bits, scaling, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    import oracle
+    from fp8_quantization_mx_b200.sharding import global_error_stats
+    r0, r1 = shard_rows(x_bits.shape[0], world, rank)
+    _, sd, sx = oracle.block_error(np.ascontiguousarray(x_bits[r0:r1]), 0, scaling, want_blocks=False)
+    mse, sqnr = global_error_stats((sd, sx), (r1 - r0) * x_bits.shape[1])
+    out.put((rank, mse, sqnr))
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_sharded_error_stats_equal_the_whole_tensor(oracle_mod, world):
+    """The one exchange on the path: each rank's {sum d^2, sum x^2, n}
+    all-reduced gives the whole tensor's MSE and SQNR."""
+    from fp8_quantization_mx_b200 import inputs
+    x = inputs.bf16_bits_numpy(inputs.heavy_tail(rows=41, cols=512, seed=10))
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_err_worker, args=(r, world, port, x, 3, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    res = [q.get(timeout=120) for _ in range(world)]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    _, sd, sx = oracle_mod.block_error(x, 0, 3, want_blocks=False)
+    mse_full, sqnr_full = sd / x.size, 10 * np.log10(sx / sd)
+    for _, mse, sqnr in res:
+        assert np.isclose(mse, mse_full, rtol=1e-12) and np.isclose(sqnr, sqnr_full, rtol=1e-12)
