@@ -261,6 +261,7 @@ def stack_ops(mx, x, reps=50, only=None):
                                                             out=(c4, sc, mac)), fp4m),
         "fp4_fake_quant_fwd": (lambda: mx.fake_quant(x, out=y), n * 4),
         "fp4_fake_quant_bwd": (lambda: mx.fake_quant_bwd(x, g, out=y), n * 6),
+        "fp4_oas_fake_quant_fwd": (lambda: mx.fake_quant(x, mx.E2M1, mx.OAS, out=y), n * 4),
         "fp4_dequantize_bf16": (lambda: mx.dequantize(c4, sc, None, mx.E2M1, out=y), fp4),
         "fp8_dequantize_bf16": (lambda: mx.dequantize(c8, sc, None, mx.E4M3, out=y), fp8),
         "fp4_block_error": (lambda: mx.block_error(x, per_block=False), n * 2),

@@ -490,8 +490,52 @@ __global__ void __launch_bounds__(kThreads) stream_kernel(StreamArgs a) {
 // block and full warps, re-reading their 64 bytes (just loaded, so from L2).
 // Without the split every warp that holds one such block pays for the exact
 // SSE comparison on all of its lanes.
-template <int FMT, int MBS, int U>
-__global__ void __launch_bounds__(kThreads) oas_quant_kernel(StreamArgs a) {
+// Output of one lane's slice once its block's codes and scale byte are
+// decided: the codes (quantize) or the dequantized bf16 values (fake-quant
+// forward), and the scale byte (quantize; fake-quant when asked for). The
+// even lane of the block's lane pair writes the byte.
+template <int OP, int FMT, int MBS>
+__device__ __forceinline__ void emit_slice(const StreamArgs& a, int64_t c, int lane, uint4 codes,
+                                           int byte, int k, bool nonfinite) {
+  if constexpr (OP == kOpQuant) {
+    if (FMT == kFmtE2M1) st_stream8(a.codes + 8 * c, make_uint2(codes.x, codes.y));
+    else st_stream16(a.codes + 16 * c, codes);
+  } else {
+    V16 o;
+    if (nonfinite) {
+#pragma unroll
+      for (int i = 0; i < 8; ++i) o.w[i] = (static_cast<uint32_t>(kNaNbf16) << 16) | kNaNbf16;
+    } else if (FMT == kFmtE2M1 && MBS == kMbsNone && e2m1_table_scale_ok(byte)) {
+      o = e2m1x16_to_bf16(make_uint2(codes.x, codes.y), e2m1_table(byte - 127));
+    } else {
+      BlockScale s;
+      s.byte = byte;
+      s.k = k;
+      s.nonfinite = false;
+      s.have_codes = true;
+      s.codes = codes;
+      const F16 y = block_values<FMT, MBS>(codes, s);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) o.w[i] = pack_bf16x2(y.v[2 * i], y.v[2 * i + 1]);
+    }
+    st_stream32(a.out + 32 * c, o);
+  }
+  if ((OP == kOpQuant || a.scales) && (lane & 1) == 0)
+    a.scales[scale_offset(a.smap, c >> 1)] = static_cast<uint8_t>(byte);
+}
+
+// OAS quantize and fake-quant forward in two phases per CTA tile: MXFP4
+// without MBS or with MBS-Static, and the one-byte float formats. Phase 1
+// handles every block whose finer exponent is already the answer (scaled
+// max inside the band of Elem<FMT>::oas_m7 -- under MBS: at most 7f --, the
+// two candidates equal, or NaN/Inf) exactly as the single-rule kernel does,
+// and appends the other blocks (a fifth or fewer for Gaussian data) to a
+// shared-memory list, with their macro factor. Phase 2 evaluates only the
+// listed blocks, two lanes per block and full warps, re-reading their 64
+// bytes (just loaded, so from L2). Without the split every warp that holds
+// one such block pays for the exact SSE comparison on all of its lanes.
+template <int OP, int FMT, int MBS, int U>
+__global__ void __launch_bounds__(kThreads) oas_kernel(StreamArgs a) {
   constexpr int kWarps = kThreads / 32;
   constexpr int kTileSlices = kWarps * 32 * U;
   // listed blocks: first-slice offset in the low 16 bits, macro k above
@@ -532,19 +576,20 @@ __global__ void __launch_bounds__(kThreads) oas_quant_kernel(StreamArgs a) {
     }
     const bool need = valid && !nonfinite && band && b2 != b1;
     if (valid && !need) {
+      uint4 codes;
       if constexpr (FMT == kFmtE2M1) {
-        uint2 codes;
-        if (nonfinite) codes = nonfinite_e2m1_16(v[j]);
-        else if (MBS == kMbsNone) codes = enc_e2m1_16(scale_slice(v[j], b1));
-        else codes = enc_mbs_cvt_16(v[j], b1, k);
-        st_stream8(a.codes + 8 * c, codes);
+        uint2 c2;
+        if (nonfinite) c2 = nonfinite_e2m1_16(v[j]);
+        else if (MBS == kMbsNone) c2 = enc_e2m1_16(scale_slice(v[j], b1));
+        else c2 = enc_mbs_cvt_16(v[j], b1, k);
+        codes = make_uint4(c2.x, c2.y, 0, 0);
       } else {
-        st_stream16(a.codes + 16 * c, nonfinite ? nonfinite_bytes_16<FMT>(v[j])
-                                                : enc_bytes_16<FMT>(scale_slice(v[j], b1)));
+        codes = nonfinite ? nonfinite_bytes_16<FMT>(v[j]) : enc_bytes_16<FMT>(scale_slice(v[j], b1));
       }
-      if ((lane & 1) == 0) a.scales[scale_offset(a.smap, c >> 1)] = static_cast<uint8_t>(nonfinite ? 255 : b1);
+      emit_slice<OP, FMT, MBS>(a, c, lane, codes, nonfinite ? 255 : b1, k, nonfinite);
     }
-    if (MBS != kMbsNone && valid && (lane & 7) == 0) a.macro[c >> 3] = static_cast<uint8_t>(k);
+    if (OP == kOpQuant && MBS != kMbsNone && valid && (lane & 7) == 0)
+      a.macro[c >> 3] = static_cast<uint8_t>(k);
     if (need && (lane & 1) == 0)
       list[atomicAdd(&count, 1)] = static_cast<uint32_t>(c - tile0) | (static_cast<uint32_t>(k) << 16);
   }
@@ -564,18 +609,19 @@ __global__ void __launch_bounds__(kThreads) oas_quant_kernel(StreamArgs a) {
     if (has) x = ld_stream32(a.x + 32 * c);
     const uint32_t pa = pair_max(amax_bits16(x));
     const int b1 = MBS == kMbsNone ? rule_byte<FMT, kFloor>(pa) : mbs_byte(pa, k, 0);
+    uint4 codes;
+    bool up;
     if constexpr (FMT == kFmtE2M1) {
       const OasEval e = MBS == kMbsNone ? oas_eval16(x, b1) : oas_eval_mbs16(x, b1, k);
-      const int d = e.delta + __shfl_xor_sync(kFull, e.delta, 1);
-      const bool up = d > 0;
-      if (has) st_stream8(a.codes + 8 * c, up ? e.c2 : e.c1);
-      if (has && (lane & 1) == 0) a.scales[scale_offset(a.smap, c >> 1)] = static_cast<uint8_t>(up ? b1 + 1 : b1);
+      up = e.delta + __shfl_xor_sync(kFull, e.delta, 1) > 0;
+      const uint2 c2 = up ? e.c2 : e.c1;
+      codes = make_uint4(c2.x, c2.y, 0, 0);
     } else {
       const OasEvalBytes e = oas_eval_bytes16<FMT>(x, b1);
-      const bool up = pair_sum_i128(e.delta) > 0;
-      if (has) st_stream16(a.codes + 16 * c, up ? e.c2 : e.c1);
-      if (has && (lane & 1) == 0) a.scales[scale_offset(a.smap, c >> 1)] = static_cast<uint8_t>(up ? b1 + 1 : b1);
+      up = pair_sum_i128(e.delta) > 0;
+      codes = up ? e.c2 : e.c1;
     }
+    if (has) emit_slice<OP, FMT, MBS>(a, c, lane, codes, up ? b1 + 1 : b1, k, false);
   }
 }
 
@@ -1108,10 +1154,10 @@ cudaError_t launch_stream(const StreamArgs& a, cudaStream_t st) {
       if (grid > cap) grid = cap;
     }
     kern<<<static_cast<int>(grid > 0 ? grid : 1), kSweepThreads, 0, st>>>(a);
-  } else if constexpr (OP == kOpQuant && RULE == kOas && FMT != kFmtE2M1B16) {
+  } else if constexpr ((OP == kOpQuant || OP == kOpFakeFwd) && RULE == kOas && FMT != kFmtE2M1B16) {
     constexpr int kTile = (kThreads / 32) * 32 * kUnroll;   // slices per CTA
     const int64_t grid = (a.nslices + kTile - 1) / kTile;
-    oas_quant_kernel<FMT, MBS, kUnroll><<<static_cast<int>(grid), kThreads, 0, st>>>(a);
+    oas_kernel<OP, FMT, MBS, kUnroll><<<static_cast<int>(grid), kThreads, 0, st>>>(a);
   } else {
     constexpr int U = (MBS == kMbsNone) ? kUnroll : 1;
     auto kern = stream_kernel<OP, FMT, RULE, MBS, U>;
