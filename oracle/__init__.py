@@ -72,6 +72,8 @@ def _load():
     lib.oracle_fake_quant_fwd.argtypes = [u16p, i64, i64, c_int, c_int, u16p, u8p]
     lib.oracle_fake_quant_bwd.argtypes = [u16p, u16p, i64, i64, c_int, c_int, u16p]
     lib.oracle_block_error.argtypes = [u16p, i64, i64, c_int, c_int, dp, dp]
+    fp = ctypes.POINTER(ctypes.c_float)
+    lib.oracle_bat_apply.argtypes = [u16p, i64, i64, c_int, fp, fp, fp, fp, u16p, fp]
     _lib = lib
     return lib
 
@@ -220,3 +222,38 @@ def block_error(x, fmt: int = E2M1, scaling: int = FLOOR, want_blocks: bool = Tr
     if bs is not None:
         bs = bs.reshape(*x.shape[:-1], cols // block_size(fmt))
     return bs, float(totals[0]), float(totals[1])
+
+
+def bat_apply(x, a: int, A, B, beta_min=None, beta_max=None, want_f32: bool = False):
+    """BATQuant apply step: y = x diag(B_j (x) A) per 32-element block, clipped
+    to [beta_min_j min y, beta_max_j max y], rounded to bf16. A: [a, a]
+    float32; B: [cols/32, b, b] float32 (b = 32 / a); beta_*: [cols/32] float32
+    or both None. Returns the bf16 bits (and the fp32 values if asked)."""
+    x = _bf16(x)
+    rows, cols = _shape(x)
+    assert a in (1, 2, 4, 8, 16, 32)
+    b = 32 // a
+    A = np.ascontiguousarray(A, dtype=np.float32)
+    B = np.ascontiguousarray(B, dtype=np.float32)
+    assert A.shape == (a, a) and B.shape == (cols // 32, b, b)
+    assert (beta_min is None) == (beta_max is None), "both clip thresholds or neither"
+    if beta_min is not None:
+        beta_min = np.ascontiguousarray(beta_min, dtype=np.float32)
+        beta_max = np.ascontiguousarray(beta_max, dtype=np.float32)
+        assert beta_min.shape == beta_max.shape == (cols // 32,)
+    y = np.zeros(rows * cols, np.uint16)
+    yf = np.zeros(rows * cols, np.float32) if want_f32 else None
+    fp = ctypes.c_float
+    _load().oracle_bat_apply(_ptr(x, ctypes.c_uint16), rows, cols, int(a), _ptr(A, fp), _ptr(B, fp),
+                             _ptr(beta_min, fp), _ptr(beta_max, fp), _ptr(y, ctypes.c_uint16),
+                             _ptr(yf, fp))
+    y = y.reshape(x.shape)
+    if want_f32:
+        return y, yf.reshape(x.shape)
+    return y
+
+
+def bat_quantize(x, a: int, A, B, beta_min=None, beta_max=None, fmt: int = E2M1,
+                 scaling: int = FLOOR):
+    """BATQuant: the apply step, then MX quantization of its bf16 result."""
+    return quantize(bat_apply(x, a, A, B, beta_min, beta_max), fmt, scaling)

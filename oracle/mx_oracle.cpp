@@ -28,6 +28,12 @@
 //        Scaling (a 1x128 macro block with an 8-bit-mantissa factor; Static =
 //        cheap approximation, Dynamic = LUT search for minimum SSE), sections 3-4
 //        (QSNR as the error figure).
+//  [BQ]  "BATQuant: Outlier-resilient MXFP4 Quantization via Learnable
+//        Block-wise Optimization", technical summary section 2 (methodology):
+//        (a) a block-diagonal affine transform whose blocks match the MX block
+//        (32 elements), (b) each block's matrix the Kronecker product of a
+//        block-private matrix B_j and a globally shared matrix A (GPK),
+//        (c) block-wise learnable clipping thresholds beta^min, beta^max.
 //  The scale rule 2^(floor(log2 amax) - emax) and round-to-nearest-even with
 //  saturation are the OCP Microscaling definition that [AX] and [VL] point to.
 //
@@ -562,6 +568,72 @@ double dequant_value(int code, int scale_byte, int k, int fmt) {
   return element_value(code, elem_fmt(fmt)) * macro_factor(k) * decode_e8m0(scale_byte);
 }
 
+// ------------------------------------------------------------- BATQuant --
+//
+// [BQ] section 2: the activation row x is multiplied on the right by the
+// block-diagonal matrix diag(P_0, P_1, ...), one 32x32 block P_j per MX
+// block j of the row, with P_j = B_j (x) A: A is a x a and shared by every
+// block, B_j is b x b and private to column block j, a * b = 32. Indexing
+// the block's 32 elements as i = p * a + q (p < b, q < a), the Kronecker
+// entry is P_j[p*a+q][r*a+s] = B_j[p][r] * A[q][s], so
+//   y[r*a+s] = sum_p B_j[p][r] * Z[p][s],  Z[p][s] = sum_q x[p*a+q] * A[q][s]
+// (the two small products the decomposition exists for). The block's values
+// are then clipped to [beta^min_j * min(y), beta^max_j * max(y)] and the
+// result, rounded to bf16, is what the MX quantizer sees.
+//
+// Readings (the pages fix neither precision nor order): fp32 arithmetic,
+// each sum an fma chain in ascending index order starting from -0 (so a
+// one-term sum is the rounded product), except that a sum whose index runs
+// over both 16-element halves of the block is the fp32 sum of the chains of
+// the two halves (lower half + upper half). That is the stage-2 sum for
+// b >= 2 and the stage-1 sum for a = 32. The clip is t = y < lo ? lo : y,
+// then t > hi ? hi : t, with lo = fl(beta^min * min y), hi = fl(beta^max *
+// max y); a block whose transformed values are not all finite is not
+// clipped (its scale is the NaN byte either way). No thresholds given: no
+// clipping.
+
+float fma_chain(const float* u, int su, const float* v, int sv, int n) {
+  float acc = -0.0f;
+  for (int t = 0; t < n; ++t) acc = std::fmaf(u[t * su], v[t * sv], acc);
+  return acc;
+}
+
+void bat_block(const float* x, int a, const float* A, const float* Bj, const float* beta_min,
+               const float* beta_max, float* y) {
+  const int b = kBlock / a;
+  float Z[kBlock];   // Z[p * a + s]
+  for (int p = 0; p < b; ++p)
+    for (int s = 0; s < a; ++s) {
+      if (a == kBlock) {
+        Z[s] = fma_chain(x, 1, A + s, a, 16) + fma_chain(x + 16, 1, A + 16 * a + s, a, 16);
+      } else {
+        Z[p * a + s] = fma_chain(x + p * a, 1, A + s, a, a);
+      }
+    }
+  for (int r = 0; r < b; ++r)
+    for (int s = 0; s < a; ++s) {
+      const int h = b / 2;
+      if (b == 1) {
+        y[s] = fma_chain(Bj, 1, Z + s, a, 1);
+      } else {
+        y[r * a + s] = fma_chain(Bj + r, b, Z + s, a, h) +
+                       fma_chain(Bj + h * b + r, b, Z + h * a + s, a, h);
+      }
+    }
+  if (!beta_min) return;
+  float mn = y[0], mx = y[0];
+  for (int i = 0; i < kBlock; ++i) {
+    if (!std::isfinite(y[i])) return;
+    if (y[i] < mn) mn = y[i];
+    if (y[i] > mx) mx = y[i];
+  }
+  const float lo = *beta_min * mn, hi = *beta_max * mx;
+  for (int i = 0; i < kBlock; ++i) {
+    const float t = y[i] < lo ? lo : y[i];
+    y[i] = t > hi ? hi : t;
+  }
+}
+
 uint32_t float_bits(float v) {
   uint32_t u;
   std::memcpy(&u, &v, 4);
@@ -746,6 +818,33 @@ void oracle_block_error(const uint16_t* x, int64_t rows, int64_t cols, int fmt, 
   }
   totals[0] = sd;
   totals[1] = sx;
+}
+
+// [BQ] section 2 apply step: the transformed, clipped rows as bf16 (round
+// to nearest even; NaN as the canonical 0x7FC0). A is [a, a] and B is
+// [cols / 32, b, b], both row-major float; beta_min / beta_max are
+// [cols / 32] or both NULL. Also returns the fp32 values before the bf16
+// rounding when y_f32 is not NULL.
+void oracle_bat_apply(const uint16_t* x, int64_t rows, int64_t cols, int a, const float* A,
+                      const float* B, const float* beta_min, const float* beta_max, uint16_t* y,
+                      float* y_f32) {
+  const int b = kBlock / a;
+  parallel_rows(rows, [&](int64_t r0, int64_t r1) {
+    std::vector<double> row(cols);
+    for (int64_t r = r0; r < r1; ++r) {
+      decode_row(x + r * cols, cols, row.data());
+      for (int64_t j = 0; j < cols / kBlock; ++j) {
+        float xb[kBlock], yb[kBlock];
+        for (int i = 0; i < kBlock; ++i) xb[i] = static_cast<float>(row[j * kBlock + i]);
+        bat_block(xb, a, A, B + j * b * b, beta_min ? beta_min + j : nullptr,
+                  beta_max ? beta_max + j : nullptr, yb);
+        for (int i = 0; i < kBlock; ++i) {
+          y[r * cols + j * kBlock + i] = encode_bf16_rne(yb[i]);
+          if (y_f32) y_f32[r * cols + j * kBlock + i] = yb[i];
+        }
+      }
+    }
+  });
 }
 
 }  // extern "C"
