@@ -52,6 +52,7 @@ BYTES_SCALES = N_ELEM // 32
 BYTES_STEP = BYTES_IN + BYTES_CODES + BYTES_SCALES            # 1,019,215,872
 FALLBACK_HBM_GBS = 6650.0
 KERNEL_SOURCES = ["fp8_quantization_mx_b200/csrc/mx_kernels.cu",
+                  "fp8_quantization_mx_b200/csrc/mx_stream.cuh",
                   "fp8_quantization_mx_b200/csrc/mx_device.cuh"]
 PROFILE = os.path.join(ROOT, "profiles", "quantize_fp4_floor_moe_w13.md")
 
@@ -252,6 +253,8 @@ def stack_ops(mx, x, reps=50, only=None):
     y = torch.empty_like(x)
     g = torch.empty_like(x).normal_()
     fp4, fp8, fp4m = n * 2.53125, n * 3.03125, n * (2.53125 + 1 / 128)
+    from fp8_quantization_mx_b200 import inputs as _inputs
+    bat = {a: _inputs.bat_params(a, cols // 32, device=dev) for a in (1, 4, 8)}
     ops = {
         "fp4_floor_quantize": (lambda: mx.quantize(x, mx.E2M1, mx.FLOOR, out=(c4, sc, None)), fp4),
         "fp8_floor_quantize": (lambda: mx.quantize(x, mx.E4M3, mx.FLOOR, out=(c8, sc, None)), fp8),
@@ -279,6 +282,11 @@ def stack_ops(mx, x, reps=50, only=None):
         "e5m2_oas_quantize": (lambda: mx.quantize(x, mx.E5M2, mx.OAS, out=(c8, sc, None)), fp8),
         "e2m3_oas_quantize": (lambda: mx.quantize(x, mx.E2M3, mx.OAS, out=(c8, sc, None)), fp8),
         "int8_dequantize_bf16": (lambda: mx.dequantize(c8, sc, None, mx.INT8, out=y), fp8),
+        # BATQuant: block transform B_j (x) A (a x a, b x b), clip, MXFP4 FLOOR
+        "fp4_bat_a8_quantize": (lambda: mx.bat_quantize(x, *bat[8], out=(c4, sc, None)), fp4),
+        "fp4_bat_a4_quantize": (lambda: mx.bat_quantize(x, *bat[4], out=(c4, sc, None)), fp4),
+        "fp4_bat_a1_quantize": (lambda: mx.bat_quantize(x, *bat[1], out=(c4, sc, None)), fp4),
+        "bat_a8_apply": (lambda: mx.bat_apply(x, *bat[8], out=y), n * 4),
         "fp4_mbs_dynamic_quantize": (lambda: mx.quantize(x, mx.E2M1, mx.MBS_DYNAMIC, out=(c4, sc, mac)),
                                      fp4m),
         "fp4_oas_mbs_dynamic_quantize": (lambda: mx.quantize(x, mx.E2M1, mx.OAS | mx.MBS_DYNAMIC,
@@ -309,7 +317,7 @@ def stack_ops(mx, x, reps=50, only=None):
         e.synchronize()
         ms = s.elapsed_time(e) / n_reps
         res[name] = {"ms": round(ms, 4), "GB/s": round(nbytes / ms / 1e6, 1)}
-    del c4, c8, sc, sc16, mac, sc_mma, y, g
+    del c4, c8, sc, sc16, mac, sc_mma, y, g, bat
     return res
 
 

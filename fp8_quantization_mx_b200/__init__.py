@@ -37,6 +37,7 @@ __all__ = [
     "mx_block_error", "mx_status_string", "mx_version", "mx_scale_bytes", "MMA_SCALES",
     "E2M1_B16", "NVFP4", "block_size",
     "quantize", "dequantize", "fake_quant", "fake_quant_bwd", "block_error", "MXFakeQuantize",
+    "mx_bat_apply", "mx_bat_quantize", "bat_apply", "bat_quantize",
     "MXFP4_FORMAT", "MXFP8_FORMAT",
 ]
 
@@ -104,6 +105,10 @@ def load_library():
     lib.mx_version.restype = c_int
     lib.mx_scale_bytes.argtypes = [i64, i64, c_int, c_int]
     lib.mx_scale_bytes.restype = i64
+    lib.mx_bat_apply.argtypes = [vp, i64, i64, c_int, vp, vp, vp, vp, vp, vp]
+    lib.mx_bat_quantize.argtypes = [vp, i64, i64, c_int, vp, vp, vp, vp, c_int, c_int, vp, vp, vp, vp]
+    lib.mx_bat_apply.restype = c_int
+    lib.mx_bat_quantize.restype = c_int
     _lib = lib
     return lib
 
@@ -129,6 +134,16 @@ def mx_fake_quant_bwd(x, grad_y, rows, cols, format, scaling, grad_x, stream=0) 
 
 def mx_block_error(x, rows, cols, format, scaling, block_sse, totals, stream=0) -> int:
     return load_library().mx_block_error(x, rows, cols, format, scaling, block_sse, totals, stream)
+
+
+def mx_bat_apply(x, rows, cols, a_dim, A, B, beta_min, beta_max, y, stream=0) -> int:
+    return load_library().mx_bat_apply(x, rows, cols, a_dim, A, B, beta_min, beta_max, y, stream)
+
+
+def mx_bat_quantize(x, rows, cols, a_dim, A, B, beta_min, beta_max, format, scaling, codes, scales,
+                    macro, stream=0) -> int:
+    return load_library().mx_bat_quantize(x, rows, cols, a_dim, A, B, beta_min, beta_max, format,
+                                          scaling, codes, scales, macro, stream)
 
 
 def mx_status_string(status: int) -> str:
@@ -373,6 +388,65 @@ def block_error(x: torch.Tensor, format: int = E2M1, scaling: int = FLOOR,
         _check(mx_block_error(_ptr(x), rows, cols, format, scaling, _ptr(bs), _ptr(totals),
                               _stream(x.device)), "mx_block_error")
     return bs, totals
+
+
+def _bat_params(x, A, B, beta_min, beta_max):
+    """Checks the BATQuant parameters against x; returns (a, cols)."""
+    rows, cols = _rows_cols(x)
+    for name, t in (("A", A), ("B", B), ("beta_min", beta_min), ("beta_max", beta_max)):
+        if t is None:
+            continue
+        if t.dtype != torch.float32 or not t.is_contiguous() or t.device != x.device:
+            raise ValueError(f"{name} must be a contiguous float32 tensor on {x.device}")
+    a = A.shape[0] if A.dim() == 2 else -1
+    if A.dim() != 2 or A.shape[1] != a or a not in (1, 2, 4, 8, 16, 32):
+        raise ValueError("A must be [a, a] with a in 1, 2, 4, 8, 16, 32")
+    b = 32 // a
+    if tuple(B.shape) != (cols // 32, b, b):
+        raise ValueError(f"B must be [cols/32, {b}, {b}], got {tuple(B.shape)}")
+    if (beta_min is None) != (beta_max is None):
+        raise ValueError("give both clip thresholds or neither")
+    if beta_min is not None and (beta_min.numel() != cols // 32 or beta_max.numel() != cols // 32):
+        raise ValueError("beta_min / beta_max must hold cols/32 values")
+    return a
+
+
+def bat_apply(x: torch.Tensor, A: torch.Tensor, B: torch.Tensor, beta_min=None, beta_max=None,
+              out=None):
+    """BATQuant apply step: each 32-element block j of every row times
+    B[j] (x) A, clipped to [beta_min[j] min, beta_max[j] max] of the block,
+    as bf16 (see mx_bat_apply in include/mx.h for the exact arithmetic)."""
+    _cuda_bf16(x, "x")
+    rows, cols = _rows_cols(x)
+    a = _bat_params(x, A, B, beta_min, beta_max)
+    y = torch.empty_like(x) if out is None else out
+    with torch.cuda.device(x.device):
+        _check(mx_bat_apply(_ptr(x), rows, cols, a, _ptr(A), _ptr(B), _ptr(beta_min), _ptr(beta_max),
+                            _ptr(y), _stream(x.device)), "mx_bat_apply")
+    return y
+
+
+def bat_quantize(x: torch.Tensor, A: torch.Tensor, B: torch.Tensor, beta_min=None, beta_max=None,
+                 format: int = E2M1, scaling: int = FLOOR, out=None):
+    """BATQuant: bat_apply fused with quantize in one kernel; returns what
+    quantize returns for the transformed rows."""
+    _cuda_bf16(x, "x")
+    rows, cols = _rows_cols(x)
+    a = _bat_params(x, A, B, beta_min, beta_max)
+    lead = x.shape[:-1]
+    mbs = ((scaling >> 4) & 3) != 0
+    if out is None:
+        ccols = cols // 2 if format in _PACKED else cols
+        codes = torch.empty(*lead, ccols, dtype=torch.uint8, device=x.device)
+        scales = _scales_buffer(lead, rows, cols, format, scaling, x.device)
+        macro = torch.empty(*lead, cols // 128, dtype=torch.uint8, device=x.device) if mbs else None
+    else:
+        codes, scales, macro = out
+    with torch.cuda.device(x.device):
+        _check(mx_bat_quantize(_ptr(x), rows, cols, a, _ptr(A), _ptr(B), _ptr(beta_min),
+                               _ptr(beta_max), format, scaling, _ptr(codes), _ptr(scales),
+                               _ptr(macro), _stream(x.device)), "mx_bat_quantize")
+    return codes, scales, macro
 
 
 class MXFakeQuantize(torch.autograd.Function):

@@ -20,8 +20,8 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libmx.so")
 
-SOURCES = ["mx_api.cu", "mx_kernels.cu"]
-HEADERS = ["mx_device.cuh", "mx_launch.h"]
+SOURCES = ["mx_api.cu", "mx_kernels.cu", "mx_bat.cu"]
+HEADERS = ["mx_device.cuh", "mx_launch.h", "mx_stream.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-ftz=false", "-prec-div=true", "-prec-sqrt=true",
               "-fmad=true", "-Xcompiler", "-fPIC,-O2", "-cudart", "static"]
@@ -43,12 +43,23 @@ def _newest_input() -> float:
 def build(force: bool = False, verbose: bool = False, extra=None) -> str:
     if not force and os.path.exists(LIB) and os.path.getmtime(LIB) >= _newest_input():
         return LIB
-    cmd = [nvcc(), *ARCH, *NVCC_FLAGS, "-shared", "-I", INCLUDE, "-I", CSRC]
+    # one nvcc per source, in parallel, then one link
+    base = [nvcc(), *ARCH, *NVCC_FLAGS, "-I", INCLUDE, "-I", CSRC]
     if verbose:
-        cmd += ["-Xptxas", "-v"]
-    cmd += list(extra or [])
-    cmd += [os.path.join(CSRC, s) for s in SOURCES] + ["-o", LIB + ".tmp"]
-    subprocess.run(cmd, check=True)
+        base += ["-Xptxas", "-v"]
+    base += list(extra or [])
+    objs, procs = [], []
+    for src in SOURCES:
+        obj = os.path.join(CSRC, src.replace(".cu", ".o"))
+        objs.append(obj)
+        procs.append((src, subprocess.Popen(base + ["-c", os.path.join(CSRC, src), "-o", obj])))
+    failed = [src for src, p in procs if p.wait() != 0]
+    if failed:
+        raise subprocess.CalledProcessError(1, f"nvcc {' '.join(failed)}")
+    subprocess.run([nvcc(), *ARCH, "-shared", "-cudart", "static", *objs, "-o", LIB + ".tmp"],
+                   check=True)
+    for obj in objs:
+        os.remove(obj)
     os.replace(LIB + ".tmp", LIB)
     return LIB
 

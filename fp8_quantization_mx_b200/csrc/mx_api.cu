@@ -194,3 +194,64 @@ int mx_block_error(const void* x, int64_t rows, int64_t cols, int format, int sc
 }
 
 }  // extern "C"
+
+namespace {
+
+// Shared checks of the BATQuant parameters.
+int check_bat(int64_t rows, int64_t cols, int a_dim, const float* A, const float* B,
+              const float* beta_min, const float* beta_max) {
+  if (a_dim != 1 && a_dim != 2 && a_dim != 4 && a_dim != 8 && a_dim != 16 && a_dim != 32)
+    return MX_ERR_INVALID_ARG;
+  if ((beta_min == nullptr) != (beta_max == nullptr)) return MX_ERR_INVALID_ARG;
+  if (rows == 0 || cols == 0) return MX_OK;
+  if (!A || !B) return MX_ERR_INVALID_ARG;
+  if (!aligned(A, 16) || !aligned(B, 16)) return MX_ERR_ALIGN;
+  if (beta_min && (!aligned(beta_min, 4) || !aligned(beta_max, 4))) return MX_ERR_ALIGN;
+  return MX_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+int mx_bat_apply(const void* x, int64_t rows, int64_t cols, int a_dim, const float* A,
+                 const float* B, const float* beta_min, const float* beta_max, void* y,
+                 void* stream) {
+  int st = check_shape(rows, cols, false);
+  if (st != MX_OK) return st;
+  st = check_bat(rows, cols, a_dim, A, B, beta_min, beta_max);
+  if (st != MX_OK) return st;
+  const int64_t n = rows * cols;
+  if (n == 0) return MX_OK;
+  if (!x || !y) return MX_ERR_INVALID_ARG;
+  if (!aligned(x, 32) || !aligned(y, 32)) return MX_ERR_ALIGN;
+  return from_cuda(mxk::launch_bat(x, rows, cols, a_dim, A, B, beta_min, beta_max, 0, 0, nullptr,
+                                   nullptr, nullptr, y, mxk::ScaleMap{0, 0, 0.0},
+                                   static_cast<cudaStream_t>(stream)));
+}
+
+int mx_bat_quantize(const void* x, int64_t rows, int64_t cols, int a_dim, const float* A,
+                    const float* B, const float* beta_min, const float* beta_max, int format,
+                    int scaling, void* codes, uint8_t* scales, uint8_t* macro, void* stream) {
+  const int layout = scaling & MX_SCALES_MMA;
+  scaling &= ~MX_SCALES_MMA;
+  int st = check_mode(format, scaling);
+  if (st != MX_OK) return st;
+  if (block_of(format) != 32 || (scaling >> 4) == 2) return MX_ERR_UNSUPPORTED;
+  const bool mbs = (scaling >> 4) != 0;
+  st = check_shape(rows, cols, mbs);
+  if (st != MX_OK) return st;
+  st = check_bat(rows, cols, a_dim, A, B, beta_min, beta_max);
+  if (st != MX_OK) return st;
+  const int64_t n = rows * cols;
+  if (n == 0) return MX_OK;
+  if (!x || !codes || !scales || (mbs && !macro)) return MX_ERR_INVALID_ARG;
+  if (!aligned(x, 32) || !aligned(codes, 16)) return MX_ERR_ALIGN;
+  const auto cs = static_cast<cudaStream_t>(stream);
+  if (clear_padding(scales, rows, cols, layout, 32, cs) != cudaSuccess) return MX_ERR_CUDA;
+  return from_cuda(mxk::launch_bat(x, rows, cols, a_dim, A, B, beta_min, beta_max, format, scaling,
+                                   codes, scales, mbs ? macro : nullptr, nullptr,
+                                   scale_map(cols, layout, 32), cs));
+}
+
+}  // extern "C"

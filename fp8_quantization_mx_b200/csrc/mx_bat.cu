@@ -1,0 +1,440 @@
+// BATQuant apply step, alone or fused with the MX quantizer, for sm_100a.
+//
+// "BATQuant: Outlier-resilient MXFP4 Quantization via Learnable Block-wise
+// Optimization", technical summary section 2: every 32-element MX block j of
+// a row is multiplied by its own matrix P_j = B_j (x) A (A is a x a and
+// shared by all blocks, B_j is b x b and private, a b = 32), clipped to
+// [beta^min_j min y, beta^max_j max y] of the block, and quantized. With the
+// element index i = p a + q the Kronecker structure gives
+//   y[r a + s] = sum_p B_j[p][r] Z[p][s],   Z[p][s] = sum_q x[p a + q] A[q][s],
+// two small contractions (a + b multiply-adds per element instead of 32).
+//
+// Lane layout: the streaming quantizer's, a lane pair per block and 16
+// elements per lane. For a <= 16 a lane holds b/2 whole rows of X and
+// computes their Z rows; stage 2 needs all b rows, so each lane sums its own
+// rows' terms into all 32 outputs and the pair swaps the partial sums of each
+// other's outputs (16 shuffles). For a = 32 the swap happens in stage 1. The
+// arithmetic order is therefore fixed as: fp32 fma chains in index order from
+// -0, and where an index runs over both halves of the block, the chain of the
+// lower half plus the chain of the upper half (fp32 addition commutes, so
+// both lanes get the same bits). The clip uses exact comparisons; a block
+// whose transformed values are not all finite is not clipped. One round to
+// bf16 (NaN canonical), then the per-slice quantizer, unchanged.
+//
+// All of it is CUDA-core work: a contraction of 32-element vectors with
+// 4 x 4 ... 32 x 32 factors whose rounding must be reproducible does not fit
+// the tensor cores (whose accumulation order is not specified), and the
+// kernel stays close to its issue-rate bound rather than to HBM.
+//
+// A CTA owns one 512-column chunk of many rows, so each lane's block column
+// and parameters are fixed: A is staged once per CTA in shared memory (and
+// copied into registers for a <= 8), a lane's terms of B_j sit in registers
+// (a >= 4) or in shared memory (a <= 2), and so do the thresholds. Rows
+// stream through a per-thread cp.async ring in shared memory.
+
+#include "mx_stream.cuh"
+
+namespace mxk {
+
+constexpr int kOpBatApply = 4;   // write the transformed bf16 rows
+
+struct BatParams {
+  const float* A;      // [a, a] row-major
+  const float* B;      // [cols / 32, b, b] row-major
+  const float* bmin;   // [cols / 32] or null (then bmax is null too: no clip)
+  const float* bmax;
+  int64_t rows;
+  int64_t spr;         // 16-element slices per row (cols / 16, even)
+  int nchunks;         // 32-slice column chunks per row, ceil(spr / 32)
+};
+
+// Row tiles in flight per thread (cp.async ring in shared memory).
+#ifndef MX_BAT_STAGES
+#define MX_BAT_STAGES 6
+#endif
+constexpr int kBatStages = MX_BAT_STAGES;
+constexpr int kBatRing = kBatStages * 32 * kThreads;   // ring bytes
+
+// Shared-memory layout of B for a <= 2 (where a lane's rows of B_j do not fit
+// in registers): the 16 blocks of the CTA's column chunk, rows of `pitch`
+// floats, blocks `stride` floats apart. The paddings put the 32 lanes'
+// addresses of one read (16 blocks x 2 halves) in 32 distinct banks.
+template <int AD> struct BatSmemB {
+  static constexpr int BD = 32 / AD;
+  static constexpr int pitch = AD == 1 ? 32 : 17;
+  static constexpr int stride = AD == 1 ? 1025 : 289;
+  static constexpr int floats = AD <= 2 ? 16 * stride : 0;
+};
+
+template <int AD>
+constexpr size_t bat_smem_bytes() {
+  return kBatRing + sizeof(float) * (AD * AD + BatSmemB<AD>::floats);
+}
+
+__device__ __forceinline__ void cp_async16(void* dst, const void* src, int src_bytes) {
+  const uint32_t d = static_cast<uint32_t>(__cvta_generic_to_shared(dst));
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(d), "l"(src), "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+__device__ __forceinline__ float max_nan(float a, float b) {
+  float d;
+  asm("max.NaN.f32 %0, %1, %2;" : "=f"(d) : "f"(a), "f"(b));
+  return d;
+}
+__device__ __forceinline__ float min_nan(float a, float b) {
+  float d;
+  asm("min.NaN.f32 %0, %1, %2;" : "=f"(d) : "f"(a), "f"(b));
+  return d;
+}
+
+// The parameters one lane needs, for its fixed block column j and half h.
+template <int AD>
+struct LaneParams {
+  static constexpr int BD = 32 / AD;
+  static constexpr int RH = BD >= 2 ? BD / 2 : 1;   // rows of X (and Y) per lane
+  static constexpr bool kRegB = AD >= 4;             // B_j's terms in registers
+  float A[AD <= 8 ? AD * AD : 1];                    // A in registers (a <= 8)
+  float bo[kRegB ? RH * RH : 1];   // B_j[h RH + pp][h RH + rl]: own outputs (a = 32: B_j[0][0])
+  float bt[kRegB ? RH * RH : 1];   // B_j[h RH + pp][(1 - h) RH + rl]: the partner's outputs
+  const float* Bl;                 // a <= 2: row h RH of B_j in shared memory
+  float bmin, bmax;
+};
+
+// The transformed, clipped 16 values of this lane (elements 16 h .. 16 h + 15
+// of its block) as packed bf16.
+template <int AD>
+__device__ __forceinline__ V16 bat_slice(const V16& v, int h, const LaneParams<AD>& L,
+                                         const float* As, bool clip) {
+  constexpr int BD = LaneParams<AD>::BD, RH = LaneParams<AD>::RH;
+  float xf[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) xf[i] = elem(v, i);
+
+  float y[16];
+  if constexpr (AD == 32) {
+    // stage 1 over this lane's half of q, for its own 16 outputs and the
+    // partner's; the partner's partial sums complete this lane's outputs
+    float zo[16], zt[16];
+    const float* Ah = As + (16 * h) * 32;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      float ao = -0.0f, at = -0.0f;
+#pragma unroll
+      for (int q = 0; q < 16; ++q) {
+        ao = fmaf(xf[q], Ah[q * 32 + 16 * h + i], ao);
+        at = fmaf(xf[q], Ah[q * 32 + 16 * (1 - h) + i], at);
+      }
+      zo[i] = ao;
+      zt[i] = at;
+    }
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const float z = __fadd_rn(zo[i], __shfl_xor_sync(kFull, zt[i], 1));
+      y[i] = fmaf(L.bo[0], z, -0.0f);
+    }
+  } else {
+    float z[16];   // Z rows h RH .. h RH + RH - 1
+#pragma unroll
+    for (int pp = 0; pp < RH; ++pp) {
+#pragma unroll
+      for (int s = 0; s < AD; ++s) {
+        float acc = -0.0f;
+#pragma unroll
+        for (int q = 0; q < AD; ++q) {
+          float aq;
+          if constexpr (AD <= 8) {
+            aq = L.A[q * AD + s];
+          } else {
+            aq = As[q * AD + s];
+          }
+          acc = fmaf(xf[pp * AD + q], aq, acc);
+        }
+        z[pp * AD + s] = acc;
+      }
+    }
+    // stage 2: this lane's rows' terms of its own outputs (rows h RH ..)
+    // and of the partner's outputs (rows (1 - h) RH ..)
+    float yo[16], yt[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) yo[i] = yt[i] = -0.0f;
+    const int co = h * RH, ct = (1 - h) * RH;
+#pragma unroll
+    for (int pp = 0; pp < RH; ++pp) {
+#pragma unroll
+      for (int rl = 0; rl < RH; ++rl) {
+        float bo, bt;
+        if constexpr (LaneParams<AD>::kRegB) {
+          bo = L.bo[pp * RH + rl];
+          bt = L.bt[pp * RH + rl];
+        } else {
+          bo = L.Bl[pp * BatSmemB<AD>::pitch + co + rl];
+          bt = L.Bl[pp * BatSmemB<AD>::pitch + ct + rl];
+        }
+#pragma unroll
+        for (int s = 0; s < AD; ++s) {
+          yo[rl * AD + s] = fmaf(bo, z[pp * AD + s], yo[rl * AD + s]);
+          yt[rl * AD + s] = fmaf(bt, z[pp * AD + s], yt[rl * AD + s]);
+        }
+      }
+    }
+    // __fadd_rn: a one-term chain (b = 2) is a rounded product, which must
+    // not be contracted with this addition into one fma
+#pragma unroll
+    for (int i = 0; i < 16; ++i) y[i] = __fadd_rn(yo[i], __shfl_xor_sync(kFull, yt[i], 1));
+    (void)BD;
+  }
+
+  if (clip) {
+    float mx = y[0], mn = y[0];
+#pragma unroll
+    for (int i = 1; i < 16; ++i) {
+      mx = max_nan(mx, y[i]);
+      mn = min_nan(mn, y[i]);
+    }
+    mx = max_nan(mx, __shfl_xor_sync(kFull, mx, 1));
+    mn = min_nan(mn, __shfl_xor_sync(kFull, mn, 1));
+    if (isfinite(mx) && isfinite(mn)) {
+      const float lo = __fmul_rn(L.bmin, mn);
+      const float hi = __fmul_rn(L.bmax, mx);
+      if (lo != 0.0f && hi != 0.0f) {
+        // a nonzero bound equals y only with the same sign: min/max are
+        // then exactly the comparisons below (a NaN bound leaves y alone)
+#pragma unroll
+        for (int i = 0; i < 16; ++i) y[i] = fminf(fmaxf(y[i], lo), hi);
+      } else {
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float t = y[i] < lo ? lo : y[i];
+          y[i] = t > hi ? hi : t;
+        }
+      }
+    }
+  }
+  V16 o;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) o.w[i] = pack_bf16x2(y[2 * i], y[2 * i + 1]);
+  return o;
+}
+
+// NaN halves of a slice -> the canonical quiet NaN 0x7FC0 (only called for
+// blocks whose max magnitude is NaN or Inf).
+__device__ __forceinline__ void canonical_nan(V16& v) {
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    uint32_t w = v.w[i];
+    if ((w & 0x7FFFu) > 0x7F80u) w = (w & 0xFFFF0000u) | kNaNbf16;
+    if (((w >> 16) & 0x7FFFu) > 0x7F80u) w = (w & 0xFFFFu) | (static_cast<uint32_t>(kNaNbf16) << 16);
+    v.w[i] = w;
+  }
+}
+
+// One CTA owns one 32-slice column chunk (16 blocks, 512 columns) of the rows
+// g * 8 + w + t * G * 8 (warp w, CTA group g of G): each lane's block column,
+// and so its parameters, never changes, and a warp reads 1 KB of one row per
+// step. Each thread streams its 32 bytes of successive rows through a ring of
+// kBatStages slots (cp.async, waited per thread: no block-wide barrier after
+// the parameters are staged).
+template <int AD, int OP, int FMT, int RULE, int MBS>
+__global__ void __launch_bounds__(kThreads) bat_kernel(StreamArgs a, BatParams p) {
+  extern __shared__ __align__(16) uint8_t smem[];
+  float* As = reinterpret_cast<float*>(smem + kBatRing);
+  float* Bs = As + AD * AD;
+  const int cc = blockIdx.x % p.nchunks;
+  const int64_t g = blockIdx.x / p.nchunks;
+  const int64_t G = gridDim.x / p.nchunks;
+  const int tid = threadIdx.x, lane = tid & 31, w = tid >> 5;
+  const int64_t cs = static_cast<int64_t>(cc) * 32 + lane;   // slice within the row
+  const bool col_ok = cs < p.spr;
+  const int h = lane & 1;
+  const int64_t nb = p.spr >> 1;
+  const int64_t j = col_ok ? (cs >> 1) : 0;
+
+  for (int i = tid; i < AD * AD; i += kThreads) As[i] = p.A[i];
+  if constexpr (AD <= 2) {
+    using SB = BatSmemB<AD>;
+    for (int i = tid; i < 16 * SB::BD * SB::BD; i += kThreads) {
+      const int jl = i / (SB::BD * SB::BD), e = i % (SB::BD * SB::BD);
+      const int64_t jj = static_cast<int64_t>(cc) * 16 + jl;
+      Bs[jl * SB::stride + (e / SB::BD) * SB::pitch + e % SB::BD] =
+          jj < nb ? p.B[jj * SB::BD * SB::BD + e] : 0.0f;
+    }
+  }
+  __syncthreads();
+
+  LaneParams<AD> L;
+  constexpr int BD = LaneParams<AD>::BD, RH = LaneParams<AD>::RH;
+  if constexpr (AD <= 8) {
+#pragma unroll
+    for (int i = 0; i < AD * AD; ++i) L.A[i] = As[i];
+  } else {
+    L.A[0] = 0.0f;
+  }
+  if constexpr (AD == 32) {
+    L.bo[0] = p.B[j];
+    L.bt[0] = 0.0f;
+  } else if constexpr (LaneParams<AD>::kRegB) {
+    const float* Bj = p.B + j * (BD * BD) + (h * RH) * BD;
+#pragma unroll
+    for (int pp = 0; pp < RH; ++pp) {
+#pragma unroll
+      for (int rl = 0; rl < RH; ++rl) {
+        L.bo[pp * RH + rl] = Bj[pp * BD + h * RH + rl];
+        L.bt[pp * RH + rl] = Bj[pp * BD + (1 - h) * RH + rl];
+      }
+    }
+  } else {
+    L.bo[0] = L.bt[0] = 0.0f;
+  }
+  L.Bl = Bs + (lane >> 1) * BatSmemB<AD>::stride + (h * RH) * BatSmemB<AD>::pitch;
+  const bool clip = p.bmin != nullptr;
+  L.bmin = clip ? p.bmin[j] : 0.0f;
+  L.bmax = clip ? p.bmax[j] : 0.0f;
+
+  uint8_t* slot0 = smem + tid * 16;   // slot s, half k at slot0 + (2 s + k) * kThreads * 16
+  const int64_t rstride = G * (kThreads / 32);
+  auto issue = [&](int64_t r, int st) {
+    const bool ok = col_ok && r < p.rows;
+    const uint8_t* src = ok ? a.x + ((r * p.spr + cs) << 5) : a.x;
+    const int n = ok ? 16 : 0;
+    cp_async16(slot0 + (2 * st) * kThreads * 16, src, n);
+    cp_async16(slot0 + (2 * st + 1) * kThreads * 16, ok ? src + 16 : src, n);
+    cp_async_commit();
+  };
+  const int64_t r0 = g * (kThreads / 32) + w;
+#pragma unroll
+  for (int d = 0; d < kBatStages - 1; ++d) issue(r0 + d * rstride, d);
+
+  double sd = 0.0, sx = 0.0;
+  int st = 0;
+  for (int64_t r = r0; r < p.rows; r += rstride) {
+    issue(r + (kBatStages - 1) * rstride, st == 0 ? kBatStages - 1 : st - 1);
+    cp_async_wait<kBatStages - 1>();
+    V16 v;
+    {
+      const uint4 lo = *reinterpret_cast<const uint4*>(slot0 + (2 * st) * kThreads * 16);
+      const uint4 hi = *reinterpret_cast<const uint4*>(slot0 + (2 * st + 1) * kThreads * 16);
+      v.w[0] = lo.x; v.w[1] = lo.y; v.w[2] = lo.z; v.w[3] = lo.w;
+      v.w[4] = hi.x; v.w[5] = hi.y; v.w[6] = hi.z; v.w[7] = hi.w;
+    }
+    st = st == kBatStages - 1 ? 0 : st + 1;
+    const int64_t c = r * p.spr + cs;
+    V16 yv = bat_slice<AD>(v, h, L, As, clip);
+    const uint32_t pa = pair_max(amax_bits16(yv));
+    if (pa >= 0x7F80u) canonical_nan(yv);
+    if constexpr (OP == kOpBatApply) {
+      if (col_ok) st_stream32(a.out + 32 * c, yv);
+    } else {
+      int k = 0;
+      if (MBS == kMbsStatic) k = mbs_static_k(oct_max(pa));
+      process_slice<kOpQuant, FMT, RULE, MBS>(a, yv, yv, c, col_ok, lane, pa, k, sd, sx);
+    }
+  }
+  cp_async_wait<0>();
+}
+
+namespace {
+
+int sm_count() {
+  int dev = 0;
+  cudaGetDevice(&dev);
+  int n = 0;
+  cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 1;
+}
+
+template <int AD, int OP, int FMT, int RULE, int MBS>
+cudaError_t launch_bat_kernel(const StreamArgs& a, const BatParams& p, cudaStream_t st) {
+  auto kern = bat_kernel<AD, OP, FMT, RULE, MBS>;
+  constexpr size_t smem = bat_smem_bytes<AD>();
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  int per_sm = 0;
+  cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, kern, kThreads, smem);
+  if (per_sm < 1) per_sm = 1;
+  // G CTA groups per column chunk: fill the resident capacity, but no group
+  // without rows
+  const int64_t cap = static_cast<int64_t>(sm_count()) * per_sm;
+  const int64_t row_groups = (p.rows + kThreads / 32 - 1) / (kThreads / 32);
+  int64_t G = cap / p.nchunks;
+  if (G < 1) G = 1;
+  if (G > row_groups) G = row_groups;
+  const int64_t grid = G * p.nchunks;
+  if (grid > 0x7FFFFFFF) return cudaErrorInvalidConfiguration;
+  kern<<<static_cast<int>(grid), kThreads, smem, st>>>(a, p);
+  return cudaGetLastError();
+}
+
+// The quantizer configurations of the single-pass streaming kernel.
+template <int AD>
+cudaError_t dispatch_bat(const StreamArgs& a, const BatParams& p, int op, int fmt, int scaling,
+                         cudaStream_t st) {
+  if (op == kOpBatApply) return launch_bat_kernel<AD, kOpBatApply, kFmtE2M1, kFloor, kMbsNone>(a, p, st);
+  const int rule = scaling & 0xF;
+  const bool mbs = (scaling >> 4) != 0;
+  switch (fmt) {
+    case kFmtE2M1:
+      if (mbs) {
+        if (rule == kOas) return launch_bat_kernel<AD, kOpQuant, kFmtE2M1, kOas, kMbsStatic>(a, p, st);
+        return launch_bat_kernel<AD, kOpQuant, kFmtE2M1, kFloor, kMbsStatic>(a, p, st);
+      }
+      switch (rule) {
+        case kCeil: return launch_bat_kernel<AD, kOpQuant, kFmtE2M1, kCeil, kMbsNone>(a, p, st);
+        case kOasRule: return launch_bat_kernel<AD, kOpQuant, kFmtE2M1, kOasRule, kMbsNone>(a, p, st);
+        case kOas: return launch_bat_kernel<AD, kOpQuant, kFmtE2M1, kOas, kMbsNone>(a, p, st);
+        default: return launch_bat_kernel<AD, kOpQuant, kFmtE2M1, kFloor, kMbsNone>(a, p, st);
+      }
+#define MXK_BAT_BYTES(F)                                                                     \
+  case F:                                                                                   \
+    if (rule == kCeil) return launch_bat_kernel<AD, kOpQuant, F, kCeil, kMbsNone>(a, p, st); \
+    if (rule == kOas) return launch_bat_kernel<AD, kOpQuant, F, kOas, kMbsNone>(a, p, st);   \
+    return launch_bat_kernel<AD, kOpQuant, F, kFloor, kMbsNone>(a, p, st);
+      MXK_BAT_BYTES(kFmtE4M3)
+      MXK_BAT_BYTES(kFmtE5M2)
+      MXK_BAT_BYTES(kFmtE3M2)
+      MXK_BAT_BYTES(kFmtE2M3)
+#undef MXK_BAT_BYTES
+    case kFmtInt8:
+      if (rule == kCeil) return launch_bat_kernel<AD, kOpQuant, kFmtInt8, kCeil, kMbsNone>(a, p, st);
+      return launch_bat_kernel<AD, kOpQuant, kFmtInt8, kFloor, kMbsNone>(a, p, st);
+    default:
+      return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace
+
+cudaError_t launch_bat(const void* x, int64_t rows, int64_t cols, int a_dim, const float* A,
+                       const float* B, const float* beta_min, const float* beta_max, int fmt,
+                       int scaling, void* codes, uint8_t* scales, uint8_t* macro, void* y,
+                       ScaleMap sm, cudaStream_t st) {
+  StreamArgs a{};
+  a.x = static_cast<const uint8_t*>(x);
+  a.nslices = rows * cols / 16;
+  a.codes = static_cast<uint8_t*>(codes);
+  a.scales = scales;
+  a.macro = macro;
+  a.out = static_cast<uint8_t*>(y);
+  a.smap = sm;
+  const int64_t spr = cols / 16;
+  if ((spr + 31) / 32 > 0x7FFFFFFF) return cudaErrorInvalidValue;
+  BatParams p{A, B, beta_min, beta_max, rows, spr, static_cast<int>((spr + 31) / 32)};
+  const int op = y ? kOpBatApply : kOpQuant;
+  switch (a_dim) {
+    case 1: return dispatch_bat<1>(a, p, op, fmt, scaling, st);
+    case 2: return dispatch_bat<2>(a, p, op, fmt, scaling, st);
+    case 4: return dispatch_bat<4>(a, p, op, fmt, scaling, st);
+    case 8: return dispatch_bat<8>(a, p, op, fmt, scaling, st);
+    case 16: return dispatch_bat<16>(a, p, op, fmt, scaling, st);
+    case 32: return dispatch_bat<32>(a, p, op, fmt, scaling, st);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+}  // namespace mxk

@@ -27,6 +27,11 @@ cudaError_t launch_fake_fwd(const void* x, int64_t n, int fmt, int scaling, void
                             uint8_t* scales_out, ScaleMap sm, cudaStream_t st);
 cudaError_t launch_fake_bwd(const void* x, const void* gy, int64_t n, int fmt, int scaling,
                             void* gx, cudaStream_t st);
+// BATQuant: y != null writes the transformed bf16 rows; else quantizes them.
+cudaError_t launch_bat(const void* x, int64_t rows, int64_t cols, int a_dim, const float* A,
+                       const float* B, const float* beta_min, const float* beta_max, int fmt,
+                       int scaling, void* codes, uint8_t* scales, uint8_t* macro, void* y,
+                       ScaleMap sm, cudaStream_t st);
 cudaError_t launch_block_error(const void* x, int64_t n, int fmt, int scaling, float* block_sse,
                                double* totals, cudaStream_t st);
 

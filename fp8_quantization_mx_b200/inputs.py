@@ -20,6 +20,9 @@ weights or datasets are used anywhere):
   positions (distinct) x20.
 * ``moe_w13``      [128, 1536, 2048] N(0, 0.02^2) times a per-expert factor
   drawn from U(0.5, 2).
+* ``bat_params``   random stand-ins for BATQuant's learned parameters (none
+  are available): A = I + s N(0,1) [a, a], B_j = I + s N(0,1) [cols/32, b, b]
+  (s = 0.1 by default), clip thresholds U(0.8, 1), all float32.
 """
 
 from __future__ import annotations
@@ -97,6 +100,19 @@ def moe_w13(experts=128, inter2=1536, hidden=2048, seed=4, device="cpu", std=0.0
     s = torch.rand(experts, 1, 1, generator=g, device=device, dtype=torch.float32) * 1.5 + 0.5
     x.mul_(s).mul_(std)
     return x.to(torch.bfloat16)
+
+
+def bat_params(a, n_blocks, seed=5, device="cpu", spread=0.1, clip=True, lo=0.8):
+    """(A [a, a], B [n_blocks, b, b], beta_min, beta_max [n_blocks] or None) float32."""
+    g = _gen(seed, device)
+    b = 32 // a
+    A = torch.eye(a, device=device) + spread * torch.randn(a, a, generator=g, device=device)
+    B = torch.eye(b, device=device) + spread * torch.randn(n_blocks, b, b, generator=g, device=device)
+    if not clip:
+        return A.contiguous(), B.contiguous(), None, None
+    bmin = lo + (1 - lo) * torch.rand(n_blocks, generator=g, device=device)
+    bmax = lo + (1 - lo) * torch.rand(n_blocks, generator=g, device=device)
+    return A.contiguous(), B.contiguous(), bmin, bmax
 
 
 def random_bf16_bits(shape, seed=0, device="cpu", finite_only=True):

@@ -15,6 +15,10 @@
  *       Quantization Error Reduction" [technical summary 1: E8M0 = 2^k only]
  *       [2.A Overflow-Aware Scaling] [2.B Macro Block Scaling] [3-4: QSNR]
  *       [5: OAS and MBS generalize to MXFP6 and MXFP8].
+ *  [BQ] "BATQuant: Outlier-resilient MXFP4 Quantization via Learnable
+ *       Block-wise Optimization" [technical summary 2: block-wise affine
+ *       transform matched to the MX block; GPK: block matrix = B_j (x) A with
+ *       A shared and B_j private; block-wise learnable clipping].
  *
  * Layout (every call): x is row-major contiguous [rows, cols] bf16, cols a
  * multiple of 32 (16 for the block-16 formats); block b of row r is elements
@@ -174,6 +178,38 @@ int mx_fake_quant_bwd(const void* x, const void* grad_y, int64_t rows, int64_t c
  * totals[0] / (rows*cols); SQNR dB = 10 log10(totals[1] / totals[0]). */
 int mx_block_error(const void* x, int64_t rows, int64_t cols, int format, int scaling,
                    float* block_sse, double* totals, void* stream);
+
+/* BATQuant apply step ([BQ] 2), alone or fused with MX quantization.
+ * Each 32-element block j of every row is multiplied on the right by
+ * P_j = B_j (x) A: with i = p*a + q (p < b, q < a, a*b = 32),
+ *   y[r*a+s] = sum_p B_j[p][r] * Z[p][s],  Z[p][s] = sum_q x[p*a+q] * A[q][s].
+ * Then, when thresholds are given and the block's 32 values are all finite,
+ * each value is clipped: t = y < lo ? lo : y; y = t > hi ? hi : t, with
+ * lo = beta_min[j] * min(block), hi = beta_max[j] * max(block) (fp32 products;
+ * thresholds >= 0 expected, e.g. a sigmoid of the learned parameter). The
+ * result is rounded to bf16 (nearest even; NaN -> 0x7FC0).
+ * Arithmetic (fixed, so that results are reproducible bit for bit): fp32,
+ * IEEE (no flush to zero); every sum is a chain of fused multiply-adds in
+ * ascending index order starting from -0, except that a sum whose index runs
+ * over both 16-element halves of the block (the sum over p when b >= 2, over
+ * q when a = 32) is the fp32 sum of the lower half's chain and the upper
+ * half's chain.
+ *   a_dim        a, one of 1, 2, 4, 8, 16, 32 (b = 32 / a).
+ *   A            device float [a, a], row-major A[q][s]; 16-byte aligned.
+ *   B            device float [cols/32, b, b], row-major B_j[p][r]; 16-byte aligned.
+ *   beta_min/max device float [cols/32], 4-byte aligned; both NULL = no clip
+ *                (exactly one NULL is MX_ERR_INVALID_ARG).
+ * mx_bat_apply writes y_bf16 [rows, cols] (32-byte aligned).
+ * mx_bat_quantize writes what mx_quantize writes for that y, for the 32-element
+ * formats and every scaling except MBS-Dynamic (MX_ERR_UNSUPPORTED; run
+ * mx_bat_apply, then mx_quantize), MX_SCALES_MMA included. Other errors as
+ * mx_quantize; a_dim not in the list or a NULL A / B is MX_ERR_INVALID_ARG. */
+int mx_bat_apply(const void* x, int64_t rows, int64_t cols, int a_dim, const float* A,
+                 const float* B, const float* beta_min, const float* beta_max, void* y_bf16,
+                 void* stream);
+int mx_bat_quantize(const void* x, int64_t rows, int64_t cols, int a_dim, const float* A,
+                    const float* B, const float* beta_min, const float* beta_max, int format,
+                    int scaling, void* codes, uint8_t* scales, uint8_t* macro, void* stream);
 
 /* Static description of a status code (never NULL). */
 const char* mx_status_string(int status);

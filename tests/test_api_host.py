@@ -152,3 +152,34 @@ def test_scale_bytes_and_mma_layout_flag(mx):
     assert mx.mx_dequantize(A, A, None, 4, 33, 0, MMA | 1, A, 0) == SHAPE
     assert mx.mx_dequantize(A, A, None, 4, 32, 0, MMA | 2, A, 0) == INVALID
     assert mx.mx_block_error(A, 4, 32, 0, MMA, None, A, 0) == UNSUPPORTED
+
+
+def test_bat_entry_points_validate(mx):
+    ap, qz = mx.mx_bat_apply, mx.mx_bat_quantize
+    # a must divide 32 as a power of two
+    for bad in (0, 3, 64, -1):
+        assert ap(A, 4, 32, bad, A, A, None, None, A, 0) == INVALID
+        assert qz(A, 4, 32, bad, A, A, None, None, 0, 0, A, A, None, 0) == INVALID
+    assert ap(A, 4, 48, 8, A, A, None, None, A, 0) == SHAPE
+    assert ap(A, 4, 32, 8, None, A, None, None, A, 0) == INVALID
+    assert ap(A, 4, 32, 8, A, None, None, None, A, 0) == INVALID
+    assert ap(A, 4, 32, 8, A, A, A, None, A, 0) == INVALID        # one threshold array alone
+    assert ap(A, 4, 32, 8, A, A, None, A, A, 0) == INVALID
+    assert ap(A, 4, 32, 8, A + 4, A, None, None, A, 0) == ALIGN   # A, B: 16 bytes
+    assert ap(A, 4, 32, 8, A, A + 8, None, None, A, 0) == ALIGN
+    assert ap(A, 4, 32, 8, A, A, A + 2, A, A, 0) == ALIGN        # thresholds: 4 bytes
+    assert ap(A + 16, 4, 32, 8, A, A, None, None, A, 0) == ALIGN
+    assert ap(A, 4, 32, 8, A, A, None, None, A + 16, 0) == ALIGN
+    assert ap(A, 4, 32, 8, A, A, None, None, None, 0) == INVALID
+    assert ap(None, 0, 32, 8, None, None, None, None, None, 0) == OK
+    # quantize: 32-element formats, no MBS-Dynamic; the mx_quantize mode rules
+    assert qz(A, 4, 128, 8, A, A, None, None, 6, 0, A, A, None, 0) == UNSUPPORTED
+    assert qz(A, 4, 128, 8, A, A, None, None, 7, 0, A, A, None, 0) == UNSUPPORTED
+    assert qz(A, 4, 128, 8, A, A, None, None, 0, 0x20, A, A, A, 0) == UNSUPPORTED
+    assert qz(A, 4, 128, 8, A, A, None, None, 0, 0x23, A, A, A, 0) == UNSUPPORTED
+    assert qz(A, 4, 128, 8, A, A, None, None, 5, 3, A, A, None, 0) == UNSUPPORTED
+    assert qz(A, 4, 96, 8, A, A, None, None, 0, 0x10, A, A, A, 0) == SHAPE
+    assert qz(A, 4, 128, 8, A, A, None, None, 0, 0x10, A, A, None, 0) == INVALID
+    assert qz(A, 4, 128, 8, A, A, None, None, 0, 0, A + 8, A, None, 0) == ALIGN
+    assert qz(A, 4, 128, 8, None, A, None, None, 0, 0, A, A, None, 0) == INVALID
+    assert qz(None, 0, 128, 8, None, None, None, None, 0, 0, None, None, None, 0) == OK

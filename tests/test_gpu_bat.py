@@ -1,0 +1,158 @@
+"""GPU parity of the BATQuant kernels ("BATQuant: Outlier-resilient MXFP4
+Quantization via Learnable Block-wise Optimization", section 2) against the
+oracle: the transformed bf16 rows and the fused quantizer's codes, scale bytes
+and macro factors, bit for bit, through the C ABI.
+
+The arithmetic order is fixed (fp32 fma chains, halves summed separately), so
+the comparison is exact, including the codes the rounding decides.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+from fp8_quantization_mx_b200 import inputs
+
+pytestmark = pytest.mark.gpu
+
+E2M1, E4M3, E5M2, E3M2, E2M3, INT8 = 0, 1, 2, 3, 4, 5
+FLOOR, CEIL, OAS_RULE, OAS, MBS_STATIC = 0, 1, 2, 3, 16
+MMA = 1 << 8
+A_DIMS = (1, 2, 4, 8, 16, 32)
+# shapes: several warp tiles with a ragged last one; rows shorter than a
+# 512-element tile (tiles wrap rows) and longer
+SHAPES = [(37, 96), (9, 2048), (130, 1152)]
+
+
+def _np(t):
+    return None if t is None else t.detach().cpu().numpy()
+
+
+def run_both(mx, oracle_mod, x, params, fmt=None, scaling=None):
+    A, B, bmin, bmax = params
+    a = A.shape[0]
+    xb = inputs.bf16_bits_numpy(x)
+    if fmt is None:
+        y = mx.bat_apply(x, A, B, bmin, bmax)
+        torch.cuda.synchronize()
+        want = oracle_mod.bat_apply(xb, a, _np(A), _np(B), _np(bmin), _np(bmax))
+        return inputs.bf16_bits_numpy(y), want
+    got = mx.bat_quantize(x, A, B, bmin, bmax, fmt, scaling)
+    torch.cuda.synchronize()
+    want = oracle_mod.bat_quantize(xb, a, _np(A), _np(B), _np(bmin), _np(bmax), fmt, scaling)
+    return [_np(t) for t in got], list(want)
+
+
+def assert_same(got, want):
+    if isinstance(got, list):
+        for g, w in zip(got, want):
+            assert (g is None) == (w is None)
+            if g is not None:
+                assert np.array_equal(g, w), np.argwhere(g != w)[:5]
+    else:
+        assert np.array_equal(got, want), np.argwhere(got != want)[:5]
+
+
+@pytest.mark.parametrize("a", A_DIMS)
+@pytest.mark.parametrize("shape", SHAPES)
+@pytest.mark.parametrize("clip", [False, True])
+def test_apply_matches_oracle(mx, oracle_mod, cuda, a, shape, clip):
+    rows, cols = shape
+    x = inputs.outlier_act(rows, cols, seed=rows + cols).to(cuda)
+    params = inputs.bat_params(a, cols // 32, seed=a + rows, device=cuda, spread=0.3, clip=clip)
+    assert_same(*run_both(mx, oracle_mod, x, params))
+
+
+@pytest.mark.parametrize("a", A_DIMS)
+def test_quantize_fp4_floor_every_a(mx, oracle_mod, cuda, a):
+    x = inputs.heavy_tail(67, 1152, seed=a).to(cuda)
+    params = inputs.bat_params(a, 1152 // 32, seed=a, device=cuda)
+    assert_same(*run_both(mx, oracle_mod, x, params, E2M1, FLOOR))
+
+
+MODES = [(E2M1, FLOOR), (E2M1, CEIL), (E2M1, OAS_RULE), (E2M1, OAS), (E2M1, MBS_STATIC),
+         (E2M1, OAS | MBS_STATIC), (E4M3, FLOOR), (E4M3, CEIL), (E4M3, OAS), (E5M2, OAS),
+         (E3M2, FLOOR), (E3M2, OAS), (E2M3, CEIL), (E2M3, OAS), (INT8, FLOOR), (INT8, CEIL)]
+
+
+@pytest.mark.parametrize("fm", MODES)
+@pytest.mark.parametrize("a", [4, 8, 32])
+def test_quantize_every_mode(mx, oracle_mod, cuda, fm, a):
+    fmt, scaling = fm
+    x = inputs.outlier_act(130, 1152, seed=fmt * 7 + scaling).to(cuda)
+    params = inputs.bat_params(a, 1152 // 32, seed=11 + a, device=cuda)
+    assert_same(*run_both(mx, oracle_mod, x, params, fmt, scaling))
+
+
+@pytest.mark.parametrize("fm", [(E2M1, FLOOR), (E2M1, OAS | MBS_STATIC), (E4M3, OAS)])
+def test_fused_equals_apply_then_quantize_with_tiled_scales(mx, cuda, fm):
+    fmt, scaling = fm
+    x = inputs.heavy_tail(300, 2048, seed=9).to(cuda)
+    A, B, bmin, bmax = inputs.bat_params(8, 64, seed=9, device=cuda)
+    y = mx.bat_apply(x, A, B, bmin, bmax)
+    for flag in (0, MMA):
+        want = mx.quantize(y, fmt, scaling | flag)
+        got = mx.bat_quantize(x, A, B, bmin, bmax, fmt, scaling | flag)
+        for g, w in zip(got, want):
+            assert (g is None and w is None) or torch.equal(g, w)
+
+
+def test_edge_blocks(mx, oracle_mod, cuda):
+    """Zero blocks, NaN / Inf inputs, values that overflow fp32 and bf16 in
+    the transform, subnormal results, thresholds 0 / NaN / > 1, negative
+    zeros: bit-exact on both outputs."""
+    rows, cols = 8, 512
+    rng = np.random.default_rng(1)
+    x = rng.standard_normal((rows, cols)).astype(np.float32)
+    x[0, :32] = 0.0
+    x[0, 32:64] = -0.0
+    x[1, 5] = np.nan
+    x[1, 40] = np.inf
+    x[1, 70] = -np.inf
+    x[2, :64] *= 2e37                     # fp32 overflow in the sums (some inputs Inf)
+    x[3, :64] *= 1e-38                    # subnormal products
+    x[4, 64:96] = 2.0 ** -126
+    xb = torch.from_numpy(x).to(torch.bfloat16).to(cuda)
+    nb = cols // 32
+    for a in A_DIMS:
+        A, B, _, _ = inputs.bat_params(a, nb, seed=a, device=cuda, spread=0.5, clip=False)
+        bmin = torch.full((nb,), 0.9, device=cuda)
+        bmax = torch.full((nb,), 0.9, device=cuda)
+        bmin[0], bmax[0] = 0.0, 0.0
+        bmin[1], bmax[1] = float("nan"), 0.5
+        bmin[2], bmax[2] = 1.5, float("inf")
+        bmin[3], bmax[3] = 0.0, 1.0
+        for params in ((A, B, bmin, bmax), (A, B, None, None)):
+            assert_same(*run_both(mx, oracle_mod, xb, params))
+            assert_same(*run_both(mx, oracle_mod, xb, params, E2M1, OAS | MBS_STATIC))
+            assert_same(*run_both(mx, oracle_mod, xb, params, E4M3, FLOOR))
+
+
+def test_identity_parameters_are_plain_quantization(mx, cuda):
+    x = inputs.heavy_tail(256, 4096, seed=4).to(cuda)
+    for a in A_DIMS:
+        A = torch.eye(a, device=cuda)
+        B = torch.eye(32 // a, device=cuda).expand(4096 // 32, -1, -1).contiguous()
+        got = mx.bat_quantize(x, A, B, format=E2M1, scaling=OAS)
+        want = mx.quantize(x, E2M1, OAS)
+        assert torch.equal(got[0], want[0]) and torch.equal(got[1], want[1])
+
+
+def test_full_moe_stack_sampled_rows(mx, oracle_mod, cuda):
+    """The bench workload (MoE w13 [128, 1536, 2048], a = 8, clipping, MXFP4
+    FLOOR) in the bench's launch configuration; 96 sampled rows against the
+    oracle."""
+    x = inputs.moe_w13(device=cuda).view(-1, 2048)
+    params = inputs.bat_params(8, 64, device=cuda)
+    A, B, bmin, bmax = params
+    codes, scales, _ = mx.bat_quantize(x, A, B, bmin, bmax, E2M1, FLOOR)
+    y = mx.bat_apply(x, A, B, bmin, bmax)
+    torch.cuda.synchronize()
+    idx = torch.randperm(x.shape[0], generator=torch.Generator().manual_seed(0))[:96]
+    xs = inputs.bf16_bits_numpy(x[idx.to(cuda)])
+    oc, os_, _ = oracle_mod.bat_quantize(xs, 8, _np(A), _np(B), _np(bmin), _np(bmax), E2M1, FLOOR)
+    assert np.array_equal(codes[idx.to(cuda)].cpu().numpy(), oc)
+    assert np.array_equal(scales[idx.to(cuda)].cpu().numpy(), os_)
+    oy = oracle_mod.bat_apply(xs, 8, _np(A), _np(B), _np(bmin), _np(bmax))
+    assert np.array_equal(inputs.bf16_bits_numpy(y[idx.to(cuda)]), oy)
+    del x, y, codes, scales
