@@ -55,6 +55,12 @@ struct BatParams {
 constexpr int kBatStages = MX_BAT_STAGES;
 constexpr int kBatRing = kBatStages * 32 * kThreads;   // ring bytes
 
+// A is copied into registers for a <= MX_BAT_REG_A (else read from shared
+// memory, two pairs per 16-byte load, shared by the lane's rows).
+#ifndef MX_BAT_REG_A
+#define MX_BAT_REG_A 4
+#endif
+
 // Shared-memory layout of B for a <= 2 (where a lane's rows of B_j do not fit
 // in registers): the 16 blocks of the CTA's column chunk, rows of `pitch`
 // floats, blocks `stride` floats apart. The paddings put the 32 lanes'
@@ -93,13 +99,39 @@ __device__ __forceinline__ float min_nan(float a, float b) {
   return d;
 }
 
+// Two fused multiply-adds in one instruction (sm_100 packed fp32): each half
+// is an IEEE fma rounded to nearest even, exactly as fmaf.
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("{\n"
+      " .reg .b64 ra, rb, rc, rd;\n"
+      " mov.b64 ra, {%2, %3};\n"
+      " mov.b64 rb, {%4, %5};\n"
+      " mov.b64 rc, {%6, %7};\n"
+      " fma.rn.f32x2 rd, ra, rb, rc;\n"
+      " mov.b64 {%0, %1}, rd;\n"
+      "}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
+}
+
+// Per-half clamp of packed bf16: min(max(v, lo), hi) (a NaN bound is ignored).
+__device__ __forceinline__ uint32_t clamp_bf16x2(uint32_t v, uint32_t lo, uint32_t hi) {
+  uint32_t d;
+  asm("max.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(v), "r"(lo));
+  asm("min.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(d), "r"(hi));
+  return d;
+}
+
 // The parameters one lane needs, for its fixed block column j and half h.
 template <int AD>
 struct LaneParams {
   static constexpr int BD = 32 / AD;
   static constexpr int RH = BD >= 2 ? BD / 2 : 1;   // rows of X (and Y) per lane
   static constexpr bool kRegB = AD >= 4;             // B_j's terms in registers
-  float A[AD <= 8 ? AD * AD : 1];                    // A in registers (a <= 8)
+  static constexpr bool kRegA = AD <= MX_BAT_REG_A;  // A in registers
+  float A[kRegA ? AD * AD : 1];
   float bo[kRegB ? RH * RH : 1];   // B_j[h RH + pp][h RH + rl]: own outputs (a = 32: B_j[0][0])
   float bt[kRegB ? RH * RH : 1];   // B_j[h RH + pp][(1 - h) RH + rl]: the partner's outputs
   const float* Bl;                 // a <= 2: row h RH of B_j in shared memory
@@ -111,7 +143,7 @@ struct LaneParams {
 template <int AD>
 __device__ __forceinline__ V16 bat_slice(const V16& v, int h, const LaneParams<AD>& L,
                                          const float* As, bool clip) {
-  constexpr int BD = LaneParams<AD>::BD, RH = LaneParams<AD>::RH;
+  constexpr int RH = LaneParams<AD>::RH;
   float xf[16];
 #pragma unroll
   for (int i = 0; i < 16; ++i) xf[i] = elem(v, i);
@@ -119,50 +151,89 @@ __device__ __forceinline__ V16 bat_slice(const V16& v, int h, const LaneParams<A
   float y[16];
   if constexpr (AD == 32) {
     // stage 1 over this lane's half of q, for its own 16 outputs and the
-    // partner's; the partner's partial sums complete this lane's outputs
-    float zo[16], zt[16];
+    // partner's (pairs of adjacent outputs per instruction); the partner's
+    // partial sums complete this lane's outputs
+    float2 zo[8], zt[8];
+#pragma unroll
+    for (int m = 0; m < 8; ++m) zo[m] = zt[m] = make_float2(-0.0f, -0.0f);
     const float* Ah = As + (16 * h) * 32;
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      float ao = -0.0f, at = -0.0f;
+    for (int q = 0; q < 16; ++q) {
+      const float2 xq = make_float2(xf[q], xf[q]);
+      const float4* ro = reinterpret_cast<const float4*>(Ah + q * 32 + 16 * h);
+      const float4* rt = reinterpret_cast<const float4*>(Ah + q * 32 + 16 * (1 - h));
 #pragma unroll
-      for (int q = 0; q < 16; ++q) {
-        ao = fmaf(xf[q], Ah[q * 32 + 16 * h + i], ao);
-        at = fmaf(xf[q], Ah[q * 32 + 16 * (1 - h) + i], at);
+      for (int m4 = 0; m4 < 4; ++m4) {
+        const float4 ao = ro[m4], at = rt[m4];
+        zo[2 * m4] = ffma2(xq, make_float2(ao.x, ao.y), zo[2 * m4]);
+        zo[2 * m4 + 1] = ffma2(xq, make_float2(ao.z, ao.w), zo[2 * m4 + 1]);
+        zt[2 * m4] = ffma2(xq, make_float2(at.x, at.y), zt[2 * m4]);
+        zt[2 * m4 + 1] = ffma2(xq, make_float2(at.z, at.w), zt[2 * m4 + 1]);
       }
-      zo[i] = ao;
-      zt[i] = at;
     }
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const float z = __fadd_rn(zo[i], __shfl_xor_sync(kFull, zt[i], 1));
-      y[i] = fmaf(L.bo[0], z, -0.0f);
+    for (int m = 0; m < 8; ++m) {
+      const float z0 = __fadd_rn(zo[m].x, __shfl_xor_sync(kFull, zt[m].x, 1));
+      const float z1 = __fadd_rn(zo[m].y, __shfl_xor_sync(kFull, zt[m].y, 1));
+      y[2 * m] = fmaf(L.bo[0], z0, -0.0f);
+      y[2 * m + 1] = fmaf(L.bo[0], z1, -0.0f);
     }
-  } else {
-    float z[16];   // Z rows h RH .. h RH + RH - 1
+  } else if constexpr (AD == 1) {
+    // Z = x A[0][0]; stage 2 is the full 32 x 32 B_j (no decomposition)
+    float z[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) z[i] = fmaf(xf[i], L.A[0], -0.0f);
+    float yo[16], yt[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) yo[i] = yt[i] = -0.0f;
+    const int co = h * RH, ct = (1 - h) * RH;
 #pragma unroll
     for (int pp = 0; pp < RH; ++pp) {
 #pragma unroll
-      for (int s = 0; s < AD; ++s) {
-        float acc = -0.0f;
+      for (int rl = 0; rl < RH; ++rl) {
+        const float bo = L.Bl[pp * BatSmemB<AD>::pitch + co + rl];
+        const float bt = L.Bl[pp * BatSmemB<AD>::pitch + ct + rl];
+        yo[rl] = fmaf(bo, z[pp], yo[rl]);
+        yt[rl] = fmaf(bt, z[pp], yt[rl]);
+      }
+    }
 #pragma unroll
-        for (int q = 0; q < AD; ++q) {
-          float aq;
-          if constexpr (AD <= 8) {
-            aq = L.A[q * AD + s];
-          } else {
-            aq = As[q * AD + s];
-          }
-          acc = fmaf(xf[pp * AD + q], aq, acc);
+    for (int i = 0; i < 16; ++i) y[i] = __fadd_rn(yo[i], __shfl_xor_sync(kFull, yt[i], 1));
+  } else {
+    // pairs (s, s + 1) of adjacent outputs per instruction in both stages;
+    // each A pair serves the lane's RH rows (the chains stay in q order)
+    constexpr int AH = AD / 2;
+    float2 z2[8];   // Z rows h RH .. h RH + RH - 1, column pairs
+#pragma unroll
+    for (int i = 0; i < 8; ++i) z2[i] = make_float2(-0.0f, -0.0f);
+#pragma unroll
+    for (int q = 0; q < AD; ++q) {
+      float2 aq[AH];
+      if constexpr (LaneParams<AD>::kRegA) {
+#pragma unroll
+        for (int m = 0; m < AH; ++m) aq[m] = make_float2(L.A[q * AD + 2 * m], L.A[q * AD + 2 * m + 1]);
+      } else if constexpr (AD >= 4) {
+#pragma unroll
+        for (int m4 = 0; m4 < AD / 4; ++m4) {
+          const float4 a4 = reinterpret_cast<const float4*>(As + q * AD)[m4];
+          aq[2 * m4] = make_float2(a4.x, a4.y);
+          aq[2 * m4 + 1] = make_float2(a4.z, a4.w);
         }
-        z[pp * AD + s] = acc;
+      } else {
+        aq[0] = *reinterpret_cast<const float2*>(As + q * AD);
+      }
+#pragma unroll
+      for (int pp = 0; pp < RH; ++pp) {
+        const float xv = xf[pp * AD + q];
+#pragma unroll
+        for (int m = 0; m < AH; ++m) z2[pp * AH + m] = ffma2(make_float2(xv, xv), aq[m], z2[pp * AH + m]);
       }
     }
     // stage 2: this lane's rows' terms of its own outputs (rows h RH ..)
     // and of the partner's outputs (rows (1 - h) RH ..)
-    float yo[16], yt[16];
+    float2 yo[8], yt[8];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) yo[i] = yt[i] = -0.0f;
+    for (int i = 0; i < 8; ++i) yo[i] = yt[i] = make_float2(-0.0f, -0.0f);
     const int co = h * RH, ct = (1 - h) * RH;
 #pragma unroll
     for (int pp = 0; pp < RH; ++pp) {
@@ -177,19 +248,23 @@ __device__ __forceinline__ V16 bat_slice(const V16& v, int h, const LaneParams<A
           bt = L.Bl[pp * BatSmemB<AD>::pitch + ct + rl];
         }
 #pragma unroll
-        for (int s = 0; s < AD; ++s) {
-          yo[rl * AD + s] = fmaf(bo, z[pp * AD + s], yo[rl * AD + s]);
-          yt[rl * AD + s] = fmaf(bt, z[pp * AD + s], yt[rl * AD + s]);
+        for (int m = 0; m < AH; ++m) {
+          yo[rl * AH + m] = ffma2(make_float2(bo, bo), z2[pp * AH + m], yo[rl * AH + m]);
+          yt[rl * AH + m] = ffma2(make_float2(bt, bt), z2[pp * AH + m], yt[rl * AH + m]);
         }
       }
     }
     // __fadd_rn: a one-term chain (b = 2) is a rounded product, which must
     // not be contracted with this addition into one fma
 #pragma unroll
-    for (int i = 0; i < 16; ++i) y[i] = __fadd_rn(yo[i], __shfl_xor_sync(kFull, yt[i], 1));
-    (void)BD;
+    for (int i = 0; i < 8; ++i) {
+      y[2 * i] = __fadd_rn(yo[i].x, __shfl_xor_sync(kFull, yt[i].x, 1));
+      y[2 * i + 1] = __fadd_rn(yo[i].y, __shfl_xor_sync(kFull, yt[i].y, 1));
+    }
   }
 
+  uint32_t lo2 = 0, hi2 = 0;
+  bool packed_clip = false;
   if (clip) {
     float mx = y[0], mn = y[0];
 #pragma unroll
@@ -202,11 +277,15 @@ __device__ __forceinline__ V16 bat_slice(const V16& v, int h, const LaneParams<A
     if (isfinite(mx) && isfinite(mn)) {
       const float lo = __fmul_rn(L.bmin, mn);
       const float hi = __fmul_rn(L.bmax, mx);
-      if (lo != 0.0f && hi != 0.0f) {
-        // a nonzero bound equals y only with the same sign: min/max are
-        // then exactly the comparisons below (a NaN bound leaves y alone)
-#pragma unroll
-        for (int i = 0; i < 16; ++i) y[i] = fminf(fmaxf(y[i], lo), hi);
+      lo2 = pack_bf16x2(lo, lo);
+      hi2 = pack_bf16x2(hi, hi);
+      if ((lo2 & 0x7FFFu) != 0 && (hi2 & 0x7FFFu) != 0) {
+        // Rounding to bf16 is monotone, so it commutes with min and max:
+        // clamping the rounded values to the rounded bounds gives the
+        // rounded clamp. With both rounded bounds nonzero a tie is between
+        // identical values, so the bits agree too (a NaN bound is ignored
+        // by both forms).
+        packed_clip = true;
       } else {
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
@@ -219,6 +298,10 @@ __device__ __forceinline__ V16 bat_slice(const V16& v, int h, const LaneParams<A
   V16 o;
 #pragma unroll
   for (int i = 0; i < 8; ++i) o.w[i] = pack_bf16x2(y[2 * i], y[2 * i + 1]);
+  if (packed_clip) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) o.w[i] = clamp_bf16x2(o.w[i], lo2, hi2);
+  }
   return o;
 }
 
@@ -240,8 +323,13 @@ __device__ __forceinline__ void canonical_nan(V16& v) {
 // step. Each thread streams its 32 bytes of successive rows through a ring of
 // kBatStages slots (cp.async, waited per thread: no block-wide barrier after
 // the parameters are staged).
+// Resident CTAs per SM the register budget is cut for (a = 8 / the others).
+#ifndef MX_BAT_MINB8
+#define MX_BAT_MINB8 3
+#endif
+
 template <int AD, int OP, int FMT, int RULE, int MBS>
-__global__ void __launch_bounds__(kThreads) bat_kernel(StreamArgs a, BatParams p) {
+__global__ void __launch_bounds__(kThreads, AD == 8 ? MX_BAT_MINB8 : 2) bat_kernel(StreamArgs a, BatParams p) {
   extern __shared__ __align__(16) uint8_t smem[];
   float* As = reinterpret_cast<float*>(smem + kBatRing);
   float* Bs = As + AD * AD;
@@ -269,11 +357,11 @@ __global__ void __launch_bounds__(kThreads) bat_kernel(StreamArgs a, BatParams p
 
   LaneParams<AD> L;
   constexpr int BD = LaneParams<AD>::BD, RH = LaneParams<AD>::RH;
-  if constexpr (AD <= 8) {
+  if constexpr (LaneParams<AD>::kRegA) {
 #pragma unroll
     for (int i = 0; i < AD * AD; ++i) L.A[i] = As[i];
   } else {
-    L.A[0] = 0.0f;
+    L.A[0] = As[0];
   }
   if constexpr (AD == 32) {
     L.bo[0] = p.B[j];
