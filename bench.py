@@ -254,7 +254,7 @@ def stack_ops(mx, x, reps=50, only=None):
     g = torch.empty_like(x).normal_()
     fp4, fp8, fp4m = n * 2.53125, n * 3.03125, n * (2.53125 + 1 / 128)
     from fp8_quantization_mx_b200 import inputs as _inputs
-    bat = {a: _inputs.bat_params(a, cols // 32, device=dev) for a in (1, 4, 8)}
+    bat = {a: _inputs.bat_params(a, cols // 32, device=dev) for a in (1, 2, 4, 8)}
     ops = {
         "fp4_floor_quantize": (lambda: mx.quantize(x, mx.E2M1, mx.FLOOR, out=(c4, sc, None)), fp4),
         "fp8_floor_quantize": (lambda: mx.quantize(x, mx.E4M3, mx.FLOOR, out=(c8, sc, None)), fp8),
@@ -285,6 +285,7 @@ def stack_ops(mx, x, reps=50, only=None):
         # BATQuant: block transform B_j (x) A (a x a, b x b), clip, MXFP4 FLOOR
         "fp4_bat_a8_quantize": (lambda: mx.bat_quantize(x, *bat[8], out=(c4, sc, None)), fp4),
         "fp4_bat_a4_quantize": (lambda: mx.bat_quantize(x, *bat[4], out=(c4, sc, None)), fp4),
+        "fp4_bat_a2_quantize": (lambda: mx.bat_quantize(x, *bat[2], out=(c4, sc, None)), fp4),
         "fp4_bat_a1_quantize": (lambda: mx.bat_quantize(x, *bat[1], out=(c4, sc, None)), fp4),
         "bat_a8_apply": (lambda: mx.bat_apply(x, *bat[8], out=y), n * 4),
         "fp4_mbs_dynamic_quantize": (lambda: mx.quantize(x, mx.E2M1, mx.MBS_DYNAMIC, out=(c4, sc, mac)),

@@ -62,19 +62,27 @@ constexpr int kBatRing = kBatStages * 32 * kThreads;   // ring bytes
 #endif
 
 // Shared-memory layout of B for a <= 2 (where a lane's rows of B_j do not fit
-// in registers): the 16 blocks of the CTA's column chunk, rows of `pitch`
-// floats, blocks `stride` floats apart. The paddings put the 32 lanes'
-// addresses of one read (16 blocks x 2 halves) in 32 distinct banks.
+// in registers): the 16 blocks of the CTA's column chunk, rows of b floats,
+// the lower-half rows (p >= b/2) 16 bytes further on, blocks `stride` floats
+// apart. A lane reads 16 bytes at a time; with stride / 4 = 2 (mod 8) and the
+// half offset, the 8 lanes of each quarter-warp phase (4 blocks x 2 halves)
+// hit 8 distinct 16-byte bank groups, for its own columns and the partner's.
 template <int AD> struct BatSmemB {
   static constexpr int BD = 32 / AD;
-  static constexpr int pitch = AD == 1 ? 32 : 17;
-  static constexpr int stride = AD == 1 ? 1025 : 289;
+  static constexpr int RH = BD / 2;
+  static constexpr int pitch = BD;
+  static constexpr int half_off = 4;
+  static constexpr int stride = AD == 1 ? 1032 : 264;
   static constexpr int floats = AD <= 2 ? 16 * stride : 0;
+  __host__ __device__ static constexpr int offset(int p, int r) { return p * pitch + (p >= RH ? half_off : 0) + r; }
 };
+
+// A's shared-memory slot, rounded up to 16 bytes so that B stays aligned.
+template <int AD> __host__ __device__ constexpr int bat_a_floats() { return (AD * AD + 3) / 4 * 4; }
 
 template <int AD>
 constexpr size_t bat_smem_bytes() {
-  return kBatRing + sizeof(float) * (AD * AD + BatSmemB<AD>::floats);
+  return kBatRing + sizeof(float) * (bat_a_floats<AD>() + BatSmemB<AD>::floats);
 }
 
 __device__ __forceinline__ void cp_async16(void* dst, const void* src, int src_bytes) {
@@ -179,26 +187,80 @@ __device__ __forceinline__ V16 bat_slice(const V16& v, int h, const LaneParams<A
       y[2 * m + 1] = fmaf(L.bo[0], z1, -0.0f);
     }
   } else if constexpr (AD == 1) {
-    // Z = x A[0][0]; stage 2 is the full 32 x 32 B_j (no decomposition)
+    // Z = x A[0][0]; stage 2 is the full 32 x 32 B_j (no decomposition), in
+    // pairs of adjacent output rows: B_j's row pairs come 4 floats per load
     float z[16];
 #pragma unroll
     for (int i = 0; i < 16; ++i) z[i] = fmaf(xf[i], L.A[0], -0.0f);
-    float yo[16], yt[16];
+    float2 yo[8], yt[8];
 #pragma unroll
-    for (int i = 0; i < 16; ++i) yo[i] = yt[i] = -0.0f;
-    const int co = h * RH, ct = (1 - h) * RH;
+    for (int i = 0; i < 8; ++i) yo[i] = yt[i] = make_float2(-0.0f, -0.0f);
+    const float* Bo = L.Bl + h * RH;
+    const float* Bt = L.Bl + (1 - h) * RH;
 #pragma unroll
     for (int pp = 0; pp < RH; ++pp) {
+      const float2 zd = make_float2(z[pp], z[pp]);
 #pragma unroll
-      for (int rl = 0; rl < RH; ++rl) {
-        const float bo = L.Bl[pp * BatSmemB<AD>::pitch + co + rl];
-        const float bt = L.Bl[pp * BatSmemB<AD>::pitch + ct + rl];
-        yo[rl] = fmaf(bo, z[pp], yo[rl]);
-        yt[rl] = fmaf(bt, z[pp], yt[rl]);
+      for (int q4 = 0; q4 < RH / 4; ++q4) {
+        const float4 bo = reinterpret_cast<const float4*>(Bo + pp * BatSmemB<AD>::pitch)[q4];
+        const float4 bt = reinterpret_cast<const float4*>(Bt + pp * BatSmemB<AD>::pitch)[q4];
+        yo[2 * q4] = ffma2(make_float2(bo.x, bo.y), zd, yo[2 * q4]);
+        yo[2 * q4 + 1] = ffma2(make_float2(bo.z, bo.w), zd, yo[2 * q4 + 1]);
+        yt[2 * q4] = ffma2(make_float2(bt.x, bt.y), zd, yt[2 * q4]);
+        yt[2 * q4 + 1] = ffma2(make_float2(bt.z, bt.w), zd, yt[2 * q4 + 1]);
       }
     }
 #pragma unroll
-    for (int i = 0; i < 16; ++i) y[i] = __fadd_rn(yo[i], __shfl_xor_sync(kFull, yt[i], 1));
+    for (int j = 0; j < 8; ++j) {
+      y[2 * j] = __fadd_rn(yo[j].x, __shfl_xor_sync(kFull, yt[j].x, 1));
+      y[2 * j + 1] = __fadd_rn(yo[j].y, __shfl_xor_sync(kFull, yt[j].y, 1));
+    }
+  } else if constexpr (AD == 2) {
+    // stage 1 in pairs (Z[p][0], Z[p][1]); stage 2 in pairs of adjacent
+    // output rows (Y[r][s], Y[r+1][s]) from 16-byte loads of B_j's rows
+    float2 z2[8];
+#pragma unroll
+    for (int pp = 0; pp < RH; ++pp) {
+      float2 acc = make_float2(-0.0f, -0.0f);
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        const float xv = xf[pp * 2 + q];
+        acc = ffma2(make_float2(xv, xv), make_float2(L.A[q * 2], L.A[q * 2 + 1]), acc);
+      }
+      z2[pp] = acc;
+    }
+    float2 yo[2][4], yt[2][4];   // [s][row pair]
+#pragma unroll
+    for (int i = 0; i < 4; ++i) yo[0][i] = yo[1][i] = yt[0][i] = yt[1][i] = make_float2(-0.0f, -0.0f);
+    const float* Bo = L.Bl + h * RH;
+    const float* Bt = L.Bl + (1 - h) * RH;
+#pragma unroll
+    for (int pp = 0; pp < RH; ++pp) {
+      const float2 zd0 = make_float2(z2[pp].x, z2[pp].x);
+      const float2 zd1 = make_float2(z2[pp].y, z2[pp].y);
+#pragma unroll
+      for (int q4 = 0; q4 < RH / 4; ++q4) {
+        const float4 bo = reinterpret_cast<const float4*>(Bo + pp * BatSmemB<AD>::pitch)[q4];
+        const float4 bt = reinterpret_cast<const float4*>(Bt + pp * BatSmemB<AD>::pitch)[q4];
+        yo[0][2 * q4] = ffma2(make_float2(bo.x, bo.y), zd0, yo[0][2 * q4]);
+        yo[0][2 * q4 + 1] = ffma2(make_float2(bo.z, bo.w), zd0, yo[0][2 * q4 + 1]);
+        yo[1][2 * q4] = ffma2(make_float2(bo.x, bo.y), zd1, yo[1][2 * q4]);
+        yo[1][2 * q4 + 1] = ffma2(make_float2(bo.z, bo.w), zd1, yo[1][2 * q4 + 1]);
+        yt[0][2 * q4] = ffma2(make_float2(bt.x, bt.y), zd0, yt[0][2 * q4]);
+        yt[0][2 * q4 + 1] = ffma2(make_float2(bt.z, bt.w), zd0, yt[0][2 * q4 + 1]);
+        yt[1][2 * q4] = ffma2(make_float2(bt.x, bt.y), zd1, yt[1][2 * q4]);
+        yt[1][2 * q4 + 1] = ffma2(make_float2(bt.z, bt.w), zd1, yt[1][2 * q4 + 1]);
+      }
+    }
+    // element r * 2 + s of this lane's half
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+#pragma unroll
+      for (int sc = 0; sc < 2; ++sc) {
+        y[(2 * j) * 2 + sc] = __fadd_rn(yo[sc][j].x, __shfl_xor_sync(kFull, yt[sc][j].x, 1));
+        y[(2 * j + 1) * 2 + sc] = __fadd_rn(yo[sc][j].y, __shfl_xor_sync(kFull, yt[sc][j].y, 1));
+      }
+    }
   } else {
     // pairs (s, s + 1) of adjacent outputs per instruction in both stages;
     // each A pair serves the lane's RH rows (the chains stay in q order)
@@ -234,19 +296,13 @@ __device__ __forceinline__ V16 bat_slice(const V16& v, int h, const LaneParams<A
     float2 yo[8], yt[8];
 #pragma unroll
     for (int i = 0; i < 8; ++i) yo[i] = yt[i] = make_float2(-0.0f, -0.0f);
-    const int co = h * RH, ct = (1 - h) * RH;
 #pragma unroll
     for (int pp = 0; pp < RH; ++pp) {
 #pragma unroll
       for (int rl = 0; rl < RH; ++rl) {
-        float bo, bt;
-        if constexpr (LaneParams<AD>::kRegB) {
-          bo = L.bo[pp * RH + rl];
-          bt = L.bt[pp * RH + rl];
-        } else {
-          bo = L.Bl[pp * BatSmemB<AD>::pitch + co + rl];
-          bt = L.Bl[pp * BatSmemB<AD>::pitch + ct + rl];
-        }
+        static_assert(LaneParams<AD>::kRegB, "a >= 4 keeps B_j's terms in registers");
+        const float bo = L.bo[pp * RH + rl];
+        const float bt = L.bt[pp * RH + rl];
 #pragma unroll
         for (int m = 0; m < AH; ++m) {
           yo[rl * AH + m] = ffma2(make_float2(bo, bo), z2[pp * AH + m], yo[rl * AH + m]);
@@ -332,7 +388,7 @@ template <int AD, int OP, int FMT, int RULE, int MBS>
 __global__ void __launch_bounds__(kThreads, AD == 8 ? MX_BAT_MINB8 : 2) bat_kernel(StreamArgs a, BatParams p) {
   extern __shared__ __align__(16) uint8_t smem[];
   float* As = reinterpret_cast<float*>(smem + kBatRing);
-  float* Bs = As + AD * AD;
+  float* Bs = As + bat_a_floats<AD>();
   const int cc = blockIdx.x % p.nchunks;
   const int64_t g = blockIdx.x / p.nchunks;
   const int64_t G = gridDim.x / p.nchunks;
@@ -349,7 +405,7 @@ __global__ void __launch_bounds__(kThreads, AD == 8 ? MX_BAT_MINB8 : 2) bat_kern
     for (int i = tid; i < 16 * SB::BD * SB::BD; i += kThreads) {
       const int jl = i / (SB::BD * SB::BD), e = i % (SB::BD * SB::BD);
       const int64_t jj = static_cast<int64_t>(cc) * 16 + jl;
-      Bs[jl * SB::stride + (e / SB::BD) * SB::pitch + e % SB::BD] =
+      Bs[jl * SB::stride + SB::offset(e / SB::BD, e % SB::BD)] =
           jj < nb ? p.B[jj * SB::BD * SB::BD + e] : 0.0f;
     }
   }
@@ -379,7 +435,8 @@ __global__ void __launch_bounds__(kThreads, AD == 8 ? MX_BAT_MINB8 : 2) bat_kern
   } else {
     L.bo[0] = L.bt[0] = 0.0f;
   }
-  L.Bl = Bs + (lane >> 1) * BatSmemB<AD>::stride + (h * RH) * BatSmemB<AD>::pitch;
+  // a <= 2: this lane's rows h RH .. of B_j in shared memory
+  L.Bl = Bs + (lane >> 1) * BatSmemB<AD>::stride + BatSmemB<AD>::offset(h * RH, 0);
   const bool clip = p.bmin != nullptr;
   L.bmin = clip ? p.bmin[j] : 0.0f;
   L.bmax = clip ? p.bmax[j] : 0.0f;
