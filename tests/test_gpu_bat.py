@@ -156,3 +156,22 @@ def test_full_moe_stack_sampled_rows(mx, oracle_mod, cuda):
     oy = oracle_mod.bat_apply(xs, 8, _np(A), _np(B), _np(bmin), _np(bmax))
     assert np.array_equal(inputs.bf16_bits_numpy(y[idx.to(cuda)]), oy)
     del x, y, codes, scales
+
+
+def test_more_than_2_31_elements(mx, oracle_mod, cuda):
+    """64-bit indexing: a tensor of 2^31 + 131072 elements (4.3 GB bf16); rows
+    past the 2^31-th element against the oracle."""
+    cols = 2048
+    rows = (1 << 31) // cols + 64
+    x = torch.empty(rows, cols, dtype=torch.bfloat16, device=cuda)
+    x.copy_(inputs.outlier_act(64, cols, seed=77).to(cuda).repeat(rows // 64, 1))
+    A, B, bmin, bmax = inputs.bat_params(8, cols // 32, seed=3, device=cuda)
+    codes, scales, _ = mx.bat_quantize(x, A, B, bmin, bmax, E2M1, FLOOR)
+    torch.cuda.synchronize()
+    tail = slice(rows - 40, rows)
+    xs = inputs.bf16_bits_numpy(x[tail])
+    oc, os_, _ = oracle_mod.bat_quantize(xs, 8, _np(A), _np(B), _np(bmin), _np(bmax), E2M1, FLOOR)
+    assert np.array_equal(codes[tail].cpu().numpy(), oc)
+    assert np.array_equal(scales[tail].cpu().numpy(), os_)
+    del x, codes, scales
+    torch.cuda.empty_cache()
