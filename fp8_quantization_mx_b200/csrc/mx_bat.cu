@@ -107,23 +107,6 @@ __device__ __forceinline__ float min_nan(float a, float b) {
   return d;
 }
 
-// Two fused multiply-adds in one instruction (sm_100 packed fp32): each half
-// is an IEEE fma rounded to nearest even, exactly as fmaf.
-__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
-  float2 d;
-  asm("{\n"
-      " .reg .b64 ra, rb, rc, rd;\n"
-      " mov.b64 ra, {%2, %3};\n"
-      " mov.b64 rb, {%4, %5};\n"
-      " mov.b64 rc, {%6, %7};\n"
-      " fma.rn.f32x2 rd, ra, rb, rc;\n"
-      " mov.b64 {%0, %1}, rd;\n"
-      "}"
-      : "=f"(d.x), "=f"(d.y)
-      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
-  return d;
-}
-
 // Per-half clamp of packed bf16: min(max(v, lo), hi) (a NaN bound is ignored).
 __device__ __forceinline__ uint32_t clamp_bf16x2(uint32_t v, uint32_t lo, uint32_t hi) {
   uint32_t d;

@@ -188,6 +188,55 @@ __device__ __forceinline__ float sq_acc_hi(uint32_t w, float acc) {
   return d;
 }
 
+// Two fused multiply-adds in one instruction (sm_100 packed fp32): each half
+// is an IEEE fma rounded to nearest even, exactly as fmaf.
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("{\n"
+      " .reg .b64 ra, rb, rc, rd;\n"
+      " mov.b64 ra, {%2, %3};\n"
+      " mov.b64 rb, {%4, %5};\n"
+      " mov.b64 rc, {%6, %7};\n"
+      " fma.rn.f32x2 rd, ra, rb, rc;\n"
+      " mov.b64 {%0, %1}, rd;\n"
+      "}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
+}
+
+// Two products in one instruction (sm_100 packed fp32): each half is an IEEE
+// product rounded to nearest even, exactly as a * b.
+__device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n"
+      " .reg .b64 ra, rb, rd;\n"
+      " mov.b64 ra, {%2, %3};\n"
+      " mov.b64 rb, {%4, %5};\n"
+      " mul.rn.f32x2 rd, ra, rb;\n"
+      " mov.b64 {%0, %1}, rd;\n"
+      "}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+
+// lo[i] = e[i] * L and hi[i] = e[i] * H for N (even) values, two per
+// instruction: the two ends of a reciprocal bracket.
+template <int N>
+__device__ __forceinline__ void bracket_products(const float* e, float L, float H, float* lo, float* hi) {
+  const float2 l2 = make_float2(L, L), h2 = make_float2(H, H);
+#pragma unroll
+  for (int i = 0; i < N / 2; ++i) {
+    const float2 p = make_float2(e[2 * i], e[2 * i + 1]);
+    const float2 a = fmul2(p, l2), b = fmul2(p, h2);
+    lo[2 * i] = a.x;
+    lo[2 * i + 1] = a.y;
+    hi[2 * i] = b.x;
+    hi[2 * i + 1] = b.y;
+  }
+}
+
 // ------------------------------------------------------- element encoding --
 
 // Two bf16x2 words (4 scaled values, element order) -> 4 E2M1 codes in the low
@@ -801,13 +850,10 @@ __device__ __forceinline__ uint32_t even_of_adjacent(uint32_t lo, uint32_t hi) {
 __device__ __forceinline__ uint2 enc_mbs_cvt_16(const V16& x, int b, int k) {
   const FactorBracket fb = factor_bracket(k);
   const V16 s = scale_slice(x, b);
-  float lo[16], hi[16];
+  float e[16], lo[16], hi[16];
 #pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    const float e = elem(s, i);
-    lo[i] = e * fb.L;
-    hi[i] = e * fb.H;
-  }
+  for (int i = 0; i < 16; ++i) e[i] = elem(s, i);
+  bracket_products<16>(e, fb.L, fb.H, lo, hi);
   return make_uint2(even_of_adjacent(cvt_e2m1_f8(lo), cvt_e2m1_f8(hi)),
                     even_of_adjacent(cvt_e2m1_f8(lo + 8), cvt_e2m1_f8(hi + 8)));
 }
@@ -822,11 +868,7 @@ __device__ __forceinline__ int small_int(float v) {
 // enc_mbs_cvt_16), and their E2M1 magnitudes as floats.
 __device__ __forceinline__ uint32_t mbs_codes8(const float* s8, float L, float H) {
   float lo[8], hi[8];
-#pragma unroll
-  for (int j = 0; j < 8; ++j) {
-    lo[j] = s8[j] * L;
-    hi[j] = s8[j] * H;
-  }
+  bracket_products<8>(s8, L, H, lo, hi);
   return even_of_adjacent(cvt_e2m1_f8(lo), cvt_e2m1_f8(hi));
 }
 // ---------------------------------------------------------------- NVFP4 --
@@ -863,13 +905,10 @@ __device__ __forceinline__ uint2 enc_e2m1_div_16(const V16& x, float s) {
   asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(inv) : "f"(s));
   const float L = inv * 0.99999904632568359375f;   // 1 - 2^-20
   const float H = inv * 1.00000095367431640625f;   // 1 + 2^-20
-  float lo[16], hi[16];
+  float e[16], lo[16], hi[16];
 #pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    const float e = elem(x, i);
-    lo[i] = e * L;
-    hi[i] = e * H;
-  }
+  for (int i = 0; i < 16; ++i) e[i] = elem(x, i);
+  bracket_products<16>(e, L, H, lo, hi);
   return make_uint2(even_of_adjacent(cvt_e2m1_f8(lo), cvt_e2m1_f8(hi)),
                     even_of_adjacent(cvt_e2m1_f8(lo + 8), cvt_e2m1_f8(hi + 8)));
 }
@@ -900,13 +939,8 @@ __device__ __forceinline__ OasEval oas_eval_mbs16(const V16& x, int b1, int k) {
   OasEval r;
   {
     float lo[16], hi[16], lo2[16], hi2[16];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      lo[i] = s[i] * fb.L;
-      hi[i] = s[i] * fb.H;
-      lo2[i] = h[i] * fb.L;
-      hi2[i] = h[i] * fb.H;
-    }
+    bracket_products<16>(s, fb.L, fb.H, lo, hi);
+    bracket_products<16>(h, fb.L, fb.H, lo2, hi2);
     r.c1 = make_uint2(even_of_adjacent(cvt_e2m1_f8(lo), cvt_e2m1_f8(hi)),
                       even_of_adjacent(cvt_e2m1_f8(lo + 8), cvt_e2m1_f8(hi + 8)));
     r.c2 = make_uint2(even_of_adjacent(cvt_e2m1_f8(lo2), cvt_e2m1_f8(hi2)),
