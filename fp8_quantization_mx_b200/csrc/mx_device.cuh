@@ -696,15 +696,20 @@ __device__ __forceinline__ OasEval oas_eval16(const V16& x, int b1) {
   r.c2 = enc_e2m1_16(s2);
   const V16 q1 = e2m1x16_to_bf16(r.c1);
   const V16 q2 = e2m1x16_to_bf16(r.c2);
-  float acc = 0.0f;
+  // d1 = s - q1, d2 = s - 2 q2, sum of (d1 - d2)(d1 + d2), two elements per
+  // packed fma; every value and partial sum is an exact multiple of 2^-9
+  // below 2^6, so the order does not matter
+  const float2 m1 = make_float2(-1.0f, -1.0f), p1 = make_float2(1.0f, 1.0f);
+  const float2 m2 = make_float2(-2.0f, -2.0f);
+  float2 acc = make_float2(0.0f, 0.0f);
 #pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    const float s = elem(s1, i);
-    const float d1 = s - elem(q1, i);
-    const float d2 = fmaf(-2.0f, elem(q2, i), s);
-    acc = fmaf(d1 - d2, d1 + d2, acc);
+  for (int w = 0; w < 8; ++w) {
+    const float2 s = make_float2(bf_lo(s1.w[w]), bf_hi(s1.w[w]));
+    const float2 d1 = ffma2(make_float2(bf_lo(q1.w[w]), bf_hi(q1.w[w])), m1, s);
+    const float2 d2 = ffma2(make_float2(bf_lo(q2.w[w]), bf_hi(q2.w[w])), m2, s);
+    acc = ffma2(ffma2(d2, m1, d1), ffma2(d2, p1, d1), acc);
   }
-  r.delta = __float2int_rn(acc * 1024.0f);   // an integer below 2^16: exact
+  r.delta = __float2int_rn((acc.x + acc.y) * 1024.0f);   // an integer below 2^16: exact
   return r;
 }
 
@@ -932,9 +937,12 @@ __device__ __forceinline__ OasEval oas_eval_mbs16(const V16& x, int b1, int k) {
   const V16 s1 = scale_slice(x, b1);
   float s[16], h[16];
 #pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    s[i] = elem(s1, i);
-    h[i] = s[i] * 0.5f;
+  for (int i = 0; i < 8; ++i) {
+    s[2 * i] = bf_lo(s1.w[i]);
+    s[2 * i + 1] = bf_hi(s1.w[i]);
+    const float2 hh = fmul2(make_float2(s[2 * i], s[2 * i + 1]), make_float2(0.5f, 0.5f));
+    h[2 * i] = hh.x;
+    h[2 * i + 1] = hh.y;
   }
   OasEval r;
   {
@@ -948,13 +956,21 @@ __device__ __forceinline__ OasEval oas_eval_mbs16(const V16& x, int b1, int k) {
   }
   const V16 q1 = e2m1x16_to_bf16(r.c1);
   const V16 q2 = e2m1x16_to_bf16(r.c2);
-  const float f2 = fb.f * 2.0f;
+  // D = 512 (s - q f), two elements per packed fma; the second fma scales
+  // by 512 (exact) and adds 1.5 * 2^23, which leaves the integer D in the
+  // low mantissa bits (as small_int)
+  const float2 nf1 = make_float2(-fb.f, -fb.f), nf2 = make_float2(-2.0f * fb.f, -2.0f * fb.f);
+  const float2 k512 = make_float2(512.0f, 512.0f), kmag = make_float2(12582912.0f, 12582912.0f);
   int acc = 0;
 #pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    const int D1 = small_int(fmaf(-elem(q1, i), fb.f, s[i]) * 512.0f);
-    const int D2 = small_int(fmaf(-elem(q2, i), f2, s[i]) * 512.0f);
-    acc += D1 * D1 - D2 * D2;
+  for (int w = 0; w < 8; ++w) {
+    const float2 sp = make_float2(s[2 * w], s[2 * w + 1]);
+    const float2 t1 = ffma2(make_float2(bf_lo(q1.w[w]), bf_hi(q1.w[w])), nf1, sp);
+    const float2 t2 = ffma2(make_float2(bf_lo(q2.w[w]), bf_hi(q2.w[w])), nf2, sp);
+    const float2 u1 = ffma2(t1, k512, kmag), u2 = ffma2(t2, k512, kmag);
+    const int a0 = __float_as_int(u1.x) - 0x4B400000, a1 = __float_as_int(u1.y) - 0x4B400000;
+    const int b0 = __float_as_int(u2.x) - 0x4B400000, b1v = __float_as_int(u2.y) - 0x4B400000;
+    acc += a0 * a0 - b0 * b0 + a1 * a1 - b1v * b1v;
   }
   r.delta = acc;
   return r;

@@ -21,7 +21,7 @@ MMA = 1 << 8
 A_DIMS = (1, 2, 4, 8, 16, 32)
 # shapes: several warp tiles with a ragged last one; rows shorter than a
 # 512-element tile (tiles wrap rows) and longer
-SHAPES = [(37, 96), (9, 2048), (130, 1152)]
+SHAPES = [(37, 96), (9, 2048), (130, 1152), (5, 32), (1, 64), (3, 8192)]
 
 
 def _np(t):
@@ -126,6 +126,15 @@ def test_edge_blocks(mx, oracle_mod, cuda):
             assert_same(*run_both(mx, oracle_mod, xb, params))
             assert_same(*run_both(mx, oracle_mod, xb, params, E2M1, OAS | MBS_STATIC))
             assert_same(*run_both(mx, oracle_mod, xb, params, E4M3, FLOOR))
+
+
+@pytest.mark.parametrize("shape", [(3, 128), (17, 640), (2, 8192)])
+def test_mbs_macro_blocks_across_chunks(mx, oracle_mod, cuda, shape):
+    # one macro block per row; a partial 512-column chunk; 16 chunks per row
+    rows, cols = shape
+    x = inputs.heavy_tail(rows, cols, seed=cols).to(cuda)
+    params = inputs.bat_params(4, cols // 32, seed=rows, device=cuda, spread=0.3)
+    assert_same(*run_both(mx, oracle_mod, x, params, E2M1, OAS | MBS_STATIC))
 
 
 def test_identity_parameters_are_plain_quantization(mx, cuda):
