@@ -723,11 +723,15 @@ __device__ __forceinline__ OasEval oas_eval16(const V16& x, int b1) {
 // smallest magnitude, so s (8 significant bits) and both grid values are
 // multiples of U and D1, D2 are exact integers below 2^41; an element that
 // rounds to the same value gives D1 == D2 whatever its size. The products
-// reach 2^82 for E5M2, so the sum is kept in 128-bit integers.
+// reach 2^82 for E5M2, so its sum is kept in 128-bit integers; for E4M3,
+// E3M2 and E2M3, |D| < 2^(emax + 11 - min_log2) <= 2^28, every product stays
+// below 2^58 and a lane's sum of 16 below 2^62: 64-bit integers hold them.
 struct OasEvalBytes {
   uint4 c1, c2;
   __int128 delta;
 };
+template <bool kWide> struct OasAcc { using T = long long; };
+template <> struct OasAcc<true> { using T = __int128; };
 template <int FMT>
 __device__ __forceinline__ OasEvalBytes oas_eval_bytes16(const V16& x, int b1) {
   const V16 s1 = scale_slice(x, b1);
@@ -738,13 +742,14 @@ __device__ __forceinline__ OasEvalBytes oas_eval_bytes16(const V16& x, int b1) {
   const F16 q1 = dec_bytes_16<FMT>(r.c1, 1.0f);
   const F16 q2 = dec_bytes_16<FMT>(r.c2, 2.0f);   // E2 values in units of the E1 scale
   const float unit = pow2f(9 - Elem<FMT>::min_log2);
-  __int128 acc = 0;
+  using Acc = typename OasAcc<FMT == kFmtE5M2>::T;
+  Acc acc = 0;
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
     const float si = elem(s1, i);
     const long long D1 = __float2ll_rn((si - q1.v[i]) * unit);
     const long long D2 = __float2ll_rn((si - q2.v[i]) * unit);
-    acc += static_cast<__int128>(D1 - D2) * static_cast<__int128>(D1 + D2);
+    acc += static_cast<Acc>(D1 - D2) * static_cast<Acc>(D1 + D2);
   }
   r.delta = acc;
   return r;
