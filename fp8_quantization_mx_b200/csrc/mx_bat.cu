@@ -362,13 +362,17 @@ __device__ __forceinline__ void canonical_nan(V16& v) {
 // step. Each thread streams its 32 bytes of successive rows through a ring of
 // kBatStages slots (cp.async, waited per thread: no block-wide barrier after
 // the parameters are staged).
-// Resident CTAs per SM the register budget is cut for (a = 8 / the others).
-#ifndef MX_BAT_MINB8
-#define MX_BAT_MINB8 3
+// Resident CTAs per SM the register budget is cut for: 3 (80 registers) where
+// that costs no or few spills, else 2.
+#ifndef MX_BAT_MINB_WIDE
+#define MX_BAT_MINB_WIDE 3
 #endif
+__host__ __device__ constexpr int bat_min_blocks(int ad) {
+  return (ad == 8 || ad == 16) ? 3 : ((ad == 2 || ad == 32) ? MX_BAT_MINB_WIDE : 2);
+}
 
 template <int AD, int OP, int FMT, int RULE, int MBS>
-__global__ void __launch_bounds__(kThreads, AD == 8 ? MX_BAT_MINB8 : 2) bat_kernel(StreamArgs a, BatParams p) {
+__global__ void __launch_bounds__(kThreads, bat_min_blocks(AD)) bat_kernel(StreamArgs a, BatParams p) {
   extern __shared__ __align__(16) uint8_t smem[];
   float* As = reinterpret_cast<float*>(smem + kBatRing);
   float* Bs = As + bat_a_floats<AD>();
