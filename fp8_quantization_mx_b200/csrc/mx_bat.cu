@@ -27,10 +27,11 @@
 // kernel stays close to its issue-rate bound rather than to HBM.
 //
 // A CTA owns one 512-column chunk of many rows, so each lane's block column
-// and parameters are fixed: A is staged once per CTA in shared memory (and
-// copied into registers for a <= 8), a lane's terms of B_j sit in registers
-// (a >= 4) or in shared memory (a <= 2), and so do the thresholds. Rows
-// stream through a per-thread cp.async ring in shared memory.
+// and parameters are fixed. A is staged once per CTA in shared memory, and
+// copied into registers for a <= 4. A lane's terms of B_j sit in registers
+// (a >= 4) or in shared memory (a <= 2), and its thresholds in registers.
+// Rows stream through a per-thread cp.async ring in shared memory. Both
+// stages issue packed fp32 fmas (two outputs per instruction).
 
 #include "mx_stream.cuh"
 
@@ -63,8 +64,8 @@ constexpr int kBatRing = kBatStages * 32 * kThreads;   // ring bytes
 
 // Shared-memory layout of B for a <= 2 (where a lane's rows of B_j do not fit
 // in registers): the 16 blocks of the CTA's column chunk, rows of b floats,
-// the lower-half rows (p >= b/2) 16 bytes further on, blocks `stride` floats
-// apart. A lane reads 16 bytes at a time; with stride / 4 = 2 (mod 8) and the
+// the rows of the block's second half (p >= b/2) 16 bytes further on, blocks
+// `stride` floats apart. A lane reads 16 bytes at a time; with stride / 4 = 2 (mod 8) and the
 // half offset, the 8 lanes of each quarter-warp phase (4 blocks x 2 halves)
 // hit 8 distinct 16-byte bank groups, for its own columns and the partner's.
 template <int AD> struct BatSmemB {
