@@ -726,6 +726,12 @@ __device__ __forceinline__ OasEval oas_eval16(const V16& x, int b1) {
 // reach 2^82 for E5M2, so its sum is kept in 128-bit integers; for E4M3,
 // E3M2 and E2M3, |D| < 2^(emax + 11 - min_log2) <= 2^28, every product stays
 // below 2^58 and a lane's sum of 16 below 2^62: 64-bit integers hold them.
+// The integer held exactly by a float v with |v| < 2^22 (no conversion unit:
+// adding 1.5 * 2^23 puts v in the low mantissa bits).
+__device__ __forceinline__ int small_int(float v) {
+  return __float_as_int(v + 12582912.0f) - 0x4B400000;
+}
+
 struct OasEvalBytes {
   uint4 c1, c2;
   __int128 delta;
@@ -747,8 +753,15 @@ __device__ __forceinline__ OasEvalBytes oas_eval_bytes16(const V16& x, int b1) {
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
     const float si = elem(s1, i);
-    const long long D1 = __float2ll_rn((si - q1.v[i]) * unit);
-    const long long D2 = __float2ll_rn((si - q2.v[i]) * unit);
+    long long D1, D2;
+    if constexpr (Elem<FMT>::emax + 11 - Elem<FMT>::min_log2 <= 22) {
+      // E3M2, E2M3: |D| < 2^22, so the float add of small_int extracts it
+      D1 = small_int((si - q1.v[i]) * unit);
+      D2 = small_int((si - q2.v[i]) * unit);
+    } else {
+      D1 = __float2ll_rn((si - q1.v[i]) * unit);
+      D2 = __float2ll_rn((si - q2.v[i]) * unit);
+    }
     acc += static_cast<Acc>(D1 - D2) * static_cast<Acc>(D1 + D2);
   }
   r.delta = acc;
@@ -866,12 +879,6 @@ __device__ __forceinline__ uint2 enc_mbs_cvt_16(const V16& x, int b, int k) {
   bracket_products<16>(e, fb.L, fb.H, lo, hi);
   return make_uint2(even_of_adjacent(cvt_e2m1_f8(lo), cvt_e2m1_f8(hi)),
                     even_of_adjacent(cvt_e2m1_f8(lo + 8), cvt_e2m1_f8(hi + 8)));
-}
-
-// The integer held exactly by a float v with |v| < 2^22 (no conversion unit:
-// adding 1.5 * 2^23 puts v in the low mantissa bits).
-__device__ __forceinline__ int small_int(float v) {
-  return __float_as_int(v + 12582912.0f) - 0x4B400000;
 }
 
 // Codes of 8 non-negative scaled values under the bracket L <= 1/f <= H (see
