@@ -758,6 +758,10 @@ __device__ __forceinline__ OasEvalBytes oas_eval_bytes16(const V16& x, int b1) {
       // E3M2, E2M3: |D| < 2^22, so the float add of small_int extracts it
       D1 = small_int((si - q1.v[i]) * unit);
       D2 = small_int((si - q2.v[i]) * unit);
+    } else if constexpr (Elem<FMT>::emax + 11 - Elem<FMT>::min_log2 <= 31) {
+      // E4M3: |D| < 2^28 fits the 32-bit converter
+      D1 = __float2int_rn((si - q1.v[i]) * unit);
+      D2 = __float2int_rn((si - q2.v[i]) * unit);
     } else {
       D1 = __float2ll_rn((si - q1.v[i]) * unit);
       D2 = __float2ll_rn((si - q2.v[i]) * unit);
