@@ -9,11 +9,14 @@ tensors are not on a CUDA device, the calls raise.
 Two layers, both exported here:
 
 * ``mx_quantize``, ``mx_dequantize``, ``mx_fake_quant_fwd``,
-  ``mx_fake_quant_bwd``, ``mx_block_error``, ``mx_status_string``: the C
+  ``mx_fake_quant_bwd``, ``mx_block_error``, ``mx_bat_apply``,
+  ``mx_bat_quantize``, ``mx_scale_bytes``, ``mx_status_string``: the C
   functions with their C names and arguments (raw pointers as ints, stream as
   an int handle), returning the status code.
 * ``quantize``, ``dequantize``, ``fake_quant``, ``fake_quant_bwd``,
-  ``block_error``: tensor-level calls that check tensors, allocate outputs
+  ``block_error``, ``bat_apply``, ``bat_quantize`` (BATQuant's block
+  transform and clip, alone or fused with quantize):
+  tensor-level calls that check tensors, allocate outputs
   with torch on the input's device, launch on the current CUDA stream and
   raise ``MXError`` on a nonzero status. ``quantize`` and ``dequantize`` also
   take CPU tensors: the binding then copies the input to the GPU, launches,
