@@ -109,3 +109,42 @@ def test_sharded_error_stats_equal_the_whole_tensor(oracle_mod, world):
     mse_full, sqnr_full = sd / x.size, 10 * np.log10(sx / sd)
     for _, mse, sqnr in res:
         assert np.isclose(mse, mse_full, rtol=1e-12) and np.isclose(sqnr, sqnr_full, rtol=1e-12)
+
+
+def _bat_worker(rank, world, port, x_bits, params, out):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    import oracle
+    r0, r1 = shard_rows(x_bits.shape[0], world, rank)
+    A, B, bmin, bmax = params
+    c, s, _ = oracle.bat_quantize(np.ascontiguousarray(x_bits[r0:r1]), A.shape[0], A, B, bmin, bmax)
+    parts = [None] * world
+    dist.all_gather_object(parts, (r0, r1, c, s))
+    if rank == 0:
+        out.put(parts)
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def test_two_rank_batquant_shards_match_whole_tensor(oracle_mod):
+    """BATQuant's parameters belong to column blocks: every rank passes the
+    same A, B and thresholds with its own rows, and the gathered result is
+    the whole tensor's."""
+    from fp8_quantization_mx_b200 import inputs
+    x = inputs.bf16_bits_numpy(inputs.outlier_act(rows=29, cols=256, seed=5))
+    params = tuple(None if t is None else t.numpy() for t in inputs.bat_params(8, 256 // 32, seed=2))
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_bat_worker, args=(r, 2, port, x, params, q)) for r in range(2)]
+    for p in procs:
+        p.start()
+    parts = q.get(timeout=120)
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    A, B, bmin, bmax = params
+    c_full, s_full, _ = oracle_mod.bat_quantize(x, 8, A, B, bmin, bmax)
+    for r0, r1, c, s in parts:
+        assert np.array_equal(c, c_full[r0:r1]) and np.array_equal(s, s_full[r0:r1])
+    assert sum(p[1] - p[0] for p in parts) == 29
