@@ -157,6 +157,17 @@ def test_clip_hand_worked():
     assert np.all(y == 0)
 
 
+def test_clip_all_negative_block_hand_worked():
+    # max y = -1: hi = 0.5 * -1 = -0.5 lies above every value (no upper clip);
+    # min y = -8: lo = 0.5 * -8 = -4, so -8 and -6 become -4
+    eye = (np.eye(8, dtype=np.float32), np.eye(4, dtype=np.float32)[None])
+    x = np.full((1, 32), -1.0)
+    x[0, :3] = [-8, -6, -2]
+    y = bits_to_f64(oracle.bat_apply(bf16_bits(x), 8, *eye, np.float32([0.5]), np.float32([0.5])))
+    assert list(y[0, :3]) == [-4, -4, -2]
+    assert np.all(y[0, 3:] == -1)
+
+
 def test_nonfinite_blocks_are_not_clipped_and_nan_is_canonical():
     eye = (np.eye(8, dtype=np.float32), np.eye(4, dtype=np.float32)[None])
     x = np.full((1, 32), 2.0)
