@@ -193,6 +193,50 @@ def _cuda_bf16(x: torch.Tensor, name: str):
         raise ValueError(f"{name} must be contiguous (row-major)")
 
 
+def _check_buf(t, name: str, device, dtype, need: int):
+    """A caller-supplied buffer must be a contiguous ``dtype`` tensor on
+    ``device`` holding at least ``need`` elements: the kernels write through
+    its raw pointer, so a host tensor, a short buffer or a narrower dtype
+    would be written out of bounds."""
+    if not isinstance(t, torch.Tensor):
+        raise ValueError(f"{name} must be a tensor")
+    if t.device != torch.device(device):
+        raise ValueError(f"{name} must be on {device}, got {t.device}")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if t.numel() < need:
+        raise ValueError(f"{name} holds {t.numel()} elements, needs at least {need}")
+
+
+def _scale_count(rows, cols, format, scaling) -> int:
+    if scaling & MMA_SCALES:
+        return mx_scale_bytes(rows, cols, format, scaling)
+    return rows * (cols // block_size(format))
+
+
+def _quantize_buffers(device, lead, rows, cols, format, scaling, out):
+    """The (codes, scales, macro) a quantize call writes: new tensors on
+    ``device`` when ``out`` is None, else ``out`` after checking each buffer
+    against what the kernels write (device, uint8, contiguous, size)."""
+    mbs = ((scaling >> 4) & 3) != 0
+    ccols = cols // 2 if format in _PACKED else cols
+    if out is None:
+        codes = torch.empty(*lead, ccols, dtype=torch.uint8, device=device)
+        scales = _scales_buffer(lead, rows, cols, format, scaling, device)
+        macro = torch.empty(*lead, cols // 128, dtype=torch.uint8, device=device) if mbs else None
+        return codes, scales, macro
+    if len(out) != 3:
+        raise ValueError("out must be (codes, scales, macro)")
+    codes, scales, macro = out
+    _check_buf(codes, "codes", device, torch.uint8, rows * ccols)
+    _check_buf(scales, "scales", device, torch.uint8, _scale_count(rows, cols, format, scaling))
+    if mbs:
+        _check_buf(macro, "macro", device, torch.uint8, rows * (cols // 128))
+    return codes, scales, macro
+
+
 def quantize(x: torch.Tensor, format: int = E2M1, scaling: int = FLOOR, out=None):
     """MX-quantizes bf16 ``x`` [..., cols] along its last dimension.
 
@@ -208,6 +252,9 @@ def quantize(x: torch.Tensor, format: int = E2M1, scaling: int = FLOOR, out=None
     like a single kernel on the current stream.
     """
     if not x.is_cuda:
+        if out is not None:
+            rows, cols = _rows_cols(x)
+            _quantize_buffers(torch.device("cpu"), x.shape[:-1], rows, cols, format, scaling, out)
         dev = torch.device("cuda", torch.cuda.current_device())
         if x.is_pinned() and x.numel() * 2 >= 2 * _CHUNK_BYTES:
             return _quantize_host_pipelined(x, format, scaling, out, dev)
@@ -221,15 +268,8 @@ def quantize(x: torch.Tensor, format: int = E2M1, scaling: int = FLOOR, out=None
         return out
     _cuda_bf16(x, "x")
     rows, cols = _rows_cols(x)
-    lead = x.shape[:-1]
-    mbs = ((scaling >> 4) & 3) != 0
-    if out is None:
-        ccols = cols // 2 if format in _PACKED else cols
-        codes = torch.empty(*lead, ccols, dtype=torch.uint8, device=x.device)
-        scales = _scales_buffer(lead, rows, cols, format, scaling, x.device)
-        macro = torch.empty(*lead, cols // 128, dtype=torch.uint8, device=x.device) if mbs else None
-    else:
-        codes, scales, macro = out
+    codes, scales, macro = _quantize_buffers(x.device, x.shape[:-1], rows, cols, format, scaling,
+                                             out)
     with torch.cuda.device(x.device):
         _check(mx_quantize(_ptr(x), rows, cols, format, scaling, _ptr(codes), _ptr(scales),
                            _ptr(macro), _stream(x.device)), "mx_quantize")
@@ -255,6 +295,8 @@ def _quantize_host_pipelined(x, format, scaling, out, dev):
     mma = (scaling & MMA_SCALES) != 0
     ccols = cols // 2 if format in _PACKED else cols
     bs = block_size(format)
+    if out is not None:
+        _quantize_buffers(torch.device("cpu"), lead, rows, cols, format, scaling, out)
     if out is None:
         hc = torch.empty(*lead, ccols, dtype=torch.uint8, pin_memory=True)
         hs = (torch.empty(mx_scale_bytes(rows, cols, format, scaling), dtype=torch.uint8,
@@ -331,14 +373,25 @@ def dequantize(codes: torch.Tensor, scales: torch.Tensor, macro=None, format: in
             return _to_host(res, pinned)
         out.copy_(res, non_blocking=out.is_pinned())
         return out
-    if codes.dtype != torch.uint8 or scales.dtype != torch.uint8:
-        raise ValueError("codes and scales must be uint8")
+    if codes.dim() == 0:
+        raise ValueError("codes must be at least 1-D")
     cols = codes.shape[-1] * 2 if format in _PACKED else codes.shape[-1]
     rows = codes.numel() * (2 if format in _PACKED else 1) // cols if cols else 0
     if out_dtype not in (torch.bfloat16, torch.float32):
         raise ValueError("out_dtype must be bfloat16 or float32")
+    dev = codes.device
+    _check_buf(codes, "codes", dev, torch.uint8, codes.numel())
+    if cols % block_size(format) == 0:
+        flags = MMA_SCALES if mma_scales else 0
+        _check_buf(scales, "scales", dev, torch.uint8, _scale_count(rows, cols, format, flags))
+    else:
+        _check_buf(scales, "scales", dev, torch.uint8, 0)   # the library rejects the shape
+    if macro is not None:
+        _check_buf(macro, "macro", dev, torch.uint8, rows * (cols // 128))
     if out is None:
-        out = torch.empty(*codes.shape[:-1], cols, dtype=out_dtype, device=codes.device)
+        out = torch.empty(*codes.shape[:-1], cols, dtype=out_dtype, device=dev)
+    else:
+        _check_buf(out, "out", dev, out_dtype, rows * cols)
     with torch.cuda.device(codes.device):
         flags = int(out_dtype == torch.float32) | (MMA_SCALES if mma_scales else 0)
         _check(mx_dequantize(_ptr(codes), _ptr(scales), _ptr(macro), rows, cols, format,
@@ -352,6 +405,8 @@ def fake_quant(x: torch.Tensor, format: int = E2M1, scaling: int = FLOOR, out=No
     """QAT forward: dequantize(quantize(x)) in one kernel, bf16 out."""
     _cuda_bf16(x, "x")
     rows, cols = _rows_cols(x)
+    if out is not None:
+        _check_buf(out, "out", x.device, torch.bfloat16, x.numel())
     y = torch.empty_like(x) if out is None else out
     scales = _scales_buffer(x.shape[:-1], rows, cols, format, scaling, x.device) if return_scales else None
     with torch.cuda.device(x.device):
@@ -367,7 +422,11 @@ def fake_quant_bwd(x: torch.Tensor, grad_y: torch.Tensor, format: int = E2M1,
     _cuda_bf16(grad_y, "grad_y")
     if grad_y.shape != x.shape:
         raise ValueError("grad_y must have the shape of x")
+    if grad_y.device != x.device:
+        raise ValueError(f"grad_y must be on {x.device}, got {grad_y.device}")
     rows, cols = _rows_cols(x)
+    if out is not None:
+        _check_buf(out, "out", x.device, torch.bfloat16, x.numel())
     gx = torch.empty_like(x) if out is None else out
     with torch.cuda.device(x.device):
         _check(mx_fake_quant_bwd(_ptr(x), _ptr(grad_y), rows, cols, format, scaling, _ptr(gx),
@@ -422,6 +481,8 @@ def bat_apply(x: torch.Tensor, A: torch.Tensor, B: torch.Tensor, beta_min=None, 
     _cuda_bf16(x, "x")
     rows, cols = _rows_cols(x)
     a = _bat_params(x, A, B, beta_min, beta_max)
+    if out is not None:
+        _check_buf(out, "out", x.device, torch.bfloat16, x.numel())
     y = torch.empty_like(x) if out is None else out
     with torch.cuda.device(x.device):
         _check(mx_bat_apply(_ptr(x), rows, cols, a, _ptr(A), _ptr(B), _ptr(beta_min), _ptr(beta_max),
@@ -436,15 +497,8 @@ def bat_quantize(x: torch.Tensor, A: torch.Tensor, B: torch.Tensor, beta_min=Non
     _cuda_bf16(x, "x")
     rows, cols = _rows_cols(x)
     a = _bat_params(x, A, B, beta_min, beta_max)
-    lead = x.shape[:-1]
-    mbs = ((scaling >> 4) & 3) != 0
-    if out is None:
-        ccols = cols // 2 if format in _PACKED else cols
-        codes = torch.empty(*lead, ccols, dtype=torch.uint8, device=x.device)
-        scales = _scales_buffer(lead, rows, cols, format, scaling, x.device)
-        macro = torch.empty(*lead, cols // 128, dtype=torch.uint8, device=x.device) if mbs else None
-    else:
-        codes, scales, macro = out
+    codes, scales, macro = _quantize_buffers(x.device, x.shape[:-1], rows, cols, format, scaling,
+                                             out)
     with torch.cuda.device(x.device):
         _check(mx_bat_quantize(_ptr(x), rows, cols, a, _ptr(A), _ptr(B), _ptr(beta_min),
                                _ptr(beta_max), format, scaling, _ptr(codes), _ptr(scales),

@@ -10,6 +10,7 @@ on a host without a GPU.
 from __future__ import annotations
 
 import argparse
+import hashlib
 import os
 import subprocess
 import sys
@@ -34,14 +35,36 @@ def nvcc() -> str:
     return "nvcc"
 
 
-def _newest_input() -> float:
+STAMP = LIB + ".srchash"
+
+
+def source_hash(extra=None) -> str:
+    """SHA-256 over every source, header and flag the library is built from."""
+    h = hashlib.sha256()
     paths = [os.path.join(CSRC, s) for s in SOURCES + HEADERS] + [os.path.join(INCLUDE, "mx.h"),
                                                                    os.path.abspath(__file__)]
-    return max(os.path.getmtime(p) for p in paths)
+    for p in paths:
+        h.update(os.path.basename(p).encode() + b"\0")
+        with open(p, "rb") as f:
+            h.update(f.read())
+    h.update(" ".join(ARCH + NVCC_FLAGS + list(extra or [])).encode())
+    return h.hexdigest()
+
+
+def _stamp() -> str:
+    try:
+        with open(STAMP) as f:
+            return f.read().strip()
+    except OSError:
+        return ""
 
 
 def build(force: bool = False, verbose: bool = False, extra=None) -> str:
-    if not force and os.path.exists(LIB) and os.path.getmtime(LIB) >= _newest_input():
+    """Builds libmx.so unless the one in place was built from these exact
+    sources and flags (its recorded source hash matches); file times are not
+    trusted, so a stale library is always rebuilt."""
+    want = source_hash(extra)
+    if not force and not verbose and os.path.exists(LIB) and _stamp() == want:
         return LIB
     # one nvcc per source, in parallel, then one link
     base = [nvcc(), *ARCH, *NVCC_FLAGS, "-I", INCLUDE, "-I", CSRC]
@@ -61,6 +84,9 @@ def build(force: bool = False, verbose: bool = False, extra=None) -> str:
     for obj in objs:
         os.remove(obj)
     os.replace(LIB + ".tmp", LIB)
+    with open(STAMP + ".tmp", "w") as f:
+        f.write(want + "\n")
+    os.replace(STAMP + ".tmp", STAMP)
     return LIB
 
 

@@ -11,7 +11,7 @@ namespace mxk {
 // the plain [rows, cols/32] array; otherwise the tiled layout of block-scaled
 // tensor-core operands (128 rows x 4 block columns per 512-byte tile, tiles
 // row-major with nct tiles per tile row, inside a tile the byte
-// (r % 32) * 16 + (r / 32) * 4 + (j % 4)).
+// (r % 32) * 16 + ((r / 32) % 4) * 4 + (j % 4)).
 struct ScaleMap {
   int64_t bpr;   // blocks per row (cols / 32), or 0 for the plain layout
   int64_t nct;   // tiles per tile row: ceil(bpr / 4)

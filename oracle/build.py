@@ -2,6 +2,7 @@
 
 from __future__ import annotations
 
+import hashlib
 import os
 import subprocess
 
@@ -13,13 +14,22 @@ def oracle_library_path() -> str:
 
 
 def build_oracle(force: bool = False) -> str:
+    """Compiles the oracle unless the library in place was built from this
+    exact source and command (recorded hash; file times are not trusted)."""
     src = os.path.join(_HERE, "mx_oracle.cpp")
     out = oracle_library_path()
-    if not force and os.path.exists(out) and os.path.getmtime(out) >= os.path.getmtime(src):
-        return out
     cmd = ["g++", "-O2", "-std=c++17", "-Wall", "-Wextra", "-shared", "-fPIC", "-pthread",
-           "-ffp-contract=off", src, "-o", out]
+           "-ffp-contract=off", src, "-o", out + ".tmp"]
+    with open(src, "rb") as f:
+        want = hashlib.sha256(f.read() + " ".join(cmd[:-3]).encode()).hexdigest()
+    stamp = out + ".srchash"
+    have = open(stamp).read().strip() if os.path.exists(stamp) else ""
+    if not force and os.path.exists(out) and have == want:
+        return out
     subprocess.run(cmd, check=True)
+    os.replace(out + ".tmp", out)
+    with open(stamp, "w") as f:
+        f.write(want + "\n")
     return out
 
 

@@ -183,3 +183,76 @@ def test_bat_entry_points_validate(mx):
     assert qz(A, 4, 128, 8, A, A, None, None, 0, 0, A + 8, A, None, 0) == ALIGN
     assert qz(A, 4, 128, 8, None, A, None, None, 0, 0, A, A, None, 0) == INVALID
     assert qz(None, 0, 128, 8, None, None, None, None, 0, 0, None, None, None, 0) == OK
+
+
+# -------------------------------------------- caller-supplied buffers ----
+
+def test_binding_checks_every_output_buffer(mx):
+    """Buffers passed as ``out`` are checked (device, dtype, contiguity,
+    size) before the C call: the kernels write through their raw pointers.
+    The checks run here against CPU tensors, with ``meta`` tensors standing
+    in for a buffer on the wrong device; nothing is launched."""
+    import torch
+    cpu = torch.device("cpu")
+    u8 = lambda *s: torch.zeros(*s, dtype=torch.uint8)
+    lead, rows, cols = (4,), 4, 256
+    chk = lambda out, fmt=0, sc=0: mx._quantize_buffers(cpu, lead, rows, cols, fmt, sc, out)
+    chk((u8(4, 128), u8(4, 8), None))                              # exact sizes pass
+    chk((u8(4, 128), u8(4, 8), u8(4, 2)), 0, mx.MBS_STATIC)
+    chk((u8(4, 256), u8(4, 8), None), mx.E4M3)
+    chk((u8(512), u8(1024), None), 0, mx.MMA_SCALES)               # two padded 128 x 4 tiles
+    bad = [
+        ((u8(4, 127), u8(4, 8), None), 0, 0),                      # codes one byte short
+        ((u8(4, 128), u8(4, 7), None), 0, 0),                      # scales short
+        ((u8(4, 128), u8(1023), None), 0, mx.MMA_SCALES),          # tiled scales need 1024
+        ((u8(4, 128), u8(4, 8), None), 0, mx.MBS_STATIC),          # macro missing
+        ((u8(4, 128), u8(4, 8), u8(4, 1)), 0, mx.MBS_DYNAMIC),     # macro short
+        ((u8(4, 128), u8(4, 8), None), mx.E4M3, 0),                # FP8 codes are 1 B/elem
+        ((torch.zeros(4, 128, dtype=torch.int16), u8(4, 8), None), 0, 0),
+        ((u8(4, 256)[:, ::2], u8(4, 8), None), 0, 0),              # not contiguous
+        ((torch.empty(4, 128, dtype=torch.uint8, device="meta"), u8(4, 8), None), 0, 0),
+        ((u8(4, 128), u8(4, 8)), 0, 0),                            # not a triple
+    ]
+    for out, fmt, sc in bad:
+        with pytest.raises(ValueError):
+            chk(out, fmt, sc)
+    with pytest.raises(ValueError):
+        mx._check_buf(torch.zeros(8, dtype=torch.bfloat16), "out", cpu, torch.float32, 8)
+    with pytest.raises(ValueError):
+        mx._check_buf(torch.zeros(7, dtype=torch.float32), "out", cpu, torch.float32, 8)
+    mx._check_buf(torch.zeros(8, dtype=torch.float32), "out", cpu, torch.float32, 8)
+
+
+def test_binding_checks_host_path_buffers(mx):
+    """A CPU input with CPU ``out`` buffers: the same checks, before any copy."""
+    import torch
+    x = torch.zeros(4, 64, dtype=torch.bfloat16)
+    short = (torch.zeros(4, 31, dtype=torch.uint8), torch.zeros(4, 2, dtype=torch.uint8), None)
+    with pytest.raises(ValueError):
+        mx.quantize(x, out=short)
+
+
+def test_launch_failure_returns_mx_err_cuda(mx):
+    """With no CUDA device visible, a call that passes validation fails at its
+    first CUDA runtime call and returns MX_ERR_CUDA (nothing is written; the
+    fake addresses are never dereferenced because no kernel can start). Runs
+    in a child process that sees no device, on a host with or without GPUs."""
+    import subprocess
+    import sys
+    code = (
+        "import ctypes, sys\n"
+        f"lib = ctypes.CDLL({mx.library_path()!r})\n"
+        "vp, i64, ci = ctypes.c_void_p, ctypes.c_int64, ctypes.c_int\n"
+        "lib.mx_quantize.argtypes = [vp, i64, i64, ci, ci, vp, vp, vp, vp]\n"
+        "lib.mx_block_error.argtypes = [vp, i64, i64, ci, ci, vp, vp, vp]\n"
+        "lib.mx_dequantize.argtypes = [vp, vp, vp, i64, i64, ci, ci, vp, vp]\n"
+        f"A = {A}\n"
+        "print(lib.mx_quantize(A, 4, 128, 0, 0, A, A, None, None),\n"
+        "      lib.mx_quantize(A, 4, 128, 0, 3 | 256, A, A, None, None),\n"
+        "      lib.mx_block_error(A, 4, 128, 0, 0, None, A, None),\n"
+        "      lib.mx_dequantize(A, A, None, 4, 128, 1, 0, A, None))\n")
+    env = dict(os.environ, CUDA_VISIBLE_DEVICES="")
+    out = subprocess.run([sys.executable, "-c", code], env=env, capture_output=True, text=True,
+                         timeout=120)
+    assert out.returncode == 0, out.stderr
+    assert out.stdout.split() == [str(CUDA_ERR)] * 4

@@ -482,3 +482,30 @@ def test_more_than_2_31_elements(mx, oracle_mod, cuda):
     torch.cuda.synchronize()
     assert np.array_equal(bits(y), oracle_mod.dequantize(host_u8(c[-4:]), host_u8(s[-4:]), None,
                                                          4, cols, E2M1))
+
+
+def test_binding_rejects_bad_out_buffers(mx, cuda):
+    """Caller buffers that do not fit what the kernels write raise ValueError
+    before any launch: a host buffer for a device input, short or narrower
+    buffers, a buffer on the wrong device."""
+    x = inputs.random_bf16_bits((4, 256), seed=12).to(cuda)
+    u8 = lambda n, dev=cuda: torch.empty(n, dtype=torch.uint8, device=dev)
+    with pytest.raises(ValueError):
+        mx.quantize(x, out=(u8(512, "cpu"), u8(32), None))           # host codes
+    with pytest.raises(ValueError):
+        mx.quantize(x, E2M1, FLOOR | (1 << 8), out=(u8(512), u8(32), None))   # tiled needs 1024
+    with pytest.raises(ValueError):
+        mx.quantize(x, E4M3, FLOOR, out=(u8(512), u8(32), None))     # FP8 codes: 1024
+    c, s, _ = mx.quantize(x)
+    with pytest.raises(ValueError):
+        mx.dequantize(c, s, out_dtype=torch.float32,
+                      out=torch.empty(4, 256, dtype=torch.bfloat16, device=cuda))
+    with pytest.raises(ValueError):
+        mx.dequantize(c, s[:, :4].contiguous())                          # short scales
+    with pytest.raises(ValueError):
+        mx.fake_quant(x, out=torch.empty(4, 255, dtype=torch.bfloat16, device=cuda))
+    with pytest.raises(ValueError):
+        mx.fake_quant_bwd(x, x.cpu())
+    with pytest.raises(ValueError):
+        mx.fake_quant_bwd(x, x, out=torch.empty(4, 256, dtype=torch.float32, device=cuda))
+    torch.cuda.synchronize()
