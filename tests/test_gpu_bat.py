@@ -4,7 +4,13 @@ oracle: the transformed bf16 rows and the fused quantizer's codes, scale bytes
 and macro factors, bit for bit, through the C ABI.
 
 The arithmetic order is fixed (fp32 fma chains, halves summed separately), so
-the comparison is exact, including the codes the rounding decides.
+the comparison with the oracle is exact, including the codes the rounding
+decides. That order is a reading of the pages (they fix no precision), so the
+GPU output is also checked against definitions that carry no summation order:
+integer cases where every order gives the same bits (an int64 Kronecker
+product), and random cases within the fp32 + bf16 rounding bound of an fp64
+product; the fused quantizer's codes are then the oracle's quantization of the
+GPU's own transformed rows.
 """
 
 import numpy as np
@@ -184,3 +190,141 @@ def test_more_than_2_31_elements(mx, oracle_mod, cuda):
     assert np.array_equal(scales[tail].cpu().numpy(), os_)
     del x, codes, scales
     torch.cuda.empty_cache()
+
+
+# ------------------------------------ structure-free definitions (fp64) ----
+
+U = 2.0 ** -24
+
+
+def _kron_product(xf, A, B):
+    """x [rows, cols] times diag(B_j (x) A) over the 32-element blocks, in the
+    dtype of the inputs (int64 or float64): numpy's Kronecker product, a
+    plain matrix product, no chosen order."""
+    rows, cols = xf.shape
+    out = np.zeros_like(xf)
+    for j in range(cols // 32):
+        out[:, 32 * j:32 * j + 32] = xf[:, 32 * j:32 * j + 32] @ np.kron(B[j], A)
+    return out
+
+
+def _clip_blocks(y, bmin, bmax):
+    """[beta_min_j min, beta_max_j max] of each row's block j, upper bound last."""
+    rows, cols = y.shape
+    yb = y.reshape(rows, cols // 32, 32)
+    lo = bmin[None, :, None] * yb.min(axis=2, keepdims=True)
+    hi = bmax[None, :, None] * yb.max(axis=2, keepdims=True)
+    return np.minimum(np.maximum(yb, lo), hi).reshape(rows, cols)
+
+
+def _bf16_bits_of_exact(v):
+    """bf16 bits of exact values below 2^24 (float32 holds them; one RNE)."""
+    return torch.from_numpy(np.ascontiguousarray(v, np.float32)).to(torch.bfloat16) \
+        .view(torch.int16).numpy().view(np.uint16)
+
+
+def _f64(bits16):
+    return torch.from_numpy(np.ascontiguousarray(bits16).view(np.int16)).view(torch.bfloat16) \
+        .double().numpy()
+
+
+@pytest.mark.parametrize("a", A_DIMS)
+@pytest.mark.parametrize("clip", [False, True])
+def test_apply_integer_cases_equal_the_kronecker_product(mx, oracle_mod, cuda, a, clip):
+    """Small integers: every fp32 partial sum is exact, so any summation order
+    gives the exact product; the clip thresholds 0.5 and 0.75 keep the bounds
+    exact. The GPU's bf16 output must be the one rounding of that exact value
+    (a zero may carry either sign: which one depends on the order the zero
+    terms are added in), and the fused codes the oracle's quantization of the
+    GPU's rows."""
+    b = 32 // a
+    rng = np.random.default_rng(40 + a)
+    rows, cols = 70, 1152
+    xi = rng.integers(-8, 9, (rows, cols))
+    Ai = rng.integers(-3, 4, (a, a))
+    Bi = rng.integers(-3, 4, (cols // 32, b, b))
+    exact = _kron_product(xi.astype(np.int64), Ai.astype(np.int64), Bi.astype(np.int64))
+    assert np.abs(exact).max() < 2 ** 24
+    bmin = bmax = None
+    want = exact.astype(np.float64)
+    if clip:
+        bmin = np.where(np.arange(cols // 32) % 2, 0.5, 0.75).astype(np.float32)
+        bmax = np.where(np.arange(cols // 32) % 3, 0.75, 0.5).astype(np.float32)
+        want = _clip_blocks(want, bmin.astype(np.float64), bmax.astype(np.float64))
+    want_bits = _bf16_bits_of_exact(want)
+    dev = lambda t: None if t is None else torch.from_numpy(np.ascontiguousarray(t, np.float32)).to(cuda)
+    x = torch.from_numpy(xi.astype(np.float32)).to(torch.bfloat16).to(cuda)
+    y = mx.bat_apply(x, dev(Ai), dev(Bi), dev(bmin), dev(bmax))
+    got = mx.bat_quantize(x, dev(Ai), dev(Bi), dev(bmin), dev(bmax), E2M1, OAS)
+    torch.cuda.synchronize()
+    yb = inputs.bf16_bits_numpy(y)
+    unsigned_zero = lambda v: np.where(v == 0x8000, 0, v)
+    assert np.array_equal(unsigned_zero(yb), want_bits)
+    oc, os_, _ = oracle_mod.quantize(yb, E2M1, OAS)
+    assert np.array_equal(_np(got[0]), oc) and np.array_equal(_np(got[1]), os_)
+
+
+@pytest.mark.parametrize("a", A_DIMS)
+@pytest.mark.parametrize("clip", [False, True])
+@pytest.mark.parametrize("shape", [(37, 96), (130, 1152)])
+def test_apply_within_the_rounding_bound_of_the_fp64_product(mx, oracle_mod, cuda, a, clip, shape):
+    """Random data and parameters: |y_gpu - y| is bounded, per element, by
+    the fp32 error of the transform and the thresholds, carried through the
+    clip (1-Lipschitz in the value and in both bounds), plus the final bf16
+    rounding (half an ulp, at most 2^-8 of the value). Chains of n products
+    err by at most n u of their absolute sum, so 2 (a + b + 2) u of the
+    absolute product bounds the transform (as for the oracle)."""
+    rows, cols = shape
+    b = 32 // a
+    x = inputs.heavy_tail(rows, cols, seed=a * 31 + rows).to(cuda)
+    A, B, bmin, bmax = inputs.bat_params(a, cols // 32, seed=a + cols, device=cuda, spread=0.3,
+                                         clip=clip, lo=0.5)
+    y = mx.bat_apply(x, A, B, bmin, bmax)
+    fused = mx.bat_quantize(x, A, B, bmin, bmax, E2M1, OAS | MBS_STATIC)
+    torch.cuda.synchronize()
+    xf = _f64(inputs.bf16_bits_numpy(x))
+    A64, B64 = _np(A).astype(np.float64), _np(B).astype(np.float64)
+    ref = _kron_product(xf, A64, B64)
+    mag = _kron_product(np.abs(xf), np.abs(A64), np.abs(B64))
+    err_t = 2 * (a + b + 2) * U * mag                          # transform, per element
+    if clip:
+        bl, bh = _np(bmin).astype(np.float64), _np(bmax).astype(np.float64)
+        ref = _clip_blocks(ref, bl, bh)
+        eb = err_t.reshape(rows, cols // 32, 32).max(axis=2, keepdims=True)   # per block
+        thr = np.maximum(bl, bh)[None, :, None]
+        big = np.abs(ref).reshape(rows, cols // 32, 32).max(axis=2, keepdims=True)
+        err_t = np.broadcast_to(np.maximum(1.0, thr) * eb + U * thr * big * (1 + 1e-6),
+                                (rows, cols // 32, 32)).reshape(rows, cols)
+    bound = err_t * (1 + 2.0 ** -8) + 2.0 ** -8 * np.abs(ref)
+    got = _f64(inputs.bf16_bits_numpy(y))
+    assert np.all(np.isfinite(got))
+    assert np.all(np.abs(got - ref) <= bound), np.max(np.abs(got - ref) / np.maximum(bound, 1e-300))
+    # the transform really is evaluated (a wrong index moves values by O(1))
+    assert np.abs(got - ref).max() > 0
+    # the fused codes are exactly the oracle's quantization of the GPU's rows
+    oc, os_, om = oracle_mod.quantize(inputs.bf16_bits_numpy(y), E2M1, OAS | MBS_STATIC)
+    assert np.array_equal(_np(fused[0]), oc)
+    assert np.array_equal(_np(fused[1]), os_)
+    assert np.array_equal(_np(fused[2]), om)
+
+
+def test_full_moe_stack_against_the_fp64_product(mx, cuda):
+    """The bench workload (MoE w13 rows, a = 8, clipping) on 256 sampled rows:
+    within the rounding bound of the fp64 product, in the bench's launch."""
+    x = inputs.moe_w13(device=cuda).view(-1, 2048)
+    A, B, bmin, bmax = inputs.bat_params(8, 64, device=cuda)
+    y = mx.bat_apply(x, A, B, bmin, bmax)
+    torch.cuda.synchronize()
+    idx = torch.randperm(x.shape[0], generator=torch.Generator().manual_seed(1))[:256].to(cuda)
+    xf = _f64(inputs.bf16_bits_numpy(x[idx]))
+    got = _f64(inputs.bf16_bits_numpy(y[idx]))
+    del x, y
+    A64, B64 = _np(A).astype(np.float64), _np(B).astype(np.float64)
+    bl, bh = _np(bmin).astype(np.float64), _np(bmax).astype(np.float64)
+    ref = _clip_blocks(_kron_product(xf, A64, B64), bl, bh)
+    mag = _kron_product(np.abs(xf), np.abs(A64), np.abs(B64))
+    rows = len(xf)
+    eb = (2 * (8 + 4 + 2) * U * mag).reshape(rows, 64, 32).max(axis=2, keepdims=True)
+    big = np.abs(ref).reshape(rows, 64, 32).max(axis=2, keepdims=True)
+    err = np.broadcast_to(eb + U * big * (1 + 1e-6), (rows, 64, 32)).reshape(rows, 2048)
+    assert np.all(np.abs(got - ref) <= err * (1 + 2.0 ** -8) + 2.0 ** -8 * np.abs(ref))

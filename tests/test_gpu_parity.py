@@ -4,8 +4,9 @@ Codes, scale bytes, macro bytes, dequantized bf16/float bits and straight-
 through gradients must be bit-identical; error statistics agree within a
 relative 1e-6 (the kernel sums per-block squares in double and atomically adds
 per-CTA double partials, the oracle sums sequentially in double). Inputs are
-seeded and synthetic (fp8_quantization_mx_b200.inputs); at the full workload
-sizes the oracle checks sampled rows and properties that hold at any size.
+seeded and synthetic (fp8_quantization_mx_b200.inputs). The whole-tensor
+comparisons at the workload sizes are in test_gpu_full_parity.py; here the
+small and edge-case inputs, and a tensor past 2^31 elements.
 """
 
 import numpy as np
@@ -287,82 +288,6 @@ def test_dequantize_roundtrip(mx, oracle_mod, cuda, fm):
                           oracle_mod.dequantize(oc, os_, omac, 256, 4096, fmt, out_fp32=True))
 
 
-# -------------------------------------------------- full-size workloads --
-
-def sample_rows(n_rows, k, seed):
-    rng = np.random.default_rng(seed)
-    r = np.sort(rng.choice(n_rows, size=min(k, n_rows), replace=False))
-    r[0], r[-1] = 0, n_rows - 1          # first and last row always
-    return np.unique(r)
-
-
-@pytest.mark.parametrize("fmt", BYTE_FMTS, ids=lambda f: FMT_NAMES[f])
-def test_full_mlp_weight_bytes(mx, oracle_mod, cuda, fmt):
-    x = inputs.mlp_weight(device=cuda)
-    c, s, _ = mx.quantize(x, fmt, FLOOR)
-    torch.cuda.synchronize()
-    r = sample_rows(x.shape[0], 48, 1)
-    xs = bits(x[r])
-    oc, os_, _ = oracle_mod.quantize(xs, fmt, FLOOR)
-    assert np.array_equal(host_u8(c[r]), oc)
-    assert np.array_equal(host_u8(s[r]), os_)
-    # property over every block: the FLOOR byte from the block amax exponent
-    amax = x.view(-1, 32).abs().amax(dim=1).view(torch.int16).to(torch.int32)
-    want = torch.clamp((amax >> 7) - EMAX[fmt], min=0).to(torch.uint8)
-    assert torch.equal(s.view(-1), want)
-
-
-def test_full_moe_w13_fp4(mx, oracle_mod, cuda):
-    x = inputs.moe_w13(device=cuda).view(-1, 2048)
-    c, s, _ = mx.quantize(x, E2M1, FLOOR)
-    y = mx.dequantize(c, s, None, E2M1)
-    torch.cuda.synchronize()
-    r = sample_rows(x.shape[0], 64, 2)
-    xs = bits(x[r])
-    oc, os_, _ = oracle_mod.quantize(xs, E2M1, FLOOR)
-    assert np.array_equal(host_u8(c[r]), oc)
-    assert np.array_equal(host_u8(s[r]), os_)
-    assert np.array_equal(bits(y[r]), oracle_mod.dequantize(oc, os_, None, len(r), 2048, E2M1))
-    amax = x.view(-1, 32).abs().amax(dim=1).view(torch.int16).to(torch.int32)
-    assert torch.equal(s.view(-1), torch.clamp((amax >> 7) - 2, min=0).to(torch.uint8))
-    # every code decodes to a value no farther from x than half the local grid step
-    err = (y.float() - x.float()).abs()
-    X = torch.pow(2.0, s.float() - 127).repeat_interleave(32, dim=1)
-    assert bool((err <= torch.maximum(X, (x.float().abs() - 6 * X).clamp(min=0))).all())
-
-
-def test_full_qat_tensors(mx, oracle_mod, cuda):
-    for gen, seed in ((inputs.qat_act, 3), (inputs.qat_weight, 4)):
-        x = gen(device=cuda)
-        g = inputs.qat_grad(*x.shape, device=cuda)
-        y = mx.fake_quant(x, E2M1, FLOOR)
-        gx = mx.fake_quant_bwd(x, g, E2M1, FLOOR)
-        torch.cuda.synchronize()
-        r = sample_rows(x.shape[0], 48, seed)
-        assert np.array_equal(bits(y[r]), oracle_mod.fake_quant_fwd(bits(x[r]), E2M1, FLOOR))
-        assert np.array_equal(bits(gx[r]), oracle_mod.fake_quant_bwd(bits(x[r]), bits(g[r]), E2M1, FLOOR))
-
-
-@pytest.mark.parametrize("m", FP4_MODES, ids=lambda m: ids((0, m)))
-def test_full_heavy_tail_modes(mx, oracle_mod, cuda, m):
-    x = inputs.heavy_tail(device=cuda)
-    c, s, mac = mx.quantize(x, E2M1, m)
-    bs, tot = mx.block_error(x, E2M1, m)
-    torch.cuda.synchronize()
-    r = sample_rows(x.shape[0], 12 if m >> 4 == 2 else 32, 5)
-    xs = bits(x[r])
-    oc, os_, omac = oracle_mod.quantize(xs, E2M1, m)
-    assert np.array_equal(host_u8(c[r]), oc)
-    assert np.array_equal(host_u8(s[r]), os_)
-    if m >> 4:
-        assert np.array_equal(host_u8(mac[r]), omac)
-    obs, _, _ = oracle_mod.block_error(xs, E2M1, m)
-    assert np.allclose(bs[r].cpu().numpy(), obs, rtol=REL, atol=0)
-    # totals equal the sum of the per-block values (both from the kernel)
-    assert np.isclose(tot[0].item(), bs.double().sum().item(), rtol=1e-5)
-    assert np.isclose(tot[1].item(), x.double().pow(2).sum().item(), rtol=REL)
-
-
 # ------------------------------------------------------ edge behaviour --
 
 def test_guard_bands(mx, cuda):
@@ -421,22 +346,6 @@ def test_autograd_function(mx, oracle_mod, cuda):
     xb = bits(x.detach())
     assert np.array_equal(bits(y.detach()), oracle_mod.fake_quant_fwd(xb))
     assert np.array_equal(bits(x.grad), oracle_mod.fake_quant_bwd(xb, bits(g)))
-
-
-@pytest.mark.parametrize("fm", [(E2M1_B16, OAS), (NVFP4, FLOOR)], ids=ids)
-def test_full_qat_act_block16(mx, oracle_mod, cuda, fm):
-    fmt, m = fm
-    x = inputs.qat_act(device=cuda)
-    c, s, _ = mx.quantize(x, fmt, m)
-    bs, tot = mx.block_error(x, fmt, m)
-    torch.cuda.synchronize()
-    r = sample_rows(x.shape[0], 32, 5)
-    xs = bits(x[r])
-    oc, os_, _ = oracle_mod.quantize(xs, fmt, m)
-    assert np.array_equal(host_u8(c[r]), oc)
-    assert np.array_equal(host_u8(s[r]), os_)
-    obs, _, _ = oracle_mod.block_error(xs, fmt, m)
-    assert np.allclose(bs[r].cpu().numpy(), obs, rtol=REL, atol=0)
 
 
 @pytest.mark.parametrize("fm", [(E2M1, FLOOR), (E2M1, OAS | MBS_STATIC), (NVFP4, FLOOR | (1 << 8))],
@@ -509,3 +418,39 @@ def test_binding_rejects_bad_out_buffers(mx, cuda):
     with pytest.raises(ValueError):
         mx.fake_quant_bwd(x, x, out=torch.empty(4, 256, dtype=torch.float32, device=cuda))
     torch.cuda.synchronize()
+
+
+def _golden_macro_cases():
+    import json
+    import os
+    with open(os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden",
+                           "hand_blocks.json")) as f:
+        g = json.load(f)
+    modes = {"MBS_STATIC": MBS_STATIC, "MBS_DYNAMIC": MBS_DYNAMIC,
+             "OAS|MBS_STATIC": OAS | MBS_STATIC, "OAS|MBS_DYNAMIC": OAS | MBS_DYNAMIC}
+    return [(f"{b['id']}-{m}", b["values"], modes[m], e) for b in g["macro_blocks"]
+            if "expect" in b for m, e in b["expect"].items()]
+
+
+@pytest.mark.parametrize("case", _golden_macro_cases(), ids=[c[0] for c in _golden_macro_cases()])
+def test_hand_macro_blocks_on_gpu(mx, cuda, case):
+    """The hand-derived macro blocks (factor k, sub-block bytes, codes,
+    dequantized values, SSE) straight against their written derivations, on
+    the GPU; each block is repeated over 3 rows x 2 macro columns."""
+    _, values, m, e = case
+    v = np.zeros(128, np.float32)
+    v[:len(values)] = values
+    x = torch.from_numpy(np.tile(v, (3, 2))).to(torch.bfloat16).to(cuda)
+    c, s, mac = mx.quantize(x, E2M1, m)
+    yf = mx.dequantize(c, s, mac, E2M1, torch.float32)
+    bs, tot = mx.block_error(x, E2M1, m)
+    torch.cuda.synchronize()
+    assert bool((mac == e["k"]).all())
+    assert host_u8(s).tolist() == [e["bytes"] * 2] * 3
+    nib = host_u8(c)[:, :len(e["codes"])]
+    got_codes = np.stack([nib & 15, nib >> 4], axis=-1).reshape(3, -1)[:, :len(e["codes"])]
+    assert got_codes.tolist() == [e["codes"]] * 3
+    y = yf.cpu().numpy().reshape(3, 2, 128)
+    assert np.all(y[:, :, :len(e["dequant"])] == np.array(e["dequant"], np.float32))
+    assert np.all(y[:, :, len(e["dequant"]):] == 0)
+    assert np.isclose(tot[0].item(), 6 * e["sse"], rtol=REL, atol=0)

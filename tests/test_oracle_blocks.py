@@ -17,7 +17,8 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 with open(os.path.join(HERE, "golden", "hand_blocks.json")) as f:
     GOLDEN = json.load(f)
 
-MODES = {"FLOOR": 0, "CEIL": 1, "OAS_RULE": 2, "OAS": 3, "MBS_STATIC": 1 << 4}
+MODES = {"FLOOR": 0, "CEIL": 1, "OAS_RULE": 2, "OAS": 3, "MBS_STATIC": 1 << 4,
+         "MBS_DYNAMIC": 2 << 4, "OAS|MBS_STATIC": 3 | 1 << 4, "OAS|MBS_DYNAMIC": 3 | 2 << 4}
 FMTS = {"E2M1": 0, "E4M3": 1, "E5M2": 2, "E3M2": 3, "E2M3": 4, "INT8": 5}
 
 
@@ -55,7 +56,35 @@ def test_hand_block(oracle_mod, blk):
             assert _codes(codes, fmt, len(exp)) == exp, mode
 
 
-@pytest.mark.parametrize("blk", GOLDEN["macro_blocks"], ids=[b["id"] for b in GOLDEN["macro_blocks"]])
+def macro_cases():
+    """(id, values, mode, expectation) of every hand-worked macro block."""
+    out = []
+    for blk in GOLDEN["macro_blocks"]:
+        if "expect" in blk:
+            out += [(f"{blk['id']}-{m}", blk["values"], m, e) for m, e in blk["expect"].items()]
+    return out
+
+
+@pytest.mark.parametrize("case", macro_cases(), ids=[c[0] for c in macro_cases()])
+def test_hand_macro_block_modes(oracle_mod, case):
+    """MBS-Static / Dynamic (with and without OAS) on hand-worked macro blocks:
+    the factor, the sub-block bytes, the first codes, their dequantized
+    values and the macro-block SSE, all derived by hand in the fixture."""
+    _, values, mode, e = case
+    x = _block(values, 128).reshape(1, 128)
+    codes, scales, macro = oracle_mod.quantize(x, 0, MODES[mode])
+    assert int(macro[0, 0]) == e["k"]
+    assert [int(s) for s in scales[0]] == e["bytes"]
+    assert _codes(codes, 0, len(e["codes"])) == e["codes"]
+    y = oracle_mod.dequantize(codes, scales, macro, 1, 128, 0, out_fp32=True).view(np.float32)[0]
+    assert [float(v) for v in y[:len(e["dequant"])]] == e["dequant"]
+    assert np.all(y[len(e["dequant"]):] == 0)
+    bs, sd, _ = oracle_mod.block_error(x, 0, MODES[mode])
+    assert sd == e["sse"] and bs.sum() == e["sse"]
+
+
+@pytest.mark.parametrize("blk", [b for b in GOLDEN["macro_blocks"] if "expect" not in b],
+                         ids=[b["id"] for b in GOLDEN["macro_blocks"] if "expect" not in b])
 def test_hand_macro_block(oracle_mod, blk):
     x = _block(blk["values"], 128)
     codes, scales, macro = oracle_mod.quantize(x.reshape(1, 128), 0, MODES[blk["scaling"]])
