@@ -41,6 +41,7 @@ __all__ = [
     "E2M1_B16", "NVFP4", "block_size",
     "quantize", "dequantize", "fake_quant", "fake_quant_bwd", "block_error", "MXFakeQuantize",
     "mx_bat_apply", "mx_bat_quantize", "bat_apply", "bat_quantize",
+    "mx_gemm", "mx_quant_gemm", "gemm", "quant_gemm",
     "MXFP4_FORMAT", "MXFP8_FORMAT",
 ]
 
@@ -112,6 +113,10 @@ def load_library():
     lib.mx_bat_quantize.argtypes = [vp, i64, i64, c_int, vp, vp, vp, vp, c_int, c_int, vp, vp, vp, vp]
     lib.mx_bat_apply.restype = c_int
     lib.mx_bat_quantize.restype = c_int
+    lib.mx_gemm.argtypes = [vp, vp, vp, vp, i64, i64, i64, c_int, vp, vp, vp]
+    lib.mx_quant_gemm.argtypes = [vp, c_int, vp, vp, i64, i64, i64, c_int, vp, vp, vp, vp, vp]
+    lib.mx_gemm.restype = c_int
+    lib.mx_quant_gemm.restype = c_int
     _lib = lib
     return lib
 
@@ -147,6 +152,17 @@ def mx_bat_quantize(x, rows, cols, a_dim, A, B, beta_min, beta_max, format, scal
                     macro, stream=0) -> int:
     return load_library().mx_bat_quantize(x, rows, cols, a_dim, A, B, beta_min, beta_max, format,
                                           scaling, codes, scales, macro, stream)
+
+
+def mx_gemm(a_codes, a_scales, b_codes, b_scales, M, N, K, out_fp32, d, status, stream=0) -> int:
+    return load_library().mx_gemm(a_codes, a_scales, b_codes, b_scales, M, N, K, out_fp32, d, status,
+                                  stream)
+
+
+def mx_quant_gemm(a, scaling, b_codes, b_scales, M, N, K, out_fp32, d, a_codes_out, a_scales_out,
+                  status, stream=0) -> int:
+    return load_library().mx_quant_gemm(a, scaling, b_codes, b_scales, M, N, K, out_fp32, d,
+                                        a_codes_out, a_scales_out, status, stream)
 
 
 def mx_status_string(status: int) -> str:
@@ -521,3 +537,80 @@ class MXFakeQuantize(torch.autograd.Function):
         (x,) = ctx.saved_tensors
         gx = fake_quant_bwd(x.contiguous(), grad_y.contiguous(), ctx.format, ctx.scaling)
         return gx, None, None
+
+
+# ---------------------------------------------------- block-scaled GEMM --
+
+def _gemm_operand_b(b_codes, b_scales, K, device):
+    """B: MXFP4 codes [N, K/2] and its scales in the MMA_SCALES layout."""
+    if b_codes.dim() != 2 or b_codes.shape[1] * 2 != K:
+        raise ValueError(f"b_codes must be [N, K/2] = [N, {K // 2}]")
+    N = b_codes.shape[0]
+    _check_buf(b_codes, "b_codes", device, torch.uint8, N * (K // 2))
+    _check_buf(b_scales, "b_scales", device, torch.uint8,
+               max(0, mx_scale_bytes(N, K, E2M1, MMA_SCALES)))
+    return N
+
+
+def _gemm_out(M, N, out_dtype, out, device):
+    if out_dtype not in (torch.bfloat16, torch.float32):
+        raise ValueError("out_dtype must be bfloat16 or float32")
+    if out is None:
+        return torch.empty(M, N, dtype=out_dtype, device=device)
+    _check_buf(out, "out", device, out_dtype, M * N)
+    return out
+
+
+def _gemm_status(status, device):
+    if status is None:
+        return None
+    _check_buf(status, "status", device, torch.int32, 1)
+    return status
+
+
+def gemm(a_codes: torch.Tensor, a_scales: torch.Tensor, b_codes: torch.Tensor,
+         b_scales: torch.Tensor, out_dtype=torch.bfloat16, out=None, status=None):
+    """D = A B^T on the tensor cores, A [M, K] and B [N, K] both MXFP4: codes
+    (as ``quantize`` writes them) and scales in the MMA_SCALES layout.
+    ``status``: an optional int32 device tensor the kernel sets nonzero if one
+    of its waits timed out. Returns D [M, N] (bf16 or float32)."""
+    if not a_codes.is_cuda:
+        raise ValueError("a_codes must be a CUDA tensor")
+    dev = a_codes.device
+    if a_codes.dim() != 2:
+        raise ValueError("a_codes must be [M, K/2]")
+    M, K = a_codes.shape[0], a_codes.shape[1] * 2
+    _check_buf(a_codes, "a_codes", dev, torch.uint8, M * (K // 2))
+    _check_buf(a_scales, "a_scales", dev, torch.uint8, max(0, mx_scale_bytes(M, K, E2M1, MMA_SCALES)))
+    N = _gemm_operand_b(b_codes, b_scales, K, dev)
+    d = _gemm_out(M, N, out_dtype, out, dev)
+    st = _gemm_status(status, dev)
+    with torch.cuda.device(dev):
+        _check(mx_gemm(_ptr(a_codes), _ptr(a_scales), _ptr(b_codes), _ptr(b_scales), M, N, K,
+                       int(out_dtype == torch.float32), _ptr(d), _ptr(st), _stream(dev)), "mx_gemm")
+    return d
+
+
+def quant_gemm(a: torch.Tensor, b_codes: torch.Tensor, b_scales: torch.Tensor,
+               scaling: int = FLOOR, out_dtype=torch.bfloat16, out=None, a_out=None, status=None):
+    """D = MXFP4(a) B^T with bf16 ``a`` [M, K] quantized inside the GEMM
+    (``scaling``: FLOOR, CEIL, OAS_RULE or OAS). ``a_out`` = (codes [M, K/2],
+    tiled scales) also receives A's quantized form when given. Returns D."""
+    _cuda_bf16(a, "a")
+    if a.dim() != 2:
+        raise ValueError("a must be [M, K]")
+    M, K = a.shape
+    dev = a.device
+    N = _gemm_operand_b(b_codes, b_scales, K, dev)
+    d = _gemm_out(M, N, out_dtype, out, dev)
+    ac = asc = None
+    if a_out is not None:
+        ac, asc = a_out
+        _check_buf(ac, "a_out codes", dev, torch.uint8, M * (K // 2))
+        _check_buf(asc, "a_out scales", dev, torch.uint8, max(0, mx_scale_bytes(M, K, E2M1, MMA_SCALES)))
+    st = _gemm_status(status, dev)
+    with torch.cuda.device(dev):
+        _check(mx_quant_gemm(_ptr(a), scaling, _ptr(b_codes), _ptr(b_scales), M, N, K,
+                             int(out_dtype == torch.float32), _ptr(d), _ptr(ac), _ptr(asc), _ptr(st),
+                             _stream(dev)), "mx_quant_gemm")
+    return d

@@ -21,8 +21,8 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libmx.so")
 
-SOURCES = ["mx_api.cu", "mx_kernels.cu", "mx_bat.cu"]
-HEADERS = ["mx_device.cuh", "mx_launch.h", "mx_stream.cuh"]
+SOURCES = ["mx_api.cu", "mx_kernels.cu", "mx_bat.cu", "mx_gemm.cu"]
+HEADERS = ["mx_device.cuh", "mx_launch.h", "mx_stream.cuh", "mx_tc.cuh"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-ftz=false", "-prec-div=true", "-prec-sqrt=true",
               "-fmad=true", "-Xcompiler", "-fPIC,-O2", "-cudart", "static"]

@@ -255,3 +255,68 @@ int mx_bat_quantize(const void* x, int64_t rows, int64_t cols, int a_dim, const 
 }
 
 }  // extern "C"
+
+namespace {
+
+// Shared checks of the block-scaled GEMM entry points. K must hold whole
+// 256-element K-blocks; N a multiple of 8 (16-byte output stores); the grid's
+// row count bounds M.
+int check_gemm(int64_t M, int64_t N, int64_t K, int out_fp32, const void* b_codes,
+               const uint8_t* b_scales, const void* d) {
+  if (M < 0 || N < 0 || K < 0) return MX_ERR_INVALID_ARG;
+  if (K % 256 != 0 || N % 8 != 0) return MX_ERR_SHAPE;
+  if (M > (int64_t(65535) * 128) || N > (int64_t(1) << 31) || K > (int64_t(1) << 31))
+    return MX_ERR_INVALID_ARG;
+  if ((M > 0 && K > kMaxElems / M) || (N > 0 && K > kMaxElems / N) ||
+      (M > 0 && N > kMaxElems / M))
+    return MX_ERR_INVALID_ARG;
+  if (out_fp32 != 0 && out_fp32 != 1) return MX_ERR_INVALID_ARG;
+  if (M == 0 || N == 0) return MX_OK;
+  if (!d) return MX_ERR_INVALID_ARG;
+  if (!aligned(d, 16)) return MX_ERR_ALIGN;
+  if (K == 0) return MX_OK;
+  if (!b_codes || !b_scales) return MX_ERR_INVALID_ARG;
+  if (!aligned(b_codes, 16) || !aligned(b_scales, 16)) return MX_ERR_ALIGN;
+  return MX_OK;
+}
+
+// K == 0: the product is all zeros.
+int gemm_zero(int64_t M, int64_t N, int out_fp32, void* d, cudaStream_t st) {
+  return from_cuda(cudaMemsetAsync(d, 0, static_cast<size_t>(M * N * (out_fp32 ? 4 : 2)), st));
+}
+
+}  // namespace
+
+extern "C" {
+
+int mx_gemm(const void* a_codes, const uint8_t* a_scales, const void* b_codes,
+            const uint8_t* b_scales, int64_t M, int64_t N, int64_t K, int out_fp32, void* d,
+            int* status, void* stream) {
+  int st = check_gemm(M, N, K, out_fp32, b_codes, b_scales, d);
+  if (st != MX_OK || M == 0 || N == 0) return st;
+  const auto cs = static_cast<cudaStream_t>(stream);
+  if (K == 0) return gemm_zero(M, N, out_fp32, d, cs);
+  if (!a_codes || !a_scales) return MX_ERR_INVALID_ARG;
+  if (!aligned(a_codes, 16) || !aligned(a_scales, 16) || (status && !aligned(status, 4)))
+    return MX_ERR_ALIGN;
+  return from_cuda(mxk::launch_gemm(a_codes, a_scales, 0, b_codes, b_scales, M, N, K, out_fp32, d,
+                                    nullptr, nullptr, status, cs));
+}
+
+int mx_quant_gemm(const void* a_bf16, int scaling, const void* b_codes, const uint8_t* b_scales,
+                  int64_t M, int64_t N, int64_t K, int out_fp32, void* d, void* a_codes_out,
+                  uint8_t* a_scales_out, int* status, void* stream) {
+  if (scaling < MX_SCALE_FLOOR || scaling > MX_SCALE_OAS) return MX_ERR_UNSUPPORTED;
+  int st = check_gemm(M, N, K, out_fp32, b_codes, b_scales, d);
+  if (st != MX_OK || M == 0 || N == 0) return st;
+  const auto cs = static_cast<cudaStream_t>(stream);
+  if (K == 0) return gemm_zero(M, N, out_fp32, d, cs);
+  if (!a_bf16) return MX_ERR_INVALID_ARG;
+  if (!aligned(a_bf16, 32) || (a_codes_out && !aligned(a_codes_out, 8)) ||
+      (status && !aligned(status, 4)))
+    return MX_ERR_ALIGN;
+  return from_cuda(mxk::launch_gemm(a_bf16, nullptr, scaling, b_codes, b_scales, M, N, K,
+                                    out_fp32, d, a_codes_out, a_scales_out, status, cs));
+}
+
+}  // extern "C"

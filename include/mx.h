@@ -211,6 +211,43 @@ int mx_bat_quantize(const void* x, int64_t rows, int64_t cols, int a_dim, const 
                     const float* B, const float* beta_min, const float* beta_max, int format,
                     int scaling, void* codes, uint8_t* scales, uint8_t* macro, void* stream);
 
+/* Block-scaled MXFP4 GEMM on the tensor cores, the consumer of the MX
+ * tensors ([UP] 2.B and 4: the scale work beside the tensor-core GEMM; [VL]
+ * MXFP4 MoE section: SM100 kernels consume MXFP4 operands with E8M0 scales):
+ *   D[M, N] = A[M, K] . B[N, K]^T,
+ * A and B MXFP4 (E2M1 elements, one E8M0 scale per 32 elements along K), the
+ * products summed in fp32 by tcgen05.mma.kind::mxf4.block_scale (the
+ * tensor cores' summation order is not specified; results agree with the
+ * exact product within fp32 rounding and are bit-exact where every partial
+ * sum is exact), D written as bf16 (nearest even) or, with out_fp32 = 1, as
+ * float. Row-major everywhere:
+ *   b_codes   device uint8 [N, K/2], as mx_quantize writes MXFP4 codes
+ *             (16-byte aligned).
+ *   b_scales  device uint8, B's scales in the MX_SCALES_MMA layout
+ *             (mx_scale_bytes(N, K, MX_FMT_E2M1, MX_SCALES_MMA) bytes;
+ *             16-byte aligned).
+ *   d         device [M, N] bf16 or float (16-byte aligned).
+ *   status    device int32 or NULL: set nonzero if one of the kernel's waits
+ *             ran out (a kernel fault, not a result; the output is then
+ *             undefined). Never cleared by the library.
+ * Shapes: K a multiple of 256, N a multiple of 8 (MX_ERR_SHAPE); M up to
+ * 8,388,480. M == 0 or N == 0 does nothing; K == 0 writes zeros.
+ * mx_gemm: A pre-quantized, a_codes [M, K/2] (16-byte aligned) and a_scales
+ * in the MX_SCALES_MMA layout (16-byte aligned).
+ * mx_quant_gemm: A given as bf16 [M, K] (32-byte aligned) and quantized to
+ * MXFP4 inside the GEMM with `scaling` (MX_SCALE_FLOOR, CEIL, OAS_RULE or
+ * OAS; no MBS: its factors are not powers of two, which a block-scaled MMA
+ * cannot apply), exactly as mx_quantize would quantize it; the quantized A
+ * is written out only if a_codes_out ([M, K/2], 8-byte aligned) and/or
+ * a_scales_out (MX_SCALES_MMA layout) are given. Other errors as
+ * mx_quantize. */
+int mx_gemm(const void* a_codes, const uint8_t* a_scales, const void* b_codes,
+            const uint8_t* b_scales, int64_t M, int64_t N, int64_t K, int out_fp32, void* d,
+            int* status, void* stream);
+int mx_quant_gemm(const void* a_bf16, int scaling, const void* b_codes, const uint8_t* b_scales,
+                  int64_t M, int64_t N, int64_t K, int out_fp32, void* d, void* a_codes_out,
+                  uint8_t* a_scales_out, int* status, void* stream);
+
 /* Static description of a status code (never NULL). */
 const char* mx_status_string(int status);
 

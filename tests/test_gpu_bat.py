@@ -266,7 +266,7 @@ def test_apply_integer_cases_equal_the_kronecker_product(mx, oracle_mod, cuda, a
 
 @pytest.mark.parametrize("a", A_DIMS)
 @pytest.mark.parametrize("clip", [False, True])
-@pytest.mark.parametrize("shape", [(37, 96), (130, 1152)])
+@pytest.mark.parametrize("shape", [(37, 384), (130, 1152)])
 def test_apply_within_the_rounding_bound_of_the_fp64_product(mx, oracle_mod, cuda, a, clip, shape):
     """Random data and parameters: |y_gpu - y| is bounded, per element, by
     the fp32 error of the transform and the thresholds, carried through the
