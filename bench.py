@@ -153,24 +153,97 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
-def oracle_baseline(x_host_rows, budget_s: float = 10.0):
-    """Times the CPU oracle on a bounded sample of the workload (rows of 2048)."""
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def _timed(fn):
+    t0 = time.perf_counter()
+    fn()
+    return time.perf_counter() - t0
+
+
+def _rows_for(fn_rows, total_rows, budget_s, probe_rows):
+    """Rows of a sample that takes about budget_s, from a timed probe."""
+    probe_rows = min(probe_rows, total_rows)
+    dt = _timed(lambda: fn_rows(probe_rows))
+    rate = probe_rows / max(dt, 1e-6)
+    return int(min(total_rows, max(probe_rows, rate * budget_s)))
+
+
+def oracle_baseline(x_host_rows, inputs_mod, budget_s: float = 8.0):
+    """The CPU oracle on the host cores: the headline workload (MoE w13 stack,
+    MXFP4 FLOOR quantize) on a bounded sample with every core and with one
+    thread, then each other workload's op(s) on a bounded sample with every
+    core. Input SHA-256 over each whole tensor's bf16 bytes."""
+    import hashlib as _hl
+    import numpy as np
     import oracle
     threads = len(os.sched_getaffinity(0))
     oracle.set_threads(threads)
-    probe = x_host_rows[:256]
-    t0 = time.perf_counter()
-    oracle.quantize(probe, 0, 0)
-    rate = probe.shape[0] / max(time.perf_counter() - t0, 1e-6)        # rows per s
-    nrows = int(min(x_host_rows.shape[0], max(256, rate * budget_s)))
-    sample = x_host_rows[:nrows]
-    t0 = time.perf_counter()
-    oracle.quantize(sample, 0, 0)
-    dt = time.perf_counter() - t0
-    nbytes = sample.size * 2 + sample.size // 2 + sample.size // 32
-    return {"value": nbytes / dt / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
-            "sample": f"first {nrows} of {x_host_rows.shape[0]} rows of 2048 ({sample.size} elements), "
-                      f"{dt:.2f} s on {threads} threads, scalar C++ oracle"}
+    q = lambda rows: oracle.quantize(x_host_rows[:rows], 0, 0)
+    nrows = _rows_for(q, x_host_rows.shape[0], budget_s, 256)
+    dt = _timed(lambda: q(nrows))
+    n = nrows * HIDDEN
+    per_elem_bytes = 2 + 0.5 + 1 / 32
+    out = {"value": n * per_elem_bytes / dt / 1e9, "unit": "GB/s", "cores": threads, "kind": "oracle",
+           "cpu_model": cpu_model(),
+           "sample": f"first {nrows} of {x_host_rows.shape[0]} rows of 2048 ({n} elements) of the "
+                     f"headline stack, {dt:.2f} s on {threads} threads, scalar C++ oracle",
+           "input_sha256": {"moe_w13_128x1536x2048": _hl.sha256(x_host_rows.tobytes()).hexdigest()},
+           "input_sha256_of": "the tensors the oracle timed: the headline stack is the bench's own "
+                              "input copied from the device; the other workloads are generated on "
+                              "the host from the same seeds (a different stream than on the device)"}
+    oracle.set_threads(1)
+    r1 = _rows_for(q, x_host_rows.shape[0], 2.0, 16)
+    d1 = _timed(lambda: q(r1))
+    out["single_thread"] = {"value": r1 * HIDDEN * per_elem_bytes / d1 / 1e9, "unit": "GB/s",
+                            "sample": f"first {r1} rows, {d1:.2f} s, 1 thread"}
+    oracle.set_threads(threads)
+    per_cfg = {}
+
+    def rec(name, arr, bytes_per_elem, fn, budget=1.5, probe=64):
+        rows = _rows_for(lambda r: fn(arr[:r]), arr.shape[0], budget, probe)
+        dtc = _timed(lambda: fn(np.ascontiguousarray(arr[:rows])))
+        ne = rows * arr.shape[1]
+        per_cfg[name] = {"GB/s": round(ne * bytes_per_elem / dtc / 1e9, 4),
+                         "elements_per_s": round(ne / dtc), "rows": rows, "of_rows": arr.shape[0],
+                         "s": round(dtc, 3)}
+
+    bits = inputs_mod.bf16_bits_numpy
+    x1 = bits(inputs_mod.outlier_act())
+    out["input_sha256"]["outlier_act_256x4096"] = _hl.sha256(x1.tobytes()).hexdigest()
+    rec("outlier_act_256x4096/fp4_floor_quantize", x1, 2.53125, lambda a: oracle.quantize(a, 0, 0))
+    c1, s1, _ = oracle.quantize(x1, 0, 0)
+    t_deq = _timed(lambda: oracle.dequantize(c1, s1, None, 256, 4096, 0))
+    per_cfg["outlier_act_256x4096/fp4_dequantize_bf16"] = {
+        "GB/s": round(256 * 4096 * 2.53125 / t_deq / 1e9, 4), "rows": 256, "of_rows": 256,
+        "s": round(t_deq, 3)}
+    x2 = bits(inputs_mod.mlp_weight())
+    out["input_sha256"]["mlp_weight_8192x3072"] = _hl.sha256(x2.tobytes()).hexdigest()
+    rec("mlp_weight_8192x3072/fp8_floor_quantize", x2, 3.03125, lambda a: oracle.quantize(a, 1, 0))
+    x3 = bits(inputs_mod.qat_act())
+    g3 = bits(inputs_mod.qat_grad(16384, 3072))
+    out["input_sha256"]["qat_act_16384x3072"] = _hl.sha256(x3.tobytes()).hexdigest()
+    rec("qat_act_16384x3072/fp4_fake_quant_fwd", x3, 4, lambda a: oracle.fake_quant_fwd(a))
+    rec("qat_act_16384x3072/fp4_fake_quant_bwd", x3, 6,
+        lambda a: oracle.fake_quant_bwd(a, np.ascontiguousarray(g3[:a.shape[0]])))
+    x4 = bits(inputs_mod.heavy_tail())
+    out["input_sha256"]["heavy_tail_8192x4096"] = _hl.sha256(x4.tobytes()).hexdigest()
+    for mname, m in (("FLOOR", 0), ("OAS", 3), ("MBS_STATIC", 16), ("MBS_DYNAMIC", 32)):
+        rec(f"heavy_tail_8192x4096/fp4_{mname}_quantize", x4, 2.53125 + (1 / 128 if m >> 4 else 0),
+            lambda a, m=m: oracle.quantize(a, 0, m), budget=1.0, probe=2 if m >> 4 == 2 else 32)
+    rec("heavy_tail_8192x4096/fp4_FLOOR_block_error", x4, 2,
+        lambda a: oracle.block_error(a, 0, 0, want_blocks=False))
+    out["per_config"] = per_cfg
+    return out
 
 
 # --------------------------------------------------------------- arms --
@@ -387,6 +460,81 @@ def other_ops(mx, inputs, dev, reps=10):
     return res
 
 
+GEMM_SHAPES = [
+    # (name, M tokens, N, K): the Llama-3.2-3B MLP weight [8192, 3072] as B
+    ("llama3.2-3b_mlp_prefill_4096tok", 4096, 8192, 3072),
+    ("llama3.2-3b_mlp_decode_128tok", 128, 8192, 3072),
+    ("square_8192", 8192, 8192, 8192),
+]
+
+
+def measured_fp4_peak():
+    """Dense FP4 tensor peak: the measured bf16 GEMM burst x 4 (the nominal
+    FP4 / bf16 ratio, 9 / 2.25 PFLOP/s)."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return 4.0 * float(json.load(f)["bf16_tflops"]), "measured bf16 burst x 4 (nominal ratio)"
+    except Exception:
+        return 4.0 * 1590.0, "fallback bf16 x 4"
+
+
+def gemm_ops(mx, inputs, dev, reps=20):
+    """The block-scaled MXFP4 GEMM D = A B^T (bf16 out) on the tensor cores:
+    A pre-quantized; A quantized inside the GEMM (fused); quantize then GEMM
+    (unfused). Median CUDA-event time of `reps`, L2 flushed before each. The
+    library's block-scaled GEMM (cuBLAS through torch) on the same operands is
+    timed beside it as context."""
+    import torch
+    F = torch.nn.functional
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+    peak, peak_src = measured_fp4_peak()
+    res = {"_peak_tflops": peak, "_peak_source": peak_src}
+    for name, M, N, K in GEMM_SHAPES:
+        a = inputs.normal_weight(M, K, seed=11, device=dev, std=1.0)
+        w = inputs.normal_weight(N, K, seed=12, device=dev)
+        bc, bs, _ = mx.quantize(w, mx.E2M1, mx.FLOOR | mx.MMA_SCALES)
+        ac, as_, _ = mx.quantize(a, mx.E2M1, mx.FLOOR | mx.MMA_SCALES)
+        d = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+        st = torch.zeros(1, dtype=torch.int32, device=dev)
+        fns = {
+            "quantize_a": lambda: mx.quantize(a, mx.E2M1, mx.FLOOR | mx.MMA_SCALES, out=(ac, as_, None)),
+            "gemm": lambda: mx.gemm(ac, as_, bc, bs, out=d, status=st),
+            "fused_quant_gemm": lambda: mx.quant_gemm(a, bc, bs, mx.FLOOR, out=d, status=st),
+            "unfused_quantize_then_gemm": lambda: (
+                mx.quantize(a, mx.E2M1, mx.FLOOR | mx.MMA_SCALES, out=(ac, as_, None)),
+                mx.gemm(ac, as_, bc, bs, out=d, status=st)),
+        }
+        r = {"M": M, "N": N, "K": K, "flop": 2.0 * M * N * K}
+        for k, fn in fns.items():
+            fn()
+            torch.cuda.synchronize()
+            ms = time_op(fn, reps, flush)
+            r[k + "_us"] = round(ms * 1e3, 2)
+            if k != "quantize_a":
+                r[k + "_tflops"] = round(r["flop"] / (ms * 1e-3) / 1e12, 1)
+        r["gemm_frac_of_peak"] = round(r["gemm_tflops"] / peak, 3)
+        r["fused_vs_unfused"] = round(r["unfused_quantize_then_gemm_us"] / r["fused_quant_gemm_us"], 3)
+        try:
+            lib = lambda: F.scaled_mm(ac.view(torch.float4_e2m1fn_x2), bc.view(torch.float4_e2m1fn_x2).t(),
+                                      as_.view(torch.float8_e8m0fnu), F.ScalingType.BlockWise1x32,
+                                      bs.view(torch.float8_e8m0fnu), F.ScalingType.BlockWise1x32,
+                                      swizzle_a=F.SwizzleType.SWIZZLE_32_4_4,
+                                      swizzle_b=F.SwizzleType.SWIZZLE_32_4_4, output_dtype=torch.bfloat16)
+            ref = lib()
+            mx.gemm(ac, as_, bc, bs, out=d, status=st)
+            torch.cuda.synchronize()
+            r["context_library_gemm_us"] = round(time_op(lib, reps, flush) * 1e3, 2)
+            r["context_library_gemm_bit_identical"] = bool(torch.equal(ref.view(torch.int16),
+                                                                       d.view(torch.int16)))
+        except Exception as e:   # the library path is context only
+            r["context_library_gemm"] = f"unavailable: {str(e).splitlines()[0][:120]}"
+        r["status"] = int(st.item())
+        res[name] = r
+        del a, w, bc, bs, ac, as_, d
+    del flush
+    return res
+
+
 def run_mx(args):
     import torch
     import torch.distributed as dist
@@ -478,10 +626,11 @@ def run_mx(args):
     if not args.no_ops and world == 1:
         ops = {"moe_w13_128x1536x2048": stack_ops(mx, x)}
         ops.update(other_ops(mx, inputs, dev))
+        ops["gemm_mxfp4"] = gemm_ops(mx, inputs, dev)
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        cpu = oracle_baseline(xh.view(torch.int16).numpy().view("uint16").reshape(-1, HIDDEN))
+        cpu = oracle_baseline(xh.view(torch.int16).numpy().view("uint16").reshape(-1, HIDDEN), inputs)
     del xh
 
     peak, peak_src = measured_peak()

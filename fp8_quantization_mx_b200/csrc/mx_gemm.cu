@@ -24,10 +24,13 @@
 //              the streaming kernels' per-slice quantizer straight from
 //              global memory into the swizzled operand tile and the scale
 //              tile in shared memory: the quantized activations never reach
-//              HBM; then the epilogue
-//   warps 2-5  (pre-quantized A) the epilogue
-// Epilogue: TMEM -> registers (tcgen05.ld, one row per thread), fp32 -> bf16
-// (or fp32) -> global.
+//              HBM; then the epilogue of the tile
+//   warps 2-9  (pre-quantized A) the epilogue
+// Epilogue: TMEM -> registers (tcgen05.ld, one row per thread, two warps
+// per 32-lane quarter splitting the columns), the accumulator released to
+// the next tile, then fp32 -> bf16 (or fp32) -> global.
+// The kernel is persistent (one CTA per SM looping over tiles), so the next
+// tile's loads overlap the previous tile's epilogue.
 //
 // Every wait is bounded in time (mbar_wait): a wait that runs out sets the
 // caller's status word and the CTA drains its in-flight copies and MMAs,
@@ -52,7 +55,7 @@ constexpr uint32_t kSfTile = 512;  // 128 rows x 4 scales
 
 // Status codes a timed-out wait leaves in *status (which role gave up).
 constexpr int kStatusProducer = 1, kStatusMmaB = 2, kStatusMmaA = 3, kStatusQuant = 4,
-              kStatusEpilogue = 5, kStatusDrain = 6;
+              kStatusEpilogue = 5, kStatusDrain = 6, kStatusStaging = 7;
 
 struct GemmArgs {
   const uint8_t* a_bf16;    // fused: bf16 A [M, K]
@@ -66,16 +69,20 @@ struct GemmArgs {
   int out_fp32;
 };
 
+// Shared-memory plan common to both kernels: S stages of (A codes, B codes,
+// A scale tiles, B scale tiles), then (fused) one bf16 staging tile of A,
+// then the barriers.
 template <int BN, int S, bool FUSED>
 struct GemmCfg {
-  static constexpr int kQuantWarps = FUSED ? 8 : 4;   // warps after the two control warps
-  static constexpr int kThreads = (2 + kQuantWarps) * 32;
+  static constexpr int kWorkWarps = 8;   // quantizer (fused) and epilogue warps
+  static constexpr int kThreads = (2 + kWorkWarps) * 32;
   static constexpr uint32_t kTileB = BN * kRowBytes;
   static constexpr uint32_t kSfA = 2 * kSfTile;                   // one band, two K-tiles
   static constexpr uint32_t kSfB = (BN / 128) * 2 * kSfTile;      // BN/128 bands
   static constexpr uint32_t kStage = kTileA + kTileB + kSfA + kSfB;
-  static constexpr uint32_t kBarBytes = 8 * (3 * S + 1) + 8;
-  static constexpr uint32_t kSmem = S * kStage + kBarBytes + 1024;   // + alignment slack
+  static constexpr uint32_t kStaging = FUSED ? kGemmBM * kGemmBK * 2 : 0;   // bf16 A tile
+  static constexpr uint32_t kBarBytes = 8 * (4 * S + 3) + 8;
+  static constexpr uint32_t kSmem = S * kStage + kStaging + kBarBytes + 1024;   // + alignment
   // TMEM: BN accumulator columns, then per stage 8 columns of A scales and
   // BN/16 of B scales (two K-tiles x bands x 4 columns)
   static constexpr uint32_t kSfCols = 8 + BN / 16;
@@ -85,171 +92,445 @@ struct GemmCfg {
   static_assert(kSmem <= 227 * 1024, "shared memory");
 };
 
-template <int BN, int S, bool FUSED, int RULE>
-__global__ void __launch_bounds__(GemmCfg<BN, S, FUSED>::kThreads, 1)
+// Addresses of one CTA's shared-memory plan.
+template <int BN, int S, bool FUSED>
+struct Smem {
+  using C = GemmCfg<BN, S, FUSED>;
+  uint32_t base, sA, sB, sSFA, sSFB, sStg, sBar;
+  uint32_t* tmem_holder;
+  volatile int* abort_flag;
+  __device__ explicit Smem(uint8_t* raw_ptr) {
+    const uint32_t raw = tc::smem_addr(raw_ptr);
+    base = (raw + 1023u) & ~1023u;   // 128-byte swizzle atoms need 1024-byte alignment
+    sA = base;
+    sB = sA + S * kTileA;
+    sSFA = sB + S * C::kTileB;
+    sSFB = sSFA + S * C::kSfA;
+    sStg = sSFB + S * C::kSfB;
+    sBar = sStg + C::kStaging;
+    tmem_holder = reinterpret_cast<uint32_t*>(raw_ptr + (sBar + 8u * (4 * S + 3) - raw));
+    abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
+  }
+  __device__ uint32_t fullB(int s) const { return sBar + 8u * s; }
+  __device__ uint32_t fullA(int s) const { return sBar + 8u * (S + s); }
+  __device__ uint32_t empty(int s) const { return sBar + 8u * (2 * S + s); }
+  __device__ uint32_t tfull() const { return sBar + 8u * (3 * S); }
+  __device__ uint32_t tempty() const { return sBar + 8u * (3 * S + 1); }
+  __device__ uint32_t stg_full() const { return sBar + 8u * (3 * S + 2); }
+  __device__ uint32_t qfree(int s) const { return sBar + 8u * (3 * S + 3 + s); }
+};
+
+// One K-block on the tensor cores (one thread): the stage's scale tiles into
+// TMEM, then four MMAs of K = 64.
+template <int BN, int S, bool FUSED>
+__device__ __forceinline__ void issue_kblock(const Smem<BN, S, FUSED>& sm, uint32_t tmem, int s,
+                                             bool first) {
+  using C = GemmCfg<BN, S, FUSED>;
+  const uint32_t sfa = tmem + BN + s * C::kSfCols;
+  const uint32_t sfb = sfa + 8;
+  tc::tmem_cp_sf(sfa, tc::sf_desc(sm.sSFA + s * C::kSfA));
+  tc::tmem_cp_sf(sfa + 4, tc::sf_desc(sm.sSFA + s * C::kSfA + kSfTile));
+#pragma unroll
+  for (int tt = 0; tt < 2; ++tt)
+#pragma unroll
+    for (int band = 0; band < BN / 128; ++band)
+      tc::tmem_cp_sf(sfb + tt * (BN / 32) + band * 4,
+                     tc::sf_desc(sm.sSFB + s * C::kSfB + band * 2 * kSfTile + tt * kSfTile));
+  const uint64_t adesc = tc::kmajor_sw128_desc(sm.sA + s * kTileA);
+  const uint64_t bdesc = tc::kmajor_sw128_desc(sm.sB + s * C::kTileB);
+#pragma unroll
+  for (int kk = 0; kk < 4; ++kk) {
+    // K = 64 per MMA: 32 code bytes further along the swizzled rows; scales:
+    // K-tile kk / 2, byte (kk % 2) * 2 of the 32-bit word
+    const int tt = kk >> 1;
+    tc::mma_mxf4(tmem, adesc + 2 * kk, bdesc + 2 * kk, tc::idesc_mxf4(kGemmBM, BN, (kk & 1) * 2),
+                 sfa + tt * 4, sfb + tt * (BN / 32), !(first && kk == 0));
+  }
+}
+
+// Epilogue of one tile by the eight work warps: warp w reads TMEM lanes
+// 32 (w % 4) .. + 31 (its quarter), warps 2-5 the first half of the columns
+// and warps 6-9 the second; the values go to registers, the accumulator is
+// released (tmem_empty), then fp32 -> bf16 (or fp32) -> global. Returns
+// false when the kernel is aborting.
+template <int BN, int S, bool FUSED>
+__device__ __forceinline__ bool epilogue_tile(const Smem<BN, S, FUSED>& sm, const GemmArgs& g,
+                                              uint32_t tmem, uint32_t tile_par, int64_t m0,
+                                              int64_t n0, int warp, int lane) {
+  const int q = warp & 3;
+  const int c_begin = ((warp - 2) / 4) * (BN / 2);
+  const bool got =
+      tc::mbar_wait(sm.tfull(), tile_par, sm.abort_flag, g.status, kStatusEpilogue, false);
+  tc::tc_fence_after();
+  // one decision for all eight warps (tcgen05.ld is a whole-warp instruction,
+  // and the fused kernel's work warps meet at named barriers afterwards)
+  if (!tc::named_all(3, GemmCfg<BN, S, FUSED>::kWorkWarps * 32, got && !*sm.abort_flag))
+    return false;
+  const int64_t m = m0 + q * 32 + lane;
+  constexpr int kCols = BN / 2;
+  uint32_t acc[kCols];
+#pragma unroll
+  for (int c0 = 0; c0 < kCols; c0 += 32) {
+    uint32_t r[32];
+    tc::tmem_ld32(tmem + (static_cast<uint32_t>(q * 32) << 16) + c_begin + c0, r);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) acc[c0 + i] = r[i];
+  }
+  tc::tc_fence_before();
+  __syncwarp();
+  if (lane == 0) tc::mbar_arrive(sm.tempty());
+  if (m < g.M) {
+#pragma unroll
+    for (int gq = 0; gq < kCols / 8; ++gq) {
+      const int64_t n = n0 + c_begin + 8 * gq;
+      if (n < g.N) {
+        if (g.out_fp32) {
+          uint4* o = reinterpret_cast<uint4*>(g.d + (m * g.N + n) * 4);
+          o[0] = make_uint4(acc[8 * gq], acc[8 * gq + 1], acc[8 * gq + 2], acc[8 * gq + 3]);
+          o[1] = make_uint4(acc[8 * gq + 4], acc[8 * gq + 5], acc[8 * gq + 6], acc[8 * gq + 7]);
+        } else {
+          uint32_t h[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            const __nv_bfloat162 b2 = __floats2bfloat162_rn(
+                __uint_as_float(acc[8 * gq + 2 * i]), __uint_as_float(acc[8 * gq + 2 * i + 1]));
+            h[i] = *reinterpret_cast<const uint32_t*>(&b2);
+          }
+          *reinterpret_cast<uint4*>(g.d + (m * g.N + n) * 2) = make_uint4(h[0], h[1], h[2], h[3]);
+        }
+      }
+    }
+  }
+  return true;
+}
+
+// ------------------------------------------- pre-quantized A: persistent --
+// CTA b takes tiles b, b + gridDim.x, ... (tile t: m-tile t / tiles_n, n-tile
+// t % tiles_n). The stage ring runs on across tiles; the accumulator is
+// handed between the MMA issuer and the epilogue by the tmem_full /
+// tmem_empty barriers, so the next tile's loads proceed while the epilogue
+// drains the accumulator.
+template <int BN, int S>
+__global__ void __launch_bounds__(GemmCfg<BN, S, false>::kThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const GemmArgs g) {
-  using C = GemmCfg<BN, S, FUSED>;
+  using C = GemmCfg<BN, S, false>;
   extern __shared__ uint8_t smem_raw[];
-  const uint32_t raw = tc::smem_addr(smem_raw);
-  const uint32_t base = (raw + 1023u) & ~1023u;   // 128-byte swizzle atoms need 1024 alignment
-  uint8_t* const gbase = smem_raw + (base - raw);
-  const uint32_t sA = base;
-  const uint32_t sB = sA + S * kTileA;
-  const uint32_t sSFA = sB + S * C::kTileB;
-  const uint32_t sSFB = sSFA + S * C::kSfA;
-  const uint32_t sBar = sSFB + S * C::kSfB;
-  auto fullB = [&](int s) { return sBar + 8u * s; };
-  auto fullA = [&](int s) { return sBar + 8u * (S + s); };
-  auto empty = [&](int s) { return sBar + 8u * (2 * S + s); };
-  const uint32_t tfull = sBar + 8u * (3 * S);
-  uint32_t* const tmem_holder = reinterpret_cast<uint32_t*>(gbase + (sBar + 8u * (3 * S + 1) - base));
-  volatile int* const abort_flag = reinterpret_cast<volatile int*>(tmem_holder + 1);
-
+  const Smem<BN, S, false> sm(smem_raw);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int64_t n0 = static_cast<int64_t>(blockIdx.x) * BN;
-  const int64_t m0 = static_cast<int64_t>(blockIdx.y) * kGemmBM;
   const int nk = static_cast<int>(g.K / kGemmBK);
   const int64_t T = g.K / 128;   // scale tiles per 128-row band
+  const int64_t tiles_n = (g.N + BN - 1) / BN;
+  const int64_t ntiles = ((g.M + kGemmBM - 1) / kGemmBM) * tiles_n;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < S; ++s) {
-      tc::mbar_init(fullB(s), 1);
-      tc::mbar_init(fullA(s), FUSED ? C::kQuantWarps : 1);
-      tc::mbar_init(empty(s), 1);
+      tc::mbar_init(sm.fullB(s), 1);
+      tc::mbar_init(sm.empty(s), 1);
     }
-    tc::mbar_init(tfull, 1);
-    *abort_flag = 0;
+    tc::mbar_init(sm.tfull(), 1);
+    tc::mbar_init(sm.tempty(), C::kWorkWarps);
+    *sm.abort_flag = 0;
     tc::fence_mbar_init();
   }
-  if (warp == 1) tc::tmem_alloc(tc::smem_addr(tmem_holder), C::kTmemCols);
+  if (warp == 1) tc::tmem_alloc(tc::smem_addr(sm.tmem_holder), C::kTmemCols);
   tc::tc_fence_before();
   __syncthreads();
   tc::tc_fence_after();
-  const uint32_t tmem = *tmem_holder;
+  const uint32_t tmem = *sm.tmem_holder;
 
   if (warp == 0) {
     // ---------------------------------------------------------- producer
     if (lane == 0) {
       tc::prefetch_tmap(&tmB);
-      if (!FUSED) tc::prefetch_tmap(&tmA);
-      // B's scale bands present in the tiled buffer (rows padded to 128)
-      const int64_t nb0 = n0 / 128;
+      tc::prefetch_tmap(&tmA);
       const int64_t bands_total = (g.N + 127) / 128;
-      const int64_t left = bands_total - nb0;
-      const int nbands = static_cast<int>(left < BN / 128 ? left : BN / 128);
-      const uint32_t tx = C::kTileB + nbands * 2 * kSfTile + (FUSED ? 0u : kTileA + 2 * kSfTile);
-      int armed = 0;
-      for (int kb = 0; kb < nk; ++kb) {
-        const int s = kb % S;
-        const uint32_t ph = (kb / S) & 1;
-        if (!tc::mbar_wait(empty(s), ph ^ 1, abort_flag, g.status, kStatusProducer)) break;
-        tc::mbar_arrive_expect_tx(fullB(s), tx);
-        tc::tma_load_2d(sB + s * C::kTileB, &tmB, kb * static_cast<int>(kRowBytes),
-                        static_cast<int>(n0), fullB(s));
-        for (int band = 0; band < nbands; ++band)
-          tc::bulk_load(sSFB + s * C::kSfB + band * 2 * kSfTile,
-                        g.b_scales + ((nb0 + band) * T + 2 * kb) * kSfTile, 2 * kSfTile, fullB(s));
-        if (!FUSED) {
-          tc::tma_load_2d(sA + s * kTileA, &tmA, kb * static_cast<int>(kRowBytes),
-                          static_cast<int>(m0), fullB(s));
-          tc::bulk_load(sSFA + s * C::kSfA, g.a_scales + ((m0 / 128) * T + 2 * kb) * kSfTile,
-                        2 * kSfTile, fullB(s));
+      int64_t it = 0;   // K-blocks issued so far (the ring position)
+      bool ok = true;
+      for (int64_t t = blockIdx.x; ok && t < ntiles; t += gridDim.x) {
+        const int64_t m0 = (t / tiles_n) * kGemmBM;
+        const int64_t n0 = (t % tiles_n) * BN;
+        // B's scale bands present in the tiled buffer (rows padded to 128)
+        const int64_t nb0 = n0 / 128;
+        const int64_t left = bands_total - nb0;
+        const int nbands = static_cast<int>(left < BN / 128 ? left : BN / 128);
+        const uint32_t tx = C::kTileB + nbands * 2 * kSfTile + kTileA + 2 * kSfTile;
+        for (int kb = 0; kb < nk; ++kb, ++it) {
+          const int s = static_cast<int>(it % S);
+          const uint32_t ph = static_cast<uint32_t>(it / S) & 1;
+          if (!tc::mbar_wait(sm.empty(s), ph ^ 1, sm.abort_flag, g.status, kStatusProducer)) {
+            ok = false;
+            break;
+          }
+          tc::mbar_arrive_expect_tx(sm.fullB(s), tx);
+          tc::tma_load_2d(sm.sB + s * C::kTileB, &tmB, kb * static_cast<int>(kRowBytes),
+                          static_cast<int>(n0), sm.fullB(s));
+          for (int band = 0; band < nbands; ++band)
+            tc::bulk_load(sm.sSFB + s * C::kSfB + band * 2 * kSfTile,
+                          g.b_scales + ((nb0 + band) * T + 2 * kb) * kSfTile, 2 * kSfTile,
+                          sm.fullB(s));
+          tc::tma_load_2d(sm.sA + s * kTileA, &tmA, kb * static_cast<int>(kRowBytes),
+                          static_cast<int>(m0), sm.fullB(s));
+          tc::bulk_load(sm.sSFA + s * C::kSfA, g.a_scales + ((m0 / 128) * T + 2 * kb) * kSfTile,
+                        2 * kSfTile, sm.fullB(s));
         }
-        armed = kb + 1;
       }
       // every copy this thread issued has landed before the CTA can exit
-      for (int kb = max(0, armed - S); kb < armed; ++kb)
-        tc::mbar_wait(fullB(kb % S), (kb / S) & 1, abort_flag, g.status, kStatusDrain, false);
+      for (int64_t j = (it > S ? it - S : 0); j < it; ++j)
+        tc::mbar_wait(sm.fullB(static_cast<int>(j % S)), static_cast<uint32_t>(j / S) & 1,
+                      sm.abort_flag, g.status, kStatusDrain, false);
     }
     __syncwarp();
   } else if (warp == 1) {
     // ------------------------------------------------------ MMA issuer
     if (lane == 0) {
-      for (int kb = 0; kb < nk; ++kb) {
-        const int s = kb % S;
-        const uint32_t ph = (kb / S) & 1;
-        if (!tc::mbar_wait(fullB(s), ph, abort_flag, g.status, kStatusMmaB)) break;
-        if (FUSED && !tc::mbar_wait(fullA(s), ph, abort_flag, g.status, kStatusMmaA)) break;
-        tc::tc_fence_after();
-        const uint32_t sfa = tmem + BN + s * C::kSfCols;
-        const uint32_t sfb = sfa + 8;
-        tc::tmem_cp_sf(sfa, tc::sf_desc(sSFA + s * C::kSfA));
-        tc::tmem_cp_sf(sfa + 4, tc::sf_desc(sSFA + s * C::kSfA + kSfTile));
-#pragma unroll
-        for (int t = 0; t < 2; ++t)
-#pragma unroll
-          for (int band = 0; band < BN / 128; ++band)
-            tc::tmem_cp_sf(sfb + t * (BN / 32) + band * 4,
-                           tc::sf_desc(sSFB + s * C::kSfB + band * 2 * kSfTile + t * kSfTile));
-        const uint64_t adesc = tc::kmajor_sw128_desc(sA + s * kTileA);
-        const uint64_t bdesc = tc::kmajor_sw128_desc(sB + s * C::kTileB);
-#pragma unroll
-        for (int kk = 0; kk < 4; ++kk) {
-          // K = 64 per MMA: 32 code bytes further along the swizzled rows;
-          // scales: K-tile kk / 2, byte (kk % 2) * 2 of the 32-bit word
-          const int t = kk >> 1;
-          tc::mma_mxf4(tmem, adesc + 2 * kk, bdesc + 2 * kk,
-                       tc::idesc_mxf4(kGemmBM, BN, (kk & 1) * 2), sfa + t * 4, sfb + t * (BN / 32),
-                       (kb | kk) != 0);
+      int64_t it = 0;
+      uint32_t tile_par = 0;
+      bool ok = true;
+      for (int64_t t = blockIdx.x; ok && t < ntiles; t += gridDim.x, tile_par ^= 1) {
+        // the epilogue has read the previous tile's accumulator
+        ok = tc::mbar_wait(sm.tempty(), tile_par ^ 1, sm.abort_flag, g.status, kStatusMmaB);
+        if (ok) tc::tc_fence_after();
+        for (int kb = 0; ok && kb < nk; ++kb, ++it) {
+          const int s = static_cast<int>(it % S);
+          const uint32_t ph = static_cast<uint32_t>(it / S) & 1;
+          if (!tc::mbar_wait(sm.fullB(s), ph, sm.abort_flag, g.status, kStatusMmaB)) {
+            ok = false;
+            break;
+          }
+          tc::tc_fence_after();
+          issue_kblock(sm, tmem, s, kb == 0);
+          tc::tc_commit(sm.empty(s));
         }
-        tc::tc_commit(empty(s));
+        // committed on every exit, so that the epilogue never waits for a
+        // commit that will not come and TMEM is never freed under an MMA
+        tc::tc_commit(sm.tfull());
       }
-      // arrives once every MMA issued above has completed (also after a
-      // break, so that TMEM is never freed under a running MMA)
-      tc::tc_commit(tfull);
     }
     __syncwarp();
   } else {
-    const int qw = warp - 2;
-    if constexpr (FUSED) {
-      // ------------------------------------------- prologue: quantize A
-      // warp qw owns rows 16 qw .. 16 qw + 15 of the tile; per pass p, lanes
-      // 0-15 take row 16 qw + 2p and lanes 16-31 the next; lane j16 = lane &
-      // 15 takes elements 16 j16 .. 16 j16 + 15 of the K-block (a lane pair
-      // is one 32-element block)
-      const int j16 = lane & 15;
-      const int64_t K2 = g.K * 2;   // bf16 row pitch in bytes
-      const bool write_a = (blockIdx.x == 0);
-      V16 v[8], nv[8];
-      auto load = [&](int kb, V16 (&dst)[8]) {
-#pragma unroll
-        for (int p = 0; p < 8; ++p) {
-          const int r = 16 * qw + 2 * p + (lane >> 4);
-          const int64_t m = m0 + r;
-          if (m < g.M) {
-            dst[p] = ld_stream32(g.a_bf16 + m * K2 + (static_cast<int64_t>(kb) * kGemmBK + 16 * j16) * 2);
-          } else {
-#pragma unroll
-            for (int i = 0; i < 8; ++i) dst[p].w[i] = 0;
+    // ---------------------------------------------------------- epilogue
+    uint32_t tile_par = 0;
+    for (int64_t t = blockIdx.x; t < ntiles; t += gridDim.x, tile_par ^= 1) {
+      if (!epilogue_tile(sm, g, tmem, tile_par, (t / tiles_n) * kGemmBM, (t % tiles_n) * BN,
+                         warp, lane))
+        break;
+    }
+    tc::tc_fence_before();
+  }
+  __syncthreads();
+  if (warp == 1) {
+    tc::tc_fence_after();
+    tc::tmem_dealloc(tmem, C::kTmemCols);
+  }
+}
+
+// ---------------------------------------- bf16 A quantized in the prologue --
+// A cluster of CL CTAs works on one m-tile and CL adjacent n-tiles at a time
+// (a "unit"; units are taken persistently, the cluster's CTAs in step). The
+// K-blocks of the unit are dealt round-robin over the cluster (K-block `it`
+// of the ring, counted across units, belongs to CTA it % CL): its owner
+// TMA-loads the 128 x 256 bf16 tile of A into a staging buffer, quantizes it
+// with the streaming kernels' per-slice quantizer into its own operand stage
+// (codes in the swizzled layout, scales in the MMA tile layout), and pushes
+// the 16 KB code tile and 1 KB scale tile into every other CTA's stage with
+// shared-to-shared bulk copies that complete on that CTA's mbarrier. Every
+// CTA's MMA commit arrives on the "empty" barrier of every CTA, so no stage is
+// refilled (locally or by a push) before all CTAs are done with it. Each CTA
+// thus quantizes 1/CL of A's tiles, and the quantized A stays on chip.
+template <int BN, int S, int CL, int RULE>
+__global__ void __launch_bounds__(GemmCfg<BN, S, true>::kThreads, 1)
+    gemm_fused_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmB,
+                      const GemmArgs g) {
+  using C = GemmCfg<BN, S, true>;
+  extern __shared__ uint8_t smem_raw[];
+  const Smem<BN, S, true> sm(smem_raw);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const uint32_t rank = CL > 1 ? tc::cluster_rank() : 0;
+  const int64_t cluster = blockIdx.x / CL;
+  const int64_t nclusters = gridDim.x / CL;
+  const int nk = static_cast<int>(g.K / kGemmBK);
+  const int64_t T = g.K / 128;   // scale tiles per 128-row band
+  const int64_t tiles_n = (g.N + BN - 1) / BN;
+  const int64_t groups_n = (tiles_n + CL - 1) / CL;
+  const int64_t units = ((g.M + kGemmBM - 1) / kGemmBM) * groups_n;
+  // ring position `it` -> (unit, K-block); this CTA's units are cluster,
+  // cluster + nclusters, ...
+  auto unit_of = [&](int64_t it) { return cluster + (it / nk) * nclusters; };
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < S; ++s) {
+      tc::mbar_init(sm.fullB(s), 1);
+      tc::mbar_init(sm.fullA(s), 1);
+      tc::mbar_init(sm.empty(s), CL);
+      tc::mbar_init(sm.qfree(s), 1);
+    }
+    tc::mbar_init(sm.tfull(), 1);
+    tc::mbar_init(sm.tempty(), C::kWorkWarps);
+    tc::mbar_init(sm.stg_full(), 1);
+    *sm.abort_flag = 0;
+    tc::fence_mbar_init();
+  }
+  if (warp == 1) tc::tmem_alloc(tc::smem_addr(sm.tmem_holder), C::kTmemCols);
+  tc::tc_fence_before();
+  __syncthreads();
+  tc::tc_fence_after();
+  if (CL > 1) tc::cluster_sync();   // peers' barriers exist before any push
+  const uint32_t tmem = *sm.tmem_holder;
+
+  if (warp == 0) {
+    // ---------------------------------------------------------- producer
+    if (lane == 0) {
+      tc::prefetch_tmap(&tmB);
+      const int64_t bands_total = (g.N + 127) / 128;
+      int64_t it = 0;
+      bool ok = true;
+      for (int64_t u = cluster; ok && u < units; u += nclusters) {
+        const int64_t n0 = ((u % groups_n) * CL + rank) * BN;   // may lie past N: zero B
+        const int64_t nb0 = n0 / 128;
+        const int64_t left = bands_total - nb0;
+        const int nbands = static_cast<int>(left <= 0 ? 0 : (left < BN / 128 ? left : BN / 128));
+        const uint32_t tx = C::kTileB + nbands * 2 * kSfTile;
+        for (int kb = 0; kb < nk; ++kb, ++it) {
+          const int s = static_cast<int>(it % S);
+          const uint32_t ph = static_cast<uint32_t>(it / S) & 1;
+          if (!tc::mbar_wait(sm.empty(s), ph ^ 1, sm.abort_flag, g.status, kStatusProducer)) {
+            ok = false;
+            break;
           }
+          tc::mbar_arrive_expect_tx(sm.fullB(s), tx);
+          tc::tma_load_2d(sm.sB + s * C::kTileB, &tmB, kb * static_cast<int>(kRowBytes),
+                          static_cast<int>(n0), sm.fullB(s));
+          for (int band = 0; band < nbands; ++band)
+            tc::bulk_load(sm.sSFB + s * C::kSfB + band * 2 * kSfTile,
+                          g.b_scales + ((nb0 + band) * T + 2 * kb) * kSfTile, 2 * kSfTile,
+                          sm.fullB(s));
+          // a K-block another CTA quantizes arrives by its push; for one of
+          // this CTA's own, the stage is handed to the quantizer. (The
+          // quantizer visits only its own K-blocks, so it cannot wait on the
+          // "empty" barrier itself: an mbarrier answers only for the parity
+          // of its last phase, and the quantizer may be several phases
+          // away. This thread waits on every phase in order.)
+          if (it % CL != rank)
+            tc::mbar_arrive_expect_tx(sm.fullA(s), kTileA + 2 * kSfTile);
+          else
+            tc::mbar_arrive(sm.qfree(s));
         }
-      };
-      if (nk > 0) load(0, v);
-      for (int kb = 0; kb < nk; ++kb) {
-        const int s = kb % S;
-        const uint32_t ph = (kb / S) & 1;
-        if (kb + 1 < nk) load(kb + 1, nv);
-        // every lane waits (acquire), and the warp leaves together: the
-        // quantizer below uses warp collectives
-        const bool ok = tc::mbar_wait(empty(s), ph ^ 1, abort_flag, g.status, kStatusQuant);
-        if (!__all_sync(kFull, ok)) break;
-#pragma unroll
+      }
+      for (int64_t j = (it > S ? it - S : 0); j < it; ++j) {
+        const int s = static_cast<int>(j % S);
+        const uint32_t ph = static_cast<uint32_t>(j / S) & 1;
+        // this thread's copies have landed, and every CTA's MMA is done with
+        // the last stages: no push into this CTA's memory, and none out of
+        // it, is still in flight when the CTA exits
+        tc::mbar_wait(sm.fullB(s), ph, sm.abort_flag, g.status, kStatusDrain, false);
+        tc::mbar_wait(sm.empty(s), ph, sm.abort_flag, g.status, kStatusDrain, false);
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int64_t it = 0;
+      uint32_t tile_par = 0;
+      bool ok = true;
+      for (int64_t u = cluster; ok && u < units; u += nclusters, tile_par ^= 1) {
+        ok = tc::mbar_wait(sm.tempty(), tile_par ^ 1, sm.abort_flag, g.status, kStatusMmaB);
+        if (ok) tc::tc_fence_after();
+        for (int kb = 0; ok && kb < nk; ++kb, ++it) {
+          const int s = static_cast<int>(it % S);
+          const uint32_t ph = static_cast<uint32_t>(it / S) & 1;
+          if (!tc::mbar_wait(sm.fullB(s), ph, sm.abort_flag, g.status, kStatusMmaB) ||
+              !tc::mbar_wait(sm.fullA(s), ph, sm.abort_flag, g.status, kStatusMmaA)) {
+            ok = false;
+            break;
+          }
+          tc::tc_fence_after();
+          issue_kblock(sm, tmem, s, kb == 0);
+          if (CL > 1)
+            tc::tc_commit_multicast(sm.empty(s), static_cast<uint16_t>((1u << CL) - 1));
+          else
+            tc::tc_commit(sm.empty(s));
+        }
+        tc::tc_commit(sm.tfull());
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------ quantizer (own K-blocks), epilogue
+    // warp ew owns rows 16 ew .. 16 ew + 15 of the tile; pass p (0..7) puts
+    // row 16 ew + 2p on lanes 0-15 and the next row on lanes 16-31; lane j16
+    // = lane & 15 takes elements 16 j16 .. 16 j16 + 15 of the K-block (a lane
+    // pair is one 32-element block)
+    const int ew = warp - 2;
+    const int j16 = lane & 15;
+    const int j = j16 >> 1;   // block column within the K-block, 0..7
+    const bool leader = (ew == 0 && lane == 0);
+    const int64_t total = static_cast<int64_t>(nk) *
+                          ((units - cluster + nclusters - 1) / nclusters);   // this CTA's ring length
+    // staging loads: issued by the leader for this CTA's K-blocks in ring order
+    auto stage_in = [&](int64_t it) {
+      const int64_t u = unit_of(it);
+      const int kb = static_cast<int>(it % nk);
+      tc::mbar_arrive_expect_tx(sm.stg_full(), C::kStaging);
+      tc::tma_load_2d(sm.sStg, &tmX, kb * kGemmBK, static_cast<int>((u / groups_n) * kGemmBM),
+                      sm.stg_full());
+    };
+    bool stg_pending = false;   // (leader) a staging load is in flight
+    if (leader && rank < total) {
+      tc::prefetch_tmap(&tmX);
+      stage_in(rank);
+      stg_pending = true;
+    }
+    int64_t it = 0;
+    uint32_t tile_par = 0, stg_par = 0;
+    uint32_t qpar = 0;   // bit s: parity of the next qfree phase of stage s
+    bool ok = true;
+    for (int64_t u = cluster; ok && u < units; u += nclusters, tile_par ^= 1) {
+      const int64_t m0 = (u / groups_n) * kGemmBM;
+      const int64_t n0 = ((u % groups_n) * CL + rank) * BN;
+      const bool write_a = (u % groups_n) == 0;   // the first n-group writes A's codes out
+      for (int kb = 0; kb < nk; ++kb, ++it) {
+        if (it % CL != rank) continue;
+        const int s = static_cast<int>(it % S);
+        // every thread waits (acquire); the eight warps then take one
+        // decision, since they meet at a named barrier below
+        const bool got_stg =
+            tc::mbar_wait(sm.stg_full(), stg_par, sm.abort_flag, g.status, kStatusStaging);
+        const bool got = got_stg && tc::mbar_wait(sm.qfree(s), (qpar >> s) & 1, sm.abort_flag,
+                                                  g.status, kStatusQuant);
+        if (got) qpar ^= 1u << s;
+        if (got_stg) {
+          stg_par ^= 1;
+          stg_pending = false;
+        }
+        if (!tc::named_all(2, C::kWorkWarps * 32, got)) {
+          ok = false;
+          break;
+        }
+#pragma unroll 2
         for (int p = 0; p < 8; ++p) {
-          const int r = 16 * qw + 2 * p + (lane >> 4);
-          const uint32_t pa = pair_max(amax_bits16(v[p]));
-          const BlockScale bs = decide_scale<kFmtE2M1, RULE, kMbsNone>(v[p], pa, 0);
-          const uint2 c = codes_fp4<kMbsNone>(v[p], bs);
-          const uint32_t dst = sA + s * kTileA + r * kRowBytes +
+          const int r = 16 * ew + 2 * p + (lane >> 4);
+          const uint32_t src = sm.sStg + r * (kGemmBK * 2) + j16 * 32;
+          V16 v;
+          asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                       : "=r"(v.w[0]), "=r"(v.w[1]), "=r"(v.w[2]), "=r"(v.w[3])
+                       : "r"(src));
+          asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                       : "=r"(v.w[4]), "=r"(v.w[5]), "=r"(v.w[6]), "=r"(v.w[7])
+                       : "r"(src + 16));
+          const uint32_t pa = pair_max(amax_bits16(v));
+          const BlockScale bs = decide_scale<kFmtE2M1, RULE, kMbsNone>(v, pa, 0);
+          const uint2 c = codes_fp4<kMbsNone>(v, bs);
+          const uint32_t dst = sm.sA + s * kTileA + r * kRowBytes +
                                ((((j16 >> 1) ^ (r & 7)) & 7) << 4) + ((j16 & 1) << 3);
           asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(dst), "r"(c.x), "r"(c.y) : "memory");
-          const int j = j16 >> 1;   // block column within the K-block, 0..7
-          if ((lane & 1) == 0) {
-            const uint32_t sdst = sSFA + s * C::kSfA + (j >> 2) * kSfTile + (r & 31) * 16 +
-                                  ((r >> 5) & 3) * 4 + (j & 3);
+          const uint32_t sdst = sm.sSFA + s * C::kSfA + (j >> 2) * kSfTile + (r & 31) * 16 +
+                                ((r >> 5) & 3) * 4 + (j & 3);
+          if ((lane & 1) == 0)
             asm volatile("st.shared.u8 [%0], %1;" ::"r"(sdst), "r"(bs.byte) : "memory");
-          }
           if (write_a) {
             const int64_t m = m0 + r;
             if (g.a_codes_out && m < g.M)
@@ -260,54 +541,29 @@ __global__ void __launch_bounds__(GemmCfg<BN, S, FUSED>::kThreads, 1)
           }
         }
         tc::fence_proxy_async_smem();
-        __syncwarp();
-        if (lane == 0) tc::mbar_arrive(fullA(s));
-        if (kb + 1 < nk) {
-#pragma unroll
-          for (int p = 0; p < 8; ++p) v[p] = nv[p];
-        }
-      }
-    }
-    // ------------------------------------------------------------ epilogue
-    // warp w reads TMEM lanes 32 (w % 4) .. + 31 (its quarter); with eight
-    // warps the two sets of four split the columns
-    constexpr int kGroups = C::kQuantWarps / 4;
-    const int q = warp & 3;
-    const int grp = qw / 4;
-    const bool got = tc::mbar_wait(tfull, 0, abort_flag, g.status, kStatusEpilogue, false);
-    tc::tc_fence_after();
-    // warp-uniform: tcgen05.ld is a whole-warp instruction
-    const bool done = __all_sync(kFull, got && !*abort_flag);
-    if (done) {
-      const int row = q * 32 + lane;
-      const int64_t m = m0 + row;
-      for (int c0 = grp * (BN / kGroups); c0 < (grp + 1) * (BN / kGroups); c0 += 32) {
-        uint32_t r[32];
-        tc::tmem_ld32(tmem + (static_cast<uint32_t>(q * 32) << 16) + c0, r);
-        if (m < g.M) {
-#pragma unroll
-          for (int gq = 0; gq < 4; ++gq) {
-            const int64_t n = n0 + c0 + 8 * gq;
-            if (n < g.N) {
-              if (g.out_fp32) {
-                uint4* o = reinterpret_cast<uint4*>(g.d + (m * g.N + n) * 4);
-                o[0] = make_uint4(r[8 * gq], r[8 * gq + 1], r[8 * gq + 2], r[8 * gq + 3]);
-                o[1] = make_uint4(r[8 * gq + 4], r[8 * gq + 5], r[8 * gq + 6], r[8 * gq + 7]);
-              } else {
-                uint32_t h[4];
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                  const __nv_bfloat162 b2 = __floats2bfloat162_rn(
-                      __uint_as_float(r[8 * gq + 2 * i]), __uint_as_float(r[8 * gq + 2 * i + 1]));
-                  h[i] = *reinterpret_cast<const uint32_t*>(&b2);
-                }
-                *reinterpret_cast<uint4*>(g.d + (m * g.N + n) * 2) = make_uint4(h[0], h[1], h[2], h[3]);
-              }
-            }
+        tc::named_sync(1, C::kWorkWarps * 32);   // the stage is written, the staging tile read
+        if (leader) {
+          if (it + CL < total) {
+            stage_in(it + CL);
+            stg_pending = true;
           }
+#pragma unroll
+          for (uint32_t p = 1; p < CL; ++p) {
+            const uint32_t peer = (rank + p) % CL;
+            const uint32_t bar = tc::mapa(sm.fullA(s), peer);
+            tc::bulk_push(tc::mapa(sm.sA + s * kTileA, peer), sm.sA + s * kTileA, kTileA, bar);
+            tc::bulk_push(tc::mapa(sm.sSFA + s * C::kSfA, peer), sm.sSFA + s * C::kSfA,
+                          2 * kSfTile, bar);
+          }
+          tc::mbar_arrive(sm.fullA(s));
         }
       }
+      if (!ok) break;
+      if (!epilogue_tile(sm, g, tmem, tile_par, m0, n0, warp, lane)) break;
     }
+    // a staging load issued but never consumed (abort) lands before the exit
+    if (leader && stg_pending)
+      tc::mbar_wait(sm.stg_full(), stg_par, sm.abort_flag, g.status, kStatusDrain, false);
     tc::tc_fence_before();
   }
   __syncthreads();
@@ -315,6 +571,7 @@ __global__ void __launch_bounds__(GemmCfg<BN, S, FUSED>::kThreads, 1)
     tc::tc_fence_after();
     tc::tmem_dealloc(tmem, C::kTmemCols);
   }
+  if (CL > 1) tc::cluster_sync();   // no CTA leaves while a peer may still address it
 }
 
 // ------------------------------------------------------------- host side --
@@ -353,25 +610,98 @@ bool code_tmap(CUtensorMap* tm, const void* codes, int64_t rows, int64_t K, int 
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-template <int BN, int S, bool FUSED, int RULE>
-cudaError_t launch_gemm_cfg(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& g,
+// Tensor map of bf16 A [M, K] read in 256-element x 128-row boxes, row-major
+// in shared memory without swizzle (rows past M read as zero).
+bool bf16_tmap(CUtensorMap* tm, const void* a, int64_t M, int64_t K) {
+  EncodeTiledFn enc = tensor_map_encoder();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {static_cast<cuuint64_t>(K), static_cast<cuuint64_t>(M)};
+  const cuuint64_t strides[1] = {static_cast<cuuint64_t>(K * 2)};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(kGemmBK), static_cast<cuuint32_t>(kGemmBM)};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(tm, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(a), dims, strides, box,
+             estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+int sm_count_of_current_device(cudaError_t* e) {
+  int dev = 0, sms = 0;
+  *e = cudaGetDevice(&dev);
+  if (*e == cudaSuccess) *e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  return sms;
+}
+
+template <int BN, int S>
+cudaError_t launch_prequant(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& g,
                             cudaStream_t st) {
-  using C = GemmCfg<BN, S, FUSED>;
-  auto kern = gemm_kernel<BN, S, FUSED, RULE>;
+  using C = GemmCfg<BN, S, false>;
+  auto kern = gemm_kernel<BN, S>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(C::kSmem));
   if (e != cudaSuccess) return e;
-  const dim3 grid(static_cast<unsigned>((g.N + BN - 1) / BN),
-                  static_cast<unsigned>((g.M + kGemmBM - 1) / kGemmBM));
+  // persistent: one CTA per SM (the shared memory allows no second), never
+  // more CTAs than tiles
+  const int64_t tiles = ((g.M + kGemmBM - 1) / kGemmBM) * ((g.N + BN - 1) / BN);
+  const int sms = sm_count_of_current_device(&e);
+  if (e != cudaSuccess) return e;
+  const unsigned grid = static_cast<unsigned>(tiles < sms ? tiles : sms);
   kern<<<grid, C::kThreads, C::kSmem, st>>>(tmA, tmB, g);
   return cudaGetLastError();
 }
 
-template <bool FUSED, int RULE>
-cudaError_t launch_gemm_bn(bool wide, const CUtensorMap& tmA, const CUtensorMap& tmB,
-                           const GemmArgs& g, cudaStream_t st) {
-  if (wide) return launch_gemm_cfg<256, 4, FUSED, RULE>(tmA, tmB, g, st);
-  return launch_gemm_cfg<128, 6, FUSED, RULE>(tmA, tmB, g, st);
+template <int BN, int S, int CL, int RULE>
+cudaError_t launch_fused(const CUtensorMap& tmX, const CUtensorMap& tmB, const GemmArgs& g,
+                         cudaStream_t st) {
+  using C = GemmCfg<BN, S, true>;
+  auto kern = gemm_fused_kernel<BN, S, CL, RULE>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(C::kSmem));
+  if (e != cudaSuccess) return e;
+  const int64_t tiles_n = (g.N + BN - 1) / BN;
+  const int64_t units = ((g.M + kGemmBM - 1) / kGemmBM) * ((tiles_n + CL - 1) / CL);
+  const int sms = sm_count_of_current_device(&e);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = CL;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.blockDim = dim3(C::kThreads);
+  cfg.dynamicSmemBytes = C::kSmem;
+  cfg.stream = st;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  // persistent clusters: as many as can be resident at once, never more than
+  // there are units
+  cfg.gridDim = dim3(static_cast<unsigned>((sms / CL) * CL));
+  int max_clusters = 0;
+  e = cudaOccupancyMaxActiveClusters(&max_clusters, kern, &cfg);
+  if (e != cudaSuccess) return e;
+  if (max_clusters < 1) return cudaErrorInvalidConfiguration;
+  const int64_t nclusters = units < max_clusters ? units : max_clusters;
+  cfg.gridDim = dim3(static_cast<unsigned>(nclusters * CL));
+  e = cudaLaunchKernelEx(&cfg, kern, tmX, tmB, g);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+// The cluster width of the fused kernel: up to 4 CTAs share each A tile, no
+// wider than the row of N tiles.
+template <int BN, int S, int RULE>
+cudaError_t launch_fused_cl(const CUtensorMap& tmX, const CUtensorMap& tmB, const GemmArgs& g,
+                            cudaStream_t st) {
+  const int64_t tiles_n = (g.N + BN - 1) / BN;
+  if (tiles_n >= 4) return launch_fused<BN, S, 4, RULE>(tmX, tmB, g, st);
+  if (tiles_n >= 2) return launch_fused<BN, S, 2, RULE>(tmX, tmB, g, st);
+  return launch_fused<BN, S, 1, RULE>(tmX, tmB, g, st);
+}
+
+template <int RULE>
+cudaError_t launch_fused_bn(bool wide, const CUtensorMap& tmX, const CUtensorMap& tmB,
+                            const GemmArgs& g, cudaStream_t st) {
+  if (wide) return launch_fused_cl<256, 3, RULE>(tmX, tmB, g, st);
+  return launch_fused_cl<128, 4, RULE>(tmX, tmB, g, st);
 }
 
 }  // namespace
@@ -385,7 +715,6 @@ cudaError_t launch_gemm(const void* a, const uint8_t* a_scales, int a_rule, cons
   const bool wide = N > 128 && ((M + kGemmBM - 1) / kGemmBM) * ((N + 255) / 256) >= 148;
   CUtensorMap tmA{}, tmB{};
   if (!code_tmap(&tmB, b_codes, N, K, wide ? 256 : 128)) return cudaErrorInvalidValue;
-  if (!fused && !code_tmap(&tmA, a, M, K, kGemmBM)) return cudaErrorInvalidValue;
   GemmArgs g{};
   g.a_bf16 = fused ? static_cast<const uint8_t*>(a) : nullptr;
   g.a_scales = a_scales;
@@ -398,12 +727,16 @@ cudaError_t launch_gemm(const void* a, const uint8_t* a_scales, int a_rule, cons
   g.N = N;
   g.K = K;
   g.out_fp32 = out_fp32;
-  if (!fused) return launch_gemm_bn<false, kFloor>(wide, tmA, tmB, g, st);
+  if (!fused) {
+    if (!code_tmap(&tmA, a, M, K, kGemmBM)) return cudaErrorInvalidValue;
+    return wide ? launch_prequant<256, 4>(tmA, tmB, g, st) : launch_prequant<128, 6>(tmA, tmB, g, st);
+  }
+  if (!bf16_tmap(&tmA, a, M, K)) return cudaErrorInvalidValue;
   switch (a_rule) {
-    case kCeil: return launch_gemm_bn<true, kCeil>(wide, tmA, tmB, g, st);
-    case kOasRule: return launch_gemm_bn<true, kOasRule>(wide, tmA, tmB, g, st);
-    case kOas: return launch_gemm_bn<true, kOas>(wide, tmA, tmB, g, st);
-    default: return launch_gemm_bn<true, kFloor>(wide, tmA, tmB, g, st);
+    case kCeil: return launch_fused_bn<kCeil>(wide, tmA, tmB, g, st);
+    case kOasRule: return launch_fused_bn<kOasRule>(wide, tmA, tmB, g, st);
+    case kOas: return launch_fused_bn<kOas>(wide, tmA, tmB, g, st);
+    default: return launch_fused_bn<kFloor>(wide, tmA, tmB, g, st);
   }
 }
 

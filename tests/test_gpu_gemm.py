@@ -34,9 +34,11 @@ MMA = 1 << 8
 RULES = [FLOOR, CEIL, OAS_RULE, OAS]
 GRID = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
 # (M, N, K): one tile; ragged M and N; a single row; several K-blocks and
-# 128-wide N tiles; the MoE w13 expert shape (N = 2I = 1536, K = H = 2048)
+# 128-wide N tiles; the MoE w13 expert shape (N = 2I = 1536, K = H = 2048);
+# more tiles than SMs, so that persistent CTAs take several tiles (256-wide,
+# one with a last N tile 8 columns wide)
 SHAPES = [(128, 128, 256), (200, 264, 512), (1, 8, 256), (300, 520, 1024), (16, 1536, 2048),
-          (260, 400, 768)]
+          (260, 400, 768), (1536, 4096, 512), (2200, 2056, 256)]
 
 
 def bits(t):
@@ -101,6 +103,40 @@ def test_integer_cases_are_exact(mx, cuda, shape, fused):
     assert np.array_equal(host(outs[torch.float32]).astype(np.float64), exact)
     want = torch.from_numpy(exact.astype(np.float32)).to(torch.bfloat16)
     assert np.array_equal(bits(outs[torch.bfloat16]), bits(want))
+
+
+# Long persistent runs: ~256 units over the clusters, each unit 12 K-blocks,
+# so every stage of the ring is refilled by changing owners many times over.
+BIG = [(4096, 8192, 3072)]
+
+
+@pytest.mark.parametrize("shape", BIG, ids=lambda s: "x".join(map(str, s)))
+def test_integer_cases_are_exact_many_units(mx, cuda, shape):
+    M, N, K = shape
+    av, a = grid_matrix(M, K, seed=5)
+    bv, b = grid_matrix(N, K, seed=6)
+    exact = av @ bv.T
+    bc, bs = weights(mx, b, cuda)
+    status = torch.zeros(1, dtype=torch.int32, device=cuda)
+    d = mx.quant_gemm(a.to(cuda), bc, bs, FLOOR, out_dtype=torch.float32, status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    assert np.array_equal(host(d).astype(np.float64), exact)
+
+
+@pytest.mark.parametrize("rule", [FLOOR, OAS], ids=["FLOOR", "OAS"])
+@pytest.mark.parametrize("shape", BIG, ids=lambda s: "x".join(map(str, s)))
+def test_fused_equals_quantize_then_gemm_many_units(mx, cuda, shape, rule):
+    M, N, K = shape
+    a = inputs.heavy_tail(M, K, seed=rule + 9).to(cuda)
+    bc, bs = weights(mx, inputs.normal_weight(N, K, seed=11), cuda)
+    status = torch.zeros(1, dtype=torch.int32, device=cuda)
+    d_fused = mx.quant_gemm(a, bc, bs, rule, out_dtype=torch.float32, status=status)
+    ac, as_, _ = mx.quantize(a, E2M1, rule | MMA)
+    d_two = mx.gemm(ac, as_, bc, bs, out_dtype=torch.float32, status=status)
+    torch.cuda.synchronize()
+    assert status.item() == 0
+    assert torch.equal(d_fused.view(torch.int32), d_two.view(torch.int32))
 
 
 @pytest.mark.parametrize("rule", RULES, ids=["FLOOR", "CEIL", "OAS_RULE", "OAS"])
