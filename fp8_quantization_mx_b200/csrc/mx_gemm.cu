@@ -150,9 +150,9 @@ __device__ __forceinline__ void issue_kblock(const Smem<BN, S, FUSED>& sm, uint3
 
 // Epilogue of one tile by the eight work warps: warp w reads TMEM lanes
 // 32 (w % 4) .. + 31 (its quarter), warps 2-5 the first half of the columns
-// and warps 6-9 the second; the values go to registers, the accumulator is
-// released (tmem_empty), then fp32 -> bf16 (or fp32) -> global. Returns
-// false when the kernel is aborting.
+// and warps 6-9 the second. bf16 out: the values are rounded into registers,
+// the accumulator released (tmem_empty), then stored; float out: stored from
+// each load, then released. Returns false when the kernel is aborting.
 template <int BN, int S, bool FUSED>
 __device__ __forceinline__ bool epilogue_tile(const Smem<BN, S, FUSED>& sm, const GemmArgs& g,
                                               uint32_t tmem, uint32_t tile_par, int64_t m0,
@@ -168,13 +168,43 @@ __device__ __forceinline__ bool epilogue_tile(const Smem<BN, S, FUSED>& sm, cons
     return false;
   const int64_t m = m0 + q * 32 + lane;
   constexpr int kCols = BN / 2;
-  uint32_t acc[kCols];
+  const uint32_t taddr = tmem + (static_cast<uint32_t>(q * 32) << 16) + c_begin;
+  if (g.out_fp32) {
+    // float out: straight from each TMEM load to global, then the release
+#pragma unroll 1
+    for (int c0 = 0; c0 < kCols; c0 += 32) {
+      uint32_t r[32];
+      tc::tmem_ld32(taddr + c0, r);
+      if (m < g.M) {
+#pragma unroll
+        for (int gq = 0; gq < 4; ++gq) {
+          const int64_t n = n0 + c_begin + c0 + 8 * gq;
+          if (n < g.N) {
+            uint4* o = reinterpret_cast<uint4*>(g.d + (m * g.N + n) * 4);
+            o[0] = make_uint4(r[8 * gq], r[8 * gq + 1], r[8 * gq + 2], r[8 * gq + 3]);
+            o[1] = make_uint4(r[8 * gq + 4], r[8 * gq + 5], r[8 * gq + 6], r[8 * gq + 7]);
+          }
+        }
+      }
+    }
+    tc::tc_fence_before();
+    __syncwarp();
+    if (lane == 0) tc::mbar_arrive(sm.tempty());
+    return true;
+  }
+  // bf16 out: the whole row share as packed bf16 pairs in registers, the
+  // accumulator released, then the stores
+  uint32_t h[kCols / 2];
 #pragma unroll
   for (int c0 = 0; c0 < kCols; c0 += 32) {
     uint32_t r[32];
-    tc::tmem_ld32(tmem + (static_cast<uint32_t>(q * 32) << 16) + c_begin + c0, r);
+    tc::tmem_ld32(taddr + c0, r);
 #pragma unroll
-    for (int i = 0; i < 32; ++i) acc[c0 + i] = r[i];
+    for (int i = 0; i < 16; ++i) {
+      const __nv_bfloat162 b2 =
+          __floats2bfloat162_rn(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
+      h[c0 / 2 + i] = *reinterpret_cast<const uint32_t*>(&b2);
+    }
   }
   tc::tc_fence_before();
   __syncwarp();
@@ -183,22 +213,9 @@ __device__ __forceinline__ bool epilogue_tile(const Smem<BN, S, FUSED>& sm, cons
 #pragma unroll
     for (int gq = 0; gq < kCols / 8; ++gq) {
       const int64_t n = n0 + c_begin + 8 * gq;
-      if (n < g.N) {
-        if (g.out_fp32) {
-          uint4* o = reinterpret_cast<uint4*>(g.d + (m * g.N + n) * 4);
-          o[0] = make_uint4(acc[8 * gq], acc[8 * gq + 1], acc[8 * gq + 2], acc[8 * gq + 3]);
-          o[1] = make_uint4(acc[8 * gq + 4], acc[8 * gq + 5], acc[8 * gq + 6], acc[8 * gq + 7]);
-        } else {
-          uint32_t h[4];
-#pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            const __nv_bfloat162 b2 = __floats2bfloat162_rn(
-                __uint_as_float(acc[8 * gq + 2 * i]), __uint_as_float(acc[8 * gq + 2 * i + 1]));
-            h[i] = *reinterpret_cast<const uint32_t*>(&b2);
-          }
-          *reinterpret_cast<uint4*>(g.d + (m * g.N + n) * 2) = make_uint4(h[0], h[1], h[2], h[3]);
-        }
-      }
+      if (n < g.N)
+        *reinterpret_cast<uint4*>(g.d + (m * g.N + n) * 2) =
+            make_uint4(h[4 * gq], h[4 * gq + 1], h[4 * gq + 2], h[4 * gq + 3]);
     }
   }
   return true;
@@ -460,10 +477,8 @@ __global__ void __launch_bounds__(GemmCfg<BN, S, true>::kThreads, 1)
     __syncwarp();
   } else {
     // ------------------------------------ quantizer (own K-blocks), epilogue
-    // warp ew owns rows 16 ew .. 16 ew + 15 of the tile; pass p (0..7) puts
-    // row 16 ew + 2p on lanes 0-15 and the next row on lanes 16-31; lane j16
-    // = lane & 15 takes elements 16 j16 .. 16 j16 + 15 of the K-block (a lane
-    // pair is one 32-element block)
+    // lane j16 = lane & 15 takes elements 16 j16 .. 16 j16 + 15 of the
+    // K-block (a lane pair is one 32-element block); the rows are below
     const int ew = warp - 2;
     const int j16 = lane & 15;
     const int j = j16 >> 1;   // block column within the K-block, 0..7
@@ -510,34 +525,68 @@ __global__ void __launch_bounds__(GemmCfg<BN, S, true>::kThreads, 1)
           ok = false;
           break;
         }
-#pragma unroll 2
-        for (int p = 0; p < 8; ++p) {
-          const int r = 16 * ew + 2 * p + (lane >> 4);
-          const uint32_t src = sm.sStg + r * (kGemmBK * 2) + j16 * 32;
-          V16 v;
-          asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-                       : "=r"(v.w[0]), "=r"(v.w[1]), "=r"(v.w[2]), "=r"(v.w[3])
-                       : "r"(src));
-          asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
-                       : "=r"(v.w[4]), "=r"(v.w[5]), "=r"(v.w[6]), "=r"(v.w[7])
-                       : "r"(src + 16));
-          const uint32_t pa = pair_max(amax_bits16(v));
-          const BlockScale bs = decide_scale<kFmtE2M1, RULE, kMbsNone>(v, pa, 0);
-          const uint2 c = codes_fp4<kMbsNone>(v, bs);
-          const uint32_t dst = sm.sA + s * kTileA + r * kRowBytes +
-                               ((((j16 >> 1) ^ (r & 7)) & 7) << 4) + ((j16 & 1) << 3);
-          asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(dst), "r"(c.x), "r"(c.y) : "memory");
-          const uint32_t sdst = sm.sSFA + s * C::kSfA + (j >> 2) * kSfTile + (r & 31) * 16 +
-                                ((r >> 5) & 3) * 4 + (j & 3);
-          if ((lane & 1) == 0)
-            asm volatile("st.shared.u8 [%0], %1;" ::"r"(sdst), "r"(bs.byte) : "memory");
-          if (write_a) {
-            const int64_t m = m0 + r;
-            if (g.a_codes_out && m < g.M)
-              st_stream8(g.a_codes_out + m * (g.K / 2) + static_cast<int64_t>(kb) * kRowBytes + 8 * j16, c);
-            if (g.a_scales_out && (lane & 1) == 0)
-              g.a_scales_out[((m0 / 128) * T + 2 * kb + (j >> 2)) * kSfTile + (r & 31) * 16 +
-                             ((r >> 5) & 3) * 4 + (j & 3)] = static_cast<uint8_t>(bs.byte);
+        // pass p: rows 16 p + 2 ew (lanes 0-15) and 16 p + 2 ew + 1 (lanes
+        // 16-31); passes wholly past M are skipped (their rows of D are never
+        // stored, so what the stage holds there does not matter)
+        const int64_t valid = g.M - m0;
+        const int npass = valid >= 128 ? 8 : static_cast<int>((valid + 15) / 16);
+        // the warp's slices are read four at a time before any is
+        // processed, so that four independent blocks' dependency chains
+        // interleave; a lane reads the two 16-byte halves of its 32 bytes in
+        // an order that spreads each quarter-warp over all 32 banks
+        const uint32_t hsw = ((lane >> 2) & 1) * 16;
+#pragma unroll
+        for (int p0 = 0; p0 < 8; p0 += 4) {
+          V16 v[4];
+#pragma unroll
+          for (int i4 = 0; i4 < 4; ++i4) {
+            const int p = p0 + i4;
+            if (p < npass) {
+              const int r = 16 * p + 2 * ew + (lane >> 4);
+              const uint32_t src = sm.sStg + r * (kGemmBK * 2) + j16 * 32;
+              uint32_t a[4], b[4];
+              asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                           : "=r"(a[0]), "=r"(a[1]), "=r"(a[2]), "=r"(a[3])
+                           : "r"(src + hsw));
+              asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                           : "=r"(b[0]), "=r"(b[1]), "=r"(b[2]), "=r"(b[3])
+                           : "r"(src + (hsw ^ 16)));
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                v[i4].w[i] = hsw ? b[i] : a[i];
+                v[i4].w[4 + i] = hsw ? a[i] : b[i];
+              }
+            }
+          }
+#pragma unroll
+          for (int i4 = 0; i4 < 4; ++i4) {
+            const int p = p0 + i4;
+            const int r = 16 * p + 2 * ew + (lane >> 4);
+            if (p >= npass) {
+              // the tiled scale buffer's padding rows hold zeros
+              if (write_a && g.a_scales_out && (lane & 1) == 0)
+                g.a_scales_out[((m0 / 128) * T + 2 * kb + (j >> 2)) * kSfTile + (r & 31) * 16 +
+                               ((r >> 5) & 3) * 4 + (j & 3)] = 0;
+              continue;
+            }
+            const uint32_t pa = pair_max(amax_bits16(v[i4]));
+            const BlockScale bs = decide_scale<kFmtE2M1, RULE, kMbsNone>(v[i4], pa, 0);
+            const uint2 c = codes_fp4<kMbsNone>(v[i4], bs);
+            const uint32_t dst = sm.sA + s * kTileA + r * kRowBytes +
+                                 ((((j16 >> 1) ^ (r & 7)) & 7) << 4) + ((j16 & 1) << 3);
+            asm volatile("st.shared.v2.u32 [%0], {%1, %2};" ::"r"(dst), "r"(c.x), "r"(c.y) : "memory");
+            const uint32_t sdst = sm.sSFA + s * C::kSfA + (j >> 2) * kSfTile + (r & 31) * 16 +
+                                  ((r >> 5) & 3) * 4 + (j & 3);
+            if ((lane & 1) == 0)
+              asm volatile("st.shared.u8 [%0], %1;" ::"r"(sdst), "r"(bs.byte) : "memory");
+            if (write_a) {
+              const int64_t m = m0 + r;
+              if (g.a_codes_out && m < g.M)
+                st_stream8(g.a_codes_out + m * (g.K / 2) + static_cast<int64_t>(kb) * kRowBytes + 8 * j16, c);
+              if (g.a_scales_out && (lane & 1) == 0)
+                g.a_scales_out[((m0 / 128) * T + 2 * kb + (j >> 2)) * kSfTile + (r & 31) * 16 +
+                               ((r >> 5) & 3) * 4 + (j & 3)] = static_cast<uint8_t>(bs.byte);
+            }
           }
         }
         tc::fence_proxy_async_smem();
