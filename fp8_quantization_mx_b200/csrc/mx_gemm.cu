@@ -735,14 +735,18 @@ cudaError_t launch_fused(const CUtensorMap& tmX, const CUtensorMap& tmB, const G
   return cudaGetLastError();
 }
 
-// The cluster width of the fused kernel: up to 4 CTAs share each A tile, no
-// wider than the row of N tiles.
+// The cluster width of the fused kernel: up to MX_GEMM_MAX_CLUSTER (a
+// build-time knob, default 4) CTAs share each A tile, no wider than the row
+// of N tiles.
+#ifndef MX_GEMM_MAX_CLUSTER
+#define MX_GEMM_MAX_CLUSTER 4
+#endif
 template <int BN, int S, int RULE>
 cudaError_t launch_fused_cl(const CUtensorMap& tmX, const CUtensorMap& tmB, const GemmArgs& g,
                             cudaStream_t st) {
   const int64_t tiles_n = (g.N + BN - 1) / BN;
-  if (tiles_n >= 4) return launch_fused<BN, S, 4, RULE>(tmX, tmB, g, st);
-  if (tiles_n >= 2) return launch_fused<BN, S, 2, RULE>(tmX, tmB, g, st);
+  if (MX_GEMM_MAX_CLUSTER >= 4 && tiles_n >= 4) return launch_fused<BN, S, 4, RULE>(tmX, tmB, g, st);
+  if (MX_GEMM_MAX_CLUSTER >= 2 && tiles_n >= 2) return launch_fused<BN, S, 2, RULE>(tmX, tmB, g, st);
   return launch_fused<BN, S, 1, RULE>(tmX, tmB, g, st);
 }
 
