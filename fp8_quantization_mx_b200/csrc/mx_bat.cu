@@ -130,6 +130,9 @@ struct LaneParams {
   float bmin, bmax;
 };
 
+template <int AD>
+__device__ __forceinline__ V16 bat_finish(float (&y)[16], const LaneParams<AD>& L, bool clip);
+
 // The transformed, clipped 16 values of this lane (elements 16 h .. 16 h + 15
 // of its block) as packed bf16.
 template <int AD>
@@ -303,6 +306,85 @@ __device__ __forceinline__ V16 bat_slice(const V16& v, int h, const LaneParams<A
     }
   }
 
+  return bat_finish<AD>(y, L, clip);
+}
+
+// a = 2 (b = 16) for two rows u, w of the same column chunk (so the same B_j)
+// at once: the transform of bat_slice, each 16-byte load of B_j's rows
+// serving both rows, every output's fma chain in the same order (so the
+// results are bat_slice's bit for bit). Stage 2 runs in two passes, this
+// lane's own outputs and then the partner's, to bound the live registers.
+__device__ __forceinline__ void bat_transform2_a2(const V16& vu, const V16& vw, int h,
+                                                  const LaneParams<2>& L, float (&yu)[16],
+                                                  float (&yw)[16]) {
+  constexpr int RH = LaneParams<2>::RH;   // 8
+  float2 zu[8], zw[8];
+#pragma unroll
+  for (int pp = 0; pp < RH; ++pp) {
+    float2 au = make_float2(-0.0f, -0.0f), aw = make_float2(-0.0f, -0.0f);
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+      const float2 aq = make_float2(L.A[q * 2], L.A[q * 2 + 1]);
+      const float xu = elem(vu, pp * 2 + q), xw = elem(vw, pp * 2 + q);
+      au = ffma2(make_float2(xu, xu), aq, au);
+      aw = ffma2(make_float2(xw, xw), aq, aw);
+    }
+    zu[pp] = au;
+    zw[pp] = aw;
+  }
+  // pass 1: own outputs (rows h RH .. of Y), pass 2: the partner's
+  float2 ou[2][4], ow[2][4];   // [s][row pair]
+#pragma unroll
+  for (int pass = 0; pass < 2; ++pass) {
+    float2 cu[2][4], cw[2][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) cu[0][i] = cu[1][i] = cw[0][i] = cw[1][i] = make_float2(-0.0f, -0.0f);
+    const float* Bc = L.Bl + (pass == 0 ? h : 1 - h) * RH;
+#pragma unroll
+    for (int pp = 0; pp < RH; ++pp) {
+      const float2 u0 = make_float2(zu[pp].x, zu[pp].x), u1 = make_float2(zu[pp].y, zu[pp].y);
+      const float2 w0 = make_float2(zw[pp].x, zw[pp].x), w1 = make_float2(zw[pp].y, zw[pp].y);
+#pragma unroll
+      for (int q4 = 0; q4 < RH / 4; ++q4) {
+        const float4 b = reinterpret_cast<const float4*>(Bc + pp * BatSmemB<2>::pitch)[q4];
+        const float2 b01 = make_float2(b.x, b.y), b23 = make_float2(b.z, b.w);
+        cu[0][2 * q4] = ffma2(b01, u0, cu[0][2 * q4]);
+        cu[0][2 * q4 + 1] = ffma2(b23, u0, cu[0][2 * q4 + 1]);
+        cu[1][2 * q4] = ffma2(b01, u1, cu[1][2 * q4]);
+        cu[1][2 * q4 + 1] = ffma2(b23, u1, cu[1][2 * q4 + 1]);
+        cw[0][2 * q4] = ffma2(b01, w0, cw[0][2 * q4]);
+        cw[0][2 * q4 + 1] = ffma2(b23, w0, cw[0][2 * q4 + 1]);
+        cw[1][2 * q4] = ffma2(b01, w1, cw[1][2 * q4]);
+        cw[1][2 * q4 + 1] = ffma2(b23, w1, cw[1][2 * q4 + 1]);
+      }
+    }
+    if (pass == 0) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        ou[0][i] = cu[0][i];
+        ou[1][i] = cu[1][i];
+        ow[0][i] = cw[0][i];
+        ow[1][i] = cw[1][i];
+      }
+    } else {
+      // element r * 2 + s of this lane's half: own chain + the partner's
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+#pragma unroll
+        for (int sc = 0; sc < 2; ++sc) {
+          yu[(2 * j) * 2 + sc] = __fadd_rn(ou[sc][j].x, __shfl_xor_sync(kFull, cu[sc][j].x, 1));
+          yu[(2 * j + 1) * 2 + sc] = __fadd_rn(ou[sc][j].y, __shfl_xor_sync(kFull, cu[sc][j].y, 1));
+          yw[(2 * j) * 2 + sc] = __fadd_rn(ow[sc][j].x, __shfl_xor_sync(kFull, cw[sc][j].x, 1));
+          yw[(2 * j + 1) * 2 + sc] = __fadd_rn(ow[sc][j].y, __shfl_xor_sync(kFull, cw[sc][j].y, 1));
+        }
+      }
+    }
+  }
+}
+
+// The clip of the lane's 16 transformed values and their rounding to bf16.
+template <int AD>
+__device__ __forceinline__ V16 bat_finish(float (&y)[16], const LaneParams<AD>& L, bool clip) {
   uint32_t lo2 = 0, hi2 = 0;
   bool packed_clip = false;
   if (clip) {
@@ -368,8 +450,12 @@ __device__ __forceinline__ void canonical_nan(V16& v) {
 #ifndef MX_BAT_MINB_WIDE
 #define MX_BAT_MINB_WIDE 3
 #endif
+// a = 2 carries two rows per step (twice the live values): 2 CTAs per SM.
+#ifndef MX_BAT_MINB_A2
+#define MX_BAT_MINB_A2 2
+#endif
 __host__ __device__ constexpr int bat_min_blocks(int ad) {
-  return (ad == 8 || ad == 16) ? 3 : ((ad == 2 || ad == 32) ? MX_BAT_MINB_WIDE : 2);
+  return (ad == 8 || ad == 16) ? 3 : (ad == 32 ? MX_BAT_MINB_WIDE : (ad == 2 ? MX_BAT_MINB_A2 : 2));
 }
 
 template <int AD, int OP, int FMT, int RULE, int MBS>
@@ -445,19 +531,16 @@ __global__ void __launch_bounds__(kThreads, bat_min_blocks(AD)) bat_kernel(Strea
 
   double sd = 0.0, sx = 0.0;
   int st = 0;
-  for (int64_t r = r0; r < p.rows; r += rstride) {
-    issue(r + (kBatStages - 1) * rstride, st == 0 ? kBatStages - 1 : st - 1);
-    cp_async_wait<kBatStages - 1>();
+  auto read_slot = [&](int sl) {
     V16 v;
-    {
-      const uint4 lo = *reinterpret_cast<const uint4*>(slot0 + (2 * st) * kThreads * 16);
-      const uint4 hi = *reinterpret_cast<const uint4*>(slot0 + (2 * st + 1) * kThreads * 16);
-      v.w[0] = lo.x; v.w[1] = lo.y; v.w[2] = lo.z; v.w[3] = lo.w;
-      v.w[4] = hi.x; v.w[5] = hi.y; v.w[6] = hi.z; v.w[7] = hi.w;
-    }
-    st = st == kBatStages - 1 ? 0 : st + 1;
+    const uint4 lo = *reinterpret_cast<const uint4*>(slot0 + (2 * sl) * kThreads * 16);
+    const uint4 hi = *reinterpret_cast<const uint4*>(slot0 + (2 * sl + 1) * kThreads * 16);
+    v.w[0] = lo.x; v.w[1] = lo.y; v.w[2] = lo.z; v.w[3] = lo.w;
+    v.w[4] = hi.x; v.w[5] = hi.y; v.w[6] = hi.z; v.w[7] = hi.w;
+    return v;
+  };
+  auto emit = [&](int64_t r, V16& yv) {
     const int64_t c = r * p.spr + cs;
-    V16 yv = bat_slice<AD>(v, h, L, As, clip);
     const uint32_t pa = pair_max(amax_bits16(yv));
     if (pa >= 0x7F80u) canonical_nan(yv);
     if constexpr (OP == kOpBatApply) {
@@ -466,6 +549,37 @@ __global__ void __launch_bounds__(kThreads, bat_min_blocks(AD)) bat_kernel(Strea
       int k = 0;
       if (MBS == kMbsStatic) k = mbs_static_k(oct_max(pa));
       process_slice<kOpQuant, FMT, RULE, MBS>(a, yv, yv, c, col_ok, lane, pa, k, sd, sx);
+    }
+  };
+  if constexpr (AD == 2) {
+    // two rows (r, r + rstride) per step: the ring's two oldest slots are
+    // read, refilled with the rows kBatStages - 1 and kBatStages strides on,
+    // and both rows go through the transform together
+    static_assert(kBatStages >= 3, "two rows per step need three slots or more");
+    for (int64_t r = r0; r < p.rows; r += 2 * rstride) {
+      cp_async_wait<kBatStages - 3>();
+      const V16 vu = read_slot(st);
+      const V16 vw = read_slot(st + 1 == kBatStages ? 0 : st + 1);
+      issue(r + (kBatStages - 1) * rstride, st == 0 ? kBatStages - 1 : st - 1);
+      issue(r + kBatStages * rstride, st);
+      st = st + 2 >= kBatStages ? st + 2 - kBatStages : st + 2;
+      float yu[16], yw[16];
+      bat_transform2_a2(vu, vw, h, L, yu, yw);
+      V16 ou = bat_finish<AD>(yu, L, clip);
+      emit(r, ou);
+      if (r + rstride < p.rows) {   // warp-uniform: rows are per warp
+        V16 ow = bat_finish<AD>(yw, L, clip);
+        emit(r + rstride, ow);
+      }
+    }
+  } else {
+    for (int64_t r = r0; r < p.rows; r += rstride) {
+      issue(r + (kBatStages - 1) * rstride, st == 0 ? kBatStages - 1 : st - 1);
+      cp_async_wait<kBatStages - 1>();
+      const V16 v = read_slot(st);
+      st = st == kBatStages - 1 ? 0 : st + 1;
+      V16 yv = bat_slice<AD>(v, h, L, As, clip);
+      emit(r, yv);
     }
   }
   cp_async_wait<0>();
