@@ -149,15 +149,8 @@ __device__ __forceinline__ void reduce_totals(double sd, double sx, double* tota
   }
 }
 
-// Resident CTAs per SM the block-error kernel is compiled for (its register
-// budget: 65536 / (256 x this)); a build-time tuning knob.
-#ifndef MX_ERROR_MIN_BLOCKS
-#define MX_ERROR_MIN_BLOCKS 1
-#endif
-
 template <int OP, int FMT, int RULE, int MBS, int U>
-__global__ void __launch_bounds__(kThreads, OP == kOpError ? MX_ERROR_MIN_BLOCKS : 1)
-    stream_kernel(StreamArgs a) {
+__global__ void __launch_bounds__(kThreads) stream_kernel(StreamArgs a) {
   const int lane = threadIdx.x & 31;
   const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
