@@ -676,8 +676,8 @@ def main():
     ap.add_argument("--no-ops", action="store_true", help="skip the per-op figures")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile-op", default=None,
-                    help="run one op of the MoE-stack table `--steps` times and print its figure "
-                         "(for profilers); no headline line")
+                    help="run one op of the MoE-stack table, or gemm_pre_MxNxK / gemm_fused_MxNxK, "
+                         "`--steps` times and print its figure (for profilers); no headline line")
     ap.add_argument("--profile-experts", type=int, default=32,
                     help="experts of the stack used by --profile-op (32: 201 MB of input, above L2)")
     args = ap.parse_args()
@@ -690,14 +690,45 @@ def main():
     return run_mx(args)
 
 
+def run_profile_gemm(args, mx, inputs):
+    """--profile-op gemm_{pre,fused}_MxNxK: `--steps` launches of the
+    pre-quantized or the fused MXFP4 GEMM on the operands gemm_ops uses."""
+    import torch
+    kind, shape = args.profile_op.split("_")[1], args.profile_op.split("_")[2]
+    M, N, K = (int(t) for t in shape.split("x"))
+    dev = torch.device("cuda", 0)
+    a = inputs.normal_weight(M, K, seed=11, device=dev, std=1.0)
+    w = inputs.normal_weight(N, K, seed=12, device=dev)
+    bc, bs, _ = mx.quantize(w, mx.E2M1, mx.FLOOR | mx.MMA_SCALES)
+    ac, as_, _ = mx.quantize(a, mx.E2M1, mx.FLOOR | mx.MMA_SCALES)
+    d = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
+    fn = ((lambda: mx.gemm(ac, as_, bc, bs, out=d)) if kind == "pre"
+          else (lambda: mx.quant_gemm(a, bc, bs, mx.FLOOR, out=d)))
+    fn()
+    torch.cuda.synchronize()
+    s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    s.record()
+    for _ in range(args.steps):
+        fn()
+    e.record()
+    e.synchronize()
+    us = s.elapsed_time(e) / args.steps * 1e3
+    print(json.dumps({"profile_op": args.profile_op, "us": round(us, 2),
+                      "TFLOP/s": round(2.0 * M * N * K / us / 1e6, 1)}), flush=True)
+    return 0
+
+
 def run_profile_op(args):
-    """One op of the MoE-stack table, alone (after the stack is generated)."""
+    """One op of the MoE-stack table, alone (after the stack is generated), or
+    one of the GEMMs (gemm_pre_MxNxK, gemm_fused_MxNxK)."""
     import torch
     import fp8_quantization_mx_b200 as mx
     from fp8_quantization_mx_b200 import build as mxbuild
     from fp8_quantization_mx_b200 import inputs
     mxbuild.build()
     mx.load_library()
+    if args.profile_op.startswith("gemm_"):
+        return run_profile_gemm(args, mx, inputs)
     x = inputs.moe_w13(experts=args.profile_experts, device="cuda").view(-1, HIDDEN)
     res = stack_ops(mx, x, reps=args.steps, only=args.profile_op)
     torch.cuda.synchronize()
