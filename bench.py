@@ -480,8 +480,9 @@ def measured_fp4_peak():
 
 def gemm_ops(mx, inputs, dev, reps=20):
     """The block-scaled MXFP4 GEMM D = A B^T (bf16 out) on the tensor cores:
-    A pre-quantized; A quantized inside the GEMM (fused); quantize then GEMM
-    (unfused). Median CUDA-event time of `reps`, L2 flushed before each. The
+    A pre-quantized; A quantized inside the GEMM on chip (fused); A quantized
+    into caller buffers and the GEMM run on them in one launch (staged);
+    quantize then GEMM (unfused). Median CUDA-event time of `reps`, L2 flushed before each. The
     library's block-scaled GEMM (cuBLAS through torch) on the same operands is
     timed beside it as context."""
     import torch
@@ -496,10 +497,13 @@ def gemm_ops(mx, inputs, dev, reps=20):
         ac, as_, _ = mx.quantize(a, mx.E2M1, mx.FLOOR | mx.MMA_SCALES)
         d = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
         st = torch.zeros(1, dtype=torch.int32, device=dev)
+        ac2, as2 = torch.empty_like(ac), torch.empty_like(as_)
         fns = {
             "quantize_a": lambda: mx.quantize(a, mx.E2M1, mx.FLOOR | mx.MMA_SCALES, out=(ac, as_, None)),
             "gemm": lambda: mx.gemm(ac, as_, bc, bs, out=d, status=st),
             "fused_quant_gemm": lambda: mx.quant_gemm(a, bc, bs, mx.FLOOR, out=d, status=st),
+            "staged_quant_gemm": lambda: mx.quant_gemm(a, bc, bs, mx.FLOOR, out=d, status=st,
+                                                       a_out=(ac2, as2)),
             "unfused_quantize_then_gemm": lambda: (
                 mx.quantize(a, mx.E2M1, mx.FLOOR | mx.MMA_SCALES, out=(ac, as_, None)),
                 mx.gemm(ac, as_, bc, bs, out=d, status=st)),
@@ -514,6 +518,7 @@ def gemm_ops(mx, inputs, dev, reps=20):
                 r[k + "_tflops"] = round(r["flop"] / (ms * 1e-3) / 1e12, 1)
         r["gemm_frac_of_peak"] = round(r["gemm_tflops"] / peak, 3)
         r["fused_vs_unfused"] = round(r["unfused_quantize_then_gemm_us"] / r["fused_quant_gemm_us"], 3)
+        r["staged_vs_unfused"] = round(r["unfused_quantize_then_gemm_us"] / r["staged_quant_gemm_us"], 3)
         try:
             lib = lambda: F.scaled_mm(ac.view(torch.float4_e2m1fn_x2), bc.view(torch.float4_e2m1fn_x2).t(),
                                       as_.view(torch.float8_e8m0fnu), F.ScalingType.BlockWise1x32,
@@ -530,7 +535,7 @@ def gemm_ops(mx, inputs, dev, reps=20):
             r["context_library_gemm"] = f"unavailable: {str(e).splitlines()[0][:120]}"
         r["status"] = int(st.item())
         res[name] = r
-        del a, w, bc, bs, ac, as_, d
+        del a, w, bc, bs, ac, as_, ac2, as2, d
     del flush
     return res
 

@@ -312,9 +312,11 @@ int mx_quant_gemm(const void* a_bf16, int scaling, const void* b_codes, const ui
   const auto cs = static_cast<cudaStream_t>(stream);
   if (K == 0) return gemm_zero(M, N, out_fp32, d, cs);
   if (!a_bf16) return MX_ERR_INVALID_ARG;
-  if (!aligned(a_bf16, 32) || (a_codes_out && !aligned(a_codes_out, 8)) ||
-      (status && !aligned(status, 4)))
+  if (!aligned(a_bf16, 32) || (a_codes_out && !aligned(a_codes_out, 16)) ||
+      (a_scales_out && a_codes_out && !aligned(a_scales_out, 16)) || (status && !aligned(status, 4)))
     return MX_ERR_ALIGN;
+  // the tiled layout's padding rows read as zero bytes
+  if (clear_padding(a_scales_out, M, K, MX_SCALES_MMA, 32, cs) != cudaSuccess) return MX_ERR_CUDA;
   return from_cuda(mxk::launch_gemm(a_bf16, nullptr, scaling, b_codes, b_scales, M, N, K,
                                     out_fp32, d, a_codes_out, a_scales_out, status, cs));
 }

@@ -36,6 +36,7 @@
 // caller's status word and the CTA drains its in-flight copies and MMAs,
 // frees its TMEM and returns.
 
+#include <cooperative_groups.h>
 #include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
@@ -228,11 +229,9 @@ __device__ __forceinline__ bool epilogue_tile(const Smem<BN, S, FUSED>& sm, cons
 // tmem_empty barriers, so the next tile's loads proceed while the epilogue
 // drains the accumulator.
 template <int BN, int S>
-__global__ void __launch_bounds__(GemmCfg<BN, S, false>::kThreads, 1)
-    gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                const GemmArgs g) {
+__device__ __forceinline__ void gemm_pre_body(const CUtensorMap* tmA, const CUtensorMap* tmB,
+                                              const GemmArgs& g, uint8_t* smem_raw) {
   using C = GemmCfg<BN, S, false>;
-  extern __shared__ uint8_t smem_raw[];
   const Smem<BN, S, false> sm(smem_raw);
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -260,8 +259,8 @@ __global__ void __launch_bounds__(GemmCfg<BN, S, false>::kThreads, 1)
   if (warp == 0) {
     // ---------------------------------------------------------- producer
     if (lane == 0) {
-      tc::prefetch_tmap(&tmB);
-      tc::prefetch_tmap(&tmA);
+      tc::prefetch_tmap(tmB);
+      tc::prefetch_tmap(tmA);
       const int64_t bands_total = (g.N + 127) / 128;
       int64_t it = 0;   // K-blocks issued so far (the ring position)
       bool ok = true;
@@ -281,13 +280,13 @@ __global__ void __launch_bounds__(GemmCfg<BN, S, false>::kThreads, 1)
             break;
           }
           tc::mbar_arrive_expect_tx(sm.fullB(s), tx);
-          tc::tma_load_2d(sm.sB + s * C::kTileB, &tmB, kb * static_cast<int>(kRowBytes),
+          tc::tma_load_2d(sm.sB + s * C::kTileB, tmB, kb * static_cast<int>(kRowBytes),
                           static_cast<int>(n0), sm.fullB(s));
           for (int band = 0; band < nbands; ++band)
             tc::bulk_load(sm.sSFB + s * C::kSfB + band * 2 * kSfTile,
                           g.b_scales + ((nb0 + band) * T + 2 * kb) * kSfTile, 2 * kSfTile,
                           sm.fullB(s));
-          tc::tma_load_2d(sm.sA + s * kTileA, &tmA, kb * static_cast<int>(kRowBytes),
+          tc::tma_load_2d(sm.sA + s * kTileA, tmA, kb * static_cast<int>(kRowBytes),
                           static_cast<int>(m0), sm.fullB(s));
           tc::bulk_load(sm.sSFA + s * C::kSfA, g.a_scales + ((m0 / 128) * T + 2 * kb) * kSfTile,
                         2 * kSfTile, sm.fullB(s));
@@ -341,6 +340,58 @@ __global__ void __launch_bounds__(GemmCfg<BN, S, false>::kThreads, 1)
     tc::tc_fence_after();
     tc::tmem_dealloc(tmem, C::kTmemCols);
   }
+}
+
+template <int BN, int S>
+__global__ void __launch_bounds__(GemmCfg<BN, S, false>::kThreads, 1)
+    gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                const GemmArgs g) {
+  extern __shared__ uint8_t smem_raw[];
+  gemm_pre_body<BN, S>(&tmA, &tmB, g, smem_raw);
+}
+
+// ------------------------------------ bf16 A staged through L2, one launch --
+// Cooperative (every CTA resident): phase 1 runs the streaming quantizer over
+// all of A with every warp of the grid, writing the codes and the tiled scales
+// into the caller's buffers (which stay in L2 at GEMM sizes); a grid-wide
+// barrier; phase 2 is the pre-quantized GEMM on them. One launch instead of
+// two, and the quantized A is read back by TMA mostly from L2.
+template <int BN, int S, int RULE>
+__global__ void __launch_bounds__(GemmCfg<BN, S, false>::kThreads, 1)
+    gemm_staged_kernel(const __grid_constant__ CUtensorMap tmA,
+                       const __grid_constant__ CUtensorMap tmB, const GemmArgs g,
+                       const StreamArgs q) {
+  extern __shared__ uint8_t smem_raw[];
+  {
+    constexpr int U = 2;   // slices per lane in flight (8 measured no faster)
+    const int lane = threadIdx.x & 31;
+    const int64_t warp = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+    const int64_t nwarps = (static_cast<int64_t>(gridDim.x) * blockDim.x) >> 5;
+    double sd = 0.0, sx = 0.0;
+    for (int64_t tile = warp; tile * 32 * U < q.nslices; tile += nwarps) {
+      const int64_t base = tile * 32 * U + lane;
+      V16 v[U];
+#pragma unroll
+      for (int j = 0; j < U; ++j) {
+        const int64_t c = base + 32 * j;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) v[j].w[i] = 0;
+        if (c < q.nslices) v[j] = ld_stream32(q.x + 32 * c);
+      }
+#pragma unroll
+      for (int j = 0; j < U; ++j) {
+        const int64_t c = base + 32 * j;
+        const uint32_t pa = pair_max(amax_bits16(v[j]));
+        process_slice<kOpQuant, kFmtE2M1, RULE, kMbsNone>(q, v[j], v[j], c, c < q.nslices, lane, pa,
+                                                           0, sd, sx);
+      }
+    }
+    // the codes were written through the generic proxy; TMA (the async
+    // proxy) reads them after the barrier
+    asm volatile("fence.proxy.async.global;" ::: "memory");
+  }
+  cooperative_groups::this_grid().sync();
+  gemm_pre_body<BN, S>(&tmA, &tmB, g, smem_raw);
 }
 
 // ---------------------------------------- bf16 A quantized in the prologue --
@@ -698,6 +749,29 @@ cudaError_t launch_prequant(const CUtensorMap& tmA, const CUtensorMap& tmB, cons
   return cudaGetLastError();
 }
 
+template <int BN, int S, int RULE>
+cudaError_t launch_staged(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& g,
+                          const StreamArgs& q, cudaStream_t st) {
+  using C = GemmCfg<BN, S, false>;
+  auto kern = gemm_staged_kernel<BN, S, RULE>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(C::kSmem));
+  if (e != cudaSuccess) return e;
+  const int64_t tiles = ((g.M + kGemmBM - 1) / kGemmBM) * ((g.N + BN - 1) / BN);
+  const int sms = sm_count_of_current_device(&e);
+  if (e != cudaSuccess) return e;
+  // every CTA resident at once (one per SM): the grid barrier needs it
+  const unsigned grid = static_cast<unsigned>(tiles < sms ? tiles : sms);
+  CUtensorMap a_map = tmA, b_map = tmB;
+  GemmArgs ga = g;
+  StreamArgs qa = q;
+  void* args[] = {&a_map, &b_map, &ga, &qa};
+  e = cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(kern), dim3(grid), dim3(C::kThreads),
+                                  args, C::kSmem, st);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
 template <int BN, int S, int CL, int RULE>
 cudaError_t launch_fused(const CUtensorMap& tmX, const CUtensorMap& tmB, const GemmArgs& g,
                          cudaStream_t st) {
@@ -783,6 +857,34 @@ cudaError_t launch_gemm(const void* a, const uint8_t* a_scales, int a_rule, cons
   if (!fused) {
     if (!code_tmap(&tmA, a, M, K, kGemmBM)) return cudaErrorInvalidValue;
     return wide ? launch_prequant<256, 4>(tmA, tmB, g, st) : launch_prequant<128, 6>(tmA, tmB, g, st);
+  }
+  if (a_codes_out && a_scales_out) {
+    // A's quantized form goes to the caller's buffers: quantize into them and
+    // run the GEMM on them in one cooperative launch
+    if (!code_tmap(&tmA, a_codes_out, M, K, kGemmBM)) return cudaErrorInvalidValue;
+    StreamArgs q{};
+    q.x = static_cast<const uint8_t*>(a);
+    q.nslices = M * K / 16;
+    q.codes = static_cast<uint8_t*>(a_codes_out);
+    q.scales = a_scales_out;
+    q.smap.bpr = K / 32;
+    q.smap.nct = (K / 32 + 3) / 4;
+    q.smap.inv = 1.0 / static_cast<double>(K / 32);
+    g.a_scales = a_scales_out;
+    switch (a_rule) {
+      case kCeil:
+        return wide ? launch_staged<256, 4, kCeil>(tmA, tmB, g, q, st)
+                    : launch_staged<128, 6, kCeil>(tmA, tmB, g, q, st);
+      case kOasRule:
+        return wide ? launch_staged<256, 4, kOasRule>(tmA, tmB, g, q, st)
+                    : launch_staged<128, 6, kOasRule>(tmA, tmB, g, q, st);
+      case kOas:
+        return wide ? launch_staged<256, 4, kOas>(tmA, tmB, g, q, st)
+                    : launch_staged<128, 6, kOas>(tmA, tmB, g, q, st);
+      default:
+        return wide ? launch_staged<256, 4, kFloor>(tmA, tmB, g, q, st)
+                    : launch_staged<128, 6, kFloor>(tmA, tmB, g, q, st);
+    }
   }
   if (!bf16_tmap(&tmA, a, M, K)) return cudaErrorInvalidValue;
   switch (a_rule) {

@@ -40,8 +40,10 @@
  * Errors: arguments are checked on the host before anything is enqueued; on
  * any error nothing is launched and no output is written. A failed launch
  * returns MX_ERR_CUDA. Faults inside a kernel surface at the caller's next
- * synchronisation, as usual for CUDA. Kernels never trap, assert or wait on
- * flags. All entry points are thread-safe.
+ * synchronisation, as usual for CUDA. Kernels never trap or assert; the
+ * streaming kernels never wait on flags, and the GEMM kernels' waits on their
+ * own barriers are bounded in time (see mx_gemm). All entry points are
+ * thread-safe.
  * Empty inputs (rows == 0 or cols == 0) are valid and launch nothing (except
  * that mx_block_error still zeroes its totals).
  * Alignment: x, grad_y, grad_x, y and out must be 32-byte aligned (the
@@ -235,12 +237,19 @@ int mx_bat_quantize(const void* x, int64_t rows, int64_t cols, int a_dim, const 
  * mx_gemm: A pre-quantized, a_codes [M, K/2] (16-byte aligned) and a_scales
  * in the MX_SCALES_MMA layout (16-byte aligned).
  * mx_quant_gemm: A given as bf16 [M, K] (32-byte aligned) and quantized to
- * MXFP4 inside the GEMM with `scaling` (MX_SCALE_FLOOR, CEIL, OAS_RULE or
+ * MXFP4 within the call with `scaling` (MX_SCALE_FLOOR, CEIL, OAS_RULE or
  * OAS; no MBS: its factors are not powers of two, which a block-scaled MMA
- * cannot apply), exactly as mx_quantize would quantize it; the quantized A
- * is written out only if a_codes_out ([M, K/2], 8-byte aligned) and/or
- * a_scales_out (MX_SCALES_MMA layout) are given. Other errors as
- * mx_quantize. */
+ * cannot apply), exactly as mx_quantize would quantize it. Two forms:
+ *  - a_codes_out ([M, K/2], 16-byte aligned) and a_scales_out (MX_SCALES_MMA
+ *    layout, 16-byte aligned, padding zeroed) both given: one cooperative
+ *    launch quantizes A into them with every SM, then (after a grid-wide
+ *    barrier) runs the GEMM on them; at GEMM sizes they are read back from
+ *    L2. They hold A's quantized form afterwards.
+ *  - otherwise: A is quantized inside the GEMM's prologue and never leaves
+ *    the chip; a thread-block cluster of up to 4 CTAs shares each quantized
+ *    tile through distributed shared memory. If exactly one of the two
+ *    buffers is given, it receives its part of A's quantized form.
+ * Other errors as mx_quantize. */
 int mx_gemm(const void* a_codes, const uint8_t* a_scales, const void* b_codes,
             const uint8_t* b_scales, int64_t M, int64_t N, int64_t K, int out_fp32, void* d,
             int* status, void* stream);

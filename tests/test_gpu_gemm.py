@@ -15,9 +15,11 @@ section: SM100 kernels consume MXFP4 operands and E8M0 scales.
 * Random cases: D against the fp64 product of the oracle's dequantized
   operands, within a bound proportional to the sum of |a_k b_k| (the tensor
   cores' accumulation order and internal precision are not specified).
-* The fused GEMM equals the unfused one (quantize, then the GEMM on the
-  quantized operands) bit for bit: both feed the same operands to the same
-  MMA sequence.
+* The fused GEMM, in both forms (A quantized on chip and shared across a
+  cluster; A quantized into the caller's buffers and the GEMM run on them in
+  the same cooperative launch), equals the unfused one (quantize, then the
+  GEMM on the quantized operands) bit for bit: both feed the same operands to
+  the same MMA sequence.
 """
 
 import numpy as np
@@ -81,7 +83,13 @@ def dequant64(oracle_mod, codes, plain_scales, rows, K):
     return y.view(np.float32).astype(np.float64)
 
 
-@pytest.mark.parametrize("fused", [True, False], ids=["fused", "prequantized"])
+def a_buffers(mx, cuda, M, K):
+    """Caller buffers for A's quantized form (codes, tiled scales)."""
+    return (torch.empty(M, K // 2, dtype=torch.uint8, device=cuda),
+            torch.empty(mx.mx_scale_bytes(M, K, E2M1, MMA), dtype=torch.uint8, device=cuda))
+
+
+@pytest.mark.parametrize("fused", ["fused", "staged", "prequantized"])
 @pytest.mark.parametrize("shape", SHAPES, ids=lambda s: "x".join(map(str, s)))
 def test_integer_cases_are_exact(mx, cuda, shape, fused):
     M, N, K = shape
@@ -93,8 +101,11 @@ def test_integer_cases_are_exact(mx, cuda, shape, fused):
     status = torch.zeros(1, dtype=torch.int32, device=cuda)
     outs = {}
     for dt in (torch.float32, torch.bfloat16):
-        if fused:
+        if fused == "fused":
             outs[dt] = mx.quant_gemm(a.to(cuda), bc, bs, FLOOR, out_dtype=dt, status=status)
+        elif fused == "staged":
+            outs[dt] = mx.quant_gemm(a.to(cuda), bc, bs, FLOOR, out_dtype=dt, status=status,
+                                     a_out=a_buffers(mx, cuda, M, K))
         else:
             ac, as_, _ = mx.quantize(a.to(cuda), E2M1, FLOOR | MMA)
             outs[dt] = mx.gemm(ac, as_, bc, bs, out_dtype=dt, status=status)
@@ -124,19 +135,23 @@ def test_integer_cases_are_exact_many_units(mx, cuda, shape):
     assert np.array_equal(host(d).astype(np.float64), exact)
 
 
+@pytest.mark.parametrize("staged", [False, True], ids=["on-chip", "staged"])
 @pytest.mark.parametrize("rule", [FLOOR, OAS], ids=["FLOOR", "OAS"])
 @pytest.mark.parametrize("shape", BIG, ids=lambda s: "x".join(map(str, s)))
-def test_fused_equals_quantize_then_gemm_many_units(mx, cuda, shape, rule):
+def test_fused_equals_quantize_then_gemm_many_units(mx, cuda, shape, rule, staged):
     M, N, K = shape
     a = inputs.heavy_tail(M, K, seed=rule + 9).to(cuda)
     bc, bs = weights(mx, inputs.normal_weight(N, K, seed=11), cuda)
     status = torch.zeros(1, dtype=torch.int32, device=cuda)
-    d_fused = mx.quant_gemm(a, bc, bs, rule, out_dtype=torch.float32, status=status)
+    buf = a_buffers(mx, cuda, M, K) if staged else None
+    d_fused = mx.quant_gemm(a, bc, bs, rule, out_dtype=torch.float32, status=status, a_out=buf)
     ac, as_, _ = mx.quantize(a, E2M1, rule | MMA)
     d_two = mx.gemm(ac, as_, bc, bs, out_dtype=torch.float32, status=status)
     torch.cuda.synchronize()
     assert status.item() == 0
     assert torch.equal(d_fused.view(torch.int32), d_two.view(torch.int32))
+    if staged:
+        assert torch.equal(buf[0], ac) and torch.equal(buf[1], as_)
 
 
 @pytest.mark.parametrize("rule", RULES, ids=["FLOOR", "CEIL", "OAS_RULE", "OAS"])
@@ -162,17 +177,21 @@ def test_fused_quantizer_writes_the_oracle_quantization(mx, oracle_mod, cuda, ru
     assert np.all(tiled[pad] == 0)
 
 
+@pytest.mark.parametrize("staged", [False, True], ids=["on-chip", "staged"])
 @pytest.mark.parametrize("rule", RULES, ids=["FLOOR", "CEIL", "OAS_RULE", "OAS"])
 @pytest.mark.parametrize("shape", SHAPES, ids=lambda s: "x".join(map(str, s)))
-def test_fused_equals_quantize_then_gemm(mx, cuda, shape, rule):
+def test_fused_equals_quantize_then_gemm(mx, cuda, shape, rule, staged):
     M, N, K = shape
     a = inputs.heavy_tail(M, K, seed=M * 3 + rule).to(cuda)
     bc, bs = weights(mx, inputs.normal_weight(N, K, seed=N), cuda)
-    d_fused = mx.quant_gemm(a, bc, bs, rule, out_dtype=torch.float32)
+    buf = a_buffers(mx, cuda, M, K) if staged else None
+    d_fused = mx.quant_gemm(a, bc, bs, rule, out_dtype=torch.float32, a_out=buf)
     ac, as_, _ = mx.quantize(a, E2M1, rule | MMA)
     d_two = mx.gemm(ac, as_, bc, bs, out_dtype=torch.float32)
     torch.cuda.synchronize()
     assert torch.equal(d_fused.view(torch.int32), d_two.view(torch.int32))
+    if staged:   # A's quantized form, padding included, is mx_quantize's
+        assert torch.equal(buf[0], ac) and torch.equal(buf[1], as_)
 
 
 @pytest.mark.parametrize("shape", SHAPES, ids=lambda s: "x".join(map(str, s)))
