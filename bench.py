@@ -480,11 +480,12 @@ def measured_fp4_peak():
 
 def gemm_ops(mx, inputs, dev, reps=20):
     """The block-scaled MXFP4 GEMM D = A B^T (bf16 out) on the tensor cores:
-    A pre-quantized; A quantized inside the GEMM on chip (fused); A quantized
-    into caller buffers and the GEMM run on them in one launch (staged);
-    quantize then GEMM (unfused). Median CUDA-event time of `reps`, L2 flushed before each. The
-    library's block-scaled GEMM (cuBLAS through torch) on the same operands is
-    timed beside it as context."""
+    A pre-quantized; A quantized within the GEMM's launch, staged through
+    scratch the library allocates (the default call: quant_gemm), through the
+    caller's buffers (staged), or on chip in the GEMM's prologue (on_chip);
+    quantize then GEMM, two launches (unfused). Median CUDA-event time of
+    `reps`, L2 flushed before each. The library's block-scaled GEMM (cuBLAS
+    through torch) on the same operands is timed beside it as context."""
     import torch
     F = torch.nn.functional
     flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
@@ -501,9 +502,11 @@ def gemm_ops(mx, inputs, dev, reps=20):
         fns = {
             "quantize_a": lambda: mx.quantize(a, mx.E2M1, mx.FLOOR | mx.MMA_SCALES, out=(ac, as_, None)),
             "gemm": lambda: mx.gemm(ac, as_, bc, bs, out=d, status=st),
-            "fused_quant_gemm": lambda: mx.quant_gemm(a, bc, bs, mx.FLOOR, out=d, status=st),
+            "quant_gemm": lambda: mx.quant_gemm(a, bc, bs, mx.FLOOR, out=d, status=st),
             "staged_quant_gemm": lambda: mx.quant_gemm(a, bc, bs, mx.FLOOR, out=d, status=st,
                                                        a_out=(ac2, as2)),
+            "on_chip_quant_gemm": lambda: mx.quant_gemm(a, bc, bs, mx.FLOOR, out=d, status=st,
+                                                        on_chip=True),
             "unfused_quantize_then_gemm": lambda: (
                 mx.quantize(a, mx.E2M1, mx.FLOOR | mx.MMA_SCALES, out=(ac, as_, None)),
                 mx.gemm(ac, as_, bc, bs, out=d, status=st)),
@@ -517,8 +520,10 @@ def gemm_ops(mx, inputs, dev, reps=20):
             if k != "quantize_a":
                 r[k + "_tflops"] = round(r["flop"] / (ms * 1e-3) / 1e12, 1)
         r["gemm_frac_of_peak"] = round(r["gemm_tflops"] / peak, 3)
-        r["fused_vs_unfused"] = round(r["unfused_quantize_then_gemm_us"] / r["fused_quant_gemm_us"], 3)
-        r["staged_vs_unfused"] = round(r["unfused_quantize_then_gemm_us"] / r["staged_quant_gemm_us"], 3)
+        for k in ("quant_gemm", "staged_quant_gemm", "on_chip_quant_gemm"):
+            r[k + "_vs_unfused"] = round(r["unfused_quantize_then_gemm_us"] / r[k + "_us"], 3)
+        # the quantization's cost inside the fused call, as a share of the GEMM
+        r["quant_gemm_overhead_of_gemm"] = round(r["quant_gemm_us"] / r["gemm_us"] - 1.0, 3)
         try:
             lib = lambda: F.scaled_mm(ac.view(torch.float4_e2m1fn_x2), bc.view(torch.float4_e2m1fn_x2).t(),
                                       as_.view(torch.float8_e8m0fnu), F.ScalingType.BlockWise1x32,
@@ -681,7 +686,7 @@ def main():
     ap.add_argument("--no-ops", action="store_true", help="skip the per-op figures")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--profile-op", default=None,
-                    help="run one op of the MoE-stack table, or gemm_pre_MxNxK / gemm_fused_MxNxK, "
+                    help="run one op of the MoE-stack table, or gemm_{pre,fused,onchip}_MxNxK, "
                          "`--steps` times and print its figure (for profilers); no headline line")
     ap.add_argument("--profile-experts", type=int, default=32,
                     help="experts of the stack used by --profile-op (32: 201 MB of input, above L2)")
@@ -696,8 +701,10 @@ def main():
 
 
 def run_profile_gemm(args, mx, inputs):
-    """--profile-op gemm_{pre,fused}_MxNxK: `--steps` launches of the
-    pre-quantized or the fused MXFP4 GEMM on the operands gemm_ops uses."""
+    """--profile-op gemm_{pre,fused,onchip}_MxNxK: `--steps` launches of the
+    pre-quantized MXFP4 GEMM, the fused one (default form: staged through
+    scratch) or the fused one with A quantized on chip, on the operands
+    gemm_ops uses."""
     import torch
     kind, shape = args.profile_op.split("_")[1], args.profile_op.split("_")[2]
     M, N, K = (int(t) for t in shape.split("x"))
@@ -707,8 +714,10 @@ def run_profile_gemm(args, mx, inputs):
     bc, bs, _ = mx.quantize(w, mx.E2M1, mx.FLOOR | mx.MMA_SCALES)
     ac, as_, _ = mx.quantize(a, mx.E2M1, mx.FLOOR | mx.MMA_SCALES)
     d = torch.empty(M, N, dtype=torch.bfloat16, device=dev)
-    fn = ((lambda: mx.gemm(ac, as_, bc, bs, out=d)) if kind == "pre"
-          else (lambda: mx.quant_gemm(a, bc, bs, mx.FLOOR, out=d)))
+    fns = {"pre": lambda: mx.gemm(ac, as_, bc, bs, out=d),
+           "fused": lambda: mx.quant_gemm(a, bc, bs, mx.FLOOR, out=d),
+           "onchip": lambda: mx.quant_gemm(a, bc, bs, mx.FLOOR, out=d, on_chip=True)}
+    fn = fns[kind]
     fn()
     torch.cuda.synchronize()
     s, e = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
@@ -725,7 +734,7 @@ def run_profile_gemm(args, mx, inputs):
 
 def run_profile_op(args):
     """One op of the MoE-stack table, alone (after the stack is generated), or
-    one of the GEMMs (gemm_pre_MxNxK, gemm_fused_MxNxK)."""
+    one of the GEMMs (gemm_pre_MxNxK, gemm_fused_MxNxK, gemm_onchip_MxNxK)."""
     import torch
     import fp8_quantization_mx_b200 as mx
     from fp8_quantization_mx_b200 import build as mxbuild

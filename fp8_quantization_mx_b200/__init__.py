@@ -41,7 +41,7 @@ __all__ = [
     "E2M1_B16", "NVFP4", "block_size",
     "quantize", "dequantize", "fake_quant", "fake_quant_bwd", "block_error", "MXFakeQuantize",
     "mx_bat_apply", "mx_bat_quantize", "bat_apply", "bat_quantize",
-    "mx_gemm", "mx_quant_gemm", "gemm", "quant_gemm",
+    "mx_gemm", "mx_quant_gemm", "gemm", "quant_gemm", "GEMM_A_ON_CHIP",
     "MXFP4_FORMAT", "MXFP8_FORMAT",
 ]
 
@@ -55,6 +55,8 @@ INT8 = 5   # MXINT8 (i * 2^-6)
 # OR into `scaling`: scale bytes in the tiled layout of block-scaled tensor-core
 # GEMMs (a flat uint8 buffer of mx_scale_bytes(rows, cols, format, scaling) bytes)
 MMA_SCALES = 1 << 8
+# OR into mx_quant_gemm's out_fp32: A quantized in the GEMM's prologue, on chip
+GEMM_A_ON_CHIP = 1 << 9
 E2M1_B16 = 6  # MXFP4 at block 16 (E8M0 scales [..., cols/16])
 NVFP4 = 7     # E2M1 at block 16 with E4M3 scales amax/6 (FLOOR only)
 _PACKED = (E2M1, E2M1_B16, NVFP4)
@@ -592,10 +594,13 @@ def gemm(a_codes: torch.Tensor, a_scales: torch.Tensor, b_codes: torch.Tensor,
 
 
 def quant_gemm(a: torch.Tensor, b_codes: torch.Tensor, b_scales: torch.Tensor,
-               scaling: int = FLOOR, out_dtype=torch.bfloat16, out=None, a_out=None, status=None):
-    """D = MXFP4(a) B^T with bf16 ``a`` [M, K] quantized inside the GEMM
-    (``scaling``: FLOOR, CEIL, OAS_RULE or OAS). ``a_out`` = (codes [M, K/2],
-    tiled scales) also receives A's quantized form when given. Returns D."""
+               scaling: int = FLOOR, out_dtype=torch.bfloat16, out=None, a_out=None, status=None,
+               on_chip: bool = False):
+    """D = MXFP4(a) B^T with bf16 ``a`` [M, K] quantized within the same
+    launch (``scaling``: FLOOR, CEIL, OAS_RULE or OAS). ``a_out`` = (codes
+    [M, K/2], tiled scales) also receives A's quantized form when given.
+    ``on_chip``: quantize inside the GEMM's prologue (thread-block clusters)
+    instead of staging A through L2. Returns D."""
     _cuda_bf16(a, "a")
     if a.dim() != 2:
         raise ValueError("a must be [M, K]")
@@ -610,7 +615,8 @@ def quant_gemm(a: torch.Tensor, b_codes: torch.Tensor, b_scales: torch.Tensor,
         _check_buf(asc, "a_out scales", dev, torch.uint8, max(0, mx_scale_bytes(M, K, E2M1, MMA_SCALES)))
     st = _gemm_status(status, dev)
     with torch.cuda.device(dev):
-        _check(mx_quant_gemm(_ptr(a), scaling, _ptr(b_codes), _ptr(b_scales), M, N, K,
-                             int(out_dtype == torch.float32), _ptr(d), _ptr(ac), _ptr(asc), _ptr(st),
-                             _stream(dev)), "mx_quant_gemm")
+        flags = int(out_dtype == torch.float32) | (GEMM_A_ON_CHIP if on_chip else 0)
+        _check(mx_quant_gemm(_ptr(a), scaling, _ptr(b_codes), _ptr(b_scales), M, N, K, flags,
+                             _ptr(d), _ptr(ac), _ptr(asc), _ptr(st), _stream(dev)),
+               "mx_quant_gemm")
     return d

@@ -299,25 +299,27 @@ int mx_gemm(const void* a_codes, const uint8_t* a_scales, const void* b_codes,
   if (!a_codes || !a_scales) return MX_ERR_INVALID_ARG;
   if (!aligned(a_codes, 16) || !aligned(a_scales, 16) || (status && !aligned(status, 4)))
     return MX_ERR_ALIGN;
-  return from_cuda(mxk::launch_gemm(a_codes, a_scales, 0, b_codes, b_scales, M, N, K, out_fp32, d,
-                                    nullptr, nullptr, status, cs));
+  return from_cuda(mxk::launch_gemm(a_codes, a_scales, 0, false, b_codes, b_scales, M, N, K,
+                                    out_fp32, d, nullptr, nullptr, status, cs));
 }
 
 int mx_quant_gemm(const void* a_bf16, int scaling, const void* b_codes, const uint8_t* b_scales,
                   int64_t M, int64_t N, int64_t K, int out_fp32, void* d, void* a_codes_out,
                   uint8_t* a_scales_out, int* status, void* stream) {
   if (scaling < MX_SCALE_FLOOR || scaling > MX_SCALE_OAS) return MX_ERR_UNSUPPORTED;
+  const bool on_chip = (out_fp32 & MX_GEMM_A_ON_CHIP) != 0;
+  out_fp32 &= ~MX_GEMM_A_ON_CHIP;
   int st = check_gemm(M, N, K, out_fp32, b_codes, b_scales, d);
   if (st != MX_OK || M == 0 || N == 0) return st;
   const auto cs = static_cast<cudaStream_t>(stream);
   if (K == 0) return gemm_zero(M, N, out_fp32, d, cs);
   if (!a_bf16) return MX_ERR_INVALID_ARG;
   if (!aligned(a_bf16, 32) || (a_codes_out && !aligned(a_codes_out, 16)) ||
-      (a_scales_out && a_codes_out && !aligned(a_scales_out, 16)) || (status && !aligned(status, 4)))
+      (a_scales_out && !aligned(a_scales_out, 16)) || (status && !aligned(status, 4)))
     return MX_ERR_ALIGN;
   // the tiled layout's padding rows read as zero bytes
   if (clear_padding(a_scales_out, M, K, MX_SCALES_MMA, 32, cs) != cudaSuccess) return MX_ERR_CUDA;
-  return from_cuda(mxk::launch_gemm(a_bf16, nullptr, scaling, b_codes, b_scales, M, N, K,
+  return from_cuda(mxk::launch_gemm(a_bf16, nullptr, scaling, on_chip, b_codes, b_scales, M, N, K,
                                     out_fp32, d, a_codes_out, a_scales_out, status, cs));
 }
 

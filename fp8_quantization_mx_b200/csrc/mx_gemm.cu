@@ -41,6 +41,8 @@
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 
+#include <mutex>
+
 #include "mx_stream.cuh"
 #include "mx_tc.cuh"
 
@@ -56,7 +58,7 @@ constexpr uint32_t kSfTile = 512;  // 128 rows x 4 scales
 
 // Status codes a timed-out wait leaves in *status (which role gave up).
 constexpr int kStatusProducer = 1, kStatusMmaB = 2, kStatusMmaA = 3, kStatusQuant = 4,
-              kStatusEpilogue = 5, kStatusDrain = 6, kStatusStaging = 7;
+              kStatusEpilogue = 5, kStatusDrain = 6, kStatusStaging = 7, kStatusReady = 8;
 
 struct GemmArgs {
   const uint8_t* a_bf16;    // fused: bf16 A [M, K]
@@ -222,15 +224,111 @@ __device__ __forceinline__ bool epilogue_tile(const Smem<BN, S, FUSED>& sm, cons
   return true;
 }
 
+// What the persistent GEMM body runs beside the GEMM. NoPrologue: nothing,
+// A arrives quantized. QuantPrologue: kWarps more warps per CTA (after the
+// epilogue warps) quantize A (bf16) into the codes and tiled scales the GEMM
+// reads, warp tiles of 32 U slices dealt over the grid in slice order, and
+// count the slices done per 128-row m-tile in `ready` (relaxed adds after a
+// proxy fence and a release fence: the GEMM reads them with TMA); the producer
+// waits (acquire, bounded) until an m-tile is complete before its first load
+// of that m-tile's A. The GEMM of the first m-tiles thus starts while the
+// rest of A is being quantized, and the epilogue warps never wait on it.
+struct NoPrologue {
+  static constexpr bool kActive = false;
+  __device__ bool wait_mtile(int64_t, volatile int*, int*) const { return true; }
+};
+
+template <int RULE>
+struct QuantPrologue {
+  static constexpr bool kActive = true;
+  static constexpr int kWarps = 6;
+  static constexpr int U = 4;   // slices per lane per warp tile (32 U slices), two tiles in flight
+  // Warps per CTA in the first round: the quantizer warps and the epilogue
+  // warps, which are idle until the first accumulator is complete; the
+  // first-round tiles are the first m-tiles, which the first wave needs.
+  static constexpr int kFirstRound = 8 + kWarps;
+  StreamArgs q;                 // the quantizer's view of A (slices of 16 elements)
+  unsigned long long* ready;    // [ceil(M / 128)], zero at launch
+  int64_t mtile_slices;         // slices per m-tile: 128 K / 16 (a multiple of 32 U)
+
+  __device__ bool wait_mtile(int64_t mt, volatile int* abort, int* status) const {
+    const int64_t left = q.nslices - mt * mtile_slices;
+    const unsigned long long target =
+        static_cast<unsigned long long>(left < mtile_slices ? left : mtile_slices);
+    if (!tc::counter_wait(ready + mt, target, abort, status, kStatusReady)) return false;
+    // acquired through the generic proxy; the loads that follow are TMA's
+    tc::fence_proxy_async_global();
+    return true;
+  }
+
+  __device__ void load_tile(int64_t tile, int lane, V16 (&v)[U]) const {
+#pragma unroll
+    for (int j = 0; j < U; ++j) {
+      const int64_t c = tile * 32 * U + lane + 32 * j;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v[j].w[i] = 0;
+      if (c < q.nslices) v[j] = ld_stream32(q.x + 32 * c);
+    }
+  }
+
+  // The slices of a finished warp tile counted to its m-tile (lane 0).
+  __device__ void count(int64_t tile) const {
+    const int64_t first = tile * 32 * U;
+    const int64_t n = q.nslices - first < 32 * U ? q.nslices - first : 32 * U;
+    tc::red_relaxed_add(ready + first / mtile_slices, static_cast<unsigned long long>(n));
+  }
+
+  // Quantizes warp tiles t0, then t1, t1 + step, t1 + 2 step, ... (t1 > t0;
+  // t1 = INT64_MAX, step 0: t0 alone) with the next tile's loads in flight
+  // while one is quantized. t0 is published on its own, the rest two at a
+  // time (one release fence, which waits for the stores, for two tiles).
+  __device__ void run(int64_t t0, int64_t t1, int64_t step, int lane) const {
+    const int64_t ntiles = (q.nslices + 32 * U - 1) / (32 * U);
+    double sd = 0.0, sx = 0.0;
+    V16 v[U], nv[U];
+    load_tile(t0, lane, v);
+    int64_t held = -1;   // a finished tile not yet published
+    bool first = true;
+    for (int64_t tile = t0, next = t1; tile < ntiles; tile = next, next += step) {
+      if (next < ntiles) load_tile(next, lane, nv);
+#pragma unroll
+      for (int j = 0; j < U; ++j) {
+        const int64_t c = tile * 32 * U + lane + 32 * j;
+        const uint32_t pa = pair_max(amax_bits16(v[j]));
+        process_slice<kOpQuant, kFmtE2M1, RULE, kMbsNone>(q, v[j], v[j], c, c < q.nslices, lane,
+                                                           pa, 0, sd, sx);
+      }
+      if (!first && held < 0 && next < ntiles) {
+        held = tile;
+      } else {
+        // the codes and scales of the held tile and this one (generic-proxy
+        // stores of all 32 lanes) are published to their m-tiles
+        tc::fence_proxy_async_global();
+        __syncwarp();
+        if (lane == 0) {
+          tc::fence_release_gpu();
+          if (held >= 0) count(held);
+          count(tile);
+        }
+        held = -1;
+      }
+      first = false;
+#pragma unroll
+      for (int j = 0; j < U; ++j) v[j] = nv[j];
+    }
+  }
+};
+
 // ------------------------------------------- pre-quantized A: persistent --
 // CTA b takes tiles b, b + gridDim.x, ... (tile t: m-tile t / tiles_n, n-tile
 // t % tiles_n). The stage ring runs on across tiles; the accumulator is
 // handed between the MMA issuer and the epilogue by the tmem_full /
 // tmem_empty barriers, so the next tile's loads proceed while the epilogue
 // drains the accumulator.
-template <int BN, int S>
+template <int BN, int S, class Pro>
 __device__ __forceinline__ void gemm_pre_body(const CUtensorMap* tmA, const CUtensorMap* tmB,
-                                              const GemmArgs& g, uint8_t* smem_raw) {
+                                              const GemmArgs& g, uint8_t* smem_raw,
+                                              const Pro& pro) {
   using C = GemmCfg<BN, S, false>;
   const Smem<BN, S, false> sm(smem_raw);
   const int warp = threadIdx.x >> 5;
@@ -263,9 +361,11 @@ __device__ __forceinline__ void gemm_pre_body(const CUtensorMap* tmA, const CUte
       tc::prefetch_tmap(tmA);
       const int64_t bands_total = (g.N + 127) / 128;
       int64_t it = 0;   // K-blocks issued so far (the ring position)
+      int64_t ready_mt = -1;   // the last m-tile known to be quantized
       bool ok = true;
       for (int64_t t = blockIdx.x; ok && t < ntiles; t += gridDim.x) {
-        const int64_t m0 = (t / tiles_n) * kGemmBM;
+        const int64_t mt = t / tiles_n;
+        const int64_t m0 = mt * kGemmBM;
         const int64_t n0 = (t % tiles_n) * BN;
         // B's scale bands present in the tiled buffer (rows padded to 128)
         const int64_t nb0 = n0 / 128;
@@ -286,10 +386,24 @@ __device__ __forceinline__ void gemm_pre_body(const CUtensorMap* tmA, const CUte
             tc::bulk_load(sm.sSFB + s * C::kSfB + band * 2 * kSfTile,
                           g.b_scales + ((nb0 + band) * T + 2 * kb) * kSfTile, 2 * kSfTile,
                           sm.fullB(s));
+          // (the stage's B is on its way while this waits for A's m-tile)
+          bool got = true;
+          if (Pro::kActive && mt != ready_mt) {
+            got = pro.wait_mtile(mt, sm.abort_flag, g.status);
+            ready_mt = mt;
+          }
+          // loaded even after a failed wait (in bounds; the result is then
+          // undefined and the status set), so that the stage completes and
+          // the drain below stays exact
           tc::tma_load_2d(sm.sA + s * kTileA, tmA, kb * static_cast<int>(kRowBytes),
                           static_cast<int>(m0), sm.fullB(s));
           tc::bulk_load(sm.sSFA + s * C::kSfA, g.a_scales + ((m0 / 128) * T + 2 * kb) * kSfTile,
                         2 * kSfTile, sm.fullB(s));
+          if (!got) {
+            ok = false;
+            ++it;
+            break;
+          }
         }
       }
       // every copy this thread issued has landed before the CTA can exit
@@ -325,8 +439,23 @@ __device__ __forceinline__ void gemm_pre_body(const CUtensorMap* tmA, const CUte
       }
     }
     __syncwarp();
+  } else if (warp >= 2 + C::kWorkWarps) {
+    // --------------------------------------------- quantizer (QuantPrologue)
+    if constexpr (Pro::kActive) {
+      const int64_t first_round = static_cast<int64_t>(gridDim.x) * Pro::kFirstRound;
+      pro.run(static_cast<int64_t>(blockIdx.x) * Pro::kFirstRound + (warp - 2),
+              first_round + static_cast<int64_t>(blockIdx.x) * Pro::kWarps +
+                  (warp - 2 - C::kWorkWarps),
+              static_cast<int64_t>(gridDim.x) * Pro::kWarps, lane);
+    }
   } else {
     // ---------------------------------------------------------- epilogue
+    if constexpr (Pro::kActive) {
+      // one first-round tile each (the epilogue waits for an MMA that waits
+      // for the first m-tiles)
+      pro.run(static_cast<int64_t>(blockIdx.x) * Pro::kFirstRound + (warp - 2), INT64_MAX, 0,
+              lane);
+    }
     uint32_t tile_par = 0;
     for (int64_t t = blockIdx.x; t < ntiles; t += gridDim.x, tile_par ^= 1) {
       if (!epilogue_tile(sm, g, tmem, tile_par, (t / tiles_n) * kGemmBM, (t % tiles_n) * BN,
@@ -347,20 +476,32 @@ __global__ void __launch_bounds__(GemmCfg<BN, S, false>::kThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                 const GemmArgs g) {
   extern __shared__ uint8_t smem_raw[];
-  gemm_pre_body<BN, S>(&tmA, &tmB, g, smem_raw);
+  gemm_pre_body<BN, S>(&tmA, &tmB, g, smem_raw, NoPrologue{});
 }
 
 // ------------------------------------ bf16 A staged through L2, one launch --
-// Cooperative (every CTA resident): phase 1 runs the streaming quantizer over
-// all of A with every warp of the grid, writing the codes and the tiled scales
-// into the caller's buffers (which stay in L2 at GEMM sizes); a grid-wide
-// barrier; phase 2 is the pre-quantized GEMM on them. One launch instead of
-// two, and the quantized A is read back by TMA mostly from L2.
+// Cooperative (every CTA resident, so that a producer's wait on another CTA's
+// quantizer warps always ends): the quantizer warps of the whole grid
+// quantize A into the caller's code and scale buffers (which stay in L2 at
+// GEMM sizes) while the GEMM runs on the m-tiles already complete.
 template <int BN, int S, int RULE>
-__global__ void __launch_bounds__(GemmCfg<BN, S, false>::kThreads, 1)
+__global__ void __launch_bounds__(GemmCfg<BN, S, false>::kThreads + 32 * QuantPrologue<RULE>::kWarps,
+                                  1)
     gemm_staged_kernel(const __grid_constant__ CUtensorMap tmA,
                        const __grid_constant__ CUtensorMap tmB, const GemmArgs g,
-                       const StreamArgs q) {
+                       const QuantPrologue<RULE> pro) {
+  extern __shared__ uint8_t smem_raw[];
+  gemm_pre_body<BN, S>(&tmA, &tmB, g, smem_raw, pro);
+}
+
+// The same when the GEMM's tiles fit in one wave: every tile needs all of A
+// before its first MMA, so nothing overlaps; every warp of the grid
+// quantizes A, a grid-wide barrier, then the GEMM (no counters to clear).
+template <int BN, int S, int RULE>
+__global__ void __launch_bounds__(GemmCfg<BN, S, false>::kThreads, 1)
+    gemm_staged_sync_kernel(const __grid_constant__ CUtensorMap tmA,
+                            const __grid_constant__ CUtensorMap tmB, const GemmArgs g,
+                            const StreamArgs q) {
   extern __shared__ uint8_t smem_raw[];
   {
     constexpr int U = 2;   // slices per lane in flight (8 measured no faster)
@@ -388,10 +529,10 @@ __global__ void __launch_bounds__(GemmCfg<BN, S, false>::kThreads, 1)
     }
     // the codes were written through the generic proxy; TMA (the async
     // proxy) reads them after the barrier
-    asm volatile("fence.proxy.async.global;" ::: "memory");
+    tc::fence_proxy_async_global();
   }
   cooperative_groups::this_grid().sync();
-  gemm_pre_body<BN, S>(&tmA, &tmB, g, smem_raw);
+  gemm_pre_body<BN, S>(&tmA, &tmB, g, smem_raw, NoPrologue{});
 }
 
 // ---------------------------------------- bf16 A quantized in the prologue --
@@ -724,6 +865,40 @@ bool bf16_tmap(CUtensorMap* tm, const void* a, int64_t M, int64_t K) {
              CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Stream-ordered scratch comes from a memory pool this library creates once
+// per device and never trims (release threshold: all), so that after the
+// first call an allocation maps no memory and costs the host microseconds;
+// the default pool gives its memory back at every synchronisation and maps it
+// again on the next call. The pools live as long as the process.
+cudaError_t scratch_pool(cudaMemPool_t* out) {
+  constexpr int kMaxDevices = 64;
+  static std::mutex mu;
+  static cudaMemPool_t pools[kMaxDevices] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!pools[dev]) {
+    cudaMemPoolProps props = {};
+    props.allocType = cudaMemAllocationTypePinned;
+    props.location.type = cudaMemLocationTypeDevice;
+    props.location.id = dev;
+    cudaMemPool_t p = nullptr;
+    e = cudaMemPoolCreate(&p, &props);
+    if (e != cudaSuccess) return e;
+    uint64_t keep = ~0ull;
+    e = cudaMemPoolSetAttribute(p, cudaMemPoolAttrReleaseThreshold, &keep);
+    if (e != cudaSuccess) {
+      cudaMemPoolDestroy(p);
+      return e;
+    }
+    pools[dev] = p;
+  }
+  *out = pools[dev];
+  return cudaSuccess;
+}
+
 int sm_count_of_current_device(cudaError_t* e) {
   int dev = 0, sms = 0;
   *e = cudaGetDevice(&dev);
@@ -751,9 +926,35 @@ cudaError_t launch_prequant(const CUtensorMap& tmA, const CUtensorMap& tmB, cons
 
 template <int BN, int S, int RULE>
 cudaError_t launch_staged(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& g,
-                          const StreamArgs& q, cudaStream_t st) {
+                          const StreamArgs& q, unsigned long long* ready, cudaStream_t st) {
   using C = GemmCfg<BN, S, false>;
   auto kern = gemm_staged_kernel<BN, S, RULE>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(C::kSmem));
+  if (e != cudaSuccess) return e;
+  const int sms = sm_count_of_current_device(&e);
+  if (e != cudaSuccess) return e;
+  // one CTA per SM, all resident at once (the producers wait on other CTAs'
+  // quantizer warps); CTAs beyond the tile count only quantize
+  CUtensorMap a_map = tmA, b_map = tmB;
+  GemmArgs ga = g;
+  QuantPrologue<RULE> pro{};
+  pro.q = q;
+  pro.ready = ready;
+  pro.mtile_slices = static_cast<int64_t>(kGemmBM) * g.K / 16;
+  void* args[] = {&a_map, &b_map, &ga, &pro};
+  e = cudaLaunchCooperativeKernel(reinterpret_cast<const void*>(kern), dim3(sms),
+                                  dim3(C::kThreads + 32 * QuantPrologue<RULE>::kWarps), args,
+                                  C::kSmem, st);
+  if (e != cudaSuccess) return e;
+  return cudaGetLastError();
+}
+
+template <int BN, int S, int RULE>
+cudaError_t launch_staged_sync(const CUtensorMap& tmA, const CUtensorMap& tmB, const GemmArgs& g,
+                               const StreamArgs& q, cudaStream_t st) {
+  using C = GemmCfg<BN, S, false>;
+  auto kern = gemm_staged_sync_kernel<BN, S, RULE>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        static_cast<int>(C::kSmem));
   if (e != cudaSuccess) return e;
@@ -770,6 +971,36 @@ cudaError_t launch_staged(const CUtensorMap& tmA, const CUtensorMap& tmB, const 
                                   args, C::kSmem, st);
   if (e != cudaSuccess) return e;
   return cudaGetLastError();
+}
+
+// The staged form for one rounding rule: the grid-barrier kernel when the
+// GEMM's tiles fit in one wave, else the overlapped kernel, its per-m-tile
+// ready counts in stream-ordered scratch (zeroed before the launch, released
+// after it).
+template <int RULE>
+cudaError_t launch_staged_rule(bool wide, const CUtensorMap& tmA, const CUtensorMap& tmB,
+                               const GemmArgs& g, const StreamArgs& q, cudaStream_t st) {
+  cudaError_t e = cudaSuccess;
+  const int sms = sm_count_of_current_device(&e);
+  if (e != cudaSuccess) return e;
+  const int64_t bn = wide ? 256 : 128;
+  const int64_t mtiles = (g.M + kGemmBM - 1) / kGemmBM;
+  if (mtiles * ((g.N + bn - 1) / bn) <= sms)
+    return wide ? launch_staged_sync<256, 4, RULE>(tmA, tmB, g, q, st)
+                : launch_staged_sync<128, 6, RULE>(tmA, tmB, g, q, st);
+  const size_t ready_bytes = static_cast<size_t>(mtiles) * 8;
+  cudaMemPool_t pool = nullptr;
+  e = scratch_pool(&pool);
+  if (e != cudaSuccess) return e;
+  unsigned long long* ready = nullptr;
+  e = cudaMallocFromPoolAsync(reinterpret_cast<void**>(&ready), ready_bytes, pool, st);
+  if (e != cudaSuccess) return e;
+  e = cudaMemsetAsync(ready, 0, ready_bytes, st);
+  if (e == cudaSuccess)
+    e = wide ? launch_staged<256, 4, RULE>(tmA, tmB, g, q, ready, st)
+             : launch_staged<128, 6, RULE>(tmA, tmB, g, q, ready, st);
+  const cudaError_t ef = cudaFreeAsync(ready, st);
+  return e != cudaSuccess ? e : ef;
 }
 
 template <int BN, int S, int CL, int RULE>
@@ -833,10 +1064,10 @@ cudaError_t launch_fused_bn(bool wide, const CUtensorMap& tmX, const CUtensorMap
 
 }  // namespace
 
-cudaError_t launch_gemm(const void* a, const uint8_t* a_scales, int a_rule, const void* b_codes,
-                        const uint8_t* b_scales, int64_t M, int64_t N, int64_t K, int out_fp32,
-                        void* d, void* a_codes_out, uint8_t* a_scales_out, int* status,
-                        cudaStream_t st) {
+cudaError_t launch_gemm(const void* a, const uint8_t* a_scales, int a_rule, bool a_on_chip,
+                        const void* b_codes, const uint8_t* b_scales, int64_t M, int64_t N,
+                        int64_t K, int out_fp32, void* d, void* a_codes_out,
+                        uint8_t* a_scales_out, int* status, cudaStream_t st) {
   const bool fused = a_scales == nullptr;
   // 256-wide tiles unless that leaves SMs idle on a small problem
   const bool wide = N > 128 && ((M + kGemmBM - 1) / kGemmBM) * ((N + 255) / 256) >= 148;
@@ -858,41 +1089,67 @@ cudaError_t launch_gemm(const void* a, const uint8_t* a_scales, int a_rule, cons
     if (!code_tmap(&tmA, a, M, K, kGemmBM)) return cudaErrorInvalidValue;
     return wide ? launch_prequant<256, 4>(tmA, tmB, g, st) : launch_prequant<128, 6>(tmA, tmB, g, st);
   }
-  if (a_codes_out && a_scales_out) {
-    // A's quantized form goes to the caller's buffers: quantize into them and
-    // run the GEMM on them in one cooperative launch
-    if (!code_tmap(&tmA, a_codes_out, M, K, kGemmBM)) return cudaErrorInvalidValue;
+  if (a_on_chip) {
+    if (!bf16_tmap(&tmA, a, M, K)) return cudaErrorInvalidValue;
+    switch (a_rule) {
+      case kCeil: return launch_fused_bn<kCeil>(wide, tmA, tmB, g, st);
+      case kOasRule: return launch_fused_bn<kOasRule>(wide, tmA, tmB, g, st);
+      case kOas: return launch_fused_bn<kOas>(wide, tmA, tmB, g, st);
+      default: return launch_fused_bn<kFloor>(wide, tmA, tmB, g, st);
+    }
+  }
+  // Staged: A is quantized into the caller's buffers, or (where the caller
+  // gives none) into stream-ordered scratch, and the GEMM runs on them in the
+  // same cooperative launch.
+  const int64_t mtiles = (M + kGemmBM - 1) / kGemmBM;
+  const size_t scale_bytes = static_cast<size_t>(mtiles * (K / 128)) * kSfTile;
+  uint8_t* codes = static_cast<uint8_t*>(a_codes_out);
+  uint8_t* scales = a_scales_out;
+  uint8_t* scratch[2] = {nullptr, nullptr};
+  cudaError_t e = cudaSuccess;
+  if (!codes || !scales) {
+    cudaMemPool_t pool = nullptr;
+    e = scratch_pool(&pool);
+    if (e != cudaSuccess) return e;
+    if (!codes) {
+      e = cudaMallocFromPoolAsync(reinterpret_cast<void**>(&scratch[0]),
+                                  static_cast<size_t>(M * K / 2), pool, st);
+      codes = scratch[0];
+    }
+    if (e == cudaSuccess && !scales) {
+      e = cudaMallocFromPoolAsync(reinterpret_cast<void**>(&scratch[1]), scale_bytes, pool, st);
+      scales = scratch[1];
+      // the padding rows of the last band are read by the MMA as zero bytes
+      if (e == cudaSuccess && M % kGemmBM != 0) {
+        const size_t band = static_cast<size_t>(K / 128) * kSfTile;
+        e = cudaMemsetAsync(scratch[1] + scale_bytes - band, 0, band, st);
+      }
+    }
+  }
+  if (e == cudaSuccess && !code_tmap(&tmA, codes, M, K, kGemmBM)) e = cudaErrorInvalidValue;
+  if (e == cudaSuccess) {
     StreamArgs q{};
     q.x = static_cast<const uint8_t*>(a);
     q.nslices = M * K / 16;
-    q.codes = static_cast<uint8_t*>(a_codes_out);
-    q.scales = a_scales_out;
+    q.codes = codes;
+    q.scales = scales;
     q.smap.bpr = K / 32;
     q.smap.nct = (K / 32 + 3) / 4;
     q.smap.inv = 1.0 / static_cast<double>(K / 32);
-    g.a_scales = a_scales_out;
+    g.a_scales = scales;
     switch (a_rule) {
-      case kCeil:
-        return wide ? launch_staged<256, 4, kCeil>(tmA, tmB, g, q, st)
-                    : launch_staged<128, 6, kCeil>(tmA, tmB, g, q, st);
-      case kOasRule:
-        return wide ? launch_staged<256, 4, kOasRule>(tmA, tmB, g, q, st)
-                    : launch_staged<128, 6, kOasRule>(tmA, tmB, g, q, st);
-      case kOas:
-        return wide ? launch_staged<256, 4, kOas>(tmA, tmB, g, q, st)
-                    : launch_staged<128, 6, kOas>(tmA, tmB, g, q, st);
-      default:
-        return wide ? launch_staged<256, 4, kFloor>(tmA, tmB, g, q, st)
-                    : launch_staged<128, 6, kFloor>(tmA, tmB, g, q, st);
+      case kCeil: e = launch_staged_rule<kCeil>(wide, tmA, tmB, g, q, st); break;
+      case kOasRule: e = launch_staged_rule<kOasRule>(wide, tmA, tmB, g, q, st); break;
+      case kOas: e = launch_staged_rule<kOas>(wide, tmA, tmB, g, q, st); break;
+      default: e = launch_staged_rule<kFloor>(wide, tmA, tmB, g, q, st);
     }
   }
-  if (!bf16_tmap(&tmA, a, M, K)) return cudaErrorInvalidValue;
-  switch (a_rule) {
-    case kCeil: return launch_fused_bn<kCeil>(wide, tmA, tmB, g, st);
-    case kOasRule: return launch_fused_bn<kOasRule>(wide, tmA, tmB, g, st);
-    case kOas: return launch_fused_bn<kOas>(wide, tmA, tmB, g, st);
-    default: return launch_fused_bn<kFloor>(wide, tmA, tmB, g, st);
+  for (uint8_t* p : scratch) {
+    if (!p) continue;
+    const cudaError_t ef = cudaFreeAsync(p, st);
+    if (e == cudaSuccess) e = ef;
   }
+  return e;
 }
 
 }  // namespace mxk

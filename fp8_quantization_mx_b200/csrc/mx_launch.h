@@ -33,12 +33,13 @@ cudaError_t launch_bat(const void* x, int64_t rows, int64_t cols, int a_dim, con
                        int scaling, void* codes, uint8_t* scales, uint8_t* macro, void* y,
                        ScaleMap sm, cudaStream_t st);
 // Block-scaled MXFP4 GEMM D = A B^T: A pre-quantized (codes + tiled scales)
-// when a_scales != null, else bf16 quantized on chip with rule a_rule (and
-// optionally written to a_codes_out / a_scales_out).
-cudaError_t launch_gemm(const void* a, const uint8_t* a_scales, int a_rule, const void* b_codes,
-                        const uint8_t* b_scales, int64_t M, int64_t N, int64_t K, int out_fp32,
-                        void* d, void* a_codes_out, uint8_t* a_scales_out, int* status,
-                        cudaStream_t st);
+// when a_scales != null, else bf16 quantized with rule a_rule within the
+// launch: staged through a_codes_out / a_scales_out (scratch for a null one),
+// or on chip (a_on_chip; a non-null buffer then receives its part).
+cudaError_t launch_gemm(const void* a, const uint8_t* a_scales, int a_rule, bool a_on_chip,
+                        const void* b_codes, const uint8_t* b_scales, int64_t M, int64_t N,
+                        int64_t K, int out_fp32, void* d, void* a_codes_out,
+                        uint8_t* a_scales_out, int* status, cudaStream_t st);
 cudaError_t launch_block_error(const void* x, int64_t n, int fmt, int scaling, float* block_sse,
                                double* totals, cudaStream_t st);
 

@@ -87,6 +87,51 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
   asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
+// The same between generic-proxy and async-proxy accesses of global memory.
+__device__ __forceinline__ void fence_proxy_async_global() {
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+}
+
+// ------------------------------------------- grid-scope counters (flags) --
+
+// A release fence followed by relaxed adds (the release pattern): every
+// write this thread has made or observed before the fence is visible to a
+// thread that acquires a value written by one of the adds.
+__device__ __forceinline__ void fence_release_gpu() {
+  asm volatile("fence.acq_rel.gpu;" ::: "memory");
+}
+
+__device__ __forceinline__ void red_relaxed_add(unsigned long long* p, unsigned long long v) {
+  asm volatile("red.relaxed.gpu.global.add.u64 [%0], %1;" ::"l"(p), "l"(v) : "memory");
+}
+
+__device__ __forceinline__ unsigned long long ld_acquire(const unsigned long long* p) {
+  unsigned long long v;
+  asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Waits until *p >= target, bounded like mbar_wait (abort flag polled, one
+// second at most: then the flag and *status are set and false returned).
+__device__ __forceinline__ bool counter_wait(const unsigned long long* p, unsigned long long target,
+                                             volatile int* abort, int* status, int code) {
+  uint64_t t0 = 0;
+  for (uint32_t it = 0;; ++it) {
+    if (ld_acquire(p) >= target) return true;
+    if ((it & 15) == 15) {
+      if (*abort) return false;
+      const uint64_t now = globaltimer();
+      if (t0 == 0) {
+        t0 = now;
+      } else if (now - t0 > kWaitLimitNs) {
+        *abort = 1;
+        if (status) atomicExch(status, code);
+        return false;
+      }
+    }
+  }
+}
+
 // -------------------------------------------------------------- copies --
 
 // 2-D TMA tile load into this CTA's shared memory; completes `bytes` on bar.

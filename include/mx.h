@@ -239,17 +239,23 @@ int mx_bat_quantize(const void* x, int64_t rows, int64_t cols, int a_dim, const 
  * mx_quant_gemm: A given as bf16 [M, K] (32-byte aligned) and quantized to
  * MXFP4 within the call with `scaling` (MX_SCALE_FLOOR, CEIL, OAS_RULE or
  * OAS; no MBS: its factors are not powers of two, which a block-scaled MMA
- * cannot apply), exactly as mx_quantize would quantize it. Two forms:
- *  - a_codes_out ([M, K/2], 16-byte aligned) and a_scales_out (MX_SCALES_MMA
- *    layout, 16-byte aligned, padding zeroed) both given: one cooperative
- *    launch quantizes A into them with every SM, then (after a grid-wide
- *    barrier) runs the GEMM on them; at GEMM sizes they are read back from
- *    L2. They hold A's quantized form afterwards.
- *  - otherwise: A is quantized inside the GEMM's prologue and never leaves
- *    the chip; a thread-block cluster of up to 4 CTAs shares each quantized
- *    tile through distributed shared memory. If exactly one of the two
- *    buffers is given, it receives its part of A's quantized form.
+ * cannot apply), exactly as mx_quantize would quantize it. a_codes_out
+ * ([M, K/2], 16-byte aligned) and a_scales_out (MX_SCALES_MMA layout,
+ * 16-byte aligned, padding zeroed), each nullable, receive A's quantized
+ * form. Two forms:
+ *  - staged (default): one cooperative launch quantizes A into those buffers
+ *    (into stream-ordered scratch for a NULL one, taken from a memory pool
+ *    the library keeps per device) and runs the GEMM on them, read back
+ *    mostly from L2. When the GEMM's tiles fit in one wave every warp
+ *    quantizes, then a grid-wide barrier; otherwise six extra warps per CTA
+ *    quantize while the GEMM runs, each 128-row band of A counted as it
+ *    completes (a per-band counter in the scratch) so that its tiles start
+ *    as soon as their band is ready.
+ *  - out_fp32 | MX_GEMM_A_ON_CHIP: A is quantized inside the GEMM's prologue
+ *    and the GEMM never reads it from memory; a thread-block cluster of up
+ *    to 4 CTAs shares each quantized tile through distributed shared memory.
  * Other errors as mx_quantize. */
+enum { MX_GEMM_A_ON_CHIP = 1 << 9 /* OR-ed into mx_quant_gemm's out_fp32 */ };
 int mx_gemm(const void* a_codes, const uint8_t* a_scales, const void* b_codes,
             const uint8_t* b_scales, int64_t M, int64_t N, int64_t K, int out_fp32, void* d,
             int* status, void* stream);

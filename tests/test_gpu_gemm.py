@@ -89,7 +89,20 @@ def a_buffers(mx, cuda, M, K):
             torch.empty(mx.mx_scale_bytes(M, K, E2M1, MMA), dtype=torch.uint8, device=cuda))
 
 
-@pytest.mark.parametrize("fused", ["fused", "staged", "prequantized"])
+# The forms of mx_quant_gemm: quantized in the GEMM's prologue on chip; staged
+# through scratch the library allocates; staged through the caller's buffers.
+FORMS = ["on-chip", "scratch", "staged"]
+
+
+def quant_gemm_form(mx, cuda, form, a, bc, bs, rule, **kw):
+    """mx_quant_gemm in one of FORMS; returns (D, the caller's A buffers or None)."""
+    M, K = a.shape
+    buf = a_buffers(mx, cuda, M, K) if form == "staged" else None
+    d = mx.quant_gemm(a, bc, bs, rule, a_out=buf, on_chip=form == "on-chip", **kw)
+    return d, buf
+
+
+@pytest.mark.parametrize("fused", FORMS + ["prequantized"])
 @pytest.mark.parametrize("shape", SHAPES, ids=lambda s: "x".join(map(str, s)))
 def test_integer_cases_are_exact(mx, cuda, shape, fused):
     M, N, K = shape
@@ -101,11 +114,9 @@ def test_integer_cases_are_exact(mx, cuda, shape, fused):
     status = torch.zeros(1, dtype=torch.int32, device=cuda)
     outs = {}
     for dt in (torch.float32, torch.bfloat16):
-        if fused == "fused":
-            outs[dt] = mx.quant_gemm(a.to(cuda), bc, bs, FLOOR, out_dtype=dt, status=status)
-        elif fused == "staged":
-            outs[dt] = mx.quant_gemm(a.to(cuda), bc, bs, FLOOR, out_dtype=dt, status=status,
-                                     a_out=a_buffers(mx, cuda, M, K))
+        if fused in FORMS:
+            outs[dt], _ = quant_gemm_form(mx, cuda, fused, a.to(cuda), bc, bs, FLOOR, out_dtype=dt,
+                                          status=status)
         else:
             ac, as_, _ = mx.quantize(a.to(cuda), E2M1, FLOOR | MMA)
             outs[dt] = mx.gemm(ac, as_, bc, bs, out_dtype=dt, status=status)
@@ -117,40 +128,43 @@ def test_integer_cases_are_exact(mx, cuda, shape, fused):
 
 
 # Long persistent runs: ~256 units over the clusters, each unit 12 K-blocks,
-# so every stage of the ring is refilled by changing owners many times over.
+# so every stage of the ring is refilled by changing owners many times over;
+# staged, 32 bands of A counted ready while seven waves of tiles run.
 BIG = [(4096, 8192, 3072)]
 
 
+@pytest.mark.parametrize("form", ["on-chip", "scratch"])
 @pytest.mark.parametrize("shape", BIG, ids=lambda s: "x".join(map(str, s)))
-def test_integer_cases_are_exact_many_units(mx, cuda, shape):
+def test_integer_cases_are_exact_many_units(mx, cuda, shape, form):
     M, N, K = shape
     av, a = grid_matrix(M, K, seed=5)
     bv, b = grid_matrix(N, K, seed=6)
     exact = av @ bv.T
     bc, bs = weights(mx, b, cuda)
     status = torch.zeros(1, dtype=torch.int32, device=cuda)
-    d = mx.quant_gemm(a.to(cuda), bc, bs, FLOOR, out_dtype=torch.float32, status=status)
+    d, _ = quant_gemm_form(mx, cuda, form, a.to(cuda), bc, bs, FLOOR, out_dtype=torch.float32,
+                           status=status)
     torch.cuda.synchronize()
     assert status.item() == 0
     assert np.array_equal(host(d).astype(np.float64), exact)
 
 
-@pytest.mark.parametrize("staged", [False, True], ids=["on-chip", "staged"])
+@pytest.mark.parametrize("form", FORMS)
 @pytest.mark.parametrize("rule", [FLOOR, OAS], ids=["FLOOR", "OAS"])
 @pytest.mark.parametrize("shape", BIG, ids=lambda s: "x".join(map(str, s)))
-def test_fused_equals_quantize_then_gemm_many_units(mx, cuda, shape, rule, staged):
+def test_fused_equals_quantize_then_gemm_many_units(mx, cuda, shape, rule, form):
     M, N, K = shape
     a = inputs.heavy_tail(M, K, seed=rule + 9).to(cuda)
     bc, bs = weights(mx, inputs.normal_weight(N, K, seed=11), cuda)
     status = torch.zeros(1, dtype=torch.int32, device=cuda)
-    buf = a_buffers(mx, cuda, M, K) if staged else None
-    d_fused = mx.quant_gemm(a, bc, bs, rule, out_dtype=torch.float32, status=status, a_out=buf)
+    d_fused, buf = quant_gemm_form(mx, cuda, form, a, bc, bs, rule, out_dtype=torch.float32,
+                                   status=status)
     ac, as_, _ = mx.quantize(a, E2M1, rule | MMA)
     d_two = mx.gemm(ac, as_, bc, bs, out_dtype=torch.float32, status=status)
     torch.cuda.synchronize()
     assert status.item() == 0
     assert torch.equal(d_fused.view(torch.int32), d_two.view(torch.int32))
-    if staged:
+    if buf is not None:
         assert torch.equal(buf[0], ac) and torch.equal(buf[1], as_)
 
 
@@ -177,21 +191,47 @@ def test_fused_quantizer_writes_the_oracle_quantization(mx, oracle_mod, cuda, ru
     assert np.all(tiled[pad] == 0)
 
 
-@pytest.mark.parametrize("staged", [False, True], ids=["on-chip", "staged"])
+@pytest.mark.parametrize("form", FORMS)
 @pytest.mark.parametrize("rule", RULES, ids=["FLOOR", "CEIL", "OAS_RULE", "OAS"])
 @pytest.mark.parametrize("shape", SHAPES, ids=lambda s: "x".join(map(str, s)))
-def test_fused_equals_quantize_then_gemm(mx, cuda, shape, rule, staged):
+def test_fused_equals_quantize_then_gemm(mx, cuda, shape, rule, form):
     M, N, K = shape
     a = inputs.heavy_tail(M, K, seed=M * 3 + rule).to(cuda)
     bc, bs = weights(mx, inputs.normal_weight(N, K, seed=N), cuda)
-    buf = a_buffers(mx, cuda, M, K) if staged else None
-    d_fused = mx.quant_gemm(a, bc, bs, rule, out_dtype=torch.float32, a_out=buf)
+    d_fused, buf = quant_gemm_form(mx, cuda, form, a, bc, bs, rule, out_dtype=torch.float32)
     ac, as_, _ = mx.quantize(a, E2M1, rule | MMA)
     d_two = mx.gemm(ac, as_, bc, bs, out_dtype=torch.float32)
     torch.cuda.synchronize()
     assert torch.equal(d_fused.view(torch.int32), d_two.view(torch.int32))
-    if staged:   # A's quantized form, padding included, is mx_quantize's
+    if buf is not None:   # A's quantized form, padding included, is mx_quantize's
         assert torch.equal(buf[0], ac) and torch.equal(buf[1], as_)
+
+
+@pytest.mark.parametrize("on_chip", [False, True], ids=["staged", "on-chip"])
+@pytest.mark.parametrize("part", ["codes", "scales"])
+@pytest.mark.parametrize("shape", [(300, 520, 1024), (1536, 4096, 512)],
+                         ids=lambda s: "x".join(map(str, s)))
+def test_one_buffer_receives_its_part(mx, cuda, shape, part, on_chip):
+    """Only one of A's buffers given: it receives mx_quantize's bytes (the
+    other part goes to scratch, staged, or stays on chip) and D is unchanged."""
+    M, N, K = shape
+    a = inputs.heavy_tail(M, K, seed=M + 5).to(cuda)
+    bc, bs = weights(mx, inputs.normal_weight(N, K, seed=N + 1), cuda)
+    ac, as_, _ = mx.quantize(a, E2M1, OAS | MMA)
+    codes, scales = a_buffers(mx, cuda, M, K)
+    buf = codes if part == "codes" else scales
+    buf.fill_(0xA5)
+    d = torch.empty(M, N, dtype=torch.float32, device=cuda)
+    flags = 1 | (mx.GEMM_A_ON_CHIP if on_chip else 0)
+    st = mx.mx_quant_gemm(a.data_ptr(), OAS, bc.data_ptr(), bs.data_ptr(), M, N, K, flags,
+                          d.data_ptr(), codes.data_ptr() if part == "codes" else None,
+                          scales.data_ptr() if part == "scales" else None, None,
+                          torch.cuda.current_stream().cuda_stream)
+    assert st == 0
+    d_two = mx.gemm(ac, as_, bc, bs, out_dtype=torch.float32)
+    torch.cuda.synchronize()
+    assert torch.equal(d.view(torch.int32), d_two.view(torch.int32))
+    assert torch.equal(buf, ac if part == "codes" else as_)
 
 
 @pytest.mark.parametrize("shape", SHAPES, ids=lambda s: "x".join(map(str, s)))
