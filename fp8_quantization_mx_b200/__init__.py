@@ -41,7 +41,7 @@ __all__ = [
     "E2M1_B16", "NVFP4", "block_size",
     "quantize", "dequantize", "fake_quant", "fake_quant_bwd", "block_error", "MXFakeQuantize",
     "mx_bat_apply", "mx_bat_quantize", "bat_apply", "bat_quantize",
-    "mx_gemm", "mx_quant_gemm", "gemm", "quant_gemm", "GEMM_A_ON_CHIP",
+    "mx_gemm", "mx_quant_gemm", "gemm", "quant_gemm", "GEMM_A_ON_CHIP", "mx_quant_gemm_noalloc",
     "MXFP4_FORMAT", "MXFP8_FORMAT",
 ]
 
@@ -72,7 +72,7 @@ FLOOR, CEIL, OAS_RULE, OAS = 0, 1, 2, 3
 MBS_STATIC, MBS_DYNAMIC = 1 << 4, 2 << 4
 
 _STATUS = {0: "MX_OK", 1: "MX_ERR_INVALID_ARG", 2: "MX_ERR_SHAPE", 3: "MX_ERR_ALIGN",
-           4: "MX_ERR_UNSUPPORTED", 5: "MX_ERR_CUDA"}
+           4: "MX_ERR_UNSUPPORTED", 5: "MX_ERR_CUDA", 6: "MX_ERR_TOO_LARGE"}
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _lib = None
@@ -119,6 +119,8 @@ def load_library():
     lib.mx_quant_gemm.argtypes = [vp, c_int, vp, vp, i64, i64, i64, c_int, vp, vp, vp, vp, vp]
     lib.mx_gemm.restype = c_int
     lib.mx_quant_gemm.restype = c_int
+    lib.mx_quant_gemm_noalloc.argtypes = [vp, c_int, vp, vp, i64, i64, i64, c_int, vp, vp, vp]
+    lib.mx_quant_gemm_noalloc.restype = c_int
     _lib = lib
     return lib
 
@@ -165,6 +167,15 @@ def mx_quant_gemm(a, scaling, b_codes, b_scales, M, N, K, out_fp32, d, a_codes_o
                   status, stream=0) -> int:
     return load_library().mx_quant_gemm(a, scaling, b_codes, b_scales, M, N, K, out_fp32, d,
                                         a_codes_out, a_scales_out, status, stream)
+
+
+def mx_quant_gemm_noalloc(a, scaling, b_codes, b_scales, M, N, K, out_fp32, d, status,
+                          stream=0) -> int:
+    """mx_quant_gemm (staged, no A buffers) with its scratch in the library's
+    fixed device array: for callers that may not allocate device memory
+    while they run. Calls that overlap on the GPU race on that array."""
+    return load_library().mx_quant_gemm_noalloc(a, scaling, b_codes, b_scales, M, N, K, out_fp32,
+                                                d, status, stream)
 
 
 def mx_status_string(status: int) -> str:

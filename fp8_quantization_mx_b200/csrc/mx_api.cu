@@ -95,6 +95,7 @@ const char* mx_status_string(int status) {
     case MX_ERR_ALIGN: return "pointer is not aligned as required";
     case MX_ERR_UNSUPPORTED: return "unsupported format / scaling combination";
     case MX_ERR_CUDA: return "CUDA launch or stream operation failed";
+    case MX_ERR_TOO_LARGE: return "problem larger than the fixed scratch of the no-allocation entry point";
     default: return "unknown status";
   }
 }
@@ -321,6 +322,23 @@ int mx_quant_gemm(const void* a_bf16, int scaling, const void* b_codes, const ui
   if (clear_padding(a_scales_out, M, K, MX_SCALES_MMA, 32, cs) != cudaSuccess) return MX_ERR_CUDA;
   return from_cuda(mxk::launch_gemm(a_bf16, nullptr, scaling, on_chip, b_codes, b_scales, M, N, K,
                                     out_fp32, d, a_codes_out, a_scales_out, status, cs));
+}
+
+// The staged quantize + GEMM for callers that may not allocate: its scratch
+// is the library's fixed device array instead of the stream-ordered pool.
+int mx_quant_gemm_noalloc(const void* a_bf16, int scaling, const void* b_codes,
+                          const uint8_t* b_scales, int64_t M, int64_t N, int64_t K, int out_fp32,
+                          void* d, int* status, void* stream) {
+  if (scaling < MX_SCALE_FLOOR || scaling > MX_SCALE_OAS) return MX_ERR_UNSUPPORTED;
+  int st = check_gemm(M, N, K, out_fp32, b_codes, b_scales, d);
+  if (st != MX_OK || M == 0 || N == 0) return st;
+  const auto cs = static_cast<cudaStream_t>(stream);
+  if (K == 0) return gemm_zero(M, N, out_fp32, d, cs);
+  if (!a_bf16) return MX_ERR_INVALID_ARG;
+  if (!aligned(a_bf16, 32) || (status && !aligned(status, 4))) return MX_ERR_ALIGN;
+  if (!mxk::noalloc_fits(M, K)) return MX_ERR_TOO_LARGE;
+  return from_cuda(mxk::launch_quant_gemm_noalloc(a_bf16, scaling, b_codes, b_scales, M, N, K,
+                                                  out_fp32, d, status, cs));
 }
 
 }  // extern "C"

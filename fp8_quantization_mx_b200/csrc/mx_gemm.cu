@@ -43,6 +43,7 @@
 
 #include <mutex>
 
+#include "mx.h"
 #include "mx_stream.cuh"
 #include "mx_tc.cuh"
 
@@ -1150,6 +1151,139 @@ cudaError_t launch_gemm(const void* a, const uint8_t* a_scales, int a_rule, bool
     if (e == cudaSuccess) e = ef;
   }
   return e;
+}
+
+// ------------------------------------ quantize + GEMM without allocation --
+// Callers that may not allocate device memory while they run (a serving
+// process that reserves its memory once at start-up and keeps it fixed, or a
+// runtime whose memory pools are unavailable) cannot use the default staged
+// form, which takes A's quantized form and the band counters from a
+// stream-ordered pool. This variant takes them from one array in the
+// library's device memory, of fixed size; every call shares it.
+
+namespace {
+
+// codes [M, K/2], then (256-byte aligned) the tiled scales, then the band
+// counters; the total must fit the array
+struct NoAllocLayout {
+  size_t scales, scale_bytes, ready, end;
+};
+
+NoAllocLayout noalloc_layout(int64_t M, int64_t K) {
+  const auto up = [](size_t v) { return (v + 255) & ~static_cast<size_t>(255); };
+  const size_t mtiles = static_cast<size_t>((M + kGemmBM - 1) / kGemmBM);
+  NoAllocLayout l{};
+  l.scales = up(static_cast<size_t>(M) * static_cast<size_t>(K / 2));
+  l.scale_bytes = mtiles * static_cast<size_t>(K / 128) * kSfTile;
+  l.ready = up(l.scales + l.scale_bytes);
+  l.end = l.ready + mtiles * 8;
+  return l;
+}
+
+template <int RULE>
+cudaError_t noalloc_rule(bool wide, bool one_wave, const CUtensorMap& tmA, const CUtensorMap& tmB,
+                         const GemmArgs& g, const StreamArgs& q, unsigned long long* ready,
+                         cudaStream_t st) {
+  if (one_wave)
+    return wide ? launch_staged_sync<256, 4, RULE>(tmA, tmB, g, q, st)
+                : launch_staged_sync<128, 6, RULE>(tmA, tmB, g, q, st);
+  return wide ? launch_staged<256, 4, RULE>(tmA, tmB, g, q, ready, st)
+              : launch_staged<128, 6, RULE>(tmA, tmB, g, q, ready, st);
+}
+
+}  // namespace
+}  // namespace mxk
+
+// The array (file scope). Host code cannot use its name as an address: the
+// device address comes from cudaGetSymbolAddress, once per device.
+static __device__ __align__(256) uint8_t mx_noalloc_scratch[MX_NOALLOC_SCRATCH_BYTES];
+
+namespace mxk {
+
+bool noalloc_fits(int64_t M, int64_t K) {
+  return noalloc_layout(M, K).end <= static_cast<size_t>(MX_NOALLOC_SCRATCH_BYTES);
+}
+
+namespace {
+
+// The array's device address on the current device, looked up on the first
+// call on that device.
+cudaError_t noalloc_scratch(uint8_t** out) {
+  constexpr int kMaxDevices = 64;
+  static std::mutex mu;
+  static uint8_t* ptrs[kMaxDevices] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!ptrs[dev]) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, mx_noalloc_scratch);
+    if (e != cudaSuccess) return e;
+    ptrs[dev] = static_cast<uint8_t*>(p);
+  }
+  *out = ptrs[dev];
+  return cudaSuccess;
+}
+
+}  // namespace
+
+cudaError_t launch_quant_gemm_noalloc(const void* a, int a_rule, const void* b_codes,
+                                      const uint8_t* b_scales, int64_t M, int64_t N, int64_t K,
+                                      int out_fp32, void* d, int* status, cudaStream_t st) {
+  if (!noalloc_fits(M, K)) return cudaErrorInvalidValue;
+  uint8_t* base = nullptr;
+  cudaError_t e = noalloc_scratch(&base);
+  if (e != cudaSuccess) return e;
+  const NoAllocLayout l = noalloc_layout(M, K);
+  uint8_t* codes = base;
+  uint8_t* scales = base + l.scales;
+  auto* ready = reinterpret_cast<unsigned long long*>(base + l.ready);
+  const bool wide = N > 128 && ((M + kGemmBM - 1) / kGemmBM) * ((N + 255) / 256) >= 148;
+  const int64_t bn = wide ? 256 : 128;
+  const int64_t mtiles = (M + kGemmBM - 1) / kGemmBM;
+  int sms = sm_count_of_current_device(&e);
+  if (e != cudaSuccess) return e;
+  const bool one_wave = mtiles * ((N + bn - 1) / bn) <= sms;
+  // the array keeps the previous call's bytes: zero what is read before it
+  // is written (the padding rows of the last band of scales, the counters)
+  if (M % kGemmBM != 0) {
+    const size_t band = static_cast<size_t>(K / 128) * kSfTile;
+    e = cudaMemsetAsync(scales + l.scale_bytes - band, 0, band, st);
+    if (e != cudaSuccess) return e;
+  }
+  if (!one_wave) {
+    e = cudaMemsetAsync(ready, 0, static_cast<size_t>(mtiles) * 8, st);
+    if (e != cudaSuccess) return e;
+  }
+  CUtensorMap tmA{}, tmB{};
+  if (!code_tmap(&tmB, b_codes, N, K, wide ? 256 : 128)) return cudaErrorInvalidValue;
+  if (!code_tmap(&tmA, codes, M, K, kGemmBM)) return cudaErrorInvalidValue;
+  GemmArgs g{};
+  g.a_bf16 = static_cast<const uint8_t*>(a);
+  g.a_scales = scales;
+  g.b_scales = b_scales;
+  g.d = static_cast<uint8_t*>(d);
+  g.status = status;
+  g.M = M;
+  g.N = N;
+  g.K = K;
+  g.out_fp32 = out_fp32;
+  StreamArgs q{};
+  q.x = static_cast<const uint8_t*>(a);
+  q.nslices = M * K / 16;
+  q.codes = codes;
+  q.scales = scales;
+  q.smap.bpr = K / 32;
+  q.smap.nct = (K / 32 + 3) / 4;
+  q.smap.inv = 1.0 / static_cast<double>(K / 32);
+  switch (a_rule) {
+    case kCeil: return noalloc_rule<kCeil>(wide, one_wave, tmA, tmB, g, q, ready, st);
+    case kOasRule: return noalloc_rule<kOasRule>(wide, one_wave, tmA, tmB, g, q, ready, st);
+    case kOas: return noalloc_rule<kOas>(wide, one_wave, tmA, tmB, g, q, ready, st);
+    default: return noalloc_rule<kFloor>(wide, one_wave, tmA, tmB, g, q, ready, st);
+  }
 }
 
 }  // namespace mxk

@@ -40,6 +40,12 @@ cudaError_t launch_gemm(const void* a, const uint8_t* a_scales, int a_rule, bool
                         const void* b_codes, const uint8_t* b_scales, int64_t M, int64_t N,
                         int64_t K, int out_fp32, void* d, void* a_codes_out,
                         uint8_t* a_scales_out, int* status, cudaStream_t st);
+// mx_quant_gemm_noalloc: the staged quantize + GEMM with its scratch in the
+// library's fixed device array (noalloc_fits: the problem fits it).
+bool noalloc_fits(int64_t M, int64_t K);
+cudaError_t launch_quant_gemm_noalloc(const void* a, int a_rule, const void* b_codes,
+                                      const uint8_t* b_scales, int64_t M, int64_t N, int64_t K,
+                                      int out_fp32, void* d, int* status, cudaStream_t st);
 cudaError_t launch_block_error(const void* x, int64_t n, int fmt, int scaling, float* block_sse,
                                double* totals, cudaStream_t st);
 

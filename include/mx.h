@@ -133,7 +133,8 @@ typedef enum {
   MX_ERR_SHAPE = 2,       /* cols % 32 != 0, or cols % 128 != 0 with MBS ([AX] 2) */
   MX_ERR_ALIGN = 3,       /* a pointer below its stated alignment */
   MX_ERR_UNSUPPORTED = 4, /* unknown format/scaling, or a scaling the format lacks */
-  MX_ERR_CUDA = 5         /* a kernel launch or stream operation failed */
+  MX_ERR_CUDA = 5,        /* a kernel launch or stream operation failed */
+  MX_ERR_TOO_LARGE = 6    /* mx_quant_gemm_noalloc: the problem exceeds its fixed scratch */
 } mx_status_t;
 
 /* Quantize ([VL] MXFP8/MXFP4 sections; [UP] 2.A/2.B for the scaling modes).
@@ -262,6 +263,33 @@ int mx_gemm(const void* a_codes, const uint8_t* a_scales, const void* b_codes,
 int mx_quant_gemm(const void* a_bf16, int scaling, const void* b_codes, const uint8_t* b_scales,
                   int64_t M, int64_t N, int64_t K, int out_fp32, void* d, void* a_codes_out,
                   uint8_t* a_scales_out, int* status, void* stream);
+
+/* mx_quant_gemm without allocation. The paper has no counterpart: this entry
+ * point serves callers that may not allocate device memory while they run,
+ * such as a serving process that reserves all its device memory at start-up
+ * and keeps it fixed, or a runtime without stream-ordered memory pools. The
+ * default mx_quant_gemm takes A's quantized form and its per-band counters
+ * from a pool; this one takes them from one array of
+ * MX_NOALLOC_SCRATCH_BYTES in the library's device memory, which every GPU
+ * that loads the library holds until the process exits. Same arguments,
+ * result and errors as mx_quant_gemm in its default (staged) form, without
+ * A's output buffers or the on-chip flag (out_fp32 is 0 or 1), and
+ *  - MX_ERR_TOO_LARGE unless the scratch fits:
+ *      M K / 2 (codes, rounded up to 256) + ceil(M / 128) K * 4 (tiled
+ *      scales, rounded up to 256) + 8 ceil(M / 128) (counters)
+ *      <= MX_NOALLOC_SCRATCH_BYTES;
+ *    e.g. 4096 x 3072 fits, 8192 x 8192 does not.
+ *  - The first call on a device looks up the array's device address
+ *    (cudaGetSymbolAddress) with that device current; make it before any
+ *    stream capture.
+ *  - Every call shares the array and leaves its bytes there; each call
+ *    clears, on its stream, the parts that must start at zero. Calls that
+ *    overlap on the GPU (other streams, other host threads) race on it and
+ *    give wrong results: order them on one stream or with events. */
+#define MX_NOALLOC_SCRATCH_BYTES (9u << 20)
+int mx_quant_gemm_noalloc(const void* a_bf16, int scaling, const void* b_codes,
+                          const uint8_t* b_scales, int64_t M, int64_t N, int64_t K, int out_fp32,
+                          void* d, int* status, void* stream);
 
 /* Static description of a status code (never NULL). */
 const char* mx_status_string(int status);

@@ -39,7 +39,7 @@ def test_library_exports_every_declared_symbol(mx):
 
 
 def test_status_strings(mx):
-    for s in range(6):
+    for s in range(7):
         assert mx.mx_status_string(s)
     assert mx.mx_status_string(99) == "unknown status"
     assert mx.mx_version() >> 16 == 1
@@ -122,6 +122,23 @@ def test_other_entry_points_validate(mx):
     assert mx.mx_block_error(A, 4, 32, 0, 0, None, A + 4, 0) == ALIGN
     assert mx.mx_block_error(A, 4, 32, 0, 0, A + 2, A, 0) == ALIGN
     assert mx.mx_block_error(A, 4, 32, 1, 0x20, None, A, 0) == UNSUPPORTED
+
+
+def test_noalloc_quant_gemm_validates_and_refuses_what_its_scratch_cannot_hold(mx):
+    """The no-allocation quantize + GEMM checks its arguments like mx_quant_gemm
+    and refuses problems whose scratch exceeds its fixed array, before any
+    CUDA call."""
+    TOO_LARGE = 6
+    f = mx.mx_quant_gemm_noalloc
+    assert f(A, 0, A, A, 8192, 64, 8192, 0, A, None, 0) == TOO_LARGE      # 32 MiB of codes
+    assert f(A, 0, A, A, 1, 64, 2 ** 22, 0, A, None, 0) == TOO_LARGE      # one padded band of scales
+    assert f(A, 0x10, A, A, 128, 64, 256, 0, A, None, 0) == UNSUPPORTED   # MBS: no
+    assert f(A, 0, A, A, 128, 60, 256, 0, A, None, 0) == SHAPE            # N % 8
+    assert f(A, 0, A, A, 128, 64, 384, 0, A, None, 0) == SHAPE            # K % 256
+    assert f(A, 0, A, A, 128, 64, 256, 1 << 9, A, None, 0) == INVALID     # no on-chip flag
+    assert f(A + 16, 0, A, A, 128, 64, 256, 0, A, None, 0) == ALIGN       # bf16 A: 32 bytes
+    assert f(None, 0, A, A, 128, 64, 256, 0, A, None, 0) == INVALID
+    assert f(A, 0, A, A, 0, 64, 256, 0, None, None, 0) == OK              # M == 0: nothing
 
 
 def test_binding_refuses_cpu_tensors_for_device_only_calls(mx):
