@@ -124,6 +124,28 @@ def test_other_entry_points_validate(mx):
     assert mx.mx_block_error(A, 4, 32, 1, 0x20, None, A, 0) == UNSUPPORTED
 
 
+def test_gemm_entry_points_validate(mx):
+    """Both GEMM entry points check shapes, flags and alignment before any
+    CUDA call; the on-chip flag is taken off out_fp32 before the check."""
+    on_chip = mx.GEMM_A_ON_CHIP
+    g, q = mx.mx_gemm, mx.mx_quant_gemm
+    assert g(A, A, A, A, 128, 64, 384, 0, A, None, 0) == SHAPE                  # K % 256
+    assert g(A, A, A, A, 128, 60, 256, 0, A, None, 0) == SHAPE                  # N % 8
+    assert g(A, A, A, A, 128, 64, 256, 2, A, None, 0) == INVALID                # out_fp32
+    assert g(A, A, A, A, 128, 64, 256, on_chip, A, None, 0) == INVALID          # no flag here
+    assert g(A + 8, A, A, A, 128, 64, 256, 0, A, None, 0) == ALIGN              # codes: 16 B
+    assert g(A, None, A, A, 128, 64, 256, 0, A, None, 0) == INVALID
+    assert g(A, A, A, A, -1, 64, 256, 0, A, None, 0) == INVALID
+    assert g(None, None, None, None, 0, 64, 256, 0, None, None, 0) == OK         # M == 0
+    assert q(A, 0x10, A, A, 128, 64, 256, 0, A, None, None, None, 0) == UNSUPPORTED   # MBS
+    assert q(A, 0, A, A, 128, 64, 384, on_chip, A, None, None, None, 0) == SHAPE
+    assert q(A, 0, A, A, 128, 64, 256, 2 | on_chip, A, None, None, None, 0) == INVALID
+    assert q(A + 16, 0, A, A, 128, 64, 256, on_chip | 1, A, None, None, None, 0) == ALIGN
+    assert q(A, 0, A, A, 128, 64, 256, 0, A, A + 8, None, None, 0) == ALIGN     # codes out
+    assert q(A, 0, A, A, 128, 64, 256, 0, A, None, A + 8, None, 0) == ALIGN     # scales out
+    assert q(A, 0, A, A, 128, 64, 256, 0, A, None, None, A + 2, 0) == ALIGN     # status
+
+
 def test_noalloc_quant_gemm_validates_and_refuses_what_its_scratch_cannot_hold(mx):
     """The no-allocation quantize + GEMM checks its arguments like mx_quant_gemm
     and refuses problems whose scratch exceeds its fixed array, before any
