@@ -975,33 +975,49 @@ cudaError_t launch_staged_sync(const CUtensorMap& tmA, const CUtensorMap& tmB, c
 }
 
 // The staged form for one rounding rule: the grid-barrier kernel when the
-// GEMM's tiles fit in one wave, else the overlapped kernel, its per-m-tile
-// ready counts in stream-ordered scratch (zeroed before the launch, released
-// after it).
+// GEMM's tiles fit in one wave, else the overlapped kernel with its per-m-tile
+// ready counts at `ready` (zero on the stream before the launch).
 template <int RULE>
-cudaError_t launch_staged_rule(bool wide, const CUtensorMap& tmA, const CUtensorMap& tmB,
-                               const GemmArgs& g, const StreamArgs& q, cudaStream_t st) {
-  cudaError_t e = cudaSuccess;
-  const int sms = sm_count_of_current_device(&e);
-  if (e != cudaSuccess) return e;
-  const int64_t bn = wide ? 256 : 128;
-  const int64_t mtiles = (g.M + kGemmBM - 1) / kGemmBM;
-  if (mtiles * ((g.N + bn - 1) / bn) <= sms)
+cudaError_t launch_staged_rule(bool wide, bool one_wave, const CUtensorMap& tmA,
+                               const CUtensorMap& tmB, const GemmArgs& g, const StreamArgs& q,
+                               unsigned long long* ready, cudaStream_t st) {
+  if (one_wave)
     return wide ? launch_staged_sync<256, 4, RULE>(tmA, tmB, g, q, st)
                 : launch_staged_sync<128, 6, RULE>(tmA, tmB, g, q, st);
-  const size_t ready_bytes = static_cast<size_t>(mtiles) * 8;
-  cudaMemPool_t pool = nullptr;
-  e = scratch_pool(&pool);
-  if (e != cudaSuccess) return e;
-  unsigned long long* ready = nullptr;
-  e = cudaMallocFromPoolAsync(reinterpret_cast<void**>(&ready), ready_bytes, pool, st);
-  if (e != cudaSuccess) return e;
-  e = cudaMemsetAsync(ready, 0, ready_bytes, st);
-  if (e == cudaSuccess)
-    e = wide ? launch_staged<256, 4, RULE>(tmA, tmB, g, q, ready, st)
-             : launch_staged<128, 6, RULE>(tmA, tmB, g, q, ready, st);
-  const cudaError_t ef = cudaFreeAsync(ready, st);
-  return e != cudaSuccess ? e : ef;
+  return wide ? launch_staged<256, 4, RULE>(tmA, tmB, g, q, ready, st)
+              : launch_staged<128, 6, RULE>(tmA, tmB, g, q, ready, st);
+}
+
+// Where a staged launch keeps A's quantized form and its band counters:
+// codes [M, K/2], then (256-byte aligned) the tiled scales, then the counters
+// (one per 128-row band), each part present only where needed.
+struct StagedScratch {
+  size_t scales, ready, end;
+};
+
+StagedScratch staged_scratch(int64_t M, int64_t K, bool codes, bool scales, bool ready) {
+  const auto up = [](size_t v) { return (v + 255) & ~static_cast<size_t>(255); };
+  const size_t mtiles = static_cast<size_t>((M + kGemmBM - 1) / kGemmBM);
+  StagedScratch l{};
+  l.scales = codes ? up(static_cast<size_t>(M) * static_cast<size_t>(K / 2)) : 0;
+  l.ready = l.scales + (scales ? up(mtiles * static_cast<size_t>(K / 128) * kSfTile) : 0);
+  l.end = l.ready + (ready ? mtiles * 8 : 0);
+  return l;
+}
+
+// Zeroes, on the stream, what a staged launch reads before writing: the
+// padding rows of the last band of `scales` (when M is not a multiple of
+// 128) and the band counters at `ready`; a NULL pointer skips its part.
+cudaError_t clear_staged(uint8_t* scales, unsigned long long* ready, int64_t M, int64_t K,
+                         cudaStream_t st) {
+  const int64_t mtiles = (M + kGemmBM - 1) / kGemmBM;
+  if (scales && M % kGemmBM != 0) {
+    const size_t band = static_cast<size_t>(K / 128) * kSfTile;
+    const cudaError_t e = cudaMemsetAsync(scales + (mtiles - 1) * band, 0, band, st);
+    if (e != cudaSuccess) return e;
+  }
+  if (ready) return cudaMemsetAsync(ready, 0, static_cast<size_t>(mtiles) * 8, st);
+  return cudaSuccess;
 }
 
 template <int BN, int S, int CL, int RULE>
@@ -1101,32 +1117,30 @@ cudaError_t launch_gemm(const void* a, const uint8_t* a_scales, int a_rule, bool
   }
   // Staged: A is quantized into the caller's buffers, or (where the caller
   // gives none) into stream-ordered scratch, and the GEMM runs on them in the
-  // same cooperative launch.
-  const int64_t mtiles = (M + kGemmBM - 1) / kGemmBM;
-  const size_t scale_bytes = static_cast<size_t>(mtiles * (K / 128)) * kSfTile;
+  // same cooperative launch; one scratch allocation holds what the caller
+  // does not give and the band counters.
+  cudaError_t e = cudaSuccess;
+  const int sms = sm_count_of_current_device(&e);
+  if (e != cudaSuccess) return e;
+  const int64_t bn = wide ? 256 : 128;
+  const bool one_wave = ((M + kGemmBM - 1) / kGemmBM) * ((N + bn - 1) / bn) <= sms;
   uint8_t* codes = static_cast<uint8_t*>(a_codes_out);
   uint8_t* scales = a_scales_out;
-  uint8_t* scratch[2] = {nullptr, nullptr};
-  cudaError_t e = cudaSuccess;
-  if (!codes || !scales) {
+  const StagedScratch l = staged_scratch(M, K, !codes, !scales, !one_wave);
+  uint8_t* scratch = nullptr;
+  if (l.end > 0) {
     cudaMemPool_t pool = nullptr;
     e = scratch_pool(&pool);
     if (e != cudaSuccess) return e;
-    if (!codes) {
-      e = cudaMallocFromPoolAsync(reinterpret_cast<void**>(&scratch[0]),
-                                  static_cast<size_t>(M * K / 2), pool, st);
-      codes = scratch[0];
-    }
-    if (e == cudaSuccess && !scales) {
-      e = cudaMallocFromPoolAsync(reinterpret_cast<void**>(&scratch[1]), scale_bytes, pool, st);
-      scales = scratch[1];
-      // the padding rows of the last band are read by the MMA as zero bytes
-      if (e == cudaSuccess && M % kGemmBM != 0) {
-        const size_t band = static_cast<size_t>(K / 128) * kSfTile;
-        e = cudaMemsetAsync(scratch[1] + scale_bytes - band, 0, band, st);
-      }
-    }
+    e = cudaMallocFromPoolAsync(reinterpret_cast<void**>(&scratch), l.end, pool, st);
+    if (e != cudaSuccess) return e;
+    if (!codes) codes = scratch;
   }
+  // (the caller's scales had their padding cleared by the API layer)
+  const bool own_scales = !scales;
+  if (own_scales) scales = scratch + l.scales;
+  auto* ready = one_wave ? nullptr : reinterpret_cast<unsigned long long*>(scratch + l.ready);
+  e = clear_staged(own_scales ? scales : nullptr, ready, M, K, st);
   if (e == cudaSuccess && !code_tmap(&tmA, codes, M, K, kGemmBM)) e = cudaErrorInvalidValue;
   if (e == cudaSuccess) {
     StreamArgs q{};
@@ -1139,15 +1153,16 @@ cudaError_t launch_gemm(const void* a, const uint8_t* a_scales, int a_rule, bool
     q.smap.inv = 1.0 / static_cast<double>(K / 32);
     g.a_scales = scales;
     switch (a_rule) {
-      case kCeil: e = launch_staged_rule<kCeil>(wide, tmA, tmB, g, q, st); break;
-      case kOasRule: e = launch_staged_rule<kOasRule>(wide, tmA, tmB, g, q, st); break;
-      case kOas: e = launch_staged_rule<kOas>(wide, tmA, tmB, g, q, st); break;
-      default: e = launch_staged_rule<kFloor>(wide, tmA, tmB, g, q, st);
+      case kCeil: e = launch_staged_rule<kCeil>(wide, one_wave, tmA, tmB, g, q, ready, st); break;
+      case kOasRule:
+        e = launch_staged_rule<kOasRule>(wide, one_wave, tmA, tmB, g, q, ready, st);
+        break;
+      case kOas: e = launch_staged_rule<kOas>(wide, one_wave, tmA, tmB, g, q, ready, st); break;
+      default: e = launch_staged_rule<kFloor>(wide, one_wave, tmA, tmB, g, q, ready, st);
     }
   }
-  for (uint8_t* p : scratch) {
-    if (!p) continue;
-    const cudaError_t ef = cudaFreeAsync(p, st);
+  if (scratch) {
+    const cudaError_t ef = cudaFreeAsync(scratch, st);
     if (e == cudaSuccess) e = ef;
   }
   return e;
@@ -1161,37 +1176,6 @@ cudaError_t launch_gemm(const void* a, const uint8_t* a_scales, int a_rule, bool
 // stream-ordered pool. This variant takes them from one array in the
 // library's device memory, of fixed size; every call shares it.
 
-namespace {
-
-// codes [M, K/2], then (256-byte aligned) the tiled scales, then the band
-// counters; the total must fit the array
-struct NoAllocLayout {
-  size_t scales, scale_bytes, ready, end;
-};
-
-NoAllocLayout noalloc_layout(int64_t M, int64_t K) {
-  const auto up = [](size_t v) { return (v + 255) & ~static_cast<size_t>(255); };
-  const size_t mtiles = static_cast<size_t>((M + kGemmBM - 1) / kGemmBM);
-  NoAllocLayout l{};
-  l.scales = up(static_cast<size_t>(M) * static_cast<size_t>(K / 2));
-  l.scale_bytes = mtiles * static_cast<size_t>(K / 128) * kSfTile;
-  l.ready = up(l.scales + l.scale_bytes);
-  l.end = l.ready + mtiles * 8;
-  return l;
-}
-
-template <int RULE>
-cudaError_t noalloc_rule(bool wide, bool one_wave, const CUtensorMap& tmA, const CUtensorMap& tmB,
-                         const GemmArgs& g, const StreamArgs& q, unsigned long long* ready,
-                         cudaStream_t st) {
-  if (one_wave)
-    return wide ? launch_staged_sync<256, 4, RULE>(tmA, tmB, g, q, st)
-                : launch_staged_sync<128, 6, RULE>(tmA, tmB, g, q, st);
-  return wide ? launch_staged<256, 4, RULE>(tmA, tmB, g, q, ready, st)
-              : launch_staged<128, 6, RULE>(tmA, tmB, g, q, ready, st);
-}
-
-}  // namespace
 }  // namespace mxk
 
 // The array (file scope). Host code cannot use its name as an address: the
@@ -1200,8 +1184,11 @@ static __device__ __align__(256) uint8_t mx_noalloc_scratch[MX_NOALLOC_SCRATCH_B
 
 namespace mxk {
 
+// codes [M, K/2], then (256-byte aligned) the tiled scales, then the band
+// counters; the total must fit the array.
 bool noalloc_fits(int64_t M, int64_t K) {
-  return noalloc_layout(M, K).end <= static_cast<size_t>(MX_NOALLOC_SCRATCH_BYTES);
+  return staged_scratch(M, K, true, true, true).end <=
+         static_cast<size_t>(MX_NOALLOC_SCRATCH_BYTES);
 }
 
 namespace {
@@ -1236,27 +1223,19 @@ cudaError_t launch_quant_gemm_noalloc(const void* a, int a_rule, const void* b_c
   uint8_t* base = nullptr;
   cudaError_t e = noalloc_scratch(&base);
   if (e != cudaSuccess) return e;
-  const NoAllocLayout l = noalloc_layout(M, K);
+  const StagedScratch l = staged_scratch(M, K, true, true, true);
   uint8_t* codes = base;
   uint8_t* scales = base + l.scales;
-  auto* ready = reinterpret_cast<unsigned long long*>(base + l.ready);
   const bool wide = N > 128 && ((M + kGemmBM - 1) / kGemmBM) * ((N + 255) / 256) >= 148;
   const int64_t bn = wide ? 256 : 128;
-  const int64_t mtiles = (M + kGemmBM - 1) / kGemmBM;
-  int sms = sm_count_of_current_device(&e);
+  const int sms = sm_count_of_current_device(&e);
   if (e != cudaSuccess) return e;
-  const bool one_wave = mtiles * ((N + bn - 1) / bn) <= sms;
+  const bool one_wave = ((M + kGemmBM - 1) / kGemmBM) * ((N + bn - 1) / bn) <= sms;
+  auto* ready = one_wave ? nullptr : reinterpret_cast<unsigned long long*>(base + l.ready);
   // the array keeps the previous call's bytes: zero what is read before it
   // is written (the padding rows of the last band of scales, the counters)
-  if (M % kGemmBM != 0) {
-    const size_t band = static_cast<size_t>(K / 128) * kSfTile;
-    e = cudaMemsetAsync(scales + l.scale_bytes - band, 0, band, st);
-    if (e != cudaSuccess) return e;
-  }
-  if (!one_wave) {
-    e = cudaMemsetAsync(ready, 0, static_cast<size_t>(mtiles) * 8, st);
-    if (e != cudaSuccess) return e;
-  }
+  e = clear_staged(scales, ready, M, K, st);
+  if (e != cudaSuccess) return e;
   CUtensorMap tmA{}, tmB{};
   if (!code_tmap(&tmB, b_codes, N, K, wide ? 256 : 128)) return cudaErrorInvalidValue;
   if (!code_tmap(&tmA, codes, M, K, kGemmBM)) return cudaErrorInvalidValue;
@@ -1279,10 +1258,10 @@ cudaError_t launch_quant_gemm_noalloc(const void* a, int a_rule, const void* b_c
   q.smap.nct = (K / 32 + 3) / 4;
   q.smap.inv = 1.0 / static_cast<double>(K / 32);
   switch (a_rule) {
-    case kCeil: return noalloc_rule<kCeil>(wide, one_wave, tmA, tmB, g, q, ready, st);
-    case kOasRule: return noalloc_rule<kOasRule>(wide, one_wave, tmA, tmB, g, q, ready, st);
-    case kOas: return noalloc_rule<kOas>(wide, one_wave, tmA, tmB, g, q, ready, st);
-    default: return noalloc_rule<kFloor>(wide, one_wave, tmA, tmB, g, q, ready, st);
+    case kCeil: return launch_staged_rule<kCeil>(wide, one_wave, tmA, tmB, g, q, ready, st);
+    case kOasRule: return launch_staged_rule<kOasRule>(wide, one_wave, tmA, tmB, g, q, ready, st);
+    case kOas: return launch_staged_rule<kOas>(wide, one_wave, tmA, tmB, g, q, ready, st);
+    default: return launch_staged_rule<kFloor>(wide, one_wave, tmA, tmB, g, q, ready, st);
   }
 }
 
