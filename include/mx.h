@@ -251,7 +251,9 @@ int mx_bat_quantize(const void* x, int64_t rows, int64_t cols, int a_dim, const 
  *    quantizes, then a grid-wide barrier; otherwise six extra warps per CTA
  *    quantize while the GEMM runs, each 128-row band of A counted as it
  *    completes (a per-band counter in the scratch) so that its tiles start
- *    as soon as their band is ready.
+ *    as soon as their band is ready. The scratch's stream-ordered
+ *    allocation costs about 2 us of GPU time per call; small, latency-bound
+ *    calls save it by passing both buffers.
  *  - out_fp32 | MX_GEMM_A_ON_CHIP: A is quantized inside the GEMM's prologue
  *    and the GEMM never reads it from memory; a thread-block cluster of up
  *    to 4 CTAs shares each quantized tile through distributed shared memory.
