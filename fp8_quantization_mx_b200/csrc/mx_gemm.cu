@@ -1,5 +1,5 @@
-// Block-scaled MXFP4 GEMM on the sm_100 tensor cores, with the MX
-// quantization of the bf16 activations fused into its prologue.
+// Block-scaled MXFP4 GEMM on the sm_100 tensor cores, and the MX
+// quantization of its bf16 activations in the same launch.
 //
 //   D[M, N] = A[M, K] . B[N, K]^T,   A and B MXFP4 (E2M1 elements, one E8M0
 //   scale per 32 elements along K), fp32 accumulation in tensor memory.
@@ -16,25 +16,29 @@
 // swizzle atom), in an S-stage shared-memory ring:
 //   warp 0     TMA: B's code tile (2-D tensor map, 128-byte swizzle) and B's
 //              scale tiles (bulk copies of the tiled layout MX_SCALES_MMA
-//              writes); A's as well when A comes pre-quantized
+//              writes); A's as well when A is in memory quantized
 //   warp 1     TMEM allocation; one thread copies the stage's scale tiles
 //              into TMEM (tcgen05.cp) and issues the four MMAs of the
 //              K-block, then commits to the stage's "empty" barrier
-//   warps 2-9  (fused) quantize A's 128 x 256 bf16 tile of the K-block with
-//              the streaming kernels' per-slice quantizer straight from
-//              global memory into the swizzled operand tile and the scale
-//              tile in shared memory: the quantized activations never reach
-//              HBM; then the epilogue of the tile
-//   warps 2-9  (pre-quantized A) the epilogue
-// Epilogue: TMEM -> registers (tcgen05.ld, one row per thread, two warps
-// per 32-lane quarter splitting the columns), the accumulator released to
-// the next tile, then fp32 -> bf16 (or fp32) -> global.
-// The kernel is persistent (one CTA per SM looping over tiles), so the next
-// tile's loads overlap the previous tile's epilogue.
+//   warps 2-9  the epilogue: TMEM -> registers (tcgen05.ld, one row per
+//              thread, two warps per 32-lane quarter splitting the columns),
+//              the accumulator released to the next tile, then fp32 -> bf16
+//              (or fp32) -> global
+// The kernels are persistent (one CTA per SM looping over tiles), so the next
+// tile's loads overlap the previous tile's epilogue. Four kernels share this
+// body:
+//   gemm_kernel              A pre-quantized
+//   gemm_staged_kernel       bf16 A: six more warps per CTA quantize A into
+//                            global codes and scales while the GEMM runs on
+//                            the 128-row bands already counted complete
+//   gemm_staged_sync_kernel  bf16 A, one wave of tiles: every warp quantizes,
+//                            a grid barrier, then the GEMM
+//   gemm_fused_kernel        bf16 A quantized on chip in the prologue by the
+//                            work warps, shared across a thread-block cluster
 //
-// Every wait is bounded in time (mbar_wait): a wait that runs out sets the
-// caller's status word and the CTA drains its in-flight copies and MMAs,
-// frees its TMEM and returns.
+// Every wait is bounded in time (mbar_wait, counter_wait): a wait that runs
+// out sets the caller's status word and the CTA drains its in-flight copies
+// and MMAs, frees its TMEM and returns.
 
 #include <cooperative_groups.h>
 #include <cuda.h>
