@@ -168,7 +168,20 @@ __device__ __forceinline__ void process_slice(const StreamArgs& a, const V16& v,
   const BlockScale s = decide_scale<FMT, RULE, MBS>(v, pa, k);
   // codes for every lane before any divergent branch (see codes_fp4)
   uint4 codes = make_uint4(0, 0, 0, 0);
-  if (OP != kOpFakeBwd) codes = lane_codes<FMT, MBS>(v, s);
+  // block error of plain E2M1: the slice is scaled once, for the codes (as
+  // codes_fp4 scales it) and for the error arithmetic below
+  constexpr bool kScaleOnce = OP == kOpError && FMT == kFmtE2M1 && MBS == kMbsNone;
+  V16 scaled;
+  if constexpr (kScaleOnce) {
+    scaled = scale_slice(v, s.nonfinite ? 127 : s.byte);
+    uint2 c;
+    if (s.nonfinite) c = nonfinite_e2m1_16(v);
+    else if (s.have_codes) c = make_uint2(s.codes.x, s.codes.y);
+    else c = enc_e2m1_16(scaled);
+    codes = make_uint4(c.x, c.y, 0, 0);
+  } else if (OP != kOpFakeBwd) {
+    codes = lane_codes<FMT, MBS>(v, s);
+  }
 
   if (OP == kOpQuant) {
     if (FMT == kFmtE2M1) {
@@ -234,7 +247,9 @@ __device__ __forceinline__ void process_slice(const StreamArgs& a, const V16& v,
     const int bs = s.nonfinite ? 127 : s.byte;
     const int E = bs - 127;
     const double p2 = __longlong_as_double(static_cast<long long>(2 * E + 1023) << 52);
-    const V16 sl = scale_slice(v, bs);
+    V16 sl;
+    if constexpr (kScaleOnce) sl = scaled;
+    else sl = scale_slice(v, bs);
     float ad[4] = {0.0f, 0.0f, 0.0f, 0.0f}, ax[4] = {0.0f, 0.0f, 0.0f, 0.0f};
     if (FMT == kFmtE2M1 && MBS == kMbsNone) {
       // |s| - |g| (the code keeps the sign of s) is exact in bf16 too: for s
