@@ -876,11 +876,15 @@ __device__ __forceinline__ uint32_t even_of_adjacent(uint32_t lo, uint32_t hi) {
 // even one is the round-to-nearest-even result.
 __device__ __forceinline__ uint2 enc_mbs_cvt_16(const V16& x, int b, int k) {
   const FactorBracket fb = factor_bracket(k);
-  const V16 s = scale_slice(x, b);
+  // 2^-E folded into the bracket: for a finite block E <= 125 (b <= 252), so
+  // L 2^-E and H 2^-E are normal floats, exact, and x (L 2^-E) rounds as
+  // (x 2^-E) L does wherever x 2^-E is a normal number; below that (an
+  // element under 2^-126 of the scale) both give a zero code of x's sign
+  const float p = inv_scale_from_byte(b);
   float e[16], lo[16], hi[16];
 #pragma unroll
-  for (int i = 0; i < 16; ++i) e[i] = elem(s, i);
-  bracket_products<16>(e, fb.L, fb.H, lo, hi);
+  for (int i = 0; i < 16; ++i) e[i] = elem(x, i);
+  bracket_products<16>(e, fb.L * p, fb.H * p, lo, hi);
   return make_uint2(even_of_adjacent(cvt_e2m1_f8(lo), cvt_e2m1_f8(hi)),
                     even_of_adjacent(cvt_e2m1_f8(lo + 8), cvt_e2m1_f8(hi + 8)));
 }
